@@ -1,0 +1,19 @@
+"""fp64 CPU oracle for the Qwen3 attention core.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the library.  It shares no code with
+the CUDA path.  Every function is pinned by `tests/test_oracle_pins.py`
+(closed forms, invariants, special cases and brute force).
+"""
+from .attention import (  # noqa: F401
+    bf16_round,
+    build_cache_k,
+    decode_ref,
+    kv_cache_values_per_token,
+    prefill_ref,
+    qk_prologue,
+    rms_norm,
+    rope,
+    rope_inv_freq,
+)
+from .loops import decode_loops, prefill_loops  # noqa: F401

@@ -1,0 +1,194 @@
+"""fp64 CPU oracle for the Qwen3 attention core (QK-Norm, RoPE, causal GQA).
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module.  It shares no code with the CUDA
+library: it is a plain restatement of the definitions on the pages, in numpy
+float64, with one matrix product per block of query rows as the only library
+step.
+
+What it computes, and where each step is defined:
+
+  1. QK-Norm, per head vector x of length d:
+        y = g * x / sqrt(mean(x^2) + eps)
+     "Qwen3 Architecture Layer-by-Layer", Primitives: Qwen3RMSNorm;
+     "Hand-Writing a Vision-Language Model, Part 1", RMSNorm (the formula is
+     stated there in words: no mean subtraction, eps inside the root);
+     "Qwen 3 From Scratch", In code.  It runs after the projection and before
+     RoPE ("Hand-Writing ... Part 1", step list 3-5).
+  2. RoPE, rotate-half pairing, for i < d/2:
+        inv_i = theta^(-2i/d),  a = pos * inv_i
+        y_i       = x_i cos a - x_{i+d/2} sin a
+        y_{i+d/2} = x_{i+d/2} cos a + x_i sin a
+     "Hand-Writing ... Part 1", RotaryEmbedding (RoPE); "Assembling a large
+     model from scratch", The complete code (rope_cos_sin, rotate_half,
+     apply_rope); "Qwen3 Architecture Layer-by-Layer", apply_rotary_pos_emb and
+     Qwen3RotaryEmbedding (inv_freq formula).  Angles are exact fp64 here.
+  3. Scores s_ij = q'_i . k'_j / sqrt(d); query head h reads KV head h // G,
+     G = Hq / Hkv ("Hand-Writing ... Part 1", repeat_kv; "Assembling a large
+     model", Attention.forward with repeat_interleave).
+  4. Causal mask on index: key j is visible to query i iff j <= i + (S - T),
+     i.e. tril(diagonal = S - T) ("Assembling a large model", Attention.forward
+     and the implementation notes below the code).
+  5. Softmax over visible keys, out_i = sum_j p_ij v_j; lse_i = natural log of
+     sum_j exp(s_ij) (the logsumexp of "Qwen3 Architecture Layer-by-Layer",
+     The cross-entropy math, applied to the scaled logits).
+  6. Decode: the new token sits at position L = cached length; its k is
+     normalised, rotated at L and appended, its v appended raw, and the query
+     attends to all L+1 keys ("Assembling a large model", KVCache.update and
+     Transformer.forward, start = cache.length).
+
+Readings where the pages leave a step open:
+  * No intermediate rounding: the pages' HF path casts to bf16 between the
+    norm and the gain; the oracle keeps everything in fp64.  `staged=True`
+    rounds q' and k' to bf16 once after RoPE, which is where the GPU path
+    rounds them before its bf16 MMAs; it is used only for the logsumexp bound.
+  * Rotate-half with theta from the argument (the page prose that speaks of
+    adjacent pairs and base 10000 contradicts every code block on the pages).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), as float64.
+
+    bfloat16 keeps 8 significant bits.  With x = m * 2^e, 0.5 <= |m| < 1, the
+    representable neighbours are multiples of 2^(e-8); rint rounds half to even.
+    Normal-range values only (the inputs here never approach under/overflow).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)
+    return np.ldexp(np.rint(m * 256.0) / 256.0, e)
+
+
+def rms_norm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """QK-Norm over the last axis: g * x / sqrt(mean(x^2) + eps)."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return np.asarray(g, dtype=np.float64) * (x / np.sqrt(ms + eps))
+
+
+def rope_inv_freq(d: int, theta: float) -> np.ndarray:
+    """inv_i = theta^(-2i/d) for i = 0 .. d/2-1."""
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(np.float64(theta), -2.0 * i / d)
+
+
+def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
+    """Rotate-half RoPE.  x [..., T, H, d]; pos broadcastable to [..., T]."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    half = d // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d, theta)  # [..., T, d/2]
+    c = np.cos(ang)[..., None, :]  # broadcast over heads
+    s = np.sin(ang)[..., None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def qk_prologue(x: np.ndarray, g: np.ndarray, pos: np.ndarray, theta: float, eps: float,
+                staged: bool = False) -> np.ndarray:
+    """QK-Norm then RoPE of raw head vectors x [..., T, H, d] at positions pos [..., T]."""
+    y = rope(rms_norm(x, g, eps), pos, theta)
+    return bf16_round(y) if staged else y
+
+
+def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray):
+    """Softmax attention of query rows over keys 0..limit[r] (inclusive).
+
+    qg [R, d] already-normed/rotated queries; kk, vv [S, d]; limit [R] int.
+    Returns out [R, d] and lse [R] (natural log, scaled logits).
+    """
+    d = qg.shape[-1]
+    s = (qg @ kk.T) / np.sqrt(np.float64(d))  # [R, S]
+    j = np.arange(kk.shape[0])
+    s = np.where(j[None, :] <= limit[:, None], s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    z = np.sum(e, axis=1, keepdims=True)
+    out = (e / z) @ vv
+    lse = (m + np.log(z))[:, 0]
+    return out, lse
+
+
+def prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, theta: float, eps: float,
+                rows=None, staged: bool = False, block: int = 256):
+    """Causal GQA prefill with the QK-Norm + RoPE prologue, in fp64.
+
+    q [B,T,Hq,d], k and v [B,T,Hkv,d], gains [d], pos [B,T] (any real arrays;
+    they are widened exactly to float64).  Returns out [B,T,Hq,d] and lse
+    [B,Hq,T].  With `rows` (a sorted int array of query indices) only those
+    rows are computed and the returned arrays are [B,len(rows),Hq,d] and
+    [B,Hq,len(rows)]; keys still run over every position the mask admits.
+    Query rows are processed in blocks so no T x T matrix is ever held.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((B, rows.size, Hq, d))
+    lse = np.zeros((B, Hq, rows.size))
+    for b in range(B):
+        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged)  # [T, Hkv, d]
+        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged)
+        for h in range(Hq):
+            hk = h // G
+            for r0 in range(0, rows.size, block):
+                rr = rows[r0:r0 + block]
+                top = int(rr.max()) + 1
+                o, l = _attend(qp[r0:r0 + block, h], kp[:top, hk], v[b, :top, hk], rr)
+                out[b, r0:r0 + block, h] = o
+                lse[b, h, r0:r0 + block] = l
+    return out, lse
+
+
+def build_cache_k(k_hist, k_norm_w, theta: float, eps: float) -> np.ndarray:
+    """Cache contents for a raw key history k_hist [L,Hkv,d]: QK-Norm and RoPE at
+    positions 0..L-1, rounded to bf16 (the cache's storage type), as float64."""
+    L = np.asarray(k_hist).shape[0]
+    return bf16_round(qk_prologue(k_hist, k_norm_w, np.arange(L), theta, eps))
+
+
+def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens,
+               theta: float, eps: float, seqs=None, staged: bool = False):
+    """One decode step over a KV cache, in fp64.
+
+    q [N,Hq,d], k_new and v_new [N,Hkv,d] raw; k_cache/v_cache indexable as
+    [n][Hkv, >=L_n, d] holding the already-normed/rotated keys and raw values;
+    cache_lens [N].  The new token sits at position L_n.  Returns out [n_sel,Hq,d]
+    and lse [n_sel,Hq] for the sequences in `seqs` (default: all).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    N, Hq, d = q.shape
+    Hkv = np.asarray(k_new).shape[1]
+    G = Hq // Hkv
+    seqs = range(N) if seqs is None else seqs
+    outs, lses = [], []
+    for n in seqs:
+        L = int(cache_lens[n])
+        qp = qk_prologue(q[n][None], q_norm_w, np.array([L]), theta, eps, staged)[0]     # [Hq, d]
+        kn = qk_prologue(np.asarray(k_new[n], dtype=np.float64)[None], k_norm_w, np.array([L]),
+                         theta, eps, staged)[0]                                            # [Hkv, d]
+        kc = np.asarray(k_cache[n], dtype=np.float64)
+        vc = np.asarray(v_cache[n], dtype=np.float64)
+        o = np.zeros((Hq, d))
+        ls = np.zeros(Hq)
+        for h in range(Hq):
+            hk = h // G
+            keys = np.concatenate([kc[hk, :L], kn[hk][None]], axis=0)
+            vals = np.concatenate([vc[hk, :L], np.asarray(v_new[n], dtype=np.float64)[hk][None]], axis=0)
+            oo, ll = _attend(qp[h][None], keys, vals, np.array([L]))
+            o[h], ls[h] = oo[0], ll[0]
+        outs.append(o)
+        lses.append(ls)
+    return np.stack(outs), np.stack(lses)
+
+
+def kv_cache_values_per_token(Hkv: int, d: int) -> int:
+    """Values one layer's cache holds per token: a key and a value per KV head
+    ("Qwen 3 From Scratch", Worked example: 2 x Hkv x d_head)."""
+    return 2 * Hkv * d

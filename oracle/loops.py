@@ -1,0 +1,82 @@
+"""Brute-force scalar-loop restatement of the attention core, for tiny shapes.
+
+TEST INFRASTRUCTURE ONLY (tests import it to pin the vectorised oracle).  Pure
+Python floats (IEEE double) and the math module; no numpy arithmetic.  Every
+step is written element by element in the order the pages give it:
+QK-Norm ("Qwen3 Architecture Layer-by-Layer", Qwen3RMSNorm), rotate-half RoPE
+("Hand-Writing a Vision-Language Model, Part 1", RotaryEmbedding), scores with
+the 1/sqrt(d) scale, the tril(diagonal=S-T) mask and an fp64 softmax
+("Assembling a large model from scratch", Attention.forward).
+"""
+from __future__ import annotations
+
+import math
+
+
+def _norm_rope(vec, gain, pos, theta, eps):
+    d = len(vec)
+    ms = sum(x * x for x in vec) / d
+    r = 1.0 / math.sqrt(ms + eps)
+    y = [gain[i] * vec[i] * r for i in range(d)]
+    half = d // 2
+    out = [0.0] * d
+    for i in range(half):
+        a = pos * theta ** (-2.0 * i / d)
+        c, s = math.cos(a), math.sin(a)
+        out[i] = y[i] * c - y[i + half] * s
+        out[i + half] = y[i + half] * c + y[i] * s
+    return out
+
+
+def prefill_loops(q, k, v, gq, gk, pos, theta, eps, S_minus_T=0):
+    """q[b][t][h][i], k/v[b][t][hk][i] nested lists (or arrays); returns
+    out[b][t][h][i] and lse[b][h][t] as nested lists."""
+    B, T, Hq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv = len(k[0][0])
+    G = Hq // Hkv
+    out = [[[[0.0] * d for _ in range(Hq)] for _ in range(T)] for _ in range(B)]
+    lse = [[[0.0] * T for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        kk = [[_norm_rope([float(x) for x in k[b][t][h]], gk, float(pos[b][t]), theta, eps)
+               for h in range(Hkv)] for t in range(T)]
+        for t in range(T):
+            for h in range(Hq):
+                qq = _norm_rope([float(x) for x in q[b][t][h]], gq, float(pos[b][t]), theta, eps)
+                hk = h // G
+                scores = []
+                for j in range(T):
+                    if j <= t + S_minus_T:
+                        scores.append(sum(qq[i] * kk[j][hk][i] for i in range(d)) / math.sqrt(d))
+                m = max(scores)
+                w = [math.exp(s - m) for s in scores]
+                z = sum(w)
+                for i in range(d):
+                    out[b][t][h][i] = sum(w[j] * float(v[b][j][hk][i]) for j in range(len(w))) / z
+                lse[b][h][t] = m + math.log(z)
+    return out, lse
+
+
+def decode_loops(q, k_new, v_new, gq, gk, k_cache, v_cache, lens, theta, eps):
+    """Decode one token per sequence, element by element.  k_cache[n][hk][j][i]
+    holds normed/rotated keys for j < lens[n]."""
+    N, Hq, d = len(q), len(q[0]), len(q[0][0])
+    Hkv = len(k_new[0])
+    G = Hq // Hkv
+    out = [[[0.0] * d for _ in range(Hq)] for _ in range(N)]
+    lse = [[0.0] * Hq for _ in range(N)]
+    for n in range(N):
+        L = int(lens[n])
+        kn = [_norm_rope([float(x) for x in k_new[n][hk]], gk, float(L), theta, eps) for hk in range(Hkv)]
+        for h in range(Hq):
+            hk = h // G
+            qq = _norm_rope([float(x) for x in q[n][h]], gq, float(L), theta, eps)
+            keys = [[float(x) for x in k_cache[n][hk][j]] for j in range(L)] + [kn[hk]]
+            vals = [[float(x) for x in v_cache[n][hk][j]] for j in range(L)] + [[float(x) for x in v_new[n][hk]]]
+            scores = [sum(qq[i] * key[i] for i in range(d)) / math.sqrt(d) for key in keys]
+            m = max(scores)
+            w = [math.exp(s - m) for s in scores]
+            z = sum(w)
+            for i in range(d):
+                out[n][h][i] = sum(w[j] * vals[j][i] for j in range(len(w))) / z
+            lse[n][h] = m + math.log(z)
+    return out, lse

@@ -1,0 +1,166 @@
+"""Seeded synthetic inputs for the Qwen3 attention core.
+
+This module only draws random numbers and rounds them to the storage dtypes.
+It holds none of the attention arithmetic (no normalisation, no rotation, no
+softmax): both the fp64 oracle and the CUDA path consume what it returns, and
+neither of them is imported here.
+
+Workload shapes follow the Qwen3 models described on the pages:
+  * Qwen3-0.6B: 16 query heads, 8 KV heads, head_dim 128 ("Qwen3 Architecture
+    Layer-by-Layer", config values; "Assembling a large model from scratch",
+    shape table).
+  * Qwen3-4B: 32 query heads, 8 KV heads, head_dim 128 ("Hand-Writing a
+    Vision-Language Model, Part 1", Attention: Grouped-Query Attention).
+  * The wide-GQA block of "Qwen 3 From Scratch", Worked example: 64 query
+    heads over 4 KV heads, head_dim 128.
+
+Value recipe (one numpy Generator, draws in this order): q, k, v ~ N(0,1);
+per-channel scales s_q, s_k with log(s) ~ U(log 0.5, log 4), shared by every
+head, token and batch row; gains g_q, g_k = 1 + 0.1 N(0,1) in fp32; then (for
+decode) the cached lengths L ~ U{1024..32768}.  q and k are multiplied by
+their scale vector, then q, k, v are rounded to bf16.  Positions are 0..T-1.
+Draws are made in float32 (numpy's float32 normal stream) to halve host memory
+on the 32768-token workload.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+HEAD_DIM = 128
+ROPE_THETA = 1.0e6
+RMS_EPS = 1.0e-6
+
+
+@dataclass(frozen=True)
+class PrefillShape:
+    name: str
+    B: int
+    T: int
+    Hq: int
+    Hkv: int
+    d: int = HEAD_DIM
+    theta: float = ROPE_THETA
+    eps: float = RMS_EPS
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    def causal_flops(self) -> float:
+        """QK^T and PV over the causal triangle only: 4*B*Hq*d*T(T+1)/2."""
+        return 4.0 * self.B * self.Hq * self.d * self.T * (self.T + 1) / 2.0
+
+
+@dataclass(frozen=True)
+class DecodeShape:
+    name: str
+    N: int
+    Hq: int
+    Hkv: int
+    d: int = HEAD_DIM
+    lmin: int = 1024
+    lmax: int = 32768
+    theta: float = ROPE_THETA
+    eps: float = RMS_EPS
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def cache_capacity(self) -> int:
+        """Slots per (sequence, KV head): the longest history plus the appended token."""
+        return self.lmax + 1
+
+
+PREFILL_SHAPES = {
+    "tiny": PrefillShape("tiny prefill B=1 T=128 Hq=16 Hkv=8", 1, 128, 16, 8),
+    "qwen3-0.6b": PrefillShape("Qwen3-0.6B-shaped prefill B=2 T=2048 Hq=16 Hkv=8", 2, 2048, 16, 8),
+    "qwen3-4b": PrefillShape("Qwen3-4B-shaped prefill B=1 T=8192 Hq=32 Hkv=8", 1, 8192, 32, 8),
+    "long-wide-gqa": PrefillShape("long-context wide-GQA prefill B=1 T=32768 Hq=64 Hkv=4", 1, 32768, 64, 4),
+}
+
+DECODE_SHAPES = {
+    "batched-decode": DecodeShape("batched decode N=64 Hq=32 Hkv=8 L~U[1024,32768]", 64, 32, 8),
+}
+
+
+def _bf16(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
+
+
+def _scales(rng: np.random.Generator, d: int) -> np.ndarray:
+    return np.exp(rng.uniform(np.log(0.5), np.log(4.0), size=d)).astype(np.float32)
+
+
+def _gains(rng: np.random.Generator, d: int) -> np.ndarray:
+    return (1.0 + 0.1 * rng.standard_normal(d)).astype(np.float32)
+
+
+def prefill_inputs(shape: PrefillShape, seed: int = 0) -> dict:
+    """Raw prefill inputs as CPU tensors.
+
+    q [B,T,Hq,d], k and v [B,T,Hkv,d] bf16; q_norm_w and k_norm_w [d] fp32;
+    pos [B,T] int32 holding 0..T-1 for every batch row.
+    """
+    B, T, Hq, Hkv, d = shape.B, shape.T, shape.Hq, shape.Hkv, shape.d
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, T, Hq, d), dtype=np.float32)
+    k = rng.standard_normal((B, T, Hkv, d), dtype=np.float32)
+    v = rng.standard_normal((B, T, Hkv, d), dtype=np.float32)
+    s_q, s_k = _scales(rng, d), _scales(rng, d)
+    g_q, g_k = _gains(rng, d), _gains(rng, d)
+    q *= s_q
+    k *= s_k
+    pos = np.broadcast_to(np.arange(T, dtype=np.int32), (B, T)).copy()
+    return {
+        "q": _bf16(q), "k": _bf16(k), "v": _bf16(v),
+        "q_norm_w": torch.from_numpy(g_q), "k_norm_w": torch.from_numpy(g_k),
+        "pos": torch.from_numpy(pos),
+    }
+
+
+def decode_step_inputs(shape: DecodeShape, seed: int = 0) -> dict:
+    """The new token of every sequence plus the cached lengths.
+
+    q [N,Hq,d], k_new and v_new [N,Hkv,d] bf16 (raw, before QK-Norm/RoPE);
+    gains [d] fp32; cache_lens [N] int32 ~ U{lmin..lmax}; the scale vector
+    s_k is returned too so that cache histories can be drawn like config k.
+    """
+    N, Hq, Hkv, d = shape.N, shape.Hq, shape.Hkv, shape.d
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((N, Hq, d), dtype=np.float32)
+    k = rng.standard_normal((N, Hkv, d), dtype=np.float32)
+    v = rng.standard_normal((N, Hkv, d), dtype=np.float32)
+    s_q, s_k = _scales(rng, d), _scales(rng, d)
+    g_q, g_k = _gains(rng, d), _gains(rng, d)
+    lens = rng.integers(shape.lmin, shape.lmax, size=N, endpoint=True).astype(np.int32)
+    q *= s_q
+    k *= s_k
+    return {
+        "q": _bf16(q), "k_new": _bf16(k), "v_new": _bf16(v),
+        "q_norm_w": torch.from_numpy(g_q), "k_norm_w": torch.from_numpy(g_k),
+        "cache_lens": torch.from_numpy(lens), "s_k": torch.from_numpy(s_k),
+    }
+
+
+def decode_history(shape: DecodeShape, n: int, length: int, s_k: torch.Tensor, seed: int = 0) -> dict:
+    """Raw history of sequence n: k_hist (scaled like k) and v_hist [length,Hkv,d] bf16.
+
+    Each sequence has its own child stream (seed, 1, n), so one sequence can be
+    drawn without drawing the others.  k_hist is raw: the cache stores it only
+    after QK-Norm and RoPE at positions 0..length-1.
+    """
+    rng = np.random.default_rng([seed, 1, n])
+    k = rng.standard_normal((length, shape.Hkv, shape.d), dtype=np.float32)
+    v = rng.standard_normal((length, shape.Hkv, shape.d), dtype=np.float32)
+    k *= s_k.numpy()
+    return {"k_hist": _bf16(k), "v_hist": _bf16(v)}
+
+
+def as_f64(t: torch.Tensor) -> np.ndarray:
+    """Exact widening of a bf16/fp32/int tensor to a float64 numpy array."""
+    return t.detach().to("cpu").to(torch.float64).numpy()

@@ -1,0 +1,285 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each check raises AssertionError on failure.  They look the oracle's functions
+up at call time (`A.<name>`), so `test_oracle_mutants.py` can plant a plausible
+mistake in the oracle and confirm that some check catches it.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle.attention as A
+import oracle.loops as Lp
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+THETA, EPS, D = 1.0e6, 1.0e-6, 128
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+def _gain(seed, d=D):
+    return 1.0 + 0.1 * np.random.default_rng(seed).standard_normal(d)
+
+
+def _inputs(B, T, Hq, Hkv, seed=0, d=D):
+    q = _rand((B, T, Hq, d), seed)
+    k = _rand((B, T, Hkv, d), seed + 1)
+    v = _rand((B, T, Hkv, d), seed + 2)
+    pos = np.broadcast_to(np.arange(T), (B, T)).copy()
+    return q, k, v, _gain(seed + 3, d), _gain(seed + 4, d), pos
+
+
+# ---------------------------------------------------------------- bf16 rounding
+def check_bf16_round_matches_torch():
+    """The oracle's own bf16 rounding equals torch's float32->bfloat16 conversion
+    (round to nearest even) on float32-representable values, ties included."""
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal(20000).astype(np.float32) * np.float32(50.0)
+    ties = (np.arange(1, 2001, dtype=np.float32) * np.float32(2 ** -8) + np.float32(1.0)).astype(np.float32)
+    x = np.concatenate([x, ties, -ties])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = A.bf16_round(x.astype(np.float64))
+    assert np.array_equal(got, ref), np.flatnonzero(got != ref)[:5]
+
+
+# ---------------------------------------------------------------- RMSNorm
+def check_rmsnorm_unit_gain_closed_form():
+    """With unit gain the output RMS is sqrt(ms / (ms + eps)) exactly."""
+    for seed, scale in [(0, 1.0), (1, 1e-3), (2, 30.0)]:
+        x = _rand((64, D), seed, scale)
+        y = A.rms_norm(x, np.ones(D), EPS)
+        ms = np.mean(x * x, axis=-1)
+        rms_y = np.sqrt(np.mean(y * y, axis=-1))
+        assert np.allclose(rms_y, np.sqrt(ms / (ms + EPS)), rtol=1e-13, atol=0)
+
+
+def check_rmsnorm_gain_and_no_centering():
+    """The gain multiplies channel-wise, and there is no mean subtraction: a
+    constant vector c*1 maps to sign(c) * g * |c|/sqrt(c^2+eps)."""
+    g = _gain(5)
+    for c in (2.0, -0.5):
+        y = A.rms_norm(np.full((1, D), c), g, EPS)
+        assert np.allclose(y[0], g * c / math.sqrt(c * c + EPS), rtol=1e-14)
+    x = _rand((3, D), 9)
+    assert np.allclose(A.rms_norm(x, g, EPS), g * A.rms_norm(x, np.ones(D), EPS), rtol=1e-14)
+
+
+# ---------------------------------------------------------------- RoPE
+def check_rope_inv_freq_golden():
+    gold = json.load(open(GOLDEN))["rope_inv_freq"]
+    inv = A.rope_inv_freq(gold["head_dim"], float(gold["rope_theta"]))
+    assert inv.shape == (gold["n_frequencies"],)
+    i = np.arange(gold["n_frequencies"])
+    assert np.allclose(inv, 10.0 ** (gold["base10_exponent_per_i"] * i), rtol=1e-13)
+    assert inv[0] == 1.0 and abs(inv[63] / 1.2409e-6 - 1) < 1e-4
+
+
+def check_rope_identity_at_pos0():
+    x = _rand((1, 4, 3, D), 11)
+    assert np.allclose(A.rope(x, np.zeros((1, 4)), THETA), x, rtol=0, atol=0)
+
+
+def check_rope_plane_rotation():
+    """Unit vector e_i (i < d/2) at position p is rotated in the (i, i+d/2) plane
+    by angle p*inv_i, counter-clockwise: the textbook matrix [[c,-s],[s,c]]."""
+    p = 37.0
+    for i in (0, 5, 31, 63):
+        a = p * THETA ** (-2.0 * i / D)
+        Rm = np.array([[math.cos(a), -math.sin(a)], [math.sin(a), math.cos(a)]])
+        for col, unit in enumerate((i, i + D // 2)):
+            x = np.zeros((1, 1, D))
+            x[0, 0, unit] = 1.0
+            y = A.rope(x, np.array([p]), THETA)[0, 0]
+            assert abs(y[i] - Rm[0, col]) < 1e-14 and abs(y[i + D // 2] - Rm[1, col]) < 1e-14
+            others = np.delete(y, [i, i + D // 2])
+            assert np.all(others == 0.0)
+
+
+def check_rope_preserves_norm():
+    x = _rand((2, 16, 4, D), 12, 3.0)
+    pos = np.random.default_rng(13).integers(0, 40000, size=(2, 16))
+    y = A.rope(x, pos, THETA)
+    assert np.allclose(np.linalg.norm(y, axis=-1), np.linalg.norm(x, axis=-1), rtol=1e-13)
+
+
+def check_rope_relative_position():
+    """<R(m) q, R(n) k> depends only on m - n."""
+    q = _rand((1, 1, D), 14)
+    k = _rand((1, 1, D), 15)
+    base = None
+    for m, n in [(10, 3), (107, 100), (32767, 32760)]:
+        dq = A.rope(q, np.array([m]), THETA)[0, 0]
+        dk = A.rope(k, np.array([n]), THETA)[0, 0]
+        val = float(dq @ dk)
+        if base is None:
+            base = val
+        assert abs(val - base) < 1e-9 * max(1.0, abs(base))
+
+
+# ---------------------------------------------------------------- attention
+def check_row0_is_v0():
+    """Prefill row 0 sees only key 0: out = v_0 of KV head h//G, lse = s_00."""
+    q, k, v, gq, gk, pos = _inputs(2, 9, 4, 2, seed=20)
+    out, lse = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    G = 2
+    for b in range(2):
+        qp = A.qk_prologue(q[b, :1], gq, pos[b, :1], THETA, EPS)[0]
+        kp = A.qk_prologue(k[b, :1], gk, pos[b, :1], THETA, EPS)[0]
+        for h in range(4):
+            assert np.array_equal(out[b, 0, h], v[b, 0, h // G])
+            assert abs(lse[b, h, 0] - qp[h] @ kp[h // G] / math.sqrt(D)) < 1e-12
+
+
+def check_constant_v():
+    """If every value vector equals c, every output equals c (rows sum to 1)."""
+    q, k, _, gq, gk, pos = _inputs(1, 40, 4, 2, seed=21)
+    c = _rand((D,), 22)
+    v = np.broadcast_to(c, (1, 40, 2, D)).copy()
+    out, _ = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, block=16)
+    assert np.allclose(out, c, rtol=0, atol=1e-13)
+
+
+def check_gqa_equals_mha_on_repeated_kv():
+    """GQA with G = Hq/Hkv equals MHA run on KV heads repeated G times each
+    (repeat_interleave along the head axis)."""
+    q, k, v, gq, gk, pos = _inputs(1, 24, 8, 2, seed=23)
+    out_g, lse_g = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    kr, vr = np.repeat(k, 4, axis=2), np.repeat(v, 4, axis=2)
+    out_m, lse_m = A.prefill_ref(q, kr, vr, gq, gk, pos, THETA, EPS)
+    assert np.allclose(out_g, out_m, rtol=0, atol=1e-14) and np.allclose(lse_g, lse_m, atol=1e-14)
+
+
+def check_against_torch_sdpa():
+    """The attention part equals torch's fp64 scaled_dot_product_attention
+    (causal, enable_gqa) applied to the oracle's normed and rotated q, k."""
+    B, T, Hq, Hkv = 2, 33, 8, 2
+    q, k, v, gq, gk, pos = _inputs(B, T, Hq, Hkv, seed=24)
+    out, _ = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, block=8)
+    qp = np.stack([A.qk_prologue(q[b], gq, pos[b], THETA, EPS) for b in range(B)])
+    kp = np.stack([A.qk_prologue(k[b], gk, pos[b], THETA, EPS) for b in range(B)])
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).transpose(1, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(t(qp), t(kp), t(v), is_causal=True, enable_gqa=True)
+    assert np.allclose(out, ref.transpose(1, 2).numpy(), rtol=0, atol=1e-12)
+
+
+def check_causality():
+    """Changing keys/values after row i leaves rows <= i unchanged."""
+    q, k, v, gq, gk, pos = _inputs(1, 30, 4, 2, seed=25)
+    out1, lse1 = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, 18:] += 5.0
+    v2[:, 18:] -= 3.0
+    out2, lse2 = A.prefill_ref(q, k2, v2, gq, gk, pos, THETA, EPS)
+    assert np.array_equal(out1[:, :18], out2[:, :18]) and np.array_equal(lse1[:, :, :18], lse2[:, :, :18])
+    assert not np.allclose(out1[:, 18:], out2[:, 18:])
+
+
+def check_brute_force_prefill():
+    for (T, Hq, Hkv, seed) in [(5, 2, 1, 30), (16, 4, 2, 31), (9, 4, 1, 32)]:
+        q, k, v, gq, gk, pos = _inputs(1, T, Hq, Hkv, seed=seed)
+        pos = pos + 3 * seed  # arbitrary, non-zero start
+        out, lse = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, block=4)
+        out_l, lse_l = Lp.prefill_loops(q.tolist(), k.tolist(), v.tolist(), gq.tolist(), gk.tolist(),
+                                        pos.tolist(), THETA, EPS)
+        assert np.allclose(out, np.array(out_l), rtol=0, atol=1e-12)
+        assert np.allclose(lse, np.array(lse_l), rtol=0, atol=1e-12)
+
+
+def _tiny_decode(seed, N=2, Hq=4, Hkv=2, lens=(5, 9)):
+    rng = np.random.default_rng(seed)
+    Lmax = max(lens) + 1
+    q = rng.standard_normal((N, Hq, D))
+    kn = rng.standard_normal((N, Hkv, D))
+    vn = rng.standard_normal((N, Hkv, D))
+    kh = rng.standard_normal((N, Lmax, Hkv, D))
+    vc = rng.standard_normal((N, Hkv, Lmax, D))
+    gq, gk = _gain(seed + 1), _gain(seed + 2)
+    kc = np.stack([A.qk_prologue(kh[n], gk, np.arange(Lmax), THETA, EPS).transpose(1, 0, 2) for n in range(N)])
+    return q, kn, vn, gq, gk, kc, vc, np.array(lens), kh
+
+
+def check_brute_force_decode():
+    q, kn, vn, gq, gk, kc, vc, lens, _ = _tiny_decode(40)
+    out, lse = A.decode_ref(q, kn, vn, gq, gk, kc, vc, lens, THETA, EPS)
+    out_l, lse_l = Lp.decode_loops(q.tolist(), kn.tolist(), vn.tolist(), gq.tolist(), gk.tolist(),
+                                   kc.tolist(), vc.tolist(), lens.tolist(), THETA, EPS)
+    assert np.allclose(out, np.array(out_l), rtol=0, atol=1e-12)
+    assert np.allclose(lse, np.array(lse_l), rtol=0, atol=1e-12)
+
+
+def check_decode_equals_last_prefill_row():
+    """Decode at cached length L over a cache of keys normed/rotated at 0..L-1
+    equals row L of a prefill over the same L+1 raw tokens."""
+    rng = np.random.default_rng(41)
+    L, Hq, Hkv = 23, 8, 2
+    q = rng.standard_normal((1, L + 1, Hq, D))
+    k = rng.standard_normal((1, L + 1, Hkv, D))
+    v = rng.standard_normal((1, L + 1, Hkv, D))
+    gq, gk = _gain(42), _gain(43)
+    pos = np.arange(L + 1)[None]
+    out_p, lse_p = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    kc = A.qk_prologue(k[0, :L], gk, np.arange(L), THETA, EPS).transpose(1, 0, 2)[None]
+    vc = v[0, :L].transpose(1, 0, 2)[None]
+    out_d, lse_d = A.decode_ref(q[:, L], k[:, L], v[:, L], gq, gk, kc, vc, np.array([L]), THETA, EPS)
+    assert np.allclose(out_d[0], out_p[0, L], rtol=0, atol=1e-13)
+    assert np.allclose(lse_d[0], lse_p[0, :, L], rtol=0, atol=1e-13)
+
+
+def check_position_shift_invariance():
+    """Shifting every position by a constant leaves outputs unchanged (RoPE is relative)."""
+    q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=50)
+    o1, l1 = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    o2, l2 = A.prefill_ref(q, k, v, gq, gk, pos + 12345, THETA, EPS)
+    assert np.allclose(o1, o2, rtol=0, atol=1e-9) and np.allclose(l1, l2, atol=1e-9)
+
+
+def check_qk_scale_invariance():
+    """Scaling raw q or k by c > 0 leaves the output unchanged up to the eps term."""
+    q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=51)
+    o1, _ = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    o2, _ = A.prefill_ref(q * 7.5, k * 0.25, v, gq, gk, pos, THETA, EPS)
+    # eps moves a normalised k by ~eps / (2 * mean(k^2)) ~ 8e-6 relative here.
+    assert np.allclose(o1, o2, rtol=0, atol=2e-4)
+    o3, _ = A.prefill_ref(q * 7.5, k * 0.25, v, gq, gk, pos, THETA, 0.0)
+    o4, _ = A.prefill_ref(q, k, v, gq, gk, pos, THETA, 0.0)
+    assert np.allclose(o3, o4, rtol=0, atol=1e-12)
+
+
+def check_row_subset_equals_full():
+    q, k, v, gq, gk, pos = _inputs(2, 50, 4, 1, seed=52)
+    out, lse = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    rows = np.array([0, 7, 31, 49])
+    out_s, lse_s = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, rows=rows, block=3)
+    assert np.allclose(out_s, out[:, rows], rtol=0, atol=1e-14)
+    assert np.allclose(lse_s, lse[:, :, rows], rtol=0, atol=1e-14)
+
+
+def check_worked_example_kv_cache():
+    gold = json.load(open(GOLDEN))["wide_gqa_block"]
+    vals = A.kv_cache_values_per_token(gold["n_kv_heads"], gold["head_dim"])
+    assert vals == gold["kv_cache_values_per_token_per_layer"]
+    mha = A.kv_cache_values_per_token(gold["n_query_heads"], gold["head_dim"])
+    assert vals / mha == gold["fraction_of_full_multi_head_cache"]
+    assert gold["key_value_projection"][1] == gold["n_kv_heads"] * gold["head_dim"]
+    assert gold["query_projection"][1] == gold["n_query_heads"] * gold["head_dim"]
+
+
+def check_worked_example_logit_scale():
+    """Unit-RMS head vectors have raw dot products of RMS ~ sqrt(128) ~ 11.3."""
+    gold = json.load(open(GOLDEN))["wide_gqa_block"]
+    x = _rand((20000, D), 60, 3.0)
+    y = _rand((20000, D), 61, 0.2)
+    qn = A.rms_norm(x, np.ones(D), EPS)
+    kn = A.rms_norm(y, np.ones(D), EPS)
+    rms = float(np.sqrt(np.mean(np.sum(qn * kn, axis=-1) ** 2)))
+    assert abs(rms - gold["raw_dot_rms_of_unit_rms_vectors"]) < 0.03 * 11.3
+
+
+ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

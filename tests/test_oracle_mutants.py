@@ -1,0 +1,95 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and confirm the pins catch
+each one: a wrong RoPE sign, adjacent-pair RoPE, a missing eps, mean-centering,
+h mod Hkv head mapping, an off-by-one causal mask, a missing 1/sqrt(d) scale,
+and a base-2 logsumexp."""
+import numpy as np
+import pytest
+
+import oracle.attention as A
+from tests import oracle_checks as C
+
+
+def _rope_wrong_sign(x, pos, theta):
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * A.rope_inv_freq(x.shape[-1], theta)
+    c, s = np.cos(ang)[..., None, :], np.sin(ang)[..., None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
+
+
+def _rope_adjacent_pairs(x, pos, theta):
+    x = np.asarray(x, dtype=np.float64)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * A.rope_inv_freq(x.shape[-1], theta)
+    c, s = np.cos(ang)[..., None, :], np.sin(ang)[..., None, :]
+    xe, xo = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = xe * c - xo * s
+    y[..., 1::2] = xo * c + xe * s
+    return y
+
+
+def _norm_no_eps(x, g, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return g * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True))
+
+
+def _norm_centered(x, g, eps):
+    x = np.asarray(x, dtype=np.float64)
+    x = x - x.mean(axis=-1, keepdims=True)
+    return g * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+
+
+def _attend_off_by_one(qg, kk, vv, limit):
+    return _ORIG_ATTEND(qg, kk, vv, limit - 1 + (limit == 0))
+
+
+def _attend_no_scale(qg, kk, vv, limit):
+    return _ORIG_ATTEND(qg * np.sqrt(qg.shape[-1]), kk, vv, limit)
+
+
+def _attend_log2(qg, kk, vv, limit):
+    o, l = _ORIG_ATTEND(qg, kk, vv, limit)
+    return o, l / np.log(2.0)
+
+
+_ORIG_ATTEND = A._attend
+
+
+def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=False, block=256):
+    # h -> h % Hkv instead of h // G: permute the query heads so the oracle's
+    # h // G lookup lands on h % Hkv, then undo the permutation on the output.
+    q = np.asarray(q, dtype=np.float64)
+    Hq, Hkv = q.shape[2], np.asarray(k).shape[2]
+    G = Hq // Hkv
+    perm = np.array([(h % Hkv) * G + h // Hkv for h in range(Hq)])
+    qq = np.empty_like(q)
+    qq[:, :, perm] = q
+    o, l = _ORIG_PREFILL(qq, k, v, gq, gk, pos, theta, eps, rows=rows, staged=staged, block=block)
+    return o[:, :, perm], l[:, perm]
+
+
+_ORIG_PREFILL = A.prefill_ref
+
+MUTANTS = [
+    ("rope", _rope_wrong_sign),
+    ("rope", _rope_adjacent_pairs),
+    ("rms_norm", _norm_no_eps),
+    ("rms_norm", _norm_centered),
+    ("_attend", _attend_off_by_one),
+    ("_attend", _attend_no_scale),
+    ("_attend", _attend_log2),
+    ("prefill_ref", _prefill_mod_mapping),
+]
+
+
+@pytest.mark.parametrize("name,fn", MUTANTS, ids=[m[1].__name__.strip("_") for m in MUTANTS])
+def test_pins_catch_planted_mistake(monkeypatch, name, fn):
+    monkeypatch.setattr(A, name, fn)
+    failed = []
+    for check in C.ALL_CHECKS:
+        try:
+            check()
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"no pin caught the planted mistake in {name}"
