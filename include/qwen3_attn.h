@@ -1,0 +1,181 @@
+/*
+ * qwen3_attn.h - C ABI of libqwen3attn.so, the Qwen3 attention core on B200 (sm_100a).
+ *
+ * The core takes projected q/k/v and computes, per head vector of head_dim d = 128:
+ *   1. QK-Norm: y = g * x / sqrt(mean(x^2) + eps), fp32 statistics, learned gain g[d]
+ *      ("Qwen3 Architecture Layer-by-Layer", Primitives: Qwen3RMSNorm; "Hand-Writing a
+ *      Vision-Language Model, Part 1", RMSNorm and the order-of-operations list).
+ *   2. RoPE, rotate-half pairing (dim i with dim i + d/2), inv_i = theta^(-2i/d), angle
+ *      pos * inv_i ("Hand-Writing ... Part 1", RotaryEmbedding (RoPE); "Qwen3 Architecture
+ *      Layer-by-Layer", apply_rotary_pos_emb and Qwen3RotaryEmbedding).
+ *   3. Causal grouped-query attention, scale 1/sqrt(d), query head h reading KV head
+ *      h / (Hq/Hkv) ("Assembling a large model from scratch", The complete code,
+ *      Attention.forward; "Qwen3 Architecture Layer-by-Layer", The attention dispatch).
+ * V is never normalised or rotated.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers to memory the caller owns; the library
+ *     never frees or retains them.  bf16 tensors are passed as `qwen3_bf16` (uint16 bit
+ *     patterns of IEEE bfloat16).  All tensors are dense row-major (C order) with the
+ *     shapes stated below; base addresses must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream) and never
+ *     synchronise, except qwen3_attn_device_status().  Host-side argument checks happen
+ *     before any launch; a failed check launches nothing.
+ *   - Functions return a qwen3_status and never abort or throw.
+ *   - Inputs must not alias outputs.
+ *   - Supported shapes: d == 128; Hkv >= 1; Hq % Hkv == 0 with G = Hq/Hkv a power of two,
+ *     G <= 128 for prefill and G <= 16 for decode.  Other shapes return
+ *     QWEN3_ERR_UNSUPPORTED.
+ *   - Device waits are bounded.  If a kernel's internal wait runs out (a hardware or
+ *     library fault, never a legal input), the kernel records QWEN3_ERR_DEVICE_TIMEOUT in a
+ *     device-side status word and returns early; qwen3_attn_device_status() reports it.
+ */
+#ifndef QWEN3_ATTN_H_
+#define QWEN3_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t qwen3_bf16;
+typedef struct CUstream_st* qwen3_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  QWEN3_OK = 0,
+  QWEN3_ERR_INVALID_ARG = 1,    /* NULL required pointer, non-positive size, misaligned pointer */
+  QWEN3_ERR_UNSUPPORTED = 2,    /* d != 128, Hq % Hkv != 0, G not a supported power of two    */
+  QWEN3_ERR_CUDA = 3,           /* a CUDA runtime/driver call or launch failed                */
+  QWEN3_ERR_DEVICE_TIMEOUT = 4, /* a bounded device-side wait ran out                         */
+  QWEN3_ERR_WORKSPACE = 5       /* workspace NULL or smaller than the *_workspace_size value  */
+} qwen3_status;
+
+/*
+ * qwen3_qk_norm_rope - QK-Norm then RoPE of raw head vectors, written in cache layout.
+ * Defined by steps 1-2 above ("Hand-Writing ... Part 1": q_norm/k_norm run right after the
+ * projection and before RoPE).
+ *   x      [B, T, H, d] bf16, raw projected head vectors (k, or q).
+ *   w      [d] fp32 gain.
+ *   pos    [B, T] int32 positions (the rotation angle of token t of row b is pos[b,t]*inv_i).
+ *   dst    [B, H, Tcap, d] bf16: token t of row b, head h is written to slot
+ *          dst[b, h, row, :] with row = t when write_at_pos == 0, row = pos[b,t] otherwise
+ *          (the decode append: the new token of sequence b goes to index cache_len = pos).
+ *   v_src  optional [B, T, H, d] bf16, copied unchanged to v_dst at the same slots
+ *          (V is never normalised or rotated); pass NULL for both to skip.
+ *   Rows must satisfy row < Tcap; an out-of-range row is skipped and recorded as
+ *   QWEN3_ERR_INVALID_ARG in the device status word.  Results are rounded once to bf16.
+ */
+int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos,
+                       qwen3_bf16* dst, const qwen3_bf16* v_src, qwen3_bf16* v_dst,
+                       int B, int T, int H, int d, int Tcap, int write_at_pos,
+                       float theta, float eps, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_prefill - causal GQA self-attention over T new tokens with the QK-Norm+RoPE
+ * prologue ("Assembling a large model from scratch", Attention.forward with S == T; the
+ * mask is tril on token index: token i sees tokens 0..i of its own batch row).
+ *   q         [B, T, Hq, d] bf16 raw projected queries.
+ *   k, v      [B, T, Hkv, d] bf16 raw projected keys and values.
+ *   q_norm_w, k_norm_w  [d] fp32 gains.
+ *   pos       [B, T] int32 RoPE positions.
+ *   out       [B, T, Hq, d] bf16 attention output (heads not merged with o_proj).
+ * The K prologue result needs B*Hkv*T*d*2 bytes of scratch, which this call obtains
+ * stream-ordered with cudaMallocAsync/cudaFreeAsync on `stream`.  Use
+ * qwen3_attn_prefill_ex to pass your own workspace or to fill a KV cache instead.
+ */
+int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                       const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                       qwen3_bf16* out, int B, int T, int Hq, int Hkv, int d,
+                       float theta, float eps, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_prefill_ex - qwen3_attn_prefill with optional outputs and caller memory.
+ *   lse       optional [B, Hq, T] fp32: natural-log logsumexp of the scaled logits of each
+ *             query row (the logsumexp of "Qwen3 Architecture Layer-by-Layer", The
+ *             cross-entropy math, applied to attention scores).  NULL to skip.
+ *   k_cache, v_cache  optional [B, Hkv, Tcap, d] bf16 (Tcap >= T).  When given (both or
+ *             neither), the normed+rotated keys and the raw values of tokens 0..T-1 are
+ *             written to slots 0..T-1 and attention reads them from there, so the cache is
+ *             ready for qwen3_attn_decode with cache_lens = T.  No workspace is needed.
+ *   workspace, ws_bytes  scratch for the keys when no cache is given; ws_bytes must be at
+ *             least qwen3_attn_prefill_workspace_size(B, T, Hkv, d), else
+ *             QWEN3_ERR_WORKSPACE.  Ignored when a cache is given.
+ */
+int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                          const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                          qwen3_bf16* out, float* lse,
+                          qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap,
+                          void* workspace, size_t ws_bytes,
+                          int B, int T, int Hq, int Hkv, int d,
+                          float theta, float eps, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_decode - one new token per sequence attending over its KV cache
+ * ("Assembling a large model from scratch", KVCache.update and Transformer.forward: the new
+ * token sits at position cache.length and sees the whole history).
+ *   q            [N, Hq, d] bf16 raw query of the new token.
+ *   k_new, v_new [N, Hkv, d] bf16 raw key and value of the new token.
+ *   q_norm_w, k_norm_w  [d] fp32 gains.
+ *   k_cache, v_cache    [N, Hkv, Lmax, d] bf16.  Slots 0..L-1 of sequence n hold its
+ *                normed+rotated keys and raw values.  This call writes the new token's
+ *                normed+rotated key and raw value into slot L (L = cache_lens[n]).
+ *   cache_lens   [N] int32 device array, L per sequence BEFORE the append; 0 <= L < Lmax.
+ *                Not modified (the caller advances it, like the cache length that grows
+ *                by the appended tokens).  A sequence with L >= Lmax is skipped and
+ *                recorded as QWEN3_ERR_INVALID_ARG in the device status word.
+ *   out          [N, Hq, d] bf16; lse optional [N, Hq] fp32 (NULL to skip).
+ *   workspace    at least qwen3_attn_decode_workspace_size(N, Hq, d, Lmax) bytes of
+ *                device scratch for the split-KV partials, else QWEN3_ERR_WORKSPACE.
+ */
+int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                      const float* q_norm_w, const float* k_norm_w,
+                      qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                      qwen3_bf16* out, float* lse,
+                      int N, int Hq, int Hkv, int d, int Lmax,
+                      float theta, float eps, void* workspace, size_t ws_bytes,
+                      qwen3_stream_t stream);
+
+/* Scratch bytes qwen3_attn_prefill_ex needs when it is given no KV cache. */
+size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d);
+
+/* Scratch bytes qwen3_attn_decode needs (split-KV partial outputs and logsumexps). */
+size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax);
+
+/* Bytes of one layer's bf16 KV cache [2][N][Hkv][Lmax][d]: 2*Hkv*d values per token
+ * ("Qwen 3 From Scratch", Worked example: 1024 values per token for Hkv=4, d=128). */
+size_t qwen3_attn_kv_cache_bytes(int N, int Hkv, int Lmax, int d);
+
+/* Static description of a status code (never NULL). */
+const char* qwen3_attn_status_string(int status);
+
+/*
+ * qwen3_attn_device_status - synchronise `stream`, then return and optionally clear the
+ * device-side status word of the current device (QWEN3_OK if no kernel recorded an
+ * error).  When `site` is not NULL it receives a code naming the wait or check that fired.
+ */
+int qwen3_attn_device_status(qwen3_stream_t stream, int clear, int* site);
+
+/*
+ * qwen3_attn_set_wait_limit - bound, in nanoseconds, on every device-side wait of later
+ * launches (default 2e9).  Returns the previous value.
+ */
+uint64_t qwen3_attn_set_wait_limit(uint64_t ns);
+
+/*
+ * qwen3_attn_set_fault_injection - test hook.  While flags == 1, every prefill launch's K/V
+ * producer skips its first key-tile load, so the consumers' bounded waits run out and the
+ * launch ends early, leaving QWEN3_ERR_DEVICE_TIMEOUT in the status word (outputs are not
+ * written).  0 turns it off.  No memory outside the call's own buffers is touched.
+ */
+void qwen3_attn_set_fault_injection(int flags);
+
+/* Library version string. */
+const char* qwen3_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QWEN3_ATTN_H_ */

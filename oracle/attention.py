@@ -42,6 +42,9 @@ Readings where the pages leave a step open:
     norm and the gain; the oracle keeps everything in fp64.  `staged=True`
     rounds q' and k' to bf16 once after RoPE, which is where the GPU path
     rounds them before its bf16 MMAs; it is used only for the logsumexp bound.
+    That rounding decides a discrete code, so it is taken from the value held
+    in float32 (the precision in which the kernels, like the pages' RMSNorm
+    with its x.float(), hold q' and k' before the cast): fp64 -> fp32 -> bf16.
   * Rotate-half with theta from the argument (the page prose that speaks of
     adjacent pairs and base 10000 contradicts every code block on the pages).
 """
@@ -89,9 +92,11 @@ def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
 
 def qk_prologue(x: np.ndarray, g: np.ndarray, pos: np.ndarray, theta: float, eps: float,
                 staged: bool = False) -> np.ndarray:
-    """QK-Norm then RoPE of raw head vectors x [..., T, H, d] at positions pos [..., T]."""
+    """QK-Norm then RoPE of raw head vectors x [..., T, H, d] at positions pos [..., T].
+
+    staged=True returns the bf16 value the result rounds to when held in float32."""
     y = rope(rms_norm(x, g, eps), pos, theta)
-    return bf16_round(y) if staged else y
+    return bf16_round(y.astype(np.float32).astype(np.float64)) if staged else y
 
 
 def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray):

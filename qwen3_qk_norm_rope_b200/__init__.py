@@ -1,0 +1,225 @@
+"""Python binding of libqwen3attn.so: the Qwen3 attention core (QK-Norm + RoPE + causal
+GQA) on B200.
+
+Argument marshalling only.  Every step of the computation runs in the library's CUDA
+kernels; torch supplies device memory and the current stream.  There is no CPU path:
+if the library is missing, or a tensor is not on a CUDA device, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqwen3attn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_WORKSPACE = range(6)
+
+HEAD_DIM = 128
+
+# Every symbol include/qwen3_attn.h declares: (name, restype, argtypes)
+_P, _I, _F, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+SIGNATURES = {
+    "qwen3_qk_norm_rope": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P]),
+    "qwen3_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
+    "qwen3_attn_prefill_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _Z,
+                                   _I, _I, _I, _I, _I, _F, _F, _P]),
+    "qwen3_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
+    "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
+    "qwen3_attn_status_string": (ctypes.c_char_p, [_I]),
+    "qwen3_attn_device_status": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int)]),
+    "qwen3_attn_set_wait_limit": (_U64, [_U64]),
+    "qwen3_attn_set_fault_injection": (None, [_I]),
+    "qwen3_attn_version": (ctypes.c_char_p, []),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqwen3attn.so (built in-tree by `qwen3_qk_norm_rope_b200.build`)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m qwen3_qk_norm_rope_b200.build` "
+                               "(there is no fallback implementation)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+class Qwen3AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def status_string(status: int) -> str:
+    return lib().qwen3_attn_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise Qwen3AttnError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device: torch.device):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device or t.device.type != "cuda":
+        raise ValueError(f"{name} must be on {device} (CUDA); got {t.device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}; got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}; got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill_workspace_size(B: int, T: int, Hkv: int, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
+
+
+def decode_workspace_size(N: int, Hq: int, Lmax: int, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_decode_workspace_size(N, Hq, d, Lmax))
+
+
+def kv_cache_bytes(N: int, Hkv: int, Lmax: int, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_kv_cache_bytes(N, Hkv, Lmax, d))
+
+
+def qk_norm_rope(x, w, pos, dst, v_src=None, v_dst=None, *, write_at_pos: bool = False,
+                 theta: float = 1.0e6, eps: float = 1.0e-6) -> torch.Tensor:
+    """QK-Norm + RoPE of x [B,T,H,d] into dst [B,H,Tcap,d] (row t, or row pos[b,t] when
+    write_at_pos); optionally copies v_src [B,T,H,d] to v_dst at the same slots."""
+    dev = x.device
+    B, T, H, d = x.shape
+    Tcap = dst.shape[2]
+    _need(x, "x", torch.bfloat16, (B, T, H, d), dev)
+    _need(w, "w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (B, T), dev)
+    _need(dst, "dst", torch.bfloat16, (B, H, Tcap, d), dev)
+    if v_src is not None:
+        _need(v_src, "v_src", torch.bfloat16, (B, T, H, d), dev)
+        _need(v_dst, "v_dst", torch.bfloat16, (B, H, Tcap, d), dev)
+    _check(lib().qwen3_qk_norm_rope(_ptr(x), _ptr(w), _ptr(pos), _ptr(dst), _ptr(v_src), _ptr(v_dst),
+                                    B, T, H, d, Tcap, int(write_at_pos), theta, eps, _stream(dev)),
+           "qwen3_qk_norm_rope")
+    return dst
+
+
+def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: float = 1.0e-6,
+            out=None, lse=None, k_cache=None, v_cache=None, workspace=None):
+    """Causal GQA prefill with the QK-Norm+RoPE prologue.  q [B,T,Hq,d], k/v [B,T,Hkv,d] bf16,
+    gains [d] fp32, pos [B,T] int32.  Returns out [B,T,Hq,d] bf16 (and writes lse [B,Hq,T]
+    fp32 and the caches [B,Hkv,Tcap,d] when given)."""
+    dev = q.device
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(q, "q", torch.bfloat16, (B, T, Hq, d), dev)
+    _need(k, "k", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(v, "v", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (B, T), dev)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, T, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq, T), dev)
+    Tcap = 0
+    if k_cache is not None or v_cache is not None:
+        Tcap = k_cache.shape[2]
+        _need(k_cache, "k_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
+        _need(v_cache, "v_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
+    elif workspace is None:
+        workspace = torch.empty(prefill_workspace_size(B, T, Hkv, d), dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().qwen3_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                       _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
+                                       _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
+           "qwen3_attn_prefill_ex")
+    return out
+
+
+def prefill_simple(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: float = 1.0e-6, out=None):
+    """qwen3_attn_prefill: the call that obtains its own stream-ordered scratch."""
+    dev = q.device
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, tuple(t.shape), dev)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _check(lib().qwen3_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                    _ptr(out), B, T, Hq, Hkv, d, theta, eps, _stream(dev)), "qwen3_attn_prefill")
+    return out
+
+
+def decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *, theta: float = 1.0e6,
+           eps: float = 1.0e-6, out=None, lse=None, workspace=None):
+    """One decode step.  q [N,Hq,d], k_new/v_new [N,Hkv,d] bf16 raw; caches [N,Hkv,Lmax,d]
+    bf16 (slot L = cache_lens[n] is written); cache_lens [N] int32 (not advanced).
+    Returns out [N,Hq,d] bf16."""
+    dev = q.device
+    N, Hq, d = q.shape
+    Hkv = k_new.shape[1]
+    Lmax = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (N, Hq, d), dev)
+    _need(k_new, "k_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(v_new, "v_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(k_cache, "k_cache", torch.bfloat16, (N, Hkv, Lmax, d), dev)
+    _need(v_cache, "v_cache", torch.bfloat16, (N, Hkv, Lmax, d), dev)
+    _need(cache_lens, "cache_lens", torch.int32, (N,), dev)
+    if out is None:
+        out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (N, Hq), dev)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(N, Hq, Lmax, d), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().qwen3_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
+                                   _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
+                                   N, Hq, Hkv, d, Lmax, theta, eps, _ptr(workspace), ws_bytes, _stream(dev)),
+           "qwen3_attn_decode")
+    return out
+
+
+def device_status(clear: bool = True, device=None) -> tuple[int, int]:
+    """Synchronise the current stream and return (status, site) of the device status word."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    site = ctypes.c_int(0)
+    st = lib().qwen3_attn_device_status(_stream(dev), int(clear), ctypes.byref(site))
+    return int(st), int(site.value)
+
+
+def set_wait_limit(ns: int) -> int:
+    return int(lib().qwen3_attn_set_wait_limit(int(ns)))
+
+
+def set_fault_injection(flags: int) -> None:
+    lib().qwen3_attn_set_fault_injection(int(flags))
+
+
+def version() -> str:
+    return lib().qwen3_attn_version().decode()

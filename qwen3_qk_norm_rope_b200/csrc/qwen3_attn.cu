@@ -1,0 +1,386 @@
+// qwen3_attn.cu - the C ABI of libqwen3attn.so: argument checks, RoPE constants, TMA
+// tensor maps and kernel launches.  All device work lives in the kernels included below;
+// this file does no arithmetic on tensor data.
+#include <cmath>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "prologue.cuh"
+
+namespace {
+
+using q3::kD;
+
+constexpr int kDecodeSplit = 1024;  // keys per split-KV CTA
+constexpr int kMaxDevices = 64;
+
+uint64_t initial_wait_ns() {
+  const char* e = std::getenv("QWEN3_ATTN_WAIT_NS");
+  if (e != nullptr) {
+    const unsigned long long v = std::strtoull(e, nullptr, 10);
+    if (v > 0) return v;
+  }
+  return 2000000000ull;
+}
+
+uint64_t g_wait_ns = initial_wait_ns();
+uint64_t g_launch_id = 0;
+int g_fault = 0;
+std::mutex g_mu;
+
+q3::WaitCfg next_wait_cfg() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return q3::WaitCfg{g_wait_ns, ++g_launch_id};
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+
+// inv_i = theta^(-2i/d) in double, split into a float and the float of its remainder.
+q3::RopeTable make_rope_table(float theta) {
+  q3::RopeTable t;
+  for (int i = 0; i < q3::kHalf; ++i) {
+    const double inv = std::pow(static_cast<double>(theta), -2.0 * i / kD);
+    t.hi[i] = static_cast<float>(inv);
+    t.lo[i] = static_cast<float>(inv - static_cast<double>(t.hi[i]));
+  }
+  return t;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tiled map, 128B swizzle, zero fill out of bounds.  dims/strides innermost first;
+// strides[i] is the byte stride of dim i+1.
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+              const cuuint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Opt the big-shared-memory kernels in once per device.
+int ensure_kernel_attrs() {
+  static bool done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QWEN3_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (done[dev]) return QWEN3_OK;
+  if (cudaFuncSetAttribute(q3::fmha_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kPrefillSmemBytes) != cudaSuccess)
+    return QWEN3_ERR_CUDA;
+  if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kDecodeSmemBytes) != cudaSuccess)
+    return QWEN3_ERR_CUDA;
+  done[dev] = true;
+  return QWEN3_OK;
+}
+
+int check_common(int Hq, int Hkv, int d) {
+  if (Hq <= 0 || Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
+  if (d != kD) return QWEN3_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0 || !is_pow2(Hq / Hkv)) return QWEN3_ERR_UNSUPPORTED;
+  return QWEN3_OK;
+}
+
+int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
+                    int B, int T, int H, int Tcap, int write_at_pos, float theta, float eps, cudaStream_t stream) {
+  q3::PrologueParams p;
+  p.x = static_cast<const uint32_t*>(x);
+  p.w = w;
+  p.pos = pos;
+  p.dst = static_cast<uint32_t*>(dst);
+  p.v_src = static_cast<const uint2*>(v_src);
+  p.v_dst = static_cast<uint2*>(v_dst);
+  p.B = B;
+  p.T = T;
+  p.H = H;
+  p.Tcap = Tcap;
+  p.write_at_pos = write_at_pos;
+  p.eps = eps;
+  p.rope = make_rope_table(theta);
+  const long long nvec = static_cast<long long>(B) * T * H;
+  const int warps = 8;
+  long long blocks = (nvec + warps - 1) / warps;
+  if (blocks > 148LL * 64) blocks = 148LL * 64;  // grid-stride beyond ~64 blocks per SM
+  q3::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qwen3_attn_version(void) { return "qwen3-attn-b200 0.1 (sm_100a)"; }
+
+const char* qwen3_attn_status_string(int status) {
+  switch (status) {
+    case QWEN3_OK: return "ok";
+    case QWEN3_ERR_INVALID_ARG: return "invalid argument";
+    case QWEN3_ERR_UNSUPPORTED: return "unsupported shape";
+    case QWEN3_ERR_CUDA: return "CUDA runtime or launch failure";
+    case QWEN3_ERR_DEVICE_TIMEOUT: return "bounded device-side wait ran out";
+    case QWEN3_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+uint64_t qwen3_attn_set_wait_limit(uint64_t ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  const uint64_t old = g_wait_ns;
+  g_wait_ns = ns;
+  return old;
+}
+
+void qwen3_attn_set_fault_injection(int flags) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_fault = flags;
+}
+
+int qwen3_attn_device_status(qwen3_stream_t stream, int clear, int* site) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QWEN3_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpyFromSymbol(h, q3::g_status, sizeof(h)) != cudaSuccess) return QWEN3_ERR_CUDA;
+  if (clear) {
+    const int z[2] = {0, 0};
+    if (cudaMemcpyToSymbol(q3::g_status, z, sizeof(z)) != cudaSuccess) return QWEN3_ERR_CUDA;
+  }
+  if (site != nullptr) *site = h[1];
+  return h[0];
+}
+
+size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d) {
+  if (B <= 0 || T <= 0 || Hkv <= 0 || d <= 0) return 0;
+  return static_cast<size_t>(B) * Hkv * T * d * 2 + 256;
+}
+
+size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax) {
+  if (N <= 0 || Hq <= 0 || d <= 0 || Lmax <= 0) return 0;
+  const size_t ns = (static_cast<size_t>(Lmax) + kDecodeSplit - 1) / kDecodeSplit;
+  const size_t o_bytes = static_cast<size_t>(N) * Hq * ns * d * 4;
+  return o_bytes + 256 + static_cast<size_t>(N) * Hq * ns * 4 + 256;
+}
+
+size_t qwen3_attn_kv_cache_bytes(int N, int Hkv, int Lmax, int d) {
+  if (N <= 0 || Hkv <= 0 || Lmax <= 0 || d <= 0) return 0;
+  return static_cast<size_t>(2) * N * Hkv * Lmax * d * sizeof(qwen3_bf16);
+}
+
+int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, qwen3_bf16* dst,
+                       const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
+                       int write_at_pos, float theta, float eps, qwen3_stream_t stream) {
+  if (x == nullptr || w == nullptr || pos == nullptr || dst == nullptr) return QWEN3_ERR_INVALID_ARG;
+  if ((v_src == nullptr) != (v_dst == nullptr)) return QWEN3_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0 || H <= 0 || Tcap <= 0) return QWEN3_ERR_INVALID_ARG;
+  if (d != kD) return QWEN3_ERR_UNSUPPORTED;
+  if (!write_at_pos && Tcap < T) return QWEN3_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(dst, 16) || !aligned(w, 8) || !aligned(pos, 4)) return QWEN3_ERR_INVALID_ARG;
+  if (v_src != nullptr && (!aligned(v_src, 16) || !aligned(v_dst, 16))) return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  return launch_prologue(x, w, pos, dst, v_src, v_dst, B, T, H, Tcap, write_at_pos, theta, eps,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                          const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
+                          qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap, void* workspace, size_t ws_bytes,
+                          int B, int T, int Hq, int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
+      pos == nullptr || out == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (B <= 0 || T <= 0) return QWEN3_ERR_INVALID_ARG;
+  int st = check_common(Hq, Hkv, d);
+  if (st != QWEN3_OK) return st;
+  if (Hq / Hkv > 128) return QWEN3_ERR_UNSUPPORTED;
+  if ((k_cache == nullptr) != (v_cache == nullptr)) return QWEN3_ERR_INVALID_ARG;
+  const bool use_cache = k_cache != nullptr;
+  if (use_cache && Tcap < T) return QWEN3_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) ||
+      !aligned(k_norm_w, 8) || !aligned(pos, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return QWEN3_ERR_INVALID_ARG;
+  if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (!use_cache) {
+    if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
+      return QWEN3_ERR_WORKSPACE;
+  }
+  if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
+    return QWEN3_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
+
+  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] (and V copied when filling a cache).
+  qwen3_bf16* kdst = use_cache ? k_cache
+                               : reinterpret_cast<qwen3_bf16*>((reinterpret_cast<uintptr_t>(workspace) + 255) &
+                                                               ~static_cast<uintptr_t>(255));
+  const int Tc = use_cache ? Tcap : T;
+  st = launch_prologue(k, k_norm_w, pos, kdst, use_cache ? v : nullptr, use_cache ? v_cache : nullptr, B, T, Hkv,
+                       Tc, 0, theta, eps, s);
+  if (st != QWEN3_OK) return st;
+
+  // 2. Tensor maps.  The key-axis extent is T (not Tcap) so slots past the prompt read as zeros.
+  CUtensorMap mk, mv;
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(T),
+                                static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(B)};
+    const cuuint64_t str[3] = {kD * 2ull, static_cast<cuuint64_t>(Tc) * kD * 2ull,
+                               static_cast<cuuint64_t>(Hkv) * Tc * kD * 2ull};
+    if (!make_map(&mk, kdst, 4, dims, str, box)) return QWEN3_ERR_CUDA;
+    if (use_cache) {
+      if (!make_map(&mv, v_cache, 4, dims, str, box)) return QWEN3_ERR_CUDA;
+    } else {
+      const cuuint64_t vstr[3] = {static_cast<cuuint64_t>(Hkv) * kD * 2ull, kD * 2ull,
+                                  static_cast<cuuint64_t>(T) * Hkv * kD * 2ull};
+      if (!make_map(&mv, v, 4, dims, vstr, box)) return QWEN3_ERR_CUDA;
+    }
+  }
+
+  // 3. Attention.
+  q3::PrefillParams p;
+  p.q = reinterpret_cast<const uint32_t*>(q);
+  p.q_norm_w = q_norm_w;
+  p.pos = pos;
+  p.out = reinterpret_cast<uint4*>(out);
+  p.lse = lse;
+  p.B = B;
+  p.T = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.log2G = ilog2(Hq / Hkv);
+  p.P = 128 >> p.log2G;
+  p.n_qt = (T + p.P - 1) / p.P;
+  p.eps = eps;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
+  p.wait = next_wait_cfg();
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    p.fault = g_fault;
+  }
+  p.rope = make_rope_table(theta);
+  const long long grid = static_cast<long long>(B) * Hkv * p.n_qt;
+  if (grid > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  q3::fmha_prefill_kernel<<<static_cast<unsigned>(grid), q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                       const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, int B, int T, int Hq, int Hkv,
+                       int d, float theta, float eps, qwen3_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
+      pos == nullptr || out == nullptr || B <= 0 || T <= 0)
+    return QWEN3_ERR_INVALID_ARG;
+  const int st0 = check_common(Hq, Hkv, d);
+  if (st0 != QWEN3_OK) return st0;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = qwen3_attn_prefill_workspace_size(B, T, Hkv, d);
+  void* ws = nullptr;
+  if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return QWEN3_ERR_CUDA;
+  const int st = qwen3_attn_prefill_ex(q, k, v, q_norm_w, k_norm_w, pos, out, nullptr, nullptr, nullptr, 0, ws,
+                                       bytes, B, T, Hq, Hkv, d, theta, eps, stream);
+  const bool freed = cudaFreeAsync(ws, s) == cudaSuccess;
+  if (st != QWEN3_OK) return st;
+  return freed ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
+                      const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                      qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta, float eps,
+                      void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
+  if (q == nullptr || k_new == nullptr || v_new == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
+      k_cache == nullptr || v_cache == nullptr || cache_lens == nullptr || out == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (N <= 0 || Lmax <= 0) return QWEN3_ERR_INVALID_ARG;
+  int st = check_common(Hq, Hkv, d);
+  if (st != QWEN3_OK) return st;
+  if (Hq / Hkv > 16 || N > 65535 || Hkv > 65535) return QWEN3_ERR_UNSUPPORTED;
+  if (static_cast<long long>(N) * Hkv * Lmax > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) ||
+      !aligned(cache_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < qwen3_attn_decode_workspace_size(N, Hq, d, Lmax)) return QWEN3_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
+
+  // 1. Append: normed+rotated k_new and raw v_new into slot L = cache_lens[n].
+  st = launch_prologue(k_new, k_norm_w, cache_lens, k_cache, v_new, v_cache, N, 1, Hkv, Lmax, 1, theta, eps, s);
+  if (st != QWEN3_OK) return st;
+
+  // 2. Split-KV attention.
+  const int ns = (Lmax + kDecodeSplit - 1) / kDecodeSplit;
+  const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
+  const size_t o_bytes = static_cast<size_t>(N) * Hq * ns * d * 4;
+  float* part_o = reinterpret_cast<float*>(w0);
+  float* part_lse = reinterpret_cast<float*>((w0 + o_bytes + 255) & ~static_cast<uintptr_t>(255));
+  CUtensorMap mk, mv;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(N) * Hkv * Lmax};
+  const cuuint64_t str[1] = {kD * 2ull};
+  const cuuint32_t box[2] = {64, 64};
+  if (!make_map(&mk, k_cache, 2, dims, str, box) || !make_map(&mv, v_cache, 2, dims, str, box)) return QWEN3_ERR_CUDA;
+  q3::DecodeParams p;
+  p.q = reinterpret_cast<const uint32_t*>(q);
+  p.q_norm_w = q_norm_w;
+  p.cache_lens = cache_lens;
+  p.part_o = part_o;
+  p.part_lse = part_lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.log2G = ilog2(Hq / Hkv);
+  p.Lmax = Lmax;
+  p.split = kDecodeSplit;
+  p.n_split_max = ns;
+  p.eps = eps;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
+  p.wait = next_wait_cfg();
+  p.rope = make_rope_table(theta);
+  q3::decode_split_kernel<<<dim3(ns, Hkv, N), q3::kDecodeThreads, q3::kDecodeSmemBytes, s>>>(mk, mv, p);
+  if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+
+  // 3. Logsumexp combine of the splits.
+  q3::CombineParams c;
+  c.part_o = part_o;
+  c.part_lse = part_lse;
+  c.cache_lens = cache_lens;
+  c.out = reinterpret_cast<uint4*>(out);
+  c.lse = lse;
+  c.Hq = Hq;
+  c.Lmax = Lmax;
+  c.split = kDecodeSplit;
+  c.n_split_max = ns;
+  q3::decode_combine_kernel<<<N * Hq, 128, 0, s>>>(c);
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+}  // extern "C"

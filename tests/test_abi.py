@@ -1,0 +1,117 @@
+"""CPU-only checks of the C-ABI library: it loads without a GPU, exports every symbol the
+header declares, and its host-side argument checks and size helpers behave as documented.
+No call here reaches a CUDA launch."""
+import ctypes
+import json
+import os
+import re
+
+import pytest
+import torch
+
+import qwen3_qk_norm_rope_b200 as qa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qwen3_attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qwen3_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = qa.lib()
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(qa.SIGNATURES) == names
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in qa.version()
+    for code in range(6):
+        assert qa.status_string(code) and qa.status_string(code) != "unknown status"
+    assert qa.status_string(99) == "unknown status"
+
+
+def test_workspace_and_cache_sizes():
+    assert qa.prefill_workspace_size(2, 2048, 8) >= 2 * 8 * 2048 * 128 * 2
+    assert qa.prefill_workspace_size(0, 10, 8) == 0
+    ns = -(-32769 // 1024)
+    assert qa.decode_workspace_size(64, 32, 32769) >= 64 * 32 * ns * (128 + 1) * 4
+    # 2*Hkv*d values per token per layer; 1024 for the wide-GQA block of the worked example
+    gold = json.load(open(os.path.join(ROOT, "tests", "golden", "worked_examples.json")))["wide_gqa_block"]
+    per_token_bytes = qa.kv_cache_bytes(1, gold["n_kv_heads"], 1, gold["head_dim"])
+    assert per_token_bytes // 2 == gold["kv_cache_values_per_token_per_layer"]
+    assert qa.kv_cache_bytes(64, 8, 32769, 128) == 2 * 64 * 8 * 32769 * 128 * 2
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every call below fails its host checks
+
+
+def _prefill_ex(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gq=FAKE, gk=FAKE, pos=FAKE, out=FAKE, lse=None, kc=None, vc=None, Tcap=0,
+             ws=None, ws_bytes=0, B=1, T=128, Hq=16, Hkv=8, d=128, theta=1e6, eps=1e-6)
+    a.update(kw)
+    return qa.lib().qwen3_attn_prefill_ex(a["q"], a["k"], a["v"], a["gq"], a["gk"], a["pos"], a["out"], a["lse"],
+                                          a["kc"], a["vc"], a["Tcap"], a["ws"], a["ws_bytes"], a["B"], a["T"],
+                                          a["Hq"], a["Hkv"], a["d"], a["theta"], a["eps"], None)
+
+
+def test_prefill_argument_checks():
+    assert _prefill_ex(q=None) == qa.ERR_INVALID_ARG
+    assert _prefill_ex(out=None) == qa.ERR_INVALID_ARG
+    assert _prefill_ex(B=0) == qa.ERR_INVALID_ARG
+    assert _prefill_ex(T=-1) == qa.ERR_INVALID_ARG
+    assert _prefill_ex(d=64) == qa.ERR_UNSUPPORTED
+    assert _prefill_ex(Hq=12, Hkv=8) == qa.ERR_UNSUPPORTED
+    assert _prefill_ex(Hq=24, Hkv=8) == qa.ERR_UNSUPPORTED  # G = 3 is not a power of two
+    assert _prefill_ex(Hq=256, Hkv=1) == qa.ERR_UNSUPPORTED  # G > 128
+    assert _prefill_ex(q=ctypes.c_void_p((1 << 20) + 2)) == qa.ERR_INVALID_ARG  # misaligned
+    assert _prefill_ex(kc=FAKE) == qa.ERR_INVALID_ARG  # k_cache without v_cache
+    assert _prefill_ex(kc=FAKE, vc=FAKE, Tcap=64) == qa.ERR_INVALID_ARG  # Tcap < T
+    assert _prefill_ex(theta=0.0, ws=FAKE, ws_bytes=1 << 30) == qa.ERR_INVALID_ARG
+    assert _prefill_ex() == qa.ERR_WORKSPACE
+    assert _prefill_ex(ws=FAKE, ws_bytes=100) == qa.ERR_WORKSPACE
+
+
+def test_decode_and_prologue_argument_checks():
+    lib = qa.lib()
+
+    def dec(**kw):
+        a = dict(q=FAKE, kn=FAKE, vn=FAKE, gq=FAKE, gk=FAKE, kc=FAKE, vc=FAKE, lens=FAKE, out=FAKE, lse=None, N=4,
+                 Hq=32, Hkv=8, d=128, Lmax=4096, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.qwen3_attn_decode(a["q"], a["kn"], a["vn"], a["gq"], a["gk"], a["kc"], a["vc"], a["lens"],
+                                     a["out"], a["lse"], a["N"], a["Hq"], a["Hkv"], a["d"], a["Lmax"], 1e6, 1e-6,
+                                     a["ws"], a["ws_bytes"], None)
+
+    assert dec(lens=None) == qa.ERR_INVALID_ARG
+    assert dec(N=0) == qa.ERR_INVALID_ARG
+    assert dec(Hq=64, Hkv=2) == qa.ERR_UNSUPPORTED  # G = 32 > 16
+    assert dec(d=256) == qa.ERR_UNSUPPORTED
+    assert dec() == qa.ERR_WORKSPACE
+    assert dec(ws=FAKE, ws_bytes=16) == qa.ERR_WORKSPACE
+    r = lib.qwen3_qk_norm_rope(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 4, 8, 128, 4, 0, 1e6, 1e-6, None)
+    assert r == qa.ERR_INVALID_ARG  # v_src without v_dst
+    r = lib.qwen3_qk_norm_rope(FAKE, FAKE, FAKE, FAKE, None, None, 1, 8, 8, 128, 4, 0, 1e6, 1e-6, None)
+    assert r == qa.ERR_INVALID_ARG  # Tcap < T when writing at t
+    r = lib.qwen3_qk_norm_rope(FAKE, FAKE, FAKE, FAKE, None, None, 1, 8, 8, 64, 8, 0, 1e6, 1e-6, None)
+    assert r == qa.ERR_UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors():
+    q = torch.zeros(1, 128, 16, 128, dtype=torch.bfloat16)
+    k = torch.zeros(1, 128, 8, 128, dtype=torch.bfloat16)
+    w = torch.ones(128)
+    pos = torch.arange(128, dtype=torch.int32)[None]
+    with pytest.raises(ValueError):
+        qa.prefill(q, k, k, w, w, pos)
+
+
+def test_wait_limit_roundtrip():
+    old = qa.set_wait_limit(123456)
+    assert qa.set_wait_limit(old) == 123456

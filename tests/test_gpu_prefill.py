@@ -1,0 +1,137 @@
+"""Prefill parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.  Full parity on the small and Qwen3-0.6B-shaped workloads and on ragged
+shapes; sampled query rows on the 4B-shaped and long wide-GQA workloads at full size."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qwen3_qk_norm_rope_b200 as qa
+from synthetic import PREFILL_SHAPES, PrefillShape, as_f64, prefill_inputs
+from tests.gpu_common import (assert_status_ok, compare, dev, prefill_gpu, prefill_oracle, to_np)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen3-0.6b"])
+def test_prefill_full_parity(name):
+    shape = PREFILL_SHAPES[name]
+    inp = prefill_inputs(shape, seed=0)
+    out, lse = prefill_gpu(inp)
+    ref, ref_lse, st_lse = prefill_oracle(inp)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, name)
+
+
+RAGGED = [
+    # (B, T, Hq, Hkv): T not a multiple of the tile, T = 1, G in {1, 2, 4, 16, 32}, B > 1
+    (1, 1, 16, 8),
+    (1, 100, 16, 8),
+    (2, 129, 8, 2),
+    (1, 200, 4, 4),
+    (1, 300, 64, 4),
+    (1, 257, 32, 1),
+    (3, 77, 8, 8),
+    (1, 1000, 32, 8),
+]
+
+
+@pytest.mark.parametrize("B,T,Hq,Hkv", RAGGED)
+def test_prefill_ragged_shapes(B, T, Hq, Hkv):
+    shape = PrefillShape("ragged", B, T, Hq, Hkv)
+    inp = prefill_inputs(shape, seed=B * 1000 + T)
+    # positions need not be 0..T-1: an arbitrary offset per row plus gaps (RoPE only)
+    rng = np.random.default_rng(T)
+    starts = rng.integers(0, 30000, size=(B, 1))
+    steps = rng.integers(1, 4, size=(B, T))
+    inp["pos"] = torch.from_numpy((starts + np.cumsum(steps, axis=1)).astype(np.int32))
+    out, lse = prefill_gpu(inp)
+    ref, ref_lse, st_lse = prefill_oracle(inp)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, f"B{B} T{T} Hq{Hq} Hkv{Hkv}")
+
+
+def _sampled_rows(T, n_first, n_rand, n_last, seed):
+    rng = np.random.default_rng(seed)
+    mid = rng.choice(np.arange(n_first, T - n_last), size=n_rand, replace=False)
+    return np.unique(np.concatenate([np.arange(n_first), mid, np.arange(T - n_last, T)]))
+
+
+@pytest.mark.parametrize("name,n_first,n_rand,n_last", [("qwen3-4b", 256, 512, 256),
+                                                         ("long-wide-gqa", 128, 192, 128)])
+def test_prefill_full_size_sampled_rows(name, n_first, n_rand, n_last):
+    shape = PREFILL_SHAPES[name]
+    inp = prefill_inputs(shape, seed=0)
+    out, lse = prefill_gpu(inp)
+    rows = _sampled_rows(shape.T, n_first, n_rand, n_last, seed=1)
+    ref, ref_lse, st_lse = prefill_oracle(inp, rows=rows)
+    o = to_np(out[:, torch.from_numpy(rows).to(out.device)])
+    l = to_np(lse[:, :, torch.from_numpy(rows).to(out.device)])
+    compare(o, l, ref, ref_lse, st_lse, name + " sampled rows")
+    # every row, not only the sampled ones, must be finite
+    assert torch.isfinite(out.float()).all()
+
+
+def test_prefill_fills_cache_and_matches_workspace_path():
+    shape = PrefillShape("cache", 2, 300, 16, 8)
+    inp = prefill_inputs(shape, seed=5)
+    d = dev()
+    Tcap = 512
+    canary = 0x7FC1  # a bf16 NaN bit pattern
+    kc = torch.empty((2, 8, Tcap, 128), dtype=torch.bfloat16, device=d)
+    vc = torch.empty_like(kc)
+    kc.view(torch.int16).fill_(canary)
+    vc.view(torch.int16).fill_(canary)
+    out_c, lse_c = prefill_gpu(inp, caches=(kc, vc))
+    out_w, lse_w = prefill_gpu(inp)
+    assert torch.equal(out_c, out_w) and torch.equal(lse_c, lse_w)
+    # cache slots 0..T-1: keys normed+rotated (one bf16 rounding), values copied bit-exactly
+    kref = oracle.qk_prologue(as_f64(inp["k"]), as_f64(inp["k_norm_w"]), inp["pos"].numpy(), 1e6, 1e-6)
+    kgot = to_np(kc[:, :, :300].permute(0, 2, 1, 3))
+    assert np.all(np.abs(kgot - kref) <= np.abs(kref) * 2.0 ** -8 + 1e-5)
+    assert torch.equal(vc[:, :, :300].permute(0, 2, 1, 3).cpu(), inp["v"])
+    # slots past T untouched
+    assert torch.equal(kc[:, :, 300:].view(torch.int16).cpu(),
+                       torch.full((2, 8, Tcap - 300, 128), canary, dtype=torch.int16))
+    assert torch.equal(vc[:, :, 300:].view(torch.int16).cpu(),
+                       torch.full((2, 8, Tcap - 300, 128), canary, dtype=torch.int16))
+    ref, ref_lse, st_lse = prefill_oracle(inp)
+    compare(to_np(out_c), to_np(lse_c), ref, ref_lse, st_lse, "cache path")
+
+
+def test_prefill_simple_call_and_guard_band():
+    shape = PREFILL_SHAPES["tiny"]
+    inp = prefill_inputs(shape, seed=3)
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items()}
+    n = 1 * 128 * 16 * 128
+    buf = torch.full((n + 4096,), -7.0, dtype=torch.bfloat16, device=d)
+    out = buf[:n].view(1, 128, 16, 128)
+    qa.prefill_simple(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], out=out)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    assert torch.all(buf[n:] == -7.0)
+    ref_out, _ = prefill_gpu(inp)
+    assert torch.equal(out, ref_out)
+    # repeated launches are bitwise reproducible
+    again, _ = prefill_gpu(inp)
+    assert torch.equal(again, ref_out)
+
+
+def test_qk_norm_rope_prologue_kernel():
+    """The standalone prologue against the oracle's QK-Norm + RoPE, positions up to 40000."""
+    d = dev()
+    rng = np.random.default_rng(9)
+    B, T, H = 2, 333, 8
+    x = torch.from_numpy((rng.standard_normal((B, T, H, 128)) * rng.uniform(0.1, 8.0, size=(B, T, H, 1)))
+                         .astype(np.float32)).to(torch.bfloat16)
+    w = torch.from_numpy((1 + 0.1 * rng.standard_normal(128)).astype(np.float32))
+    pos = torch.from_numpy(rng.integers(0, 40000, size=(B, T)).astype(np.int32))
+    dst = torch.zeros((B, H, T, 128), dtype=torch.bfloat16, device=d)
+    qa.qk_norm_rope(x.to(d), w.to(d), pos.to(d), dst)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    ref = oracle.qk_prologue(as_f64(x), as_f64(w), pos.numpy(), 1e6, 1e-6)
+    got = to_np(dst.permute(0, 2, 1, 3))
+    # one bf16 rounding of an fp32 result (angle error <~ 5e-7 rad)
+    assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 2e-5), np.abs(got - ref).max()
+    staged = oracle.bf16_round(ref)
+    assert np.mean(got != staged) < 0.01  # nearly every element rounds to the same bf16
