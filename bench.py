@@ -1,0 +1,461 @@
+"""Benchmark of the Qwen3 attention core on B200: prints ONE JSON line.
+
+One step is one pass of the whole hot path over one batch of synthetic input:
+  * prefill of the Qwen3-0.6B-shaped workload (B=2, T=2048, Hq=16, Hkv=8, d=128):
+    QK-Norm + RoPE prologue and causal GQA attention, and
+  * one batched decode step (64 sequences, cached lengths ~ U[1024, 32768], Hq=32,
+    Hkv=8): append of the new normed/rotated key, split-KV attention, LSE combine.
+`value` is the prefill throughput in TFLOP/s (causal flops 4*B*Hq*d*T(T+1)/2; the
+prologue is counted as free work); the decode throughput in GB/s rides along under
+"decode".  Inputs are resident in HBM before the timed region; L2 is flushed (a
+256 MiB write) before every step, outside the per-step CUDA-event windows.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of the step
+(weak scaling, no collective on the data path); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import DECODE_SHAPES, PREFILL_SHAPES, decode_step_inputs, prefill_inputs  # noqa: E402
+
+METRIC = "causal GQA attn TFLOP/s (+QK-Norm/RoPE) % bf16 peak; decode HBM GB/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in PEAKS_FALLBACK}, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
+    """Algorithmic HBM bytes of one decode step: every cached K and V row read once
+    (L per sequence), the new token's q read, out written, k/v_new read and written."""
+    lens = lens.astype(np.int64)
+    kv = int(lens.sum()) * Hkv * d * 2 * 2
+    qo = lens.size * Hq * d * 2 * 2
+    new = lens.size * Hkv * d * 2 * 2 * 2
+    return kv + qo + new
+
+
+def decode_flops(lens: np.ndarray, Hq: int, d: int = 128) -> float:
+    return 4.0 * Hq * d * float((lens.astype(np.int64) + 1).sum())
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), float(f[3]), f[4], f[5], f[6], f[7], f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [r[0] for r in rows]
+        loaded = [r for r in rows if r[2] > 200.0] or rows
+        reasons = set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            for name, flag in zip(names, r[4:8]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median([r[0] for r in loaded])), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "sm_mhz_min": min(sm)}
+
+
+# ------------------------------------------------------------------------------ workload
+class Workload:
+    """Device-resident inputs of one step, built once."""
+
+    def __init__(self, dev: torch.device, seed: int = 0, prefill: str = "qwen3-0.6b", decode_seqs: int = 64):
+        import dataclasses
+
+        import qwen3_qk_norm_rope_b200 as qa
+
+        self.qa = qa
+        self.dev = dev
+        self.ps = PREFILL_SHAPES[prefill]
+        full = DECODE_SHAPES["batched-decode"]
+        self.ds = full if decode_seqs == full.N else dataclasses.replace(
+            full, name=f"first {decode_seqs} sequences of the {full.name}", N=decode_seqs)
+        p = prefill_inputs(self.ps, seed=seed)
+        self.p_host = p
+        self.p = {k: v.to(dev) for k, v in p.items()}
+        self.p_out = torch.empty_like(self.p["q"])
+        self.p_ws = torch.empty(qa.prefill_workspace_size(self.ps.B, self.ps.T, self.ps.Hkv), dtype=torch.uint8,
+                                device=dev)
+        d = decode_step_inputs(full, seed=seed)
+        d = {k: (v[:decode_seqs].contiguous() if k in ("q", "k_new", "v_new", "cache_lens") else v)
+             for k, v in d.items()}
+        self.d_host = d
+        self.d = {k: v.to(dev) for k, v in d.items()}
+        self.lens = d["cache_lens"].numpy()
+        N, Hkv, Lmax = self.ds.N, self.ds.Hkv, self.ds.cache_capacity
+        self.Lmax = Lmax
+        self.kc = torch.empty((N, Hkv, Lmax, 128), dtype=torch.bfloat16, device=dev)
+        self.vc = torch.empty_like(self.kc)
+        # Cache history: raw keys drawn like the prefill keys (N(0,1) times the per-channel
+        # scale s_k), normed and rotated at positions 0..L-1 by the library's own prologue;
+        # raw values N(0,1).  Drawn on the device with a seeded generator.
+        g = torch.Generator(device=dev)
+        g.manual_seed(seed + 1)
+        s_k = d["s_k"].to(dev)
+        Lmax_hist = int(self.lens.max())
+        pos = torch.arange(Lmax_hist, dtype=torch.int32, device=dev)[None]
+        for n in range(N):
+            L = int(self.lens[n])
+            kh = (torch.randn((1, L, Hkv, 128), generator=g, device=dev) * s_k).to(torch.bfloat16)
+            vh = torch.randn((1, L, Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
+            qa.qk_norm_rope(kh, self.d["k_norm_w"], pos[:, :L].contiguous(), self.kc[n:n + 1], v_src=vh,
+                            v_dst=self.vc[n:n + 1], theta=self.ds.theta, eps=self.ds.eps)
+        self.d_out = torch.empty_like(self.d["q"])
+        self.d_ws = torch.empty(qa.decode_workspace_size(N, self.ds.Hq, Lmax), dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize(dev)
+        st, site = qa.device_status(clear=True, device=dev)
+        if st != qa.OK:
+            raise RuntimeError(f"cache build failed: {qa.status_string(st)} at site {site}")
+
+    def prefill(self):
+        p = self.p
+        self.qa.prefill(p["q"], p["k"], p["v"], p["q_norm_w"], p["k_norm_w"], p["pos"], out=self.p_out,
+                        workspace=self.p_ws)
+
+    def decode(self):
+        d = self.d
+        self.qa.decode(d["q"], d["k_new"], d["v_new"], d["q_norm_w"], d["k_norm_w"], self.kc, self.vc,
+                       d["cache_lens"], out=self.d_out, workspace=self.d_ws)
+
+    def flush_l2(self):
+        self.flush.fill_(1.0)
+
+    # launches of this library's kernels per step: prefill (prologue + attention) and
+    # decode (append + split-KV attention + combine)
+    LAUNCHES_PER_STEP = 5
+
+
+def time_steps(w: Workload, steps: int):
+    """Per-step CUDA events on the launching stream; the L2 flush sits between windows."""
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(steps):
+        w.flush_l2()
+        ev[i][0].record()
+        w.prefill()
+        ev[i][1].record()
+        w.decode()
+        ev[i][2].record()
+    torch.cuda.synchronize(w.dev)
+    pre = sum(e[0].elapsed_time(e[1]) for e in ev)
+    dec = sum(e[1].elapsed_time(e[2]) for e in ev)
+    return pre, dec
+
+
+def time_e2e(w: Workload, steps: int):
+    """The same step through the public API with host buffers: pinned host -> device copies
+    of the step's inputs, the calls, and device -> host copies of the outputs, all inside
+    the event window."""
+    ph = {k: v.pin_memory() for k, v in w.p_host.items()}
+    dh = {k: w.d_host[k].pin_memory() for k in ("q", "k_new", "v_new", "q_norm_w", "k_norm_w", "cache_lens")}
+    out_p = torch.empty(w.p_out.shape, dtype=torch.bfloat16).pin_memory()
+    out_d = torch.empty(w.d_out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in ph.values()) + sum(t.numel() * t.element_size()
+                                                                       for t in dh.values())
+    d2h = out_p.numel() * 2 + out_d.numel() * 2
+    pre_ms = 0.0
+    tot_ms = 0.0
+    for i in range(steps):
+        w.flush_l2()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        for k, v in ph.items():
+            w.p[k].copy_(v, non_blocking=True)
+        w.prefill()
+        out_p.copy_(w.p_out, non_blocking=True)
+        e1.record()
+        for k, v in dh.items():
+            w.d[k].copy_(v, non_blocking=True)
+        w.decode()
+        out_d.copy_(w.d_out, non_blocking=True)
+        e2.record()
+        torch.cuda.synchronize(w.dev)
+        pre_ms += e0.elapsed_time(e1)
+        tot_ms += e0.elapsed_time(e2)
+    return pre_ms, tot_ms, h2d, d2h
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seqs: int = 16, seed: int = 0):
+    """The fp64 oracle, as it stands, on a bounded sample of the same workload: the last
+    `rows_per_head` query rows (every head) of the first `batch_rows` batch rows of the
+    Qwen3-0.6B-shaped prefill (the defaults are the whole prefill), and the first
+    `decode_seqs` sequences of the batched decode.  Returns TFLOP/s on the prefill sample,
+    GB/s on the decode sample, the seconds each took and the BLAS thread count."""
+    import oracle
+    from synthetic import as_f64, decode_history
+
+    ps = PREFILL_SHAPES["qwen3-0.6b"]
+    inp = prefill_inputs(ps, seed=seed)
+    rows = np.arange(ps.T - rows_per_head, ps.T)
+    args = (as_f64(inp["q"][:batch_rows]), as_f64(inp["k"][:batch_rows]), as_f64(inp["v"][:batch_rows]),
+            as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][:batch_rows].numpy(), ps.theta, ps.eps)
+    t0 = time.perf_counter()
+    oracle.prefill_ref(*args, rows=rows)
+    t_pre = time.perf_counter() - t0
+    flops = batch_rows * 4.0 * ps.Hq * ps.d * float((rows + 1).sum())
+    t_dec, gbs, lens_sel = 0.0, 0.0, []
+    if decode_seqs > 0:
+        ds = DECODE_SHAPES["batched-decode"]
+        step = decode_step_inputs(ds, seed=seed)
+        lens = step["cache_lens"].numpy()
+        sel = list(range(decode_seqs))
+        kh, vh = [], []
+        for n in sel:
+            h = decode_history(ds, n, int(lens[n]), step["s_k"], seed=seed)
+            kh.append(oracle.build_cache_k(as_f64(h["k_hist"]), as_f64(step["k_norm_w"]), ds.theta,
+                                           ds.eps).transpose(1, 0, 2))
+            vh.append(as_f64(h["v_hist"]).transpose(1, 0, 2))
+        t0 = time.perf_counter()
+        oracle.decode_ref(as_f64(step["q"])[sel], as_f64(step["k_new"])[sel], as_f64(step["v_new"])[sel],
+                          as_f64(step["q_norm_w"]), as_f64(step["k_norm_w"]), kh, vh, lens[sel], ds.theta, ds.eps)
+        t_dec = time.perf_counter() - t0
+        gbs = decode_bytes(lens[sel], ds.Hq, ds.Hkv) / t_dec / 1e9
+        lens_sel = [int(lens[n]) for n in sel]
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    sample = (f"prefill: last {rows_per_head} of {ps.T} query rows x {ps.Hq} heads of {batch_rows} of {ps.B} "
+              f"batch rows of the Qwen3-0.6B-shaped workload ({flops:.3g} causal flops); decode: first "
+              f"{decode_seqs} of 64 sequences ({sum(lens_sel)} cached tokens)")
+    return {"tflops": flops / t_pre / 1e12, "gbs": gbs, "t_prefill_s": t_pre, "t_decode_s": t_dec,
+            "threads": threads, "sample": sample, "flops": flops}
+
+
+# ------------------------------------------------------------------------------ main
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(world, vals, dev):
+    if world == 1:
+        return vals
+    import torch.distributed as dist
+
+    t = torch.tensor(vals, dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle on the host cores, as it stands.  Each step is a
+    bounded sample of the workload (the last rows of one prefill batch row and one decode
+    sequence), sized from a calibration run so all K steps take about two minutes."""
+    if rank != 0:
+        return
+    cal = cpu_oracle_sample(rows_per_head=64, batch_rows=1, decode_seqs=1)  # warm-up + calibration
+    per_row = cal["t_prefill_s"] / 64
+    budget = 120.0 / max(args.steps, 1) - cal["t_decode_s"]
+    rows = int(max(4, min(2048, budget / max(per_row, 1e-6))))
+    t_pre = t_tot = flops = 0.0
+    res = None
+    for _ in range(args.steps):
+        res = cpu_oracle_sample(rows_per_head=rows, batch_rows=1, decode_seqs=1)
+        t_pre += res["t_prefill_s"]
+        t_tot += res["t_prefill_s"] + res["t_decode_s"]
+        flops += res["flops"]
+    value = flops / t_pre / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
+                             "sample": "per step, " + res["sample"]},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "decode": {"value": res["gbs"], "unit": "GB/s"}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(ps=None, ds=None):
+    ps = ps or PREFILL_SHAPES["qwen3-0.6b"]
+    ds = ds or DECODE_SHAPES["batched-decode"]
+    return {"workload": f"{ps.name} + {ds.name}",
+            "prefill": {"B": ps.B, "T": ps.T, "Hq": ps.Hq, "Hkv": ps.Hkv, "d": ps.d, "causal": True},
+            "decode": {"N": ds.N, "Hq": ds.Hq, "Hkv": ds.Hkv, "d": ds.d, "L": f"U[{ds.lmin},{ds.lmax}]",
+                       "Lmax": ds.cache_capacity},
+            "rope_theta": ps.theta, "rms_eps": ps.eps, "seed": 0,
+            "l2": "flushed before every step (256 MiB write, outside the timed windows); decode K/V 4.4 GB > L2",
+            "parallelism": "replicas (one independent workload per GPU)"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", default="qwen3-0.6b", choices=sorted(PREFILL_SHAPES),
+                    help="prefill workload of the step (profiling of the other shapes)")
+    ap.add_argument("--decode-seqs", type=int, default=64,
+                    help="decode the first n of the 64 sequences (small cases for ncu captures)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = Workload(dev, prefill=args.prefill, decode_seqs=args.decode_seqs)
+    for _ in range(args.warmup):
+        w.flush_l2()
+        w.prefill()
+        w.decode()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        pre_ms, dec_ms = time_steps(w, args.steps)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+    st, site = w.qa.device_status(clear=True, device=dev)
+    if st != w.qa.OK:
+        raise RuntimeError(f"device status {w.qa.status_string(st)} at site {site}")
+    pre_ms, dec_ms = max_over_ranks(world, [pre_ms, dec_ms], dev)
+    e2e = None
+    if not args.no_e2e:
+        e_pre, e_tot, h2d, d2h = time_e2e(w, max(1, min(args.steps, 200)))
+        e_pre, e_tot = max_over_ranks(world, [e_pre, e_tot], dev)
+        e_steps = max(1, min(args.steps, 200))
+        e2e = {"value": world * w.ps.causal_flops() * e_steps / (e_pre * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": e_tot / e_steps}
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+    K = args.steps
+    pre_s, dec_s = pre_ms * 1e-3 / K, dec_ms * 1e-3 / K
+    tflops = world * w.ps.causal_flops() / pre_s / 1e12
+    dbytes = decode_bytes(w.lens, w.ds.Hq, w.ds.Hkv)
+    gbs = world * dbytes / dec_s / 1e9
+    clocks = clk.summary()
+    dominant_is_decode = dec_s >= pre_s
+    rl_dec = {"bound": "hbm", "achieved": dbytes / dec_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+              "frac": dbytes / dec_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+              "kernel": "decode call (append + split-KV attention + combine)",
+              "algorithmic_bytes": dbytes, "peak_source": peak_src}
+    rl_pre = {"bound": "tensor", "achieved": w.ps.causal_flops() / pre_s / 1e12, "peak": peaks["bf16_tflops"],
+              "unit": "TFLOP/s", "frac": w.ps.causal_flops() / pre_s / 1e12 / peaks["bf16_tflops"],
+              "traffic": None, "kernel": "prefill call (K prologue + attention)",
+              "algorithmic_flops": w.ps.causal_flops(), "peak_source": peak_src + " burst"}
+    line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_dict(w.ps, w.ds),
+            "prefill": {"value": tflops, "unit": "TFLOP/s", "ms": pre_s * 1e3, "frac_of_peak": rl_pre["frac"]},
+            "decode": {"value": gbs, "unit": "GB/s", "ms": dec_s * 1e3, "frac_of_peak": rl_dec["frac"],
+                       "bytes": dbytes, "tflops": world * decode_flops(w.lens, w.ds.Hq) / dec_s / 1e12},
+            "roofline": rl_dec if dominant_is_decode else rl_pre,
+            "roofline_other": rl_pre if dominant_is_decode else rl_dec,
+            "gpu_launches": Workload.LAUNCHES_PER_STEP * K,
+            "clocks": clocks, "e2e": e2e}
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_sample(rows_per_head=2048, batch_rows=2, decode_seqs=16)
+        line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
+                                "sample": cb["sample"], "decode_gbs": cb["gbs"],
+                                "seconds": cb["t_prefill_s"] + cb["t_decode_s"]}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
