@@ -137,6 +137,36 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
                       float theta, float eps, void* workspace, size_t ws_bytes,
                       qwen3_stream_t stream);
 
+/*
+ * qwen3_attn_decode_noalloc - qwen3_attn_decode for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call; it exists for the host programs,
+ * not for the method.  Some callers own no allocator: a plug-in that an inference engine
+ * hands only its input and output buffers, or a serving loop whose device pool is managed
+ * elsewhere and which must not call cudaMalloc on its hot path (cudaMalloc can
+ * synchronise the device and bypasses that pool).  This call takes the same arguments as
+ * qwen3_attn_decode minus the workspace and allocates nothing: its split-KV partials live
+ * in one fixed region of QWEN3_ATTN_NOALLOC_SCRATCH_BYTES (48 MiB) of device memory that
+ * the library declares statically, which every GPU that loads the library holds until
+ * the process exits.
+ *   - Limit: qwen3_attn_decode_workspace_size(N, Hq, d, Lmax) must not exceed
+ *     QWEN3_ATTN_NOALLOC_SCRATCH_BYTES (64 sequences x 32 heads x Lmax 32769 need 34.9
+ *     MB); larger requests return QWEN3_ERR_WORKSPACE and launch nothing.
+ *   - The first call on a device looks up the region's device address (with that device
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one region, and a call leaves its partials there.
+ *     Nothing in it needs to start at zero (each split writes its partial before the
+ *     combine reads it).  Calls whose kernels overlap on the GPU (other streams, other
+ *     host threads) race on the region: serialise them.
+ * All other arguments, outputs and errors are those of qwen3_attn_decode.
+ */
+#define QWEN3_ATTN_NOALLOC_SCRATCH_BYTES ((size_t)48 << 20)
+int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                              const float* q_norm_w, const float* k_norm_w,
+                              qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                              qwen3_bf16* out, float* lse,
+                              int N, int Hq, int Hkv, int d, int Lmax,
+                              float theta, float eps, qwen3_stream_t stream);
+
 /* Scratch bytes qwen3_attn_prefill_ex needs when it is given no KV cache. */
 size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d);
 

@@ -28,6 +28,7 @@ SIGNATURES = {
     "qwen3_attn_prefill_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _Z,
                                    _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
+    "qwen3_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
@@ -202,6 +203,40 @@ def decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *,
                                    _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
                                    N, Hq, Hkv, d, Lmax, theta, eps, _ptr(workspace), ws_bytes, _stream(dev)),
            "qwen3_attn_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 48 << 20
+
+
+def decode_noalloc(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *, theta: float = 1.0e6,
+                   eps: float = 1.0e-6, out=None, lse=None):
+    """qwen3_attn_decode_noalloc: `decode` for callers that cannot allocate device memory.
+    The split-KV partials live in the library's fixed 48 MiB device region (shared by
+    every call on the device; overlapping calls race).  `out`/`lse` are still the
+    caller's; pass preallocated ones to keep this call free of allocation on the Python
+    side too."""
+    dev = q.device
+    N, Hq, d = q.shape
+    Hkv = k_new.shape[1]
+    Lmax = k_cache.shape[2]
+    _need(q, "q", torch.bfloat16, (N, Hq, d), dev)
+    _need(k_new, "k_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(v_new, "v_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(k_cache, "k_cache", torch.bfloat16, (N, Hkv, Lmax, d), dev)
+    _need(v_cache, "v_cache", torch.bfloat16, (N, Hkv, Lmax, d), dev)
+    _need(cache_lens, "cache_lens", torch.int32, (N,), dev)
+    if out is None:
+        out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (N, Hq), dev)
+    _check(lib().qwen3_attn_decode_noalloc(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
+                                           _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
+                                           N, Hq, Hkv, d, Lmax, theta, eps, _stream(dev)),
+           "qwen3_attn_decode_noalloc")
     return out
 
 

@@ -384,3 +384,44 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Decode without any device allocation: the split-KV partials go to a region the library
+// declares statically instead of a caller workspace (see qwen3_attn_decode_noalloc in
+// include/qwen3_attn.h).  In host code `g_noalloc_scratch` names a host-side stand-in, not
+// device memory, so it is never passed to a kernel directly: its device address is looked
+// up once per device with cudaGetSymbolAddress, with that device current.
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[QWEN3_ATTN_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of this device's scratch region, or nullptr when the lookup failed.
+void* noalloc_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                                         const float* q_norm_w, const float* k_norm_w, qwen3_bf16* k_cache,
+                                         qwen3_bf16* v_cache, const int32_t* cache_lens, qwen3_bf16* out,
+                                         float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta,
+                                         float eps, qwen3_stream_t stream) {
+  const size_t need = qwen3_attn_decode_workspace_size(N, Hq, d, Lmax);
+  if (need > QWEN3_ATTN_NOALLOC_SCRATCH_BYTES) return QWEN3_ERR_WORKSPACE;
+  void* scratch = noalloc_scratch_for_current_device();
+  if (scratch == nullptr) return QWEN3_ERR_CUDA;
+  return qwen3_attn_decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq,
+                           Hkv, d, Lmax, theta, eps, scratch, QWEN3_ATTN_NOALLOC_SCRATCH_BYTES, stream);
+}
