@@ -9,20 +9,31 @@
 // axis be tiled is the technique named for the fused cross-entropy in "Qwen3 Architecture
 // Layer-by-Layer", Liger fused linear cross-entropy.
 //
-// One CTA owns one 128-row query tile of one (batch row, KV head): rows are P = 128/G
-// consecutive positions x the G query heads of the group, so each K/V tile is loaded once
-// per GQA group and feeds 128 MMA rows.  Six warps:
+// Work decomposition.  A query tile is 128 MMA rows: P = 128/G consecutive positions x the
+// G query heads of one KV group, so every K/V tile feeds all heads that share it.  A work
+// item is a pair of adjacent query tiles (A = 2i, B = 2i+1) of one (batch row, KV head):
+// both read the same K/V tiles, so each K/V tile is loaded once per pair and feeds 256
+// rows.  CTAs are persistent (one per SM) and take items in heaviest-first order.
+//
+// Ten warps:
 //   warp 0      TMA producer: K'/V tiles (128 keys x 128 dims, two 128B-swizzled boxes
 //               each) into a 2-stage ring; owns the TMEM allocation.
-//   warp 1      MMA issuer (one thread): S = Q K^T into one of two TMEM S buffers, then
-//               O += P V into the TMEM O accumulator; tcgen05.commit signals completion.
-//   warps 2-5   one thread per query row: Q prologue (warp-cooperative, into swizzled
-//               smem), then per key tile: tcgen05.ld of its S row, causal mask, exp2 online
-//               softmax with a lazy rescale (O is rescaled only when the running max grows
-//               by more than 2^8), bf16 P into swizzled smem; finally O/l and the LSE.
-// TMEM: S0 cols [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
-// Every wait is bounded (see mbar_wait); on a timeout every role stops, copies and MMAs
-// in flight are drained, TMEM is freed and the error is left in the status word.
+//   warp 1      MMA issuer (one thread).  Per key tile j it issues PV_A(j-1), S_A(j),
+//               PV_B(j-1), S_B(j), so the tensor core works on one tile while the softmax
+//               warpgroup of the other tile runs.
+//   warps 2-5   softmax warpgroup of tile A, one thread per row (TMEM lane quadrant =
+//   warps 6-9   warp % 4); softmax warpgroup of tile B.  Each runs the Q prologue of its
+//               tile into swizzled smem, then per key tile: tcgen05.ld of its S row,
+//               causal mask, exp2 online softmax with a lazy rescale (O is rescaled only
+//               when the running max grows by more than 2^8), bf16 P written back into TMEM
+//               over its own S columns; finally O/l and the LSE.
+// TMEM (512 columns): S_A [0,128) with P_A at [32,96), O_A [128,256), S_B [256,384) with
+// P_B at [288,352), O_B [384,512).  PV reads P from TMEM (the TS form of tcgen05.mma).
+// Ordering: one thread issues every MMA and they complete in issue order, so the commit
+// that signals S_X(j) also covers PV_X(j-1): once a softmax thread sees S_X(j) it may
+// overwrite P_X and rescale O_X without a further wait.
+// Every wait is bounded (see mbar_wait); on a timeout every role stops, copies and MMAs in
+// flight are drained, TMEM is freed and the error is left in the status word.
 #pragma once
 #include "common.cuh"
 
@@ -34,7 +45,7 @@ struct PrefillParams {
   const int* pos;  // [B, T]
   uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
-  int B, T, Hq, Hkv, log2G, P, n_qt;
+  int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
   float eps, scale_log2;
   WaitCfg wait;
   int fault;
@@ -43,22 +54,56 @@ struct PrefillParams {
 
 constexpr uint32_t kPfTile = 32768;  // 128 rows x 128 bf16
 constexpr uint32_t kPfBox = 16384;   // 128 rows x 64 bf16: one 128B-swizzled TMA box
-constexpr uint32_t kPfQ = 0;
-constexpr uint32_t kPfK = kPfTile;       // 2 stages
-constexpr uint32_t kPfV = 3 * kPfTile;   // 2 stages
-constexpr uint32_t kPfP = 5 * kPfTile;
+constexpr uint32_t kPfQ = 0;         // Q'_A, Q'_B
+constexpr uint32_t kPfK = 2 * kPfTile;  // 2 stages
+constexpr uint32_t kPfV = 4 * kPfTile;  // 2 stages
 constexpr uint32_t kPfBar = 6 * kPfTile;
-// barrier block (byte offsets from kPfBar)
+// barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage
 constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
-                   kBOFull = 88, kBQReady = 96, kBDone = 104, kBTmemSlot = 112, kBAbort = 116;
-constexpr uint32_t kPrefillSmemBytes = kPfBar + 128 + 1024;  // + slack to align the base to 1024
-constexpr int kPrefillThreads = 192;
+                   kBOFull = 96, kBQReady = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140;
+constexpr uint32_t kPrefillSmemBytes = kPfBar + 256 + 1024;  // + slack to align the base to 1024
+constexpr int kPrefillThreads = 320;
+constexpr uint32_t kTmPOff = 32;  // P within S
 constexpr float kLn2 = 0.693147180559945309f;
+
+__device__ __forceinline__ uint32_t tm_s(int X) { return X == 0 ? 0u : 256u; }
+__device__ __forceinline__ uint32_t tm_o(int X) { return X == 0 ? 128u : 384u; }
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// D[tmem] (+)= A[tmem] * B[smem desc]: the TS form, A (here P) read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+struct TileInfo {
+  int t0, nkv;  // first position; key tiles (0 = the tile lies past T)
+};
+
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt) {
+  TileInfo ti;
+  ti.t0 = qt * p.P;
+  ti.nkv = (ti.t0 < p.T) ? (min(ti.t0 + p.P, p.T) - 1) / 128 + 1 : 0;
+  return ti;
+}
+
+// Work item -> (pair, batch row, KV head); items are numbered heaviest pair first.
+__device__ __forceinline__ void item_coords(const PrefillParams& p, int item, int& pair, int& b, int& hkv) {
+  const int BH = p.B * p.Hkv;
+  pair = p.n_pairs - 1 - item / BH;
+  const int bh = item % BH;
+  b = bh / p.Hkv;
+  hkv = bh % p.Hkv;
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
@@ -68,19 +113,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sb - raw);
-  const uint32_t sQ = sb + kPfQ, sK = sb + kPfK, sV = sb + kPfV, sP = sb + kPfP, bar = sb + kPfBar;
+  const uint32_t sK = sb + kPfK, sV = sb + kPfV, bar = sb + kPfBar;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kPfBar + kBAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + kPfBar + kBTmemSlot);
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int BH = p.B * p.Hkv;
-  const int qt = p.n_qt - 1 - static_cast<int>(blockIdx.x) / BH;  // heaviest tiles first
-  const int bh = static_cast<int>(blockIdx.x) % BH;
-  const int b = bh / p.Hkv, hkv = bh % p.Hkv;
-  const int G = 1 << p.log2G;
-  const int t0 = qt * p.P;
-  const int t_end = min(t0 + p.P, p.T);
-  const int nkv = (t_end - 1) / 128 + 1;  // key tiles 0..nkv-1 hold every key some row sees
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -89,10 +125,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar + kBVFull + 8 * s, 1);
       mbar_init(bar + kBVEmpty + 8 * s, 1);
       mbar_init(bar + kBSFull + 8 * s, 1);
+      mbar_init(bar + kBPReady + 8 * s, 128);
+      mbar_init(bar + kBOFull + 8 * s, 1);
+      mbar_init(bar + kBQReady + 8 * s, 128);
     }
-    mbar_init(bar + kBPReady, 128);
-    mbar_init(bar + kBOFull, 1);
-    mbar_init(bar + kBQReady, 128);
     mbar_init(bar + kBDone, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -113,21 +149,34 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
-      for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (j >= 2 && !mbar_wait(bar + kBKEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillKEmpty)) break;
-        if (!(p.fault != 0 && j == 0)) {
-          mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
-          tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, j * 128, hkv, b);
-          tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, j * 128, hkv, b);
-          k_last[st] = j;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int pair, b, hkv;
+        item_coords(p, item, pair, b, hkv);
+        const int n = max(tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv);
+        for (int j = 0; j < n; ++j, ++it) {
+          const int st = it & 1;
+          const uint32_t ph = (it >> 1) & 1;
+          if (it >= 2 && !mbar_wait(bar + kBKEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillKEmpty)) {
+            ok = false;
+            break;
+          }
+          if (!(p.fault != 0 && it == 0)) {
+            mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
+            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, j * 128, hkv, b);
+            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, j * 128, hkv, b);
+            k_last[st] = static_cast<int>(it);
+          }
+          if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
+          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, j * 128, hkv, b);
+          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, j * 128, hkv, b);
+          v_last[st] = static_cast<int>(it);
         }
-        if (j >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) break;
-        mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
-        tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, j * 128, hkv, b);
-        tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, j * 128, hkv, b);
-        v_last[st] = j;
       }
       // Every issued copy must land before this CTA's shared memory is released.
       for (int s = 0; s < 2; ++s) {
@@ -140,168 +189,223 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       constexpr uint32_t kIdQK = idesc_bf16(128, 128, false);  // B = K rows, K-major
       constexpr uint32_t kIdPV = idesc_bf16(128, 128, true);   // B = V, dims contiguous (MN-major)
-      const uint32_t tO = tmem + 256;
-      bool ok = mbar_wait(bar + kBQReady, 0, p.wait, abort_flag, kSitePrefillQReady);
-      auto issue_s = [&](int j) {
-        const int st = j & 1;
-        ok = ok && mbar_wait(bar + kBKFull + 8 * st, (j >> 1) & 1, p.wait, abort_flag, kSitePrefillKFull);
-        if (!ok) return;
-        tc_fence_after();
-        const uint32_t tS = tmem + (j & 1) * 128;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
-          tc_mma_ss(tS, smem_desc_sw128(sQ + koff, 16, 1024), smem_desc_sw128(sK + st * kPfTile + koff, 16, 1024),
-                    kIdQK, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar + kBSFull + 8 * (j & 1));
-        tc_commit(bar + kBKEmpty + 8 * st);
-      };
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv) issue_s(j + 1);
+      uint32_t it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int pair, b, hkv;
+        item_coords(p, item, pair, b, hkv);
+        const int nX[2] = {tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv};
+        const int n = max(nX[0], nX[1]);
+        for (int X = 0; X < 2 && ok; ++X)
+          if (nX[X] > 0) {
+            ok = mbar_wait(bar + kBQReady + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQReady);
+            ++q_cnt[X];
+          }
         if (!ok) break;
-        const int st = j & 1;
-        ok = mbar_wait(bar + kBPReady, j & 1, p.wait, abort_flag, kSitePrefillPReady) &&
-             mbar_wait(bar + kBVFull + 8 * st, (j >> 1) & 1, p.wait, abort_flag, kSitePrefillVFull);
+        // j = 0: S_A(0), S_B(0)
+        ok = mbar_wait(bar + kBKFull + 8 * (it & 1), (it >> 1) & 1, p.wait, abort_flag, kSitePrefillKFull);
         if (!ok) break;
         tc_fence_after();
+        for (int X = 0; X < 2; ++X)
+          if (nX[X] > 0) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * kPfBox + (kk & 3) * 32;
-          tc_mma_ss(tO, smem_desc_sw128(sP + aoff, 16, 1024),
-                    smem_desc_sw128(sV + st * kPfTile + kk * 2048, kPfBox, 1024), kIdPV,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
+              tc_mma_ss(tmem + tm_s(X), smem_desc_sw128(sb + kPfQ + X * kPfTile + koff, 16, 1024),
+                        smem_desc_sw128(sK + (it & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar + kBSFull + 8 * X);
+          }
+        tc_commit(bar + kBKEmpty + 8 * (it & 1));
+        // j >= 1: PV_X(j-1) then S_X(j), for X = A, B
+        for (int j = 1; j <= n && ok; ++j) {
+          const uint32_t prev = it + j - 1, cur = it + j;
+          if (j < n) {
+            ok = mbar_wait(bar + kBKFull + 8 * (cur & 1), (cur >> 1) & 1, p.wait, abort_flag, kSitePrefillKFull);
+            if (!ok) break;
+          }
+          ok = mbar_wait(bar + kBVFull + 8 * (prev & 1), (prev >> 1) & 1, p.wait, abort_flag, kSitePrefillVFull);
+          if (!ok) break;
+          for (int X = 0; X < 2; ++X) {
+            if (j - 1 < nX[X]) {
+              ok = mbar_wait(bar + kBPReady + 8 * X, p_cnt[X] & 1, p.wait, abort_flag, kSitePrefillPReady);
+              ++p_cnt[X];
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk)
+                tc_mma_ts(tmem + tm_o(X), tmem + tm_s(X) + kTmPOff + kk * 8,
+                          smem_desc_sw128(sV + (prev & 1) * kPfTile + kk * 2048, kPfBox, 1024), kIdPV,
+                          (j > 1 || kk > 0) ? 1u : 0u);
+              if (j == nX[X]) tc_commit(bar + kBOFull + 8 * X);
+            }
+            if (j < nX[X]) {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
+                tc_mma_ss(tmem + tm_s(X), smem_desc_sw128(sb + kPfQ + X * kPfTile + koff, 16, 1024),
+                          smem_desc_sw128(sK + (cur & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+              }
+              tc_commit(bar + kBSFull + 8 * X);
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar + kBVEmpty + 8 * (prev & 1));
+          if (j < n) tc_commit(bar + kBKEmpty + 8 * (cur & 1));
         }
-        tc_commit(bar + kBOFull);
-        tc_commit(bar + kBVEmpty + 8 * st);
+        it += n;
       }
       // Drain: every MMA issued above has completed once this arrives.
       tc_commit(bar + kBDone);
       mbar_wait(bar + kBDone, 0, p.wait, nullptr, kSitePrefillDrain);
     }
   } else {
-    // ------------------------------------------------------------------ softmax warpgroup
-    const int wq = warp & 3;          // TMEM lane quadrant this warp may access
-    const int row = wq * 32 + lane;   // query-tile row owned by this thread
-    {
-      // Q prologue: warp (warp-2) normalises and rotates rows [32*(warp-2), +32).
-      const float2 ga = reinterpret_cast<const float2*>(p.q_norm_w)[lane];
-      const float2 gb = reinterpret_cast<const float2*>(p.q_norm_w)[32 + lane];
-      const float hi0 = p.rope.hi[2 * lane], lo0 = p.rope.lo[2 * lane];
-      const float hi1 = p.rope.hi[2 * lane + 1], lo1 = p.rope.lo[2 * lane + 1];
-      float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
-      int cur_t = -1;
-      const int rbase = (warp - 2) * 32;
-      for (int rr = 0; rr < 32; ++rr) {
-        const int r = rbase + rr;
-        const int t = t0 + (r >> p.log2G);
-        uint32_t wa = 0u, wb = 0u;
-        if (t < p.T) {  // uniform across the warp
-          if (t != cur_t) {
-            const int ps = p.pos[static_cast<long long>(b) * p.T + t];
-            rope_sincos(ps, hi0, lo0, s0, c0);
-            rope_sincos(ps, hi1, lo1, s1, c1);
-            cur_t = t;
-          }
-          const int h = hkv * G + (r & (G - 1));
-          const uint32_t* qs = p.q + (static_cast<long long>(b * p.T + t) * p.Hq + h) * (kD / 2);
-          const uint32_t ua = qs[lane], ub = qs[32 + lane];
-          float2 ya, yb;
-          norm_rope_pairs(make_float2(bf16lo(ua), bf16hi(ua)), make_float2(bf16lo(ub), bf16hi(ub)), ga, gb, s0, c0,
-                          s1, c1, p.eps, ya, yb);
-          wa = pack_bf16x2(ya.x, ya.y);
-          wb = pack_bf16x2(yb.x, yb.y);
-        }
-        const uint32_t off = sw128_offset(r, lane >> 2) + (lane & 3) * 4;
-        st_shared_u32(sQ + off, wa);
-        st_shared_u32(sQ + kPfBox + off, wb);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(bar + kBQReady);
-    }
-
-    const int t_row = t0 + (row >> p.log2G);
-    const int lim = min(t_row, p.T - 1);  // last key index this row may see
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int X = (warp - 2) >> 2;     // 0: tile A, 1: tile B
+    const int wq = warp & 3;           // TMEM lane quadrant this warp may access
+    const int row = wq * 32 + lane;    // query-tile row owned by this thread
+    const int rbase = ((warp - 2) & 3) * 32;  // rows this warp normalises in the Q prologue
+    const uint32_t sQ = sb + kPfQ + X * kPfTile;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tO = tmem + 256 + lane_off;
+    const uint32_t tS = tmem + lane_off + tm_s(X), tO = tmem + lane_off + tm_o(X);
     const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
+    const int G = 1 << p.log2G;
+    const float2 ga = reinterpret_cast<const float2*>(p.q_norm_w)[lane];
+    const float2 gb = reinterpret_cast<const float2*>(p.q_norm_w)[32 + lane];
+    const float hi0 = p.rope.hi[2 * lane], lo0 = p.rope.lo[2 * lane];
+    const float hi1 = p.rope.hi[2 * lane + 1], lo1 = p.rope.lo[2 * lane + 1];
+    uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      ok = mbar_wait(bar + kBSFull + 8 * (j & 1), (j >> 1) & 1, p.wait, abort_flag, kSitePrefillSFull);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      float s[128];
-      const uint32_t tS = tmem + lane_off + (j & 1) * 128;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      int pair, b, hkv;
+      item_coords(p, item, pair, b, hkv);
+      const TileInfo ti = tile_info(p, 2 * pair + X);
+      if (ti.nkv == 0) continue;
+      const int t0 = ti.t0;
+      {
+        // Q prologue: this warp's 32 rows, in two batches of 16 whose loads are all issued
+        // before any arithmetic.
+        const int tl = t0 + ((rbase + lane) >> p.log2G);
+        const int pos_l = (tl < p.T) ? p.pos[static_cast<long long>(b) * p.T + tl] : 0;
+        float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
+        int cur_pos = 0x7fffffff;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          uint32_t ua[16], ub[16];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + c * 32, r);
+          for (int rr = 0; rr < 16; ++rr) {
+            const int r = rbase + half * 16 + rr;
+            const int t = t0 + (r >> p.log2G);
+            ua[rr] = ub[rr] = 0u;
+            if (t < p.T) {
+              const uint32_t* qs =
+                  p.q + (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (r & (G - 1))) * (kD / 2);
+              ua[rr] = __ldg(qs + lane);
+              ub[rr] = __ldg(qs + 32 + lane);
+            }
+          }
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+          for (int rr = 0; rr < 16; ++rr) {
+            const int r = rbase + half * 16 + rr;
+            const int t = t0 + (r >> p.log2G);
+            uint32_t wa = 0u, wb = 0u;
+            const int ps = __shfl_sync(0xffffffffu, pos_l, half * 16 + rr);
+            if (t < p.T) {  // uniform across the warp
+              if (ps != cur_pos) {
+                rope_sincos(ps, hi0, lo0, s0, c0);
+                rope_sincos(ps, hi1, lo1, s1, c1);
+                cur_pos = ps;
+              }
+              float2 ya, yb;
+              norm_rope_pairs(make_float2(bf16lo(ua[rr]), bf16hi(ua[rr])),
+                              make_float2(bf16lo(ub[rr]), bf16hi(ub[rr])), ga, gb, s0, c0, s1, c1, p.eps, ya, yb);
+              wa = pack_bf16x2(ya.x, ya.y);
+              wb = pack_bf16x2(yb.x, yb.y);
+            }
+            const uint32_t off = sw128_offset(r, lane >> 2) + (lane & 3) * 4;
+            st_shared_u32(sQ + off, wa);
+            st_shared_u32(sQ + kPfBox + off, wb);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar + kBQReady + 8 * X);
       }
-      const int kv0 = j * 128;
-      if (kv0 + 127 > t0) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = (kv0 + c <= lim) ? s[c] : -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float mt = mx * sl2;
-      float m_new = m;
-      bool resc = false;
-      if (mt > m + 8.0f) {  // lazy rescale: keep a stale max while p stays <= 2^8
-        m_new = mt;
-        resc = (j > 0);
-      }
-      uint32_t pk[64];
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = ex2(fmaf(s[c], sl2, -m_new));
-        const float p1 = ex2(fmaf(s[c + 1], sl2, -m_new));
-        sum += p0 + p1;  // fp32 row sum; P.V uses the bf16-rounded p
-        pk[c >> 1] = pack_bf16x2(p0, p1);
-      }
-      if (j > 0) {
-        ok = mbar_wait(bar + kBOFull, (j - 1) & 1, p.wait, abort_flag, kSitePrefillOFull);
+
+      const int t_row = t0 + (row >> p.log2G);
+      const int lim = min(t_row, p.T - 1);  // last key index this row may see
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < ti.nkv; ++j) {
+        ok = mbar_wait(bar + kBSFull + 8 * X, s_cnt & 1, p.wait, abort_flag, kSitePrefillSFull);
+        ++s_cnt;
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-      }
-      if (__any_sync(0xffffffffu, resc)) {
-        const float alpha = resc ? ex2(m - m_new) : 1.0f;
+        float s[128];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
+          tmem_ld32(tS + c * 32, r);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + c * 32, r);
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
         }
-        l *= alpha;
-      }
-      l += sum;
-      m = m_new;
+        const int kv0 = j * 128;
+        if (kv0 + 127 > t0) {
 #pragma unroll
-      for (int cb = 0; cb < 16; ++cb)
-        st_shared_v4(sP + (cb >> 3) * kPfBox + sw128_offset(row, cb & 7), pk[4 * cb], pk[4 * cb + 1], pk[4 * cb + 2],
-                     pk[4 * cb + 3]);
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar + kBPReady);
-    }
-    if (ok) {
-      ok = mbar_wait(bar + kBOFull, (nkv - 1) & 1, p.wait, abort_flag, kSitePrefillOFull);
+          for (int c = 0; c < 128; ++c) s[c] = (kv0 + c <= lim) ? s[c] : -INFINITY;
+        }
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float mt = mx * sl2;
+        float m_new = m;
+        bool resc = false;
+        if (mt > m + 8.0f) {  // lazy rescale: keep a stale max while p stays <= 2^8
+          m_new = mt;
+          resc = (j > 0);
+        }
+        // p = 2^(s*scale*log2(e) - m): bf16 pairs go straight to P's TMEM columns, 16 at a
+        // time, so the packed tile is never live in registers all at once.
+        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, -m_new));
+            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -m_new));
+            sum4[i & 3] += p0 + p1;  // fp32 row sum; P.V uses the bf16-rounded p
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16_nowait(tS + kTmPOff + 16 * c, pk);
+        }
+        if (__any_sync(0xffffffffu, resc)) {
+          // PV_X(j-1) has completed: the commit that signalled S_X(j) covers it.
+          const float alpha = resc ? ex2(m - m_new) : 1.0f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + c * 32, r);
+          }
+          l *= alpha;
+        }
+        tmem_wait_st();
+        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        m = m_new;
+        tc_fence_before();
+        mbar_arrive(bar + kBPReady + 8 * X);
+      }
+      if (!ok) break;
+      ok = mbar_wait(bar + kBOFull + 8 * X, o_cnt & 1, p.wait, abort_flag, kSitePrefillOFull);
+      ++o_cnt;
       ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) break;
       tc_fence_after();
       const int h = hkv * G + (row & (G - 1));
       const bool valid = t_row < p.T;

@@ -105,6 +105,19 @@ int ensure_kernel_attrs() {
   return QWEN3_OK;
 }
 
+// Streaming multiprocessors of the current device (148 on B200), cached per device.
+int num_sms() {
+  static int sms[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
 int check_common(int Hq, int Hkv, int d) {
   if (Hq <= 0 || Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
   if (d != kD) return QWEN3_ERR_UNSUPPORTED;
@@ -130,8 +143,10 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.rope = make_rope_table(theta);
   const long long nvec = static_cast<long long>(B) * T * H;
   const int warps = 8;
-  long long blocks = (nvec + warps - 1) / warps;
-  if (blocks > 148LL * 64) blocks = 148LL * 64;  // grid-stride beyond ~64 blocks per SM
+  const long long per_block = static_cast<long long>(warps) * q3::kPrologueUnroll;
+  long long blocks = (nvec + per_block - 1) / per_block;
+  const long long cap = static_cast<long long>(num_sms()) * 16;  // grid-stride beyond 16 blocks per SM
+  if (blocks > cap) blocks = cap;
   q3::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
@@ -279,6 +294,10 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   p.log2G = ilog2(Hq / Hkv);
   p.P = 128 >> p.log2G;
   p.n_qt = (T + p.P - 1) / p.P;
+  p.n_pairs = (p.n_qt + 1) / 2;
+  const long long n_items = static_cast<long long>(p.n_pairs) * B * Hkv;
+  if (n_items > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  p.n_items = static_cast<int>(n_items);
   p.eps = eps;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
   p.wait = next_wait_cfg();
@@ -287,9 +306,8 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
     p.fault = g_fault;
   }
   p.rope = make_rope_table(theta);
-  const long long grid = static_cast<long long>(B) * Hkv * p.n_qt;
-  if (grid > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
-  q3::fmha_prefill_kernel<<<static_cast<unsigned>(grid), q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
+  const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
+  q3::fmha_prefill_kernel<<<grid, q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
