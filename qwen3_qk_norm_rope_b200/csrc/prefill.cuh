@@ -27,8 +27,8 @@
 //               causal mask, exp2 online softmax with a lazy rescale (O is rescaled only
 //               when the running max grows by more than 2^8), bf16 P written back into TMEM
 //               over its own S columns; finally O/l and the LSE.
-// TMEM (512 columns): S_A [0,128) with P_A at [32,96), O_A [128,256), S_B [256,384) with
-// P_B at [288,352), O_B [384,512).  PV reads P from TMEM (the TS form of tcgen05.mma).
+// TMEM (512 columns): S_A [0,128) with P_A at [0,64), O_A [128,256), S_B [256,384) with
+// P_B at [256,320), O_B [384,512).  PV reads P from TMEM (the TS form of tcgen05.mma).
 // Ordering: one thread issues every MMA and they complete in issue order, so the commit
 // that signals S_X(j) also covers PV_X(j-1): once a softmax thread sees S_X(j) it may
 // overwrite P_X and rescale O_X without a further wait.
@@ -63,7 +63,7 @@ constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSF
                    kBOFull = 96, kBQReady = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140;
 constexpr uint32_t kPrefillSmemBytes = kPfBar + 256 + 1024;  // + slack to align the base to 1024
 constexpr int kPrefillThreads = 320;
-constexpr uint32_t kTmPOff = 32;  // P within S
+constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
 constexpr float kLn2 = 0.693147180559945309f;
 
 __device__ __forceinline__ uint32_t tm_s(int X) { return X == 0 ? 0u : 256u; }
@@ -73,6 +73,23 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for part of the exponentials so the MUFU unit (16/clk/SM) stops
+// being the softmax bottleneck.  Cody-Waite style split x = n + r, n = rint(x) (by adding
+// and subtracting 1.5*2^23), |r| <= 1/2; 2^r by a degree-4 polynomial whose coefficients
+// were fitted here for minimal relative error on [-1/2, 1/2] (max 2.7e-6 in fp32, against
+// bf16's 2^-9 for P); 2^n by adding n to the exponent field.  x is clamped at -126 so the
+// result stays a normal float (masked entries give 2^-126 instead of 0: negligible).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = __fadd_rn(x, 12582912.0f);
+  const float r = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
+  float q = fmaf(0.00956961140036583f, r, 0.05591781809926033f);
+  q = fmaf(q, r, 0.24024756252765656f);
+  q = fmaf(q, r, 0.6931218504905701f);
+  q = fmaf(q, r, 0.9999992847442627f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]: the TS form, A (here P) read from tensor memory.
@@ -95,6 +112,14 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt) {
   ti.t0 = qt * p.P;
   ti.nkv = (ti.t0 < p.T) ? (min(ti.t0 + p.P, p.T) - 1) / 128 + 1 : 0;
   return ti;
+}
+
+// Item this CTA takes in round k: snake order (left to right in even rounds, right to left
+// in odd ones) over the heaviest-first numbering, so the heaviest and lightest items of
+// consecutive rounds land on the same CTA.
+__device__ __forceinline__ int round_item(int k) {
+  return (k & 1) ? k * static_cast<int>(gridDim.x) + static_cast<int>(gridDim.x - 1 - blockIdx.x)
+                 : k * static_cast<int>(gridDim.x) + static_cast<int>(blockIdx.x);
 }
 
 // Work item -> (pair, batch row, KV head); items are numbered heaviest pair first.
@@ -151,7 +176,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
       uint32_t it = 0;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
         const int n = max(tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv);
@@ -191,7 +216,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t kIdPV = idesc_bf16(128, 128, true);   // B = V, dims contiguous (MN-major)
       uint32_t it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
         const int nX[2] = {tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv};
@@ -276,7 +301,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const float hi1 = p.rope.hi[2 * lane + 1], lo1 = p.rope.lo[2 * lane + 1];
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
       int pair, b, hkv;
       item_coords(p, item, pair, b, hkv);
       const TileInfo ti = tile_info(p, 2 * pair + X);
@@ -340,47 +365,63 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tS + c * 32, r);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
-        }
+        // Pass 1: the row max over all 128 keys (one TMEM load).  Pass 2 re-reads S in
+        // 32-column chunks, so only one chunk is live while its exponentials are formed.
         const int kv0 = j * 128;
-        if (kv0 + 127 > t0) {
+        const bool diag = kv0 + 127 > t0;  // some key of this tile lies past some row's position
+        float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = (kv0 + c <= lim) ? s[c] : -INFINITY;
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t sr[64];
+          tmem_ld64(tS + 64 * hh, sr);
+          if (diag) {
+#pragma unroll
+            for (int c = 0; c < 64; ++c) sr[c] = (kv0 + 64 * hh + c <= lim) ? sr[c] : 0xff800000u;  // -inf
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 2)
+            mx4[(c >> 1) & 3] = fmax3(mx4[(c >> 1) & 3], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
         }
-        float mx8[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = s[i];
-#pragma unroll
-        for (int c = 8; c < 128; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float mt = mx * sl2;
+        const float mt = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl2;
         float m_new = m;
         bool resc = false;
         if (mt > m + 8.0f) {  // lazy rescale: keep a stale max while p stays <= 2^8
           m_new = mt;
           resc = (j > 0);
         }
-        // p = 2^(s*scale*log2(e) - m): bf16 pairs go straight to P's TMEM columns, 16 at a
-        // time, so the packed tile is never live in registers all at once.
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        // Pass 2: p = 2^(s*scale*log2(e) - m) on pairs; bf16 pairs go straight to P's TMEM
+        // columns.  P occupies S columns [0,64): chunk c of P (columns [16c,16c+16)) only
+        // overwrites S columns that chunks 0..c have already read.
+        const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(-m_new, -m_new);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
+          uint32_t sr[32];
+          tmem_ld32(tS + 32 * c, sr);
+          if (diag) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sr[i] = (kv0 + 32 * c + i <= lim) ? sr[i] : 0xff800000u;
+          }
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, -m_new));
-            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, -m_new));
-            sum4[i & 3] += p0 + p1;  // fp32 row sum; P.V uses the bf16-rounded p
+            float x0, x1;
+            f2unpack(ffma2(f2pack(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sl2x2, negm2), x0,
+                     x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));  // fp32 row sum; P.V uses bf16 p
             pk[i] = pack_bf16x2(p0, p1);
           }
           tmem_st16_nowait(tS + kTmPOff + 16 * c, pk);
+        }
+        float sum;
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2unpack(acc[0], a0, a1);
+          f2unpack(acc[1], b0, b1);
+          f2unpack(acc[2], c0, c1);
+          f2unpack(acc[3], d0, d1);
+          sum = ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
         }
         if (__any_sync(0xffffffffu, resc)) {
           // PV_X(j-1) has completed: the commit that signalled S_X(j) covers it.
@@ -396,7 +437,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           l *= alpha;
         }
         tmem_wait_st();
-        l += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        l += sum;
         m = m_new;
         tc_fence_before();
         mbar_arrive(bar + kBPReady + 8 * X);

@@ -141,10 +141,10 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.write_at_pos = write_at_pos;
   p.eps = eps;
   p.rope = make_rope_table(theta);
-  const long long nvec = static_cast<long long>(B) * T * H;
+  const long long ntok = static_cast<long long>(B) * T;
+  if (ntok > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   const int warps = 8;
-  const long long per_block = static_cast<long long>(warps) * q3::kPrologueUnroll;
-  long long blocks = (nvec + per_block - 1) / per_block;
+  long long blocks = (ntok + warps - 1) / warps;  // one warp per token
   const long long cap = static_cast<long long>(num_sms()) * 16;  // grid-stride beyond 16 blocks per SM
   if (blocks > cap) blocks = cap;
   q3::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
