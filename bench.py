@@ -291,7 +291,9 @@ def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seq
 
 
 # ------------------------------------------------------------------------------ main
-def dist_setup(n_gpus: int):
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (torchrun env).  The process group only carries the timing
+    plumbing (barriers and the max over ranks); the data path has no collective."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -300,9 +302,12 @@ def dist_setup(n_gpus: int):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return world, rank, local
 
 
@@ -378,7 +383,7 @@ def main():
                     help="decode the first n of the 64 sequences (small cases for ncu captures)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = dist_setup("nccl")
     if args.impl == "reference":
         run_reference(args, world, rank)
         if world > 1:

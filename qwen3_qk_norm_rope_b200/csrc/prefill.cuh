@@ -75,23 +75,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for part of the exponentials so the MUFU unit (16/clk/SM) stops
-// being the softmax bottleneck.  Cody-Waite style split x = n + r, n = rint(x) (by adding
-// and subtracting 1.5*2^23), |r| <= 1/2; 2^r by a degree-4 polynomial whose coefficients
-// were fitted here for minimal relative error on [-1/2, 1/2] (max 2.7e-6 in fp32, against
-// bf16's 2^-9 for P); 2^n by adding n to the exponent field.  x is clamped at -126 so the
-// result stays a normal float (masked entries give 2^-126 instead of 0: negligible).
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = __fadd_rn(x, 12582912.0f);
-  const float r = __fsub_rn(x, __fsub_rn(t, 12582912.0f));
-  float q = fmaf(0.00956961140036583f, r, 0.05591781809926033f);
-  q = fmaf(q, r, 0.24024756252765656f);
-  q = fmaf(q, r, 0.6931218504905701f);
-  q = fmaf(q, r, 0.9999992847442627f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-
 // D[tmem] (+)= A[tmem] * B[smem desc]: the TS form, A (here P) read from tensor memory.
 __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
                                           uint32_t accumulate) {
