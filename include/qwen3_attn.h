@@ -81,9 +81,10 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos,
  *   q_norm_w, k_norm_w  [d] fp32 gains.
  *   pos       [B, T] int32 RoPE positions.
  *   out       [B, T, Hq, d] bf16 attention output (heads not merged with o_proj).
- * The K prologue result needs B*Hkv*T*d*2 bytes of scratch, which this call obtains
- * stream-ordered with cudaMallocAsync/cudaFreeAsync on `stream`.  Use
- * qwen3_attn_prefill_ex to pass your own workspace or to fill a KV cache instead.
+ * The call needs qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes of scratch (the
+ * normed+rotated keys and each token's RoPE cos/sin), which it obtains stream-ordered with
+ * cudaMallocAsync/cudaFreeAsync on `stream`.  Use qwen3_attn_prefill_ex to pass your own
+ * workspace or to fill a KV cache instead.
  */
 int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
                        const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
@@ -98,10 +99,11 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
  *   k_cache, v_cache  optional [B, Hkv, Tcap, d] bf16 (Tcap >= T).  When given (both or
  *             neither), the normed+rotated keys and the raw values of tokens 0..T-1 are
  *             written to slots 0..T-1 and attention reads them from there, so the cache is
- *             ready for qwen3_attn_decode with cache_lens = T.  No workspace is needed.
- *   workspace, ws_bytes  scratch for the keys when no cache is given; ws_bytes must be at
- *             least qwen3_attn_prefill_workspace_size(B, T, Hkv, d), else
- *             QWEN3_ERR_WORKSPACE.  Ignored when a cache is given.
+ *             ready for qwen3_attn_decode with cache_lens = T.
+ *   workspace, ws_bytes  device scratch of at least
+ *             qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes, else
+ *             QWEN3_ERR_WORKSPACE.  It holds the normed+rotated keys (unused when a cache is
+ *             given) and every token's RoPE cos/sin, shared by the key and query prologues.
  */
 int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
                           const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
@@ -167,7 +169,8 @@ int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
                               int N, int Hq, int Hkv, int d, int Lmax,
                               float theta, float eps, qwen3_stream_t stream);
 
-/* Scratch bytes qwen3_attn_prefill_ex needs when it is given no KV cache. */
+/* Scratch bytes qwen3_attn_prefill_ex needs: B*Hkv*T*d*2 (keys) + B*T*512 (RoPE cos/sin),
+ * plus alignment slack. */
 size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d);
 
 /* Scratch bytes qwen3_attn_decode needs (split-KV partial outputs and logsumexps). */

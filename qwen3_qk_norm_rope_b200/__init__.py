@@ -150,9 +150,9 @@ def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: floa
         Tcap = k_cache.shape[2]
         _need(k_cache, "k_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
         _need(v_cache, "v_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
-    elif workspace is None:
+    if workspace is None:
         workspace = torch.empty(prefill_workspace_size(B, T, Hkv, d), dtype=torch.uint8, device=dev)
-    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qwen3_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
                                        _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
                                        _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),

@@ -121,32 +121,52 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
-// Bounded wait on an mbarrier phase.  Returns false when the wait ran out (the error is
-// recorded, *abort is raised so the other roles of this CTA stop, and the launch is marked
-// so the other CTAs stop too), or when this CTA or launch has already aborted.  Pass
-// abort == nullptr to wait regardless (used when draining copies still in flight).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCfg& w, volatile int* abort,
-                                       int site) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Non-blocking probe of an mbarrier phase (no suspension).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// The waiting part of mbar_wait, out of line so the common already-complete case costs
+// one inline probe rather than a call.
+__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, uint64_t limit_ns, uint64_t launch_id,
+                                            volatile int* abort, int site) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 15u) == 0u) {
       if (abort != nullptr) {
         if (*abort != 0) return false;
-        if (*reinterpret_cast<volatile unsigned long long*>(&g_abort_launch) == w.launch_id) {
+        if (*reinterpret_cast<volatile unsigned long long*>(&g_abort_launch) == launch_id) {
           *abort = 1;
           return false;
         }
       }
-      if (global_timer_ns() - t0 > w.limit_ns) {
+      if (global_timer_ns() - t0 > limit_ns) {
         record_error(QWEN3_ERR_DEVICE_TIMEOUT, site);
-        atomicExch(&g_abort_launch, static_cast<unsigned long long>(w.launch_id));
+        atomicExch(&g_abort_launch, static_cast<unsigned long long>(launch_id));
         if (abort != nullptr) *abort = 1;
         return false;
       }
     }
   }
+}
+
+// Bounded wait on an mbarrier phase.  Returns false when the wait ran out (the error is
+// recorded, *abort is raised so the other roles of this CTA stop, and the launch is marked
+// so the other CTAs stop too), or when this CTA or launch has already aborted.  Pass
+// abort == nullptr to wait regardless (used when draining copies still in flight).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const WaitCfg& w, volatile int* abort,
+                                          int site) {
+  if (mbar_test(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, w.limit_ns, w.launch_id, abort, site);
 }
 
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, tcgen05.mma).
@@ -247,6 +267,33 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
+// 32 lanes x 32 columns, no wait: the registers are not valid until tmem_wait_ld_dep(r).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : Q3_R8(0), Q3_R8(8), Q3_R8(16), Q3_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+#define Q3_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]), \
+                  "+r"(r[i + 6]), "+r"(r[i + 7])
+// Wait for outstanding TMEM loads; naming r as read-write keeps every use of r below it.
+__device__ __forceinline__ void tmem_wait_ld_dep(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" : Q3_RW8(0), Q3_RW8(8), Q3_RW8(16), Q3_RW8(24) : : "memory");
+}
+// 32 lanes x 16 columns, with its wait.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : Q3_R8(0), Q3_R8(8)
+      : "r"(taddr)
+      : "memory");
+}
+
 // 32 lanes x 64 consecutive fp32 columns in one load, with its wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
   asm volatile(
@@ -297,6 +344,11 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

@@ -23,7 +23,8 @@
 //               warpgroup of the other tile runs.
 //   warps 2-5   softmax warpgroup of tile A, one thread per row (TMEM lane quadrant =
 //   warps 6-9   warp % 4); softmax warpgroup of tile B.  Each runs the Q prologue of its
-//               tile into swizzled smem, then per key tile: tcgen05.ld of its S row,
+//               tile (thread per row, angles from the table the K prologue wrote) into
+//               swizzled smem, then per key tile: tcgen05.ld of its S row,
 //               causal mask, exp2 online softmax with a lazy rescale (O is rescaled only
 //               when the running max grows by more than 2^8), bf16 P written back into TMEM
 //               over its own S columns; finally O/l and the LSE.
@@ -42,14 +43,13 @@ namespace q3 {
 struct PrefillParams {
   const uint32_t* q;  // [B, T, Hq, d] bf16 pairs
   const float* q_norm_w;
-  const int* pos;  // [B, T]
+  const float4* rope_tab;  // [B*T][32]: (cos, sin) of frequencies 2i, 2i+1 at each token's position
   uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
   int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
   float eps, scale_log2;
   WaitCfg wait;
   int fault;
-  RopeTable rope;
 };
 
 constexpr uint32_t kPfTile = 32768;  // 128 rows x 128 bf16
@@ -272,16 +272,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int X = (warp - 2) >> 2;     // 0: tile A, 1: tile B
     const int wq = warp & 3;           // TMEM lane quadrant this warp may access
     const int row = wq * 32 + lane;    // query-tile row owned by this thread
-    const int rbase = ((warp - 2) & 3) * 32;  // rows this warp normalises in the Q prologue
     const uint32_t sQ = sb + kPfQ + X * kPfTile;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + tm_s(X), tO = tmem + lane_off + tm_o(X);
     const float sl2 = p.scale_log2;
     const int G = 1 << p.log2G;
-    const float2 ga = reinterpret_cast<const float2*>(p.q_norm_w)[lane];
-    const float2 gb = reinterpret_cast<const float2*>(p.q_norm_w)[32 + lane];
-    const float hi0 = p.rope.hi[2 * lane], lo0 = p.rope.lo[2 * lane];
-    const float hi1 = p.rope.hi[2 * lane + 1], lo1 = p.rope.lo[2 * lane + 1];
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
     for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
@@ -291,50 +286,49 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (ti.nkv == 0) continue;
       const int t0 = ti.t0;
       {
-        // Q prologue: this warp's 32 rows, in two batches of 16 whose loads are all issued
-        // before any arithmetic.
-        const int tl = t0 + ((rbase + lane) >> p.log2G);
-        const int pos_l = (tl < p.T) ? p.pos[static_cast<long long>(b) * p.T + tl] : 0;
-        float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
-        int cur_pos = 0x7fffffff;
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
-          uint32_t ua[16], ub[16];
+        // Q prologue, one thread per row: QK-Norm of the raw row (a register-local sum of
+        // squares), gain, and rotate-half RoPE with the (cos, sin) of the row's position that
+        // the K-prologue kernel left in rope_tab; then the row goes to swizzled smem as 16
+        // chunks of 16 bytes (row r, chunk c at c ^ (r % 8): conflict-free across a warp).
+        const int t = t0 + (row >> p.log2G);
+        uint32_t w[64];  // bf16 pairs: w[i] = dims (2i, 2i+1)
+        if (t < p.T) {   // rows past T get Q' = 0
+          const uint4* qs = reinterpret_cast<const uint4*>(p.q) +
+                            (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 8);
 #pragma unroll
-          for (int rr = 0; rr < 16; ++rr) {
-            const int r = rbase + half * 16 + rr;
-            const int t = t0 + (r >> p.log2G);
-            ua[rr] = ub[rr] = 0u;
-            if (t < p.T) {
-              const uint32_t* qs =
-                  p.q + (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (r & (G - 1))) * (kD / 2);
-              ua[rr] = __ldg(qs + lane);
-              ub[rr] = __ldg(qs + 32 + lane);
-            }
+          for (int i = 0; i < 16; ++i) {
+            const uint4 u = __ldg(qs + i);
+            w[4 * i] = u.x;
+            w[4 * i + 1] = u.y;
+            w[4 * i + 2] = u.z;
+            w[4 * i + 3] = u.w;
           }
+          float ss4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int rr = 0; rr < 16; ++rr) {
-            const int r = rbase + half * 16 + rr;
-            const int t = t0 + (r >> p.log2G);
-            uint32_t wa = 0u, wb = 0u;
-            const int ps = __shfl_sync(0xffffffffu, pos_l, half * 16 + rr);
-            if (t < p.T) {  // uniform across the warp
-              if (ps != cur_pos) {
-                rope_sincos(ps, hi0, lo0, s0, c0);
-                rope_sincos(ps, hi1, lo1, s1, c1);
-                cur_pos = ps;
-              }
-              float2 ya, yb;
-              norm_rope_pairs(make_float2(bf16lo(ua[rr]), bf16hi(ua[rr])),
-                              make_float2(bf16lo(ub[rr]), bf16hi(ub[rr])), ga, gb, s0, c0, s1, c1, p.eps, ya, yb);
-              wa = pack_bf16x2(ya.x, ya.y);
-              wb = pack_bf16x2(yb.x, yb.y);
-            }
-            const uint32_t off = sw128_offset(r, lane >> 2) + (lane & 3) * 4;
-            st_shared_u32(sQ + off, wa);
-            st_shared_u32(sQ + kPfBox + off, wb);
+          for (int i = 0; i < 64; ++i) {
+            const float x0 = bf16lo(w[i]), x1 = bf16hi(w[i]);
+            ss4[i & 3] = fmaf(x0, x0, fmaf(x1, x1, ss4[i & 3]));
           }
+          const float r = rsqrtf(fmaf((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), 1.0f / kD, p.eps));
+          const float4* tab = p.rope_tab + static_cast<size_t>(b * p.T + t) * 32;
+          const float2* g2 = reinterpret_cast<const float2*>(p.q_norm_w);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
+            const float4 cs = __ldg(tab + i);  // (cos f0, sin f0, cos f1, sin f1)
+            const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
+            const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
+            const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
+            w[i] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
+            w[32 + i] = pack_bf16x2(b0 * cs.x + a0 * cs.y, b1 * cs.z + a1 * cs.w);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) w[i] = 0u;
         }
+#pragma unroll
+        for (int cb = 0; cb < 16; ++cb)
+          st_shared_v4(sQ + (cb >> 3) * kPfBox + sw128_offset(row, cb & 7), w[4 * cb], w[4 * cb + 1], w[4 * cb + 2],
+                       w[4 * cb + 3]);
         fence_proxy_async_smem();
         mbar_arrive(bar + kBQReady + 8 * X);
       }

@@ -19,6 +19,7 @@ struct PrologueParams {
   uint32_t* dst;       // [B, H, Tcap, d] bf16 pairs
   const uint2* v_src;  // optional [B, T, H, d], 4 bf16 per lane
   uint2* v_dst;        // optional [B, H, Tcap, d]
+  float4* rope_tab;    // optional [B*T][32]: (cos, sin) of frequencies 2i, 2i+1 at pos[b,t]
   int B, T, H, Tcap, write_at_pos;
   float eps;
   RopeTable rope;
@@ -27,7 +28,8 @@ struct PrologueParams {
 constexpr int kPrologueHeads = 8;  // head vectors of one token in flight per warp
 
 // One warp per token (b, t): its position and the sin/cos of its 64 angles are computed
-// once and shared by the token's H head vectors, whose loads are all issued first.
+// once and shared by the token's H head vectors, whose loads are all issued first.  The
+// prefill also keeps the angles (rope_tab) for the query tiles of the attention kernel.
 __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant__ PrologueParams p) {
   // The RoPE constants go through shared memory once per block: read from parameter space
   // with a lane-dependent index they would serialise.
@@ -54,6 +56,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     float s0, c0, s1, c1;
     rope_sincos(ps, hi0, lo0, s0, c0);
     rope_sincos(ps, hi1, lo1, s1, c1);
+    if (p.rope_tab != nullptr) p.rope_tab[static_cast<size_t>(bt) * 32 + lane] = make_float4(c0, s0, c1, s1);
     for (int h0 = 0; h0 < p.H; h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
       uint2 vv[kPrologueHeads];

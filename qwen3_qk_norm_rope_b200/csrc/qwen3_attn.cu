@@ -118,6 +118,11 @@ int num_sms() {
   return sms[dev];
 }
 
+// Bytes of the K' region of the prefill workspace (rounded to keep what follows aligned).
+size_t kspace_bytes(int B, int T, int Hkv, int d) {
+  return (static_cast<size_t>(B) * Hkv * T * d * 2 + 255) & ~static_cast<size_t>(255);
+}
+
 int check_common(int Hq, int Hkv, int d) {
   if (Hq <= 0 || Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
   if (d != kD) return QWEN3_ERR_UNSUPPORTED;
@@ -126,7 +131,8 @@ int check_common(int Hq, int Hkv, int d) {
 }
 
 int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
-                    int B, int T, int H, int Tcap, int write_at_pos, float theta, float eps, cudaStream_t stream) {
+                    int B, int T, int H, int Tcap, int write_at_pos, float theta, float eps, cudaStream_t stream,
+                    void* rope_tab = nullptr) {
   q3::PrologueParams p;
   p.x = static_cast<const uint32_t*>(x);
   p.w = w;
@@ -134,6 +140,7 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.dst = static_cast<uint32_t*>(dst);
   p.v_src = static_cast<const uint2*>(v_src);
   p.v_dst = static_cast<uint2*>(v_dst);
+  p.rope_tab = static_cast<float4*>(rope_tab);
   p.B = B;
   p.T = T;
   p.H = H;
@@ -195,7 +202,8 @@ int qwen3_attn_device_status(qwen3_stream_t stream, int clear, int* site) {
 
 size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d) {
   if (B <= 0 || T <= 0 || Hkv <= 0 || d <= 0) return 0;
-  return static_cast<size_t>(B) * Hkv * T * d * 2 + 256;
+  // K' [B, Hkv, T, d] bf16, then the per-token cos/sin table [B*T][64] float2
+  return kspace_bytes(B, T, Hkv, d) + static_cast<size_t>(B) * T * 64 * 8 + 256;
 }
 
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax) {
@@ -244,22 +252,21 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
     return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
-  if (!use_cache) {
-    if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
-      return QWEN3_ERR_WORKSPACE;
-  }
+  if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
+    return QWEN3_ERR_WORKSPACE;
   if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
     return QWEN3_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
 
-  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] (and V copied when filling a cache).
-  qwen3_bf16* kdst = use_cache ? k_cache
-                               : reinterpret_cast<qwen3_bf16*>((reinterpret_cast<uintptr_t>(workspace) + 255) &
-                                                               ~static_cast<uintptr_t>(255));
+  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] (and V copied when filling a cache);
+  //    it also leaves every token's RoPE cos/sin in the workspace for the query tiles.
+  const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
+  qwen3_bf16* kdst = use_cache ? k_cache : reinterpret_cast<qwen3_bf16*>(w0);
+  void* rope_tab = reinterpret_cast<void*>(w0 + kspace_bytes(B, T, Hkv, d));
   const int Tc = use_cache ? Tcap : T;
   st = launch_prologue(k, k_norm_w, pos, kdst, use_cache ? v : nullptr, use_cache ? v_cache : nullptr, B, T, Hkv,
-                       Tc, 0, theta, eps, s);
+                       Tc, 0, theta, eps, s, rope_tab);
   if (st != QWEN3_OK) return st;
 
   // 2. Tensor maps.  The key-axis extent is T (not Tcap) so slots past the prompt read as zeros.
@@ -284,7 +291,7 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   q3::PrefillParams p;
   p.q = reinterpret_cast<const uint32_t*>(q);
   p.q_norm_w = q_norm_w;
-  p.pos = pos;
+  p.rope_tab = static_cast<const float4*>(rope_tab);
   p.out = reinterpret_cast<uint4*>(out);
   p.lse = lse;
   p.B = B;
@@ -305,7 +312,6 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
     std::lock_guard<std::mutex> lk(g_mu);
     p.fault = g_fault;
   }
-  p.rope = make_rope_table(theta);
   const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
   q3::fmha_prefill_kernel<<<grid, q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
