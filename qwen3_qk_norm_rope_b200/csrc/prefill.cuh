@@ -277,61 +277,98 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const uint32_t tS = tmem + lane_off + tm_s(X), tO = tmem + lane_off + tm_o(X);
     const float sl2 = p.scale_log2;
     const int G = 1 << p.log2G;
+    // Q prologue of the query tile at (b, hkv, t0) into Q'_X, then signal qready_X.
+    auto q_prologue = [&](int b, int hkv, int t0) {
+      // Q prologue, one thread per row: QK-Norm of the raw row (a register-local sum of
+      // squares), gain, and rotate-half RoPE with the (cos, sin) of the row's position that
+      // the K-prologue kernel left in rope_tab; then the row goes to swizzled smem as 16
+      // chunks of 16 bytes (row r, chunk c at c ^ (r % 8): conflict-free across a warp).
+      const int t = t0 + (row >> p.log2G);
+      uint32_t w[64];  // bf16 pairs: w[i] = dims (2i, 2i+1)
+      if (t < p.T) {   // rows past T get Q' = 0
+        const uint4* qs = reinterpret_cast<const uint4*>(p.q) +
+                          (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 8);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint4 u = __ldg(qs + i);
+          w[4 * i] = u.x;
+          w[4 * i + 1] = u.y;
+          w[4 * i + 2] = u.z;
+          w[4 * i + 3] = u.w;
+        }
+        float ss4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float x0 = bf16lo(w[i]), x1 = bf16hi(w[i]);
+          ss4[i & 3] = fmaf(x0, x0, fmaf(x1, x1, ss4[i & 3]));
+        }
+        const float r = rsqrtf(fmaf((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), 1.0f / kD, p.eps));
+        const float4* tab = p.rope_tab + static_cast<size_t>(b * p.T + t) * 32;
+        const float2* g2 = reinterpret_cast<const float2*>(p.q_norm_w);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
+          const float4 cs = __ldg(tab + i);  // (cos f0, sin f0, cos f1, sin f1)
+          const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
+          const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
+          const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
+          w[i] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
+          w[32 + i] = pack_bf16x2(b0 * cs.x + a0 * cs.y, b1 * cs.z + a1 * cs.w);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) w[i] = 0u;
+      }
+#pragma unroll
+      for (int cb = 0; cb < 16; ++cb)
+        st_shared_v4(sQ + (cb >> 3) * kPfBox + sw128_offset(row, cb & 7), w[4 * cb], w[4 * cb + 1], w[4 * cb + 2],
+                     w[4 * cb + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(bar + kBQReady + 8 * X);
+    };
+    // Pull a tile's raw query rows and its rows' angles toward L2 ahead of its prologue.
+    auto prefetch_tile = [&](int b, int hkv, int t0) {
+      const int t = t0 + (row >> p.log2G);
+      if (t >= p.T) return;
+      const char* qrow = reinterpret_cast<const char*>(
+          p.q + (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 2));
+      const char* trow = reinterpret_cast<const char*>(p.rope_tab + static_cast<size_t>(b * p.T + t) * 32);
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128));
+      if ((row & (G - 1)) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(trow + 128 * i));
+      }
+    };
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
+    // The Q prologue of the next item runs as soon as this item's last S_X has been read
+    // (Q'_X is then free), before the epilogue: the tensor core can start the next item
+    // while this one's outputs are stored.  O_X stays safe: the next item's first PV_X
+    // waits for a P that is only written after this epilogue.
+    int k = 0, item = round_item(0);
+    if (item < p.n_items) {
       int pair, b, hkv;
       item_coords(p, item, pair, b, hkv);
       const TileInfo ti = tile_info(p, 2 * pair + X);
-      if (ti.nkv == 0) continue;
-      const int t0 = ti.t0;
-      {
-        // Q prologue, one thread per row: QK-Norm of the raw row (a register-local sum of
-        // squares), gain, and rotate-half RoPE with the (cos, sin) of the row's position that
-        // the K-prologue kernel left in rope_tab; then the row goes to swizzled smem as 16
-        // chunks of 16 bytes (row r, chunk c at c ^ (r % 8): conflict-free across a warp).
-        const int t = t0 + (row >> p.log2G);
-        uint32_t w[64];  // bf16 pairs: w[i] = dims (2i, 2i+1)
-        if (t < p.T) {   // rows past T get Q' = 0
-          const uint4* qs = reinterpret_cast<const uint4*>(p.q) +
-                            (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 8);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const uint4 u = __ldg(qs + i);
-            w[4 * i] = u.x;
-            w[4 * i + 1] = u.y;
-            w[4 * i + 2] = u.z;
-            w[4 * i + 3] = u.w;
-          }
-          float ss4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float x0 = bf16lo(w[i]), x1 = bf16hi(w[i]);
-            ss4[i & 3] = fmaf(x0, x0, fmaf(x1, x1, ss4[i & 3]));
-          }
-          const float r = rsqrtf(fmaf((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), 1.0f / kD, p.eps));
-          const float4* tab = p.rope_tab + static_cast<size_t>(b * p.T + t) * 32;
-          const float2* g2 = reinterpret_cast<const float2*>(p.q_norm_w);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
-            const float4 cs = __ldg(tab + i);  // (cos f0, sin f0, cos f1, sin f1)
-            const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
-            const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
-            const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
-            w[i] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
-            w[32 + i] = pack_bf16x2(b0 * cs.x + a0 * cs.y, b1 * cs.z + a1 * cs.w);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) w[i] = 0u;
-        }
-#pragma unroll
-        for (int cb = 0; cb < 16; ++cb)
-          st_shared_v4(sQ + (cb >> 3) * kPfBox + sw128_offset(row, cb & 7), w[4 * cb], w[4 * cb + 1], w[4 * cb + 2],
-                       w[4 * cb + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive(bar + kBQReady + 8 * X);
+      if (ti.nkv > 0) q_prologue(b, hkv, ti.t0);
+    }
+    for (; item < p.n_items && ok; item = round_item(++k)) {
+      int pair, b, hkv;
+      item_coords(p, item, pair, b, hkv);
+      const TileInfo ti = tile_info(p, 2 * pair + X);
+      const int next = round_item(k + 1);
+      int npair = 0, nb = 0, nhkv = 0;
+      TileInfo tn{0, 0};
+      if (next < p.n_items) {
+        item_coords(p, next, npair, nb, nhkv);
+        tn = tile_info(p, 2 * npair + X);
       }
+      if (ti.nkv == 0) {  // this item has no tile X (its prologue was skipped too)
+        if (tn.nkv > 0) q_prologue(nb, nhkv, tn.t0);
+        continue;
+      }
+      if (tn.nkv > 0) prefetch_tile(nb, nhkv, tn.t0);
+      const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
       const int lim = min(t_row, p.T - 1);  // last key index this row may see
@@ -420,6 +457,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_arrive(bar + kBPReady + 8 * X);
       }
       if (!ok) break;
+      if (tn.nkv > 0) q_prologue(nb, nhkv, tn.t0);  // every S_X of this item has been read
       ok = mbar_wait(bar + kBOFull + 8 * X, o_cnt & 1, p.wait, abort_flag, kSitePrefillOFull);
       ++o_cnt;
       ok = __all_sync(0xffffffffu, ok);
@@ -435,13 +473,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tmem_ld32(tO + c * 32, r);
         if (valid) {
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
+          for (int u = 0; u < 4; ++u) {
             uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r[8 * k + 0]) * inv_l, __uint_as_float(r[8 * k + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(r[8 * k + 2]) * inv_l, __uint_as_float(r[8 * k + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(r[8 * k + 4]) * inv_l, __uint_as_float(r[8 * k + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(r[8 * k + 6]) * inv_l, __uint_as_float(r[8 * k + 7]) * inv_l);
-            dst[c * 4 + k] = w;
+            w.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * inv_l, __uint_as_float(r[8 * u + 1]) * inv_l);
+            w.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv_l, __uint_as_float(r[8 * u + 3]) * inv_l);
+            w.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv_l, __uint_as_float(r[8 * u + 5]) * inv_l);
+            w.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv_l, __uint_as_float(r[8 * u + 7]) * inv_l);
+            dst[c * 4 + u] = w;
           }
         }
       }
