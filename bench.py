@@ -56,6 +56,28 @@ def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
     return kv + qo + new
 
 
+# DRAM traffic of the decode split-KV kernel per cached token (dram__bytes_read.sum +
+# dram__bytes_write.sum of one ncu capture of a smaller case, divided by its cached tokens),
+# valid only for the kernel source it was measured on.  Refreshed with each new capture.
+DECODE_TRAFFIC = {"src_sha256": "bd2c84e9ee529b80e5f1797279784c54abfecf2b695386d38f6a4e4de3731d07",
+                  "bytes_per_cached_token": (630.624512e6 + 6.021376e6) / 153639}
+
+
+def decode_src_sha256() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("decode.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "qwen3_qk_norm_rope_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def decode_traffic(lens: np.ndarray):
+    if DECODE_TRAFFIC["src_sha256"] is None or DECODE_TRAFFIC["src_sha256"] != decode_src_sha256():
+        return None
+    return DECODE_TRAFFIC["bytes_per_cached_token"] * float(lens.astype(np.int64).sum())
+
+
 def decode_flops(lens: np.ndarray, Hq: int, d: int = 128) -> float:
     return 4.0 * Hq * d * float((lens.astype(np.int64) + 1).sum())
 
@@ -432,7 +454,7 @@ def main():
     clocks = clk.summary()
     dominant_is_decode = dec_s >= pre_s
     rl_dec = {"bound": "hbm", "achieved": dbytes / dec_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-              "frac": dbytes / dec_s / 1e9 / peaks["hbm_gbs"], "traffic": None,
+              "frac": dbytes / dec_s / 1e9 / peaks["hbm_gbs"], "traffic": decode_traffic(w.lens),
               "kernel": "decode call (append + split-KV attention + combine)",
               "algorithmic_bytes": dbytes, "peak_source": peak_src}
     rl_pre = {"bound": "tensor", "achieved": w.ps.causal_flops() / pre_s / 1e12, "peak": peaks["bf16_tflops"],
