@@ -43,6 +43,7 @@ namespace q3 {
 struct PrefillParams {
   const uint32_t* q;  // [B, T, Hq, d] bf16 pairs
   const float* q_norm_w;
+  const float* k_norm_w;  // only its max |g| is used here (the logit bound)
   const float4* rope_tab;  // [B*T][32]: (cos, sin) of frequencies 2i, 2i+1 at each token's position
   uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
@@ -60,7 +61,8 @@ constexpr uint32_t kPfV = 4 * kPfTile;  // 2 stages
 constexpr uint32_t kPfBar = 6 * kPfTile;
 // barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage
 constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
-                   kBOFull = 96, kBQReady = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140;
+                   kBOFull = 96, kBQReady = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
+                   kBRed = 144;  // 2 groups x 4 warps x (max|g_q|, max|g_k|)
 constexpr uint32_t kPrefillSmemBytes = kPfBar + 256 + 1024;  // + slack to align the base to 1024
 constexpr int kPrefillThreads = 320;
 constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
@@ -339,6 +341,32 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(trow + 128 * i));
       }
     };
+    // Reference for the exponentials.  QK-Norm bounds every logit: by Cauchy-Schwarz on the
+    // normalised, rotated (norm-preserving) vectors, |q'.k'|/sqrt(d) <= sqrt(d) max|g_q|
+    // max|g_k| (times 1 + 2^-7 for their bf16 rounding).  With that bound bnd (in log2
+    // units) at most 60, p = 2^(s*scale*log2(e) - bnd) lies in [2^-120, 1] for every key, so
+    // a fixed reference needs no row max, no rescale and can neither overflow nor go
+    // subnormal; l and O stay bounded by the key count.  Larger gains take the running-max
+    // path.  The choice is uniform per CTA.
+    float bnd;
+    {
+      float gq = fabsf(p.q_norm_w[row]), gk = fabsf(p.k_norm_w[row]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        gq = fmaxf(gq, __shfl_xor_sync(0xffffffffu, gq, o));
+        gk = fmaxf(gk, __shfl_xor_sync(0xffffffffu, gk, o));
+      }
+      volatile float* red = reinterpret_cast<volatile float*>(sgen + kPfBar + kBRed) + X * 8;
+      if (lane == 0) {
+        red[2 * wq] = gq;
+        red[2 * wq + 1] = gk;
+      }
+      asm volatile("bar.sync %0, 128;" ::"r"(1 + X) : "memory");
+      gq = fmaxf(fmaxf(red[0], red[2]), fmaxf(red[4], red[6]));
+      gk = fmaxf(fmaxf(red[1], red[3]), fmaxf(red[5], red[7]));
+      bnd = gq * gk * (11.3137085f * (1.0f + 0.0078125f) * 1.44269504f);
+    }
+    const bool fast = bnd <= 60.0f;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
     // The Q prologue of the next item runs as soon as this item's last S_X has been read
@@ -372,17 +400,59 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 
       const int t_row = t0 + (row >> p.log2G);
       const int lim = min(t_row, p.T - 1);  // last key index this row may see
-      float m = -INFINITY, l = 0.f;
+      float m = fast ? bnd : -INFINITY, l = 0.f;
       for (int j = 0; j < ti.nkv; ++j) {
         ok = mbar_wait(bar + kBSFull + 8 * X, s_cnt & 1, p.wait, abort_flag, kSitePrefillSFull);
         ++s_cnt;
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        // Pass 1: the row max over all 128 keys (one TMEM load).  Pass 2 re-reads S in
-        // 32-column chunks, so only one chunk is live while its exponentials are formed.
         const int kv0 = j * 128;
         const bool diag = kv0 + 127 > t0;  // some key of this tile lies past some row's position
+        if (fast) {
+          // One pass in four 32-column chunks, the next chunk's TMEM load in flight while the
+          // current one is processed.  bf16 P goes to S columns [0,64): chunk c of P
+          // overwrites only columns [16c,16c+16), which chunks 0..c have already read.
+          const uint64_t sl2x2 = f2pack(sl2, sl2), negb2 = f2pack(-bnd, -bnd);
+          uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+          uint32_t cur[32];
+          tmem_ld32(tS, cur);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t nxt[32];
+            if (c < 3) tmem_ld32_nowait(tS + 32 * (c + 1), nxt);
+            if (diag) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) cur[i] = (kv0 + 32 * c + i <= lim) ? cur[i] : 0xff800000u;  // -inf
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              f2unpack(ffma2(f2pack(__uint_as_float(cur[2 * i]), __uint_as_float(cur[2 * i + 1])), sl2x2, negb2), x0,
+                       x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              acc[i & 3] = fadd2(acc[i & 3], f2pack(p0, p1));
+              pk[i] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16_nowait(tS + kTmPOff + 16 * c, pk);
+            if (c < 3) {
+              tmem_wait_ld_dep(nxt);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) cur[i] = nxt[i];
+            }
+          }
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2unpack(acc[0], a0, a1);
+          f2unpack(acc[1], b0, b1);
+          f2unpack(acc[2], c0, c1);
+          f2unpack(acc[3], d0, d1);
+          tmem_wait_st();
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        } else {
+        // Running-max path.  Pass 1: the row max over all 128 keys (two TMEM loads).  Pass 2
+        // re-reads S in 32-column chunks, so only one chunk is live while its exponentials
+        // are formed.
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
@@ -453,6 +523,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tmem_wait_st();
         l += sum;
         m = m_new;
+        }
         tc_fence_before();
         mbar_arrive(bar + kBPReady + 8 * X);
       }

@@ -291,6 +291,7 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   q3::PrefillParams p;
   p.q = reinterpret_cast<const uint32_t*>(q);
   p.q_norm_w = q_norm_w;
+  p.k_norm_w = k_norm_w;
   p.rope_tab = static_cast<const float4*>(rope_tab);
   p.out = reinterpret_cast<uint4*>(out);
   p.lse = lse;
