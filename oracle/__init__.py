@@ -8,6 +8,7 @@ the CUDA path.  Every function is pinned by `tests/test_oracle_pins.py`
 from .attention import (  # noqa: F401
     bf16_round,
     build_cache_k,
+    chunk_prefill_ref,
     decode_ref,
     kv_cache_values_per_token,
     prefill_ref,
@@ -16,4 +17,4 @@ from .attention import (  # noqa: F401
     rope,
     rope_inv_freq,
 )
-from .loops import decode_loops, prefill_loops  # noqa: F401
+from .loops import chunk_prefill_loops, decode_loops, prefill_loops  # noqa: F401

@@ -151,6 +151,47 @@ def prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, theta: float, eps: float,
     return out, lse
 
 
+def chunk_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int,
+                      theta: float, eps: float, rows=None, staged: bool = False, block: int = 256):
+    """T new tokens per batch row over a cache that already holds `start` tokens, in fp64.
+
+    "Assembling a large model from scratch", Attention.forward and the notes below
+    the code: the new q and k get QK-Norm and RoPE at their positions, the new k and
+    v are appended after the cached ones (S = start + T keys), and new row i sees key
+    j iff j <= i + (S - T) = i + start, the mask tril(diagonal = S - T).
+
+    q [B,T,Hq,d], k and v [B,T,Hkv,d] raw new tokens at positions pos [B,T];
+    k_cache and v_cache indexable as [b][Hkv, >=start, d]: cached keys as stored
+    (already normed and rotated), cached values raw.  Returns out [B,len(rows),Hq,d]
+    and lse [B,Hq,len(rows)] for the new rows in `rows` (default: all T).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    G = Hq // Hkv
+    rows = np.arange(T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.zeros((B, rows.size, Hq, d))
+    lse = np.zeros((B, Hq, rows.size))
+    for b in range(B):
+        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged)  # [T, Hkv, d]
+        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged)
+        kc = np.asarray(k_cache[b], dtype=np.float64)[:, :start]     # [Hkv, start, d]
+        vc = np.asarray(v_cache[b], dtype=np.float64)[:, :start]
+        for h in range(Hq):
+            hk = h // G
+            keys = np.concatenate([kc[hk], kp[:, hk]], axis=0)          # [start + T, d]
+            vals = np.concatenate([vc[hk], v[b, :, hk]], axis=0)
+            for r0 in range(0, rows.size, block):
+                rr = rows[r0:r0 + block]
+                top = start + int(rr.max()) + 1
+                o, l = _attend(qp[r0:r0 + block, h], keys[:top], vals[:top], rr + start)
+                out[b, r0:r0 + block, h] = o
+                lse[b, h, r0:r0 + block] = l
+    return out, lse
+
+
 def build_cache_k(k_hist, k_norm_w, theta: float, eps: float) -> np.ndarray:
     """Cache contents for a raw key history k_hist [L,Hkv,d]: QK-Norm and RoPE at
     positions 0..L-1, rounded to bf16 (the cache's storage type), as float64."""

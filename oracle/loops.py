@@ -80,3 +80,33 @@ def decode_loops(q, k_new, v_new, gq, gk, k_cache, v_cache, lens, theta, eps):
                 out[n][h][i] = sum(w[j] * vals[j][i] for j in range(len(w))) / z
             lse[n][h] = m + math.log(z)
     return out, lse
+
+
+def chunk_prefill_loops(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps):
+    """T new tokens per batch row over `start` cached ones, element by element.
+    k_cache[b][hk][j][i] holds normed/rotated keys and v_cache[b][hk][j][i] raw
+    values for j < start; new key t sits at index start + t and new row t sees
+    keys 0..start + t."""
+    B, T, Hq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
+    Hkv = len(k[0][0])
+    G = Hq // Hkv
+    out = [[[[0.0] * d for _ in range(Hq)] for _ in range(T)] for _ in range(B)]
+    lse = [[[0.0] * T for _ in range(Hq)] for _ in range(B)]
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            keys = [[float(x) for x in k_cache[b][hk][j]] for j in range(start)]
+            vals = [[float(x) for x in v_cache[b][hk][j]] for j in range(start)]
+            for t in range(T):
+                keys.append(_norm_rope([float(x) for x in k[b][t][hk]], gk, float(pos[b][t]), theta, eps))
+                vals.append([float(x) for x in v[b][t][hk]])
+            for t in range(T):
+                qq = _norm_rope([float(x) for x in q[b][t][h]], gq, float(pos[b][t]), theta, eps)
+                scores = [sum(qq[i] * keys[j][i] for i in range(d)) / math.sqrt(d) for j in range(start + t + 1)]
+                m = max(scores)
+                w = [math.exp(s - m) for s in scores]
+                z = sum(w)
+                for i in range(d):
+                    out[b][t][h][i] = sum(w[j] * vals[j][i] for j in range(len(w))) / z
+                lse[b][h][t] = m + math.log(z)
+    return out, lse

@@ -232,6 +232,64 @@ def check_decode_equals_last_prefill_row():
     assert np.allclose(lse_d[0], lse_p[0, :, L], rtol=0, atol=1e-13)
 
 
+# ---------------------------------------------------------------- chunked prefill
+def _chunk_split(q, k, v, gk, pos, start):
+    """Split a full prompt into a cache of its first `start` tokens (keys normed and
+    rotated at their positions, kept in fp64) and the remaining new tokens."""
+    B = q.shape[0]
+    kc = np.stack([A.qk_prologue(k[b, :start], gk, pos[b, :start], THETA, EPS).transpose(1, 0, 2) for b in range(B)])
+    vc = v[:, :start].transpose(0, 2, 1, 3)
+    return q[:, start:], k[:, start:], v[:, start:], pos[:, start:], kc, vc
+
+
+def check_brute_force_chunk_prefill():
+    for (start, T, Hq, Hkv, seed) in [(3, 4, 2, 1, 70), (7, 5, 4, 2, 71), (0, 6, 4, 1, 72), (9, 1, 4, 2, 73)]:
+        q, k, v, gq, gk, pos = _inputs(2, start + T, Hq, Hkv, seed=seed)
+        pos = pos + seed
+        qn, kn, vn, pn, kc, vc = _chunk_split(q, k, v, gk, pos, start)
+        out, lse = A.chunk_prefill_ref(qn, kn, vn, gq, gk, pn, kc, vc, start, THETA, EPS, block=2)
+        out_l, lse_l = Lp.chunk_prefill_loops(qn.tolist(), kn.tolist(), vn.tolist(), gq.tolist(), gk.tolist(),
+                                              pn.tolist(), kc.tolist(), vc.tolist(), start, THETA, EPS)
+        assert np.allclose(out, np.array(out_l), rtol=0, atol=1e-12)
+        assert np.allclose(lse, np.array(lse_l), rtol=0, atol=1e-12)
+
+
+def check_chunk_equals_tail_of_full_prefill():
+    """tril(diagonal = S - T) lets the new tokens see the whole history, so a chunk over
+    a cache of the first `start` tokens reproduces rows start.. of a prefill over all
+    of them ("Assembling a large model from scratch", notes below the code)."""
+    for (start, T, Hq, Hkv, seed) in [(37, 29, 8, 2, 74), (64, 64, 4, 4, 75), (5, 70, 8, 1, 76)]:
+        q, k, v, gq, gk, pos = _inputs(2, start + T, Hq, Hkv, seed=seed)
+        full_o, full_l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+        qn, kn, vn, pn, kc, vc = _chunk_split(q, k, v, gk, pos, start)
+        out, lse = A.chunk_prefill_ref(qn, kn, vn, gq, gk, pn, kc, vc, start, THETA, EPS, block=16)
+        assert np.allclose(out, full_o[:, start:], rtol=0, atol=1e-13)
+        assert np.allclose(lse, full_l[:, :, start:], rtol=0, atol=1e-13)
+        rows = np.array([0, T // 2, T - 1])
+        out_s, lse_s = A.chunk_prefill_ref(qn, kn, vn, gq, gk, pn, kc, vc, start, THETA, EPS, rows=rows, block=2)
+        assert np.allclose(out_s, full_o[:, start + rows], rtol=0, atol=1e-13)
+        assert np.allclose(lse_s, full_l[:, :, start + rows], rtol=0, atol=1e-13)
+
+
+def check_chunk_of_one_token_is_decode():
+    """A chunk of one new token over a cache of L tokens is one decode step at L."""
+    q, kn, vn, gq, gk, kc, vc, lens, _ = _tiny_decode(77, N=1, lens=(11,))
+    L = int(lens[0])
+    out_d, lse_d = A.decode_ref(q, kn, vn, gq, gk, kc, vc, lens, THETA, EPS)
+    out_c, lse_c = A.chunk_prefill_ref(q[:, None], kn[:, None], vn[:, None], gq, gk, np.array([[L]]), kc, vc, L,
+                                       THETA, EPS)
+    assert np.allclose(out_c[:, 0], out_d, rtol=0, atol=1e-13)
+    assert np.allclose(lse_c[:, :, 0], lse_d, rtol=0, atol=1e-13)
+
+
+def check_chunk_over_empty_cache_is_prefill():
+    q, k, v, gq, gk, pos = _inputs(2, 33, 8, 2, seed=78)
+    empty = np.zeros((2, 2, 0, D))
+    out, lse = A.chunk_prefill_ref(q, k, v, gq, gk, pos, empty, empty, 0, THETA, EPS)
+    ref_o, ref_l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    assert np.allclose(out, ref_o, rtol=0, atol=1e-14) and np.allclose(lse, ref_l, rtol=0, atol=1e-14)
+
+
 def check_position_shift_invariance():
     """Shifting every position by a constant leaves outputs unchanged (RoPE is relative)."""
     q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=50)

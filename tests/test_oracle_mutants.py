@@ -1,7 +1,8 @@
 """Plant plausible mistakes in the oracle (on the CPU) and confirm the pins catch
 each one: a wrong RoPE sign, adjacent-pair RoPE, a missing eps, mean-centering,
 h mod Hkv head mapping, an off-by-one causal mask, a missing 1/sqrt(d) scale,
-and a base-2 logsumexp."""
+a base-2 logsumexp, and in the chunked prefill a mask without the cached-prefix
+offset or cached keys rotated a second time."""
 import numpy as np
 import pytest
 
@@ -69,6 +70,34 @@ def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=Fal
     return o[:, :, perm], l[:, perm]
 
 
+_ORIG_CHUNK = A.chunk_prefill_ref
+
+
+def _chunk_no_offset(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps, rows=None, staged=False, block=256):
+    # the mask forgets the cached prefix: new row i sees keys 0..i of the concatenation
+    q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
+    B, T, Hq, d = q.shape
+    G = Hq // k.shape[2]
+    rows = np.arange(T) if rows is None else np.asarray(rows)
+    out, lse = np.zeros((B, rows.size, Hq, d)), np.zeros((B, Hq, rows.size))
+    for b in range(B):
+        kp = A.qk_prologue(k[b], gk, pos[b], theta, eps, staged)
+        qp = A.qk_prologue(q[b, rows], gq, np.asarray(pos[b])[rows], theta, eps, staged)
+        for h in range(Hq):
+            keys = np.concatenate([np.asarray(k_cache[b])[h // G, :start], kp[:, h // G]])
+            vals = np.concatenate([np.asarray(v_cache[b])[h // G, :start], v[b, :, h // G]])
+            o, l = A._attend(qp[:, h], keys, vals, rows)
+            out[b, :, h], lse[b, h] = o, l
+    return out, lse
+
+
+def _chunk_rerotates_cache(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps, **kw):
+    # the cached keys get RoPE a second time at their positions 0..start-1
+    kc = np.stack([A.rope(np.asarray(k_cache[b])[:, :start].transpose(1, 0, 2), np.arange(start), theta)
+                   .transpose(1, 0, 2) for b in range(len(k_cache))])
+    return _ORIG_CHUNK(q, k, v, gq, gk, pos, kc, v_cache, start, theta, eps, **kw)
+
+
 _ORIG_PREFILL = A.prefill_ref
 
 MUTANTS = [
@@ -80,6 +109,8 @@ MUTANTS = [
     ("_attend", _attend_no_scale),
     ("_attend", _attend_log2),
     ("prefill_ref", _prefill_mod_mapping),
+    ("chunk_prefill_ref", _chunk_no_offset),
+    ("chunk_prefill_ref", _chunk_rerotates_cache),
 ]
 
 
