@@ -114,6 +114,35 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
                           float theta, float eps, qwen3_stream_t stream);
 
 /*
+ * qwen3_attn_prefill_chunk - T new tokens per batch row over a KV cache that already holds
+ * `start` tokens (chunked prefill).  "Assembling a large model from scratch",
+ * Attention.forward with a cache and the notes below the code: the new keys are normed,
+ * rotated and appended after the cached ones, S = start + T keys in all, and new token i
+ * sees keys 0..start+i (the mask tril(diagonal = S - T)).  With start == 0 this is
+ * qwen3_attn_prefill_ex with a cache; with T == 1 it is one decode step at length start.
+ *   q, k, v, gains  as in qwen3_attn_prefill, for the T new tokens only.
+ *   pos       [B, T] int32 RoPE positions of the new tokens (normally start..start+T-1;
+ *             the mask uses the key index start+i, never pos).
+ *   k_cache, v_cache  required [B, Hkv, Tcap, d] bf16.  Slots 0..start-1 are read: keys
+ *             already normed and rotated, values raw, as qwen3_attn_prefill_ex and
+ *             qwen3_attn_decode leave them.  The new keys' k' and raw v are written to slots
+ *             start..start+T-1.  No other slot is touched.
+ *   out       [B, T, Hq, d] bf16; lse optional [B, Hq, T] fp32 (NULL to skip).
+ *   start     cached tokens, the same for every batch row; 0 <= start and
+ *             start + T <= Tcap, else QWEN3_ERR_INVALID_ARG.
+ *   workspace, ws_bytes  at least qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes,
+ *             else QWEN3_ERR_WORKSPACE.
+ * Other errors as in qwen3_attn_prefill_ex.  The caches must not alias q, k, v or out.
+ */
+int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                             const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                             qwen3_bf16* out, float* lse,
+                             qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap,
+                             void* workspace, size_t ws_bytes,
+                             int B, int T, int Hq, int Hkv, int d,
+                             float theta, float eps, qwen3_stream_t stream);
+
+/*
  * qwen3_attn_decode - one new token per sequence attending over its KV cache
  * ("Assembling a large model from scratch", KVCache.update and Transformer.forward: the new
  * token sits at position cache.length and sees the whole history).

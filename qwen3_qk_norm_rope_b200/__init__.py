@@ -27,6 +27,8 @@ SIGNATURES = {
     "qwen3_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_prefill_ex": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _Z,
                                    _I, _I, _I, _I, _I, _F, _F, _P]),
+    "qwen3_attn_prefill_chunk": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _Z,
+                                      _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
     "qwen3_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I]),
@@ -157,6 +159,38 @@ def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: floa
                                        _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
                                        _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
            "qwen3_attn_prefill_ex")
+    return out
+
+
+def prefill_chunk(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int, *, theta: float = 1.0e6,
+                  eps: float = 1.0e-6, out=None, lse=None, workspace=None):
+    """Chunked prefill: T new tokens per batch row over caches [B,Hkv,Tcap,d] that already
+    hold `start` tokens.  The new keys (normed, rotated) and values are written to slots
+    start..start+T-1, and new token i attends to keys 0..start+i.  Returns out [B,T,Hq,d]."""
+    dev = q.device
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(q, "q", torch.bfloat16, (B, T, Hq, d), dev)
+    _need(k, "k", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(v, "v", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (B, T), dev)
+    Tcap = k_cache.shape[2]
+    _need(k_cache, "k_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
+    _need(v_cache, "v_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, T, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq, T), dev)
+    if workspace is None:
+        workspace = torch.empty(prefill_workspace_size(B, T, Hkv, d), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().qwen3_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                          _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), int(start), Tcap,
+                                          _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
+           "qwen3_attn_prefill_chunk")
     return out
 
 

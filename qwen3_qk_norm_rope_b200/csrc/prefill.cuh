@@ -48,6 +48,7 @@ struct PrefillParams {
   uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
   int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
+  int start;  // cached keys before the first query row: query t is key index start + t
   float eps, scale_log2;
   WaitCfg wait;
   int fault;
@@ -89,13 +90,13 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 }
 
 struct TileInfo {
-  int t0, nkv;  // first position; key tiles (0 = the tile lies past T)
+  int t0, nkv;  // first query row; key tiles it reads (0 = the tile lies past T)
 };
 
 __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt) {
   TileInfo ti;
   ti.t0 = qt * p.P;
-  ti.nkv = (ti.t0 < p.T) ? (min(ti.t0 + p.P, p.T) - 1) / 128 + 1 : 0;
+  ti.nkv = (ti.t0 < p.T) ? (p.start + min(ti.t0 + p.P, p.T) - 1) / 128 + 1 : 0;
   return ti;
 }
 
@@ -399,7 +400,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
-      const int lim = min(t_row, p.T - 1);  // last key index this row may see
+      const int lim = p.start + min(t_row, p.T - 1);  // last key index this row may see
       float m = fast ? bnd : -INFINITY, l = 0.f;
       for (int j = 0; j < ti.nkv; ++j) {
         ok = mbar_wait(bar + kBSFull + 8 * X, s_cnt & 1, p.wait, abort_flag, kSitePrefillSFull);
@@ -408,7 +409,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const int kv0 = j * 128;
-        const bool diag = kv0 + 127 > t0;  // some key of this tile lies past some row's position
+        const bool diag = kv0 + 127 > p.start + t0;  // some key of this tile lies past some row's limit
         if (fast) {
           // One pass in four 32-column chunks, the next chunk's TMEM load in flight while the
           // current one is processed.  bf16 P goes to S columns [0,64): chunk c of P

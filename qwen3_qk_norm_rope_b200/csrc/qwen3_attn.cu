@@ -233,10 +233,13 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, 
                          reinterpret_cast<cudaStream_t>(stream));
 }
 
-int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
-                          const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
-                          qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap, void* workspace, size_t ws_bytes,
-                          int B, int T, int Hq, int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+namespace {
+
+// Prefill of T new tokens per batch row after `start` cached ones (start > 0 needs the caches).
+int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                 const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse, qwen3_bf16* k_cache,
+                 qwen3_bf16* v_cache, int start, int Tcap, void* workspace, size_t ws_bytes, int B, int T, int Hq,
+                 int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       pos == nullptr || out == nullptr)
     return QWEN3_ERR_INVALID_ARG;
@@ -246,7 +249,8 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   if (Hq / Hkv > 128) return QWEN3_ERR_UNSUPPORTED;
   if ((k_cache == nullptr) != (v_cache == nullptr)) return QWEN3_ERR_INVALID_ARG;
   const bool use_cache = k_cache != nullptr;
-  if (use_cache && Tcap < T) return QWEN3_ERR_INVALID_ARG;
+  if (start < 0 || (start > 0 && !use_cache)) return QWEN3_ERR_INVALID_ARG;
+  if (use_cache && (Tcap <= 0 || static_cast<long long>(start) + T > Tcap)) return QWEN3_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) ||
       !aligned(k_norm_w, 8) || !aligned(pos, 4) || (lse != nullptr && !aligned(lse, 4)))
     return QWEN3_ERR_INVALID_ARG;
@@ -259,21 +263,24 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
 
-  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] (and V copied when filling a cache);
-  //    it also leaves every token's RoPE cos/sin in the workspace for the query tiles.
+  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] from slot `start` on (and V copied
+  //    when filling a cache); it also leaves every new token's RoPE cos/sin in the workspace
+  //    for the query tiles.  Shifting the base by start rows puts token t at slot start + t.
   const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
   qwen3_bf16* kdst = use_cache ? k_cache : reinterpret_cast<qwen3_bf16*>(w0);
   void* rope_tab = reinterpret_cast<void*>(w0 + kspace_bytes(B, T, Hkv, d));
   const int Tc = use_cache ? Tcap : T;
-  st = launch_prologue(k, k_norm_w, pos, kdst, use_cache ? v : nullptr, use_cache ? v_cache : nullptr, B, T, Hkv,
-                       Tc, 0, theta, eps, s, rope_tab);
+  const size_t shift = static_cast<size_t>(start) * kD;
+  st = launch_prologue(k, k_norm_w, pos, kdst + shift, use_cache ? v : nullptr, use_cache ? v_cache + shift : nullptr,
+                       B, T, Hkv, Tc, 0, theta, eps, s, rope_tab);
   if (st != QWEN3_OK) return st;
 
-  // 2. Tensor maps.  The key-axis extent is T (not Tcap) so slots past the prompt read as zeros.
+  // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
+  //    read as zeros.
   CUtensorMap mk, mv;
   const cuuint32_t box[4] = {64, 128, 1, 1};
   {
-    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(T),
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(start) + T,
                                 static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(B)};
     const cuuint64_t str[3] = {kD * 2ull, static_cast<cuuint64_t>(Tc) * kD * 2ull,
                                static_cast<cuuint64_t>(Hkv) * Tc * kD * 2ull};
@@ -306,6 +313,7 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   const long long n_items = static_cast<long long>(p.n_pairs) * B * Hkv;
   if (n_items > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   p.n_items = static_cast<int>(n_items);
+  p.start = start;
   p.eps = eps;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
   p.wait = next_wait_cfg();
@@ -316,6 +324,26 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
   const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
   q3::fmha_prefill_kernel<<<grid, q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+}  // namespace
+
+int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                          const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
+                          qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap, void* workspace, size_t ws_bytes,
+                          int B, int T, int Hq, int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+  return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, k_cache, v_cache, 0, Tcap, workspace, ws_bytes,
+                      B, T, Hq, Hkv, d, theta, eps, stream);
+}
+
+int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                             const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
+                             qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap, void* workspace,
+                             size_t ws_bytes, int B, int T, int Hq, int Hkv, int d, float theta, float eps,
+                             qwen3_stream_t stream) {
+  if (k_cache == nullptr || v_cache == nullptr) return QWEN3_ERR_INVALID_ARG;
+  return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, k_cache, v_cache, start, Tcap, workspace,
+                      ws_bytes, B, T, Hq, Hkv, d, theta, eps, stream);
 }
 
 int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,

@@ -76,6 +76,28 @@ class DecodeShape:
         return self.lmax + 1
 
 
+@dataclass(frozen=True)
+class ChunkShape:
+    """T new tokens per batch row after `start` cached ones (chunked prefill)."""
+    name: str
+    B: int
+    start: int
+    T: int
+    Hq: int
+    Hkv: int
+    d: int = HEAD_DIM
+    theta: float = ROPE_THETA
+    eps: float = RMS_EPS
+
+    @property
+    def group(self) -> int:
+        return self.Hq // self.Hkv
+
+    def causal_flops(self) -> float:
+        """QK^T and PV over the visible keys: new row i sees start + i + 1 of them."""
+        return 4.0 * self.B * self.Hq * self.d * (self.T * self.start + self.T * (self.T + 1) / 2.0)
+
+
 PREFILL_SHAPES = {
     "tiny": PrefillShape("tiny prefill B=1 T=128 Hq=16 Hkv=8", 1, 128, 16, 8),
     "qwen3-0.6b": PrefillShape("Qwen3-0.6B-shaped prefill B=2 T=2048 Hq=16 Hkv=8", 2, 2048, 16, 8),
@@ -85,6 +107,12 @@ PREFILL_SHAPES = {
 
 DECODE_SHAPES = {
     "batched-decode": DecodeShape("batched decode N=64 Hq=32 Hkv=8 L~U[1024,32768]", 64, 32, 8),
+}
+
+
+CHUNK_SHAPES = {
+    "qwen3-4b-second-chunk": ChunkShape("Qwen3-4B-shaped chunked prefill B=1 start=4096 T=4096 Hq=32 Hkv=8",
+                                        1, 4096, 4096, 32, 8),
 }
 
 
@@ -120,6 +148,21 @@ def prefill_inputs(shape: PrefillShape, seed: int = 0) -> dict:
         "q": _bf16(q), "k": _bf16(k), "v": _bf16(v),
         "q_norm_w": torch.from_numpy(g_q), "k_norm_w": torch.from_numpy(g_k),
         "pos": torch.from_numpy(pos),
+    }
+
+
+def chunk_inputs(shape: ChunkShape, seed: int = 0) -> dict:
+    """A prompt of start + T tokens drawn exactly as prefill_inputs draws it, split in two:
+    the raw history k_hist, v_hist [B,start,Hkv,d] (the cache stores k_hist only after
+    QK-Norm and RoPE at positions 0..start-1) and the T new tokens q, k, v at positions
+    start..start+T-1, with the gains."""
+    full = prefill_inputs(PrefillShape(shape.name, shape.B, shape.start + shape.T, shape.Hq, shape.Hkv,
+                                       shape.d, shape.theta, shape.eps), seed)
+    s = shape.start
+    return {
+        "q": full["q"][:, s:].contiguous(), "k": full["k"][:, s:].contiguous(), "v": full["v"][:, s:].contiguous(),
+        "pos": full["pos"][:, s:].contiguous(), "q_norm_w": full["q_norm_w"], "k_norm_w": full["k_norm_w"],
+        "k_hist": full["k"][:, :s].contiguous(), "v_hist": full["v"][:, :s].contiguous(),
     }
 
 

@@ -78,6 +78,30 @@ def test_prefill_argument_checks():
     assert _prefill_ex(ws=FAKE, ws_bytes=100) == qa.ERR_WORKSPACE
 
 
+def _chunk(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, gq=FAKE, gk=FAKE, pos=FAKE, out=FAKE, lse=None, kc=FAKE, vc=FAKE, start=256,
+             Tcap=512, ws=None, ws_bytes=0, B=1, T=128, Hq=16, Hkv=8, d=128, theta=1e6, eps=1e-6)
+    a.update(kw)
+    return qa.lib().qwen3_attn_prefill_chunk(a["q"], a["k"], a["v"], a["gq"], a["gk"], a["pos"], a["out"],
+                                             a["lse"], a["kc"], a["vc"], a["start"], a["Tcap"], a["ws"],
+                                             a["ws_bytes"], a["B"], a["T"], a["Hq"], a["Hkv"], a["d"], a["theta"],
+                                             a["eps"], None)
+
+
+def test_chunked_prefill_argument_checks():
+    assert _chunk(kc=None, vc=None) == qa.ERR_INVALID_ARG  # the chunk needs the caches
+    assert _chunk(vc=None) == qa.ERR_INVALID_ARG
+    assert _chunk(start=-1) == qa.ERR_INVALID_ARG
+    assert _chunk(start=385) == qa.ERR_INVALID_ARG  # start + T > Tcap
+    assert _chunk(Tcap=0, start=0) == qa.ERR_INVALID_ARG
+    assert _chunk(Hq=24) == qa.ERR_UNSUPPORTED
+    assert _chunk(kc=ctypes.c_void_p((1 << 20) + 8)) == qa.ERR_INVALID_ARG  # misaligned cache
+    assert _chunk(start=384) == qa.ERR_WORKSPACE  # start + T == Tcap is valid; no workspace given
+    assert _chunk(ws=FAKE, ws_bytes=100) == qa.ERR_WORKSPACE
+    # prefill_ex has no start: a cached prefix needs the chunked call
+    assert _prefill_ex(kc=FAKE, vc=FAKE, Tcap=128) == qa.ERR_WORKSPACE
+
+
 def test_decode_and_prologue_argument_checks():
     lib = qa.lib()
 

@@ -1,0 +1,154 @@
+"""Chunked prefill parity: T new tokens over a KV cache that already holds `start` tokens
+("Assembling a large model from scratch", Attention.forward with a cache: the mask
+tril(diagonal = S - T)).  The cached prefix is built by the oracle (QK-Norm + RoPE of the
+raw history, rounded to bf16); the CUDA path runs through the C ABI and is compared with
+the fp64 oracle on the same inputs.  The caches are checked slot by slot afterwards."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qwen3_qk_norm_rope_b200 as qa
+from synthetic import CHUNK_SHAPES, ChunkShape, PrefillShape, as_f64, chunk_inputs, prefill_inputs
+from tests.gpu_common import assert_status_ok, compare, dev, prefill_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+CANARY = 0x7FC1  # a bf16 NaN bit pattern in every slot the call must not write
+
+
+def _caches(inp: dict, shape: ChunkShape, Tcap: int):
+    """bf16 caches [B,Hkv,Tcap,d]: slots < start hold the oracle's cache contents (keys
+    normed and rotated at 0..start-1, raw values), every other slot the canary."""
+    B, Hkv, s = shape.B, shape.Hkv, shape.start
+    kc = torch.empty((B, Hkv, Tcap, shape.d), dtype=torch.bfloat16)
+    kc.view(torch.int16).fill_(CANARY)
+    vc = kc.clone()
+    gk = as_f64(inp["k_norm_w"])
+    for b in range(B):
+        if s:
+            kb = oracle.build_cache_k(as_f64(inp["k_hist"][b]), gk, shape.theta, shape.eps)  # [s,Hkv,d]
+            kc[b, :, :s] = torch.from_numpy(kb.transpose(1, 0, 2).copy()).to(torch.bfloat16)
+            vc[b, :, :s] = inp["v_hist"][b].permute(1, 0, 2)
+    return kc, vc
+
+
+def _run(inp: dict, shape: ChunkShape, kc: torch.Tensor, vc: torch.Tensor):
+    d = dev()
+    t = {k: inp[k].to(d) for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
+    kcd, vcd = kc.to(d), vc.to(d)
+    lse = torch.full((shape.B, shape.Hq, shape.T), float("nan"), dtype=torch.float32, device=d)
+    out = qa.prefill_chunk(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], kcd, vcd, shape.start,
+                           theta=shape.theta, eps=shape.eps, lse=lse)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    return out, lse, kcd, vcd
+
+
+def _oracle(inp: dict, shape: ChunkShape, kc: torch.Tensor, vc: torch.Tensor, rows=None):
+    s = shape.start
+    args = (as_f64(inp["q"]), as_f64(inp["k"]), as_f64(inp["v"]), as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]),
+            inp["pos"].numpy(), as_f64(kc[:, :, :s]), as_f64(vc[:, :, :s]), s, shape.theta, shape.eps)
+    ref, ref_lse = oracle.chunk_prefill_ref(*args, rows=rows)
+    ref_st, st_lse = oracle.chunk_prefill_ref(*args, rows=rows, staged=True)
+    return ref, ref_lse, ref_st, st_lse
+
+
+def _check_caches(inp, shape, kc_before, vc_before, kc_after, vc_after):
+    s, T = shape.start, shape.T
+    ka, va = kc_after.cpu(), vc_after.cpu()
+    # the cached prefix and the slots past the chunk are untouched
+    assert torch.equal(ka[:, :, :s].view(torch.int16), kc_before[:, :, :s].view(torch.int16))
+    assert torch.equal(va[:, :, :s].view(torch.int16), vc_before[:, :, :s].view(torch.int16))
+    assert torch.equal(ka[:, :, s + T:].view(torch.int16), kc_before[:, :, s + T:].view(torch.int16))
+    assert torch.equal(va[:, :, s + T:].view(torch.int16), vc_before[:, :, s + T:].view(torch.int16))
+    # the new keys: QK-Norm + RoPE at their positions, one bf16 rounding; values bit-exact
+    kref = oracle.qk_prologue(as_f64(inp["k"]), as_f64(inp["k_norm_w"]), inp["pos"].numpy(), shape.theta, shape.eps)
+    kgot = to_np(ka[:, :, s:s + T].permute(0, 2, 1, 3))
+    assert np.all(np.abs(kgot - kref) <= np.abs(kref) * 2.0 ** -8 + 2e-5), np.abs(kgot - kref).max()
+    assert torch.equal(va[:, :, s:s + T].permute(0, 2, 1, 3), inp["v"])
+
+
+CASES = [
+    # (B, start, T, Hq, Hkv, slack): start and T off the tile grid, G in {1, 2, 4, 16, 32},
+    # one-token chunks (a decode step through the prefill kernel), a short chunk over a long
+    # prefix (few work items, many key tiles each), B > 1
+    (2, 200, 300, 16, 8, 40),
+    (1, 128, 128, 8, 8, 0),
+    (1, 1000, 77, 32, 1, 5),
+    (3, 1500, 1, 32, 8, 3),
+    (1, 9000, 40, 32, 8, 100),
+    (2, 333, 517, 64, 4, 11),
+]
+
+
+@pytest.mark.parametrize("B,start,T,Hq,Hkv,slack", CASES)
+def test_chunk_parity(B, start, T, Hq, Hkv, slack):
+    shape = ChunkShape("chunk", B, start, T, Hq, Hkv)
+    inp = chunk_inputs(shape, seed=start + T)
+    kc, vc = _caches(inp, shape, start + T + slack)
+    out, lse, kca, vca = _run(inp, shape, kc, vc)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, f"chunk B{B} start{start} T{T} Hq{Hq} Hkv{Hkv}")
+    _check_caches(inp, shape, kc, vc, kca, vca)
+
+
+def test_chunk_full_size_sampled_rows():
+    shape = CHUNK_SHAPES["qwen3-4b-second-chunk"]
+    inp = chunk_inputs(shape, seed=0)
+    kc, vc = _caches(inp, shape, shape.start + shape.T)
+    out, lse, _, _ = _run(inp, shape, kc, vc)
+    rng = np.random.default_rng(2)
+    rows = np.unique(np.concatenate([np.arange(128), rng.choice(np.arange(128, shape.T - 128), 256, replace=False),
+                                     np.arange(shape.T - 128, shape.T)]))
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc, rows=rows)
+    idx = torch.from_numpy(rows).to(out.device)
+    compare(to_np(out[:, idx]), to_np(lse[:, :, idx]), ref, ref_lse, st_lse, "4B second chunk, sampled rows")
+    assert torch.isfinite(out.float()).all()
+
+
+def test_chunk_over_empty_cache_equals_prefill_into_cache():
+    shape = ChunkShape("empty prefix", 2, 0, 300, 16, 8)
+    inp = chunk_inputs(shape, seed=8)
+    kc, vc = _caches(inp, shape, 320)
+    out, lse, kca, vca = _run(inp, shape, kc, vc)
+    pinp = {k: inp[k] for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
+    kc2, vc2 = kc.to(dev()), vc.to(dev())
+    out_p, lse_p = prefill_gpu(pinp, caches=(kc2, vc2))
+    assert torch.equal(out, out_p) and torch.equal(lse, lse_p)
+    assert torch.equal(kca.view(torch.int16), kc2.view(torch.int16))
+    assert torch.equal(vca.view(torch.int16), vc2.view(torch.int16))
+
+
+def test_two_chunks_equal_one_prefill():
+    """Prefill of the first 256 tokens into a cache, then a chunk of the next 300 over it,
+    gives the rows a single prefill of all 556 tokens gives: same key tiles in the same
+    order, same per-row limits, same softmax reference, so the same bits."""
+    d = dev()
+    full = prefill_inputs(PrefillShape("two chunks", 1, 556, 32, 8), seed=12)
+    kc = torch.zeros((1, 8, 600, 128), dtype=torch.bfloat16, device=d)
+    vc = torch.zeros_like(kc)
+    first = {k: (v[:, :256].contiguous() if v.dim() > 1 else v) for k, v in full.items()}
+    prefill_gpu(first, caches=(kc, vc))
+    t = {k: v.to(d) for k, v in full.items()}
+    lse2 = torch.empty((1, 32, 300), dtype=torch.float32, device=d)
+    out2 = qa.prefill_chunk(t["q"][:, 256:].contiguous(), t["k"][:, 256:].contiguous(), t["v"][:, 256:].contiguous(),
+                            t["q_norm_w"], t["k_norm_w"], t["pos"][:, 256:].contiguous(), kc, vc, 256, lse=lse2)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    out_f, lse_f = prefill_gpu(full)
+    diff = (out2.float() - out_f[:, 256:].float()).abs().max().item()
+    assert torch.equal(out2, out_f[:, 256:]), f"max diff {diff:.3e}"
+    assert torch.equal(lse2, lse_f[:, :, 256:])
+
+
+def test_chunk_large_gains_running_max_path():
+    shape = ChunkShape("large gains", 1, 450, 260, 16, 8)
+    inp = chunk_inputs(shape, seed=31)
+    inp["q_norm_w"] = inp["q_norm_w"] * 1.6
+    inp["k_norm_w"] = inp["k_norm_w"] * 1.6
+    kc, vc = _caches(inp, shape, 710)
+    out, lse, _, _ = _run(inp, shape, kc, vc)
+    _, _, ref_st, st_lse = _oracle(inp, shape, kc, vc)
+    # the same staged comparison and gain-scaled LSE bound as the prefill large-gains test
+    compare(to_np(out), to_np(lse), ref_st, st_lse, st_lse, "chunk large gains (staged)", lse_tol=1e-3 * 1.6 ** 2)
