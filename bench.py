@@ -11,6 +11,11 @@ prologue is counted as free work); the decode throughput in GB/s rides along und
 256 MiB write) before every step, outside the per-step CUDA-event windows.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --workload chunked-prefill    # the chunked-prefill call alone
+
+The chunked-prefill workload times qwen3_attn_prefill_chunk on the Qwen3-4B-shaped
+second chunk (B=1, 4096 new tokens over 4096 cached, Hq=32, Hkv=8) and prints its own
+line in the same format (causal flops: new row i sees start + i + 1 keys).
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs its own replica of the step
 (weak scaling, no collective on the data path); time is the max over ranks.
@@ -31,7 +36,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import DECODE_SHAPES, PREFILL_SHAPES, decode_step_inputs, prefill_inputs  # noqa: E402
+from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, chunk_inputs, decode_step_inputs, \
+    prefill_inputs  # noqa: E402
 
 METRIC = "causal GQA attn TFLOP/s (+QK-Norm/RoPE) % bf16 peak; decode HBM GB/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -312,6 +318,166 @@ def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seq
             "threads": threads, "sample": sample, "flops": flops}
 
 
+# ------------------------------------------------------------------------------ chunked prefill
+CHUNK_METRIC = "chunked-prefill causal GQA attn TFLOP/s (+QK-Norm/RoPE, cache append) % bf16 peak"
+
+
+class ChunkWorkload:
+    """Device-resident inputs of the chunked-prefill call: the new tokens, and caches whose
+    first `start` slots hold the prefix (normed and rotated by the library's prologue)."""
+
+    LAUNCHES_PER_STEP = 2  # K prologue (cache append) + attention
+
+    def __init__(self, dev: torch.device, name: str = "qwen3-4b-second-chunk", seed: int = 0):
+        import qwen3_qk_norm_rope_b200 as qa
+
+        self.qa, self.dev = qa, dev
+        self.cs = cs = CHUNK_SHAPES[name]
+        inp = chunk_inputs(cs, seed=seed)
+        self.host = {k: inp[k] for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
+        self.t = {k: v.to(dev) for k, v in self.host.items()}
+        Tcap = cs.start + cs.T
+        self.kc = torch.zeros((cs.B, cs.Hkv, Tcap, cs.d), dtype=torch.bfloat16, device=dev)
+        self.vc = torch.zeros_like(self.kc)
+        pos = torch.arange(cs.start, dtype=torch.int32, device=dev)[None].expand(cs.B, cs.start).contiguous()
+        qa.qk_norm_rope(inp["k_hist"].to(dev), self.t["k_norm_w"], pos, self.kc, v_src=inp["v_hist"].to(dev),
+                        v_dst=self.vc, theta=cs.theta, eps=cs.eps)
+        self.out = torch.empty_like(self.t["q"])
+        self.ws = torch.empty(qa.prefill_workspace_size(cs.B, cs.T, cs.Hkv), dtype=torch.uint8, device=dev)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+        torch.cuda.synchronize(dev)
+        st, site = qa.device_status(clear=True, device=dev)
+        if st != qa.OK:
+            raise RuntimeError(f"cache build failed: {qa.status_string(st)} at site {site}")
+
+    def step(self):
+        t, cs = self.t, self.cs
+        self.qa.prefill_chunk(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], self.kc, self.vc,
+                              cs.start, out=self.out, workspace=self.ws, theta=cs.theta, eps=cs.eps)
+
+    def config(self):
+        cs = self.cs
+        return {"workload": cs.name, "B": cs.B, "start": cs.start, "T": cs.T, "Hq": cs.Hq, "Hkv": cs.Hkv,
+                "d": cs.d, "rope_theta": cs.theta, "rms_eps": cs.eps, "seed": 0,
+                "l2": "flushed before every step (256 MiB write, outside the timed windows)",
+                "parallelism": "replicas (one independent workload per GPU)"}
+
+
+def cpu_oracle_chunk_sample(name: str = "qwen3-4b-second-chunk", rows: int = 512, seed: int = 0):
+    """The oracle's chunked prefill on the last `rows` new rows (every head) of the chunk."""
+    import oracle
+    from synthetic import as_f64
+
+    cs = CHUNK_SHAPES[name]
+    inp = chunk_inputs(cs, seed=seed)
+    kc = np.stack([oracle.build_cache_k(as_f64(inp["k_hist"][b]), as_f64(inp["k_norm_w"]), cs.theta, cs.eps)
+                   .transpose(1, 0, 2) for b in range(cs.B)])
+    vc = as_f64(inp["v_hist"]).transpose(0, 2, 1, 3)
+    sel = np.arange(cs.T - rows, cs.T)
+    t0 = time.perf_counter()
+    oracle.chunk_prefill_ref(as_f64(inp["q"]), as_f64(inp["k"]), as_f64(inp["v"]), as_f64(inp["q_norm_w"]),
+                             as_f64(inp["k_norm_w"]), inp["pos"].numpy(), kc, vc, cs.start, cs.theta, cs.eps,
+                             rows=sel)
+    secs = time.perf_counter() - t0
+    flops = cs.B * 4.0 * cs.Hq * cs.d * float((cs.start + sel + 1).sum())
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    sample = (f"last {rows} of {cs.T} new rows x {cs.Hq} heads of the {cs.name} ({flops:.3g} causal flops)")
+    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "sample": sample, "flops": flops}
+
+
+def run_chunk(args, world, rank, local):
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cal = cpu_oracle_chunk_sample(rows=16)
+        rows = int(max(4, min(4096, (120.0 / max(args.steps, 1)) / max(cal["seconds"] / 16, 1e-6))))
+        secs = flops = 0.0
+        res = None
+        for _ in range(args.steps):
+            res = cpu_oracle_chunk_sample(rows=rows)
+            secs += res["seconds"]
+            flops += res["flops"]
+        value = flops / secs / 1e12
+        cs = CHUNK_SHAPES["qwen3-4b-second-chunk"]
+        line = {"impl": "reference", "metric": CHUNK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": cs.name},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
+                                 "sample": "per step, " + res["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    w = ChunkWorkload(dev)
+    for _ in range(args.warmup):
+        w.flush.fill_(1.0)
+        w.step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            w.flush.fill_(1.0)
+            ev[i][0].record()
+            w.step()
+            ev[i][1].record()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+    st, site = w.qa.device_status(clear=True, device=dev)
+    if st != w.qa.OK:
+        raise RuntimeError(f"device status {w.qa.status_string(st)} at site {site}")
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    # e2e: pinned host inputs in, the call, the output back, inside one event window
+    ph = {k: v.pin_memory() for k, v in w.host.items()}
+    out_h = torch.empty(w.out.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in ph.values())
+    e_steps = max(1, min(K, 200))
+    e_ms = 0.0
+    for _ in range(e_steps):
+        w.flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k, v in ph.items():
+            w.t[k].copy_(v, non_blocking=True)
+        w.step()
+        out_h.copy_(w.out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        e_ms += e0.elapsed_time(e1)
+    ms, e_ms = max_over_ranks(world, [ms, e_ms], dev)
+    if rank != 0:
+        return
+    flops = w.cs.causal_flops()
+    per_s = ms * 1e-3 / K
+    achieved = flops / per_s / 1e12
+    line = {"metric": CHUNK_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": w.config(),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "chunked-prefill call (K prologue + cache append + attention)",
+                         "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
+            "gpu_launches": ChunkWorkload.LAUNCHES_PER_STEP * K, "clocks": clk.summary(),
+            "e2e": {"value": world * flops * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
+                    "ms_per_step": e_ms / e_steps}}
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_chunk_sample(rows=2048)
+        line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
+                                "sample": cb["sample"], "seconds": cb["seconds"]}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------------------ main
 def dist_setup(backend: str = "nccl"):
     """One process per GPU (torchrun env).  The process group only carries the timing
@@ -403,9 +569,18 @@ def main():
                     help="prefill workload of the step (profiling of the other shapes)")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="decode the first n of the 64 sequences (small cases for ncu captures)")
+    ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill"],
+                    help="step: 0.6B prefill + batched decode (default); chunked-prefill: the chunk call alone")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup("nccl")
+    if args.workload == "chunked-prefill":
+        run_chunk(args, world, rank, local)
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         if world > 1:

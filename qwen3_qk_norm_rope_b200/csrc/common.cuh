@@ -76,6 +76,24 @@ __device__ __forceinline__ void rope_sincos(int pos, float hi, float lo, float& 
   sincosf(r, &s, &c);
 }
 
+// A 16-byte global load issued where it stands (volatile: kept in program order with the
+// other volatile loads of its batch, so a batch is in flight together).
+__device__ __forceinline__ float4 ld_global_v4f(const float4* ptr) {
+  float4 v;
+  asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(ptr));
+  return v;
+}
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization
+// may start while the previous kernel in the stream still runs; griddep_wait() blocks the
+// calling thread until that kernel has completed and its memory writes are visible (a
+// no-op when there is no such kernel).  griddep_launch_dependents() lets the next kernel
+// start once every CTA of this grid has issued it or exited.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------- bf16
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   // cvt.rn.bf16x2.f32 d, a, b puts a in the upper half and b in the lower half.

@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     if (lane == 0) {
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
+      griddep_wait();  // K' (and a cache's V) come from the K-prologue kernel before this one
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
       uint32_t it = 0;
       bool ok = true;
@@ -306,16 +307,25 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           ss4[i & 3] = fmaf(x0, x0, fmaf(x1, x1, ss4[i & 3]));
         }
         const float r = rsqrtf(fmaf((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), 1.0f / kD, p.eps));
+        griddep_wait();  // rope_tab is written by the K-prologue kernel (a no-op after the first)
         const float4* tab = p.rope_tab + static_cast<size_t>(b * p.T + t) * 32;
         const float2* g2 = reinterpret_cast<const float2*>(p.q_norm_w);
+        // The row's 32 (cos, sin) pairs come in four batches of eight loads each, all in
+        // flight together: one memory latency per batch, not one per frequency.
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
-          const float4 cs = __ldg(tab + i);  // (cos f0, sin f0, cos f1, sin f1)
-          const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
-          const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
-          const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
-          w[i] = pack_bf16x2(a0 * cs.x - b0 * cs.y, a1 * cs.z - b1 * cs.w);
-          w[32 + i] = pack_bf16x2(b0 * cs.x + a0 * cs.y, b1 * cs.z + a1 * cs.w);
+        for (int i0 = 0; i0 < 32; i0 += 8) {
+          float4 cs[8];  // (cos f0, sin f0, cos f1, sin f1) of frequencies 2i, 2i+1
+#pragma unroll
+          for (int u = 0; u < 8; ++u) cs[u] = ld_global_v4f(tab + i0 + u);
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
+            const int i = i0 + u;
+            const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
+            const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
+            const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
+            w[i] = pack_bf16x2(a0 * cs[u].x - b0 * cs[u].y, a1 * cs[u].z - b1 * cs[u].w);
+            w[32 + i] = pack_bf16x2(b0 * cs[u].x + a0 * cs[u].y, b1 * cs[u].z + a1 * cs[u].w);
+          }
         }
       } else {
 #pragma unroll

@@ -34,6 +34,9 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
   // The RoPE constants go through shared memory once per block: read from parameter space
   // with a lane-dependent index they would serialise.
   __shared__ float s_rope[2 * kHalf];
+  // The attention kernel that follows may be scheduled now: it waits (griddep_wait) for
+  // this grid's results before it reads them, and meanwhile sets up and loads its queries.
+  griddep_launch_dependents();
   if (threadIdx.x < 2 * kHalf)
     s_rope[threadIdx.x] = threadIdx.x < kHalf ? p.rope.hi[threadIdx.x] : p.rope.lo[threadIdx.x - kHalf];
   __syncthreads();

@@ -322,7 +322,23 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     p.fault = g_fault;
   }
   const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
-  q3::fmha_prefill_kernel<<<grid, q3::kPrefillThreads, q3::kPrefillSmemBytes, s>>>(mk, mv, p);
+  // Programmatic dependent launch: the attention CTAs may be scheduled while the K prologue
+  // finishes; they set up, load their raw query rows, and wait (griddepcontrol.wait) before
+  // reading K', the cache or the RoPE table.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(q3::kPrefillThreads);
+  cfg.dynamicSmemBytes = q3::kPrefillSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mk, mv, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
