@@ -168,7 +168,7 @@ class Workload:
         self.p_host = p
         self.p = {k: v.to(dev) for k, v in p.items()}
         self.p_out = torch.empty_like(self.p["q"])
-        self.p_ws = torch.empty(qa.prefill_workspace_size(self.ps.B, self.ps.T, self.ps.Hkv), dtype=torch.uint8,
+        self.p_ws = torch.empty(qa.prefill_workspace_size(self.ps.B, self.ps.T, self.ps.Hq, self.ps.Hkv), dtype=torch.uint8,
                                 device=dev)
         d = decode_step_inputs(full, seed=seed)
         d = {k: (v[:decode_seqs].contiguous() if k in ("q", "k_new", "v_new", "cache_lens") else v)
@@ -343,7 +343,7 @@ class ChunkWorkload:
         qa.qk_norm_rope(inp["k_hist"].to(dev), self.t["k_norm_w"], pos, self.kc, v_src=inp["v_hist"].to(dev),
                         v_dst=self.vc, theta=cs.theta, eps=cs.eps)
         self.out = torch.empty_like(self.t["q"])
-        self.ws = torch.empty(qa.prefill_workspace_size(cs.B, cs.T, cs.Hkv), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(qa.prefill_workspace_size(cs.B, cs.T, cs.Hq, cs.Hkv), dtype=torch.uint8, device=dev)
         self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
         st, site = qa.device_status(clear=True, device=dev)

@@ -81,8 +81,8 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos,
  *   q_norm_w, k_norm_w  [d] fp32 gains.
  *   pos       [B, T] int32 RoPE positions.
  *   out       [B, T, Hq, d] bf16 attention output (heads not merged with o_proj).
- * The call needs qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes of scratch (the
- * normed+rotated keys and each token's RoPE cos/sin), which it obtains stream-ordered with
+ * The call needs qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d) bytes of scratch (the
+ * normed+rotated keys and queries), which it obtains stream-ordered with
  * cudaMallocAsync/cudaFreeAsync on `stream`.  Use qwen3_attn_prefill_ex to pass your own
  * workspace or to fill a KV cache instead.
  */
@@ -101,9 +101,10 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
  *             written to slots 0..T-1 and attention reads them from there, so the cache is
  *             ready for qwen3_attn_decode with cache_lens = T.
  *   workspace, ws_bytes  device scratch of at least
- *             qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes, else
+ *             qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d) bytes, else
  *             QWEN3_ERR_WORKSPACE.  It holds the normed+rotated keys (unused when a cache is
- *             given) and every token's RoPE cos/sin, shared by the key and query prologues.
+ *             given) and queries, which one prologue pass per token writes before the
+ *             attention kernel reads them.
  */
 int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
                           const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
@@ -130,7 +131,7 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
  *   out       [B, T, Hq, d] bf16; lse optional [B, Hq, T] fp32 (NULL to skip).
  *   start     cached tokens, the same for every batch row; 0 <= start and
  *             start + T <= Tcap, else QWEN3_ERR_INVALID_ARG.
- *   workspace, ws_bytes  at least qwen3_attn_prefill_workspace_size(B, T, Hkv, d) bytes,
+ *   workspace, ws_bytes  at least qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d) bytes,
  *             else QWEN3_ERR_WORKSPACE.
  * Other errors as in qwen3_attn_prefill_ex.  The caches must not alias q, k, v or out.
  */
@@ -198,9 +199,10 @@ int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
                               int N, int Hq, int Hkv, int d, int Lmax,
                               float theta, float eps, qwen3_stream_t stream);
 
-/* Scratch bytes qwen3_attn_prefill_ex needs: B*Hkv*T*d*2 (keys) + B*T*512 (RoPE cos/sin),
- * plus alignment slack. */
-size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d);
+/* Scratch bytes qwen3_attn_prefill_ex and qwen3_attn_prefill_chunk need: B*T*Hkv*d*2
+ * (normed, rotated keys) + B*T*Hq*d*2 (normed, rotated queries), plus alignment slack;
+ * 0 when a size is not positive. */
+size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d);
 
 /* Scratch bytes qwen3_attn_decode needs (split-KV partial outputs and logsumexps). */
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax);

@@ -31,7 +31,7 @@ SIGNATURES = {
                                       _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
     "qwen3_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
-    "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I]),
+    "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_status_string": (ctypes.c_char_p, [_I]),
@@ -96,8 +96,8 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device: 
         raise ValueError(f"{name} must be contiguous")
 
 
-def prefill_workspace_size(B: int, T: int, Hkv: int, d: int = HEAD_DIM) -> int:
-    return int(lib().qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
+def prefill_workspace_size(B: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
 
 
 def decode_workspace_size(N: int, Hq: int, Lmax: int, d: int = HEAD_DIM) -> int:
@@ -153,7 +153,7 @@ def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: floa
         _need(k_cache, "k_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
         _need(v_cache, "v_cache", torch.bfloat16, (B, Hkv, Tcap, d), dev)
     if workspace is None:
-        workspace = torch.empty(prefill_workspace_size(B, T, Hkv, d), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(prefill_workspace_size(B, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qwen3_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
                                        _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
@@ -185,7 +185,7 @@ def prefill_chunk(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int
     if lse is not None:
         _need(lse, "lse", torch.float32, (B, Hq, T), dev)
     if workspace is None:
-        workspace = torch.empty(prefill_workspace_size(B, T, Hkv, d), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(prefill_workspace_size(B, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().qwen3_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
                                           _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), int(start), Tcap,

@@ -18,7 +18,7 @@ constexpr int kHalf = kD / 2;    // RoPE pairs dim i with dim i + 64
 enum Site : int {
   kSiteNone = 0,
   kSitePrologueRow = 10,
-  kSitePrefillQReady = 20,
+  kSitePrefillQFull = 20,
   kSitePrefillKFull = 21,
   kSitePrefillVFull = 22,
   kSitePrefillKEmpty = 23,
@@ -27,6 +27,7 @@ enum Site : int {
   kSitePrefillPReady = 26,
   kSitePrefillOFull = 27,
   kSitePrefillDrain = 28,
+  kSitePrefillQEmpty = 29,
   kSiteDecodeFull = 40,
   kSiteDecodeEmpty = 41,
   kSiteDecodeLen = 42,
@@ -74,14 +75,6 @@ __device__ __forceinline__ void rope_sincos(int pos, float hi, float lo, float& 
   r = fmaf(-n, kC2, r);
   r = __fadd_rn(r, t);
   sincosf(r, &s, &c);
-}
-
-// A 16-byte global load issued where it stands (volatile: kept in program order with the
-// other volatile loads of its batch, so a batch is in flight together).
-__device__ __forceinline__ float4 ld_global_v4f(const float4* ptr) {
-  float4 v;
-  asm volatile("ld.global.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(ptr));
-  return v;
 }
 
 // Programmatic dependent launch.  A kernel launched with programmatic stream serialization

@@ -1,5 +1,5 @@
-// prefill.cuh - causal GQA flash attention for sm_100a with the Q half of the QK-Norm+RoPE
-// prologue fused into the Q-tile load.
+// prefill.cuh - causal GQA flash attention for sm_100a over the normed, rotated queries and
+// keys that the QK-Norm+RoPE prologue kernel leaves in the workspace (or the KV cache).
 //
 // What it computes: for every query row, softmax over keys j <= i of (q'.k'_j)/sqrt(d),
 // times v_j, where q' and k' are the QK-Normed and rotated vectors and query head h reads
@@ -16,15 +16,16 @@
 // rows.  CTAs are persistent (one per SM) and take items in heaviest-first order.
 //
 // Ten warps:
-//   warp 0      TMA producer: K'/V tiles (128 keys x 128 dims, two 128B-swizzled boxes
-//               each) into a 2-stage ring; owns the TMEM allocation.
+//   warp 0      TMA producer: the item's two Q' tiles (the prologue kernel wrote Q' in the
+//               tiles' row order, so a tile is one 2-D box pair), then K'/V tiles (128 keys
+//               x 128 dims, two 128B-swizzled boxes each) into a 2-stage ring; owns the TMEM
+//               allocation.  Q'_X of the next item is loaded as soon as the last S_X MMA of
+//               the current item has read the buffer, so it is resident before it is needed.
 //   warp 1      MMA issuer (one thread).  Per key tile j it issues PV_A(j-1), S_A(j),
 //               PV_B(j-1), S_B(j), so the tensor core works on one tile while the softmax
 //               warpgroup of the other tile runs.
 //   warps 2-5   softmax warpgroup of tile A, one thread per row (TMEM lane quadrant =
-//   warps 6-9   warp % 4); softmax warpgroup of tile B.  Each runs the Q prologue of its
-//               tile (thread per row, angles from the table the K prologue wrote) into
-//               swizzled smem, then per key tile: tcgen05.ld of its S row,
+//   warps 6-9   warp % 4); softmax warpgroup of tile B.  Per key tile: tcgen05.ld of its S row,
 //               causal mask, exp2 online softmax with a lazy rescale (O is rescaled only
 //               when the running max grows by more than 2^8), bf16 P written back into TMEM
 //               over its own S columns; finally O/l and the LSE.
@@ -41,10 +42,8 @@
 namespace q3 {
 
 struct PrefillParams {
-  const uint32_t* q;  // [B, T, Hq, d] bf16 pairs
-  const float* q_norm_w;
-  const float* k_norm_w;  // only its max |g| is used here (the logit bound)
-  const float4* rope_tab;  // [B*T][32]: (cos, sin) of frequencies 2i, 2i+1 at each token's position
+  const float* q_norm_w;  // the gains: only their max |g| is used here (the logit bound)
+  const float* k_norm_w;
   uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
   int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
@@ -62,8 +61,9 @@ constexpr uint32_t kPfV = 4 * kPfTile;  // 2 stages
 constexpr uint32_t kPfBar = 6 * kPfTile;
 // barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage
 constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
-                   kBOFull = 96, kBQReady = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
-                   kBRed = 144;  // 2 groups x 4 warps x (max|g_q|, max|g_k|)
+                   kBOFull = 96, kBQFull = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
+                   kBRed = 144,     // 2 groups x 4 warps x (max|g_q|, max|g_k|): 64 bytes
+                   kBQEmpty = 208;  // [X]: the last S_X MMA of an item has read Q'_X
 constexpr uint32_t kPrefillSmemBytes = kPfBar + 256 + 1024;  // + slack to align the base to 1024
 constexpr int kPrefillThreads = 320;
 constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
@@ -118,8 +118,8 @@ __device__ __forceinline__ void item_coords(const PrefillParams& p, int item, in
 }
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
-    fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ PrefillParams p) {
+    fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -138,7 +138,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar + kBSFull + 8 * s, 1);
       mbar_init(bar + kBPReady + 8 * s, 128);
       mbar_init(bar + kBOFull + 8 * s, 1);
-      mbar_init(bar + kBQReady + 8 * s, 128);
+      mbar_init(bar + kBQFull + 8 * s, 1);
+      mbar_init(bar + kBQEmpty + 8 * s, 1);
     }
     mbar_init(bar + kBDone, 1);
     *abort_flag = 0;
@@ -157,17 +158,33 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
-      griddep_wait();  // K' (and a cache's V) come from the K-prologue kernel before this one
-      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
-      uint32_t it = 0;
+      griddep_wait();  // Q', K' (and a cache's V) come from the prologue kernel before this one
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last[2] = {-1, -1};
+      uint32_t it = 0, q_use[2] = {0, 0};
       bool ok = true;
       for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
-        const int n = max(tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv);
-        for (int j = 0; j < n; ++j, ++it) {
+        const int nX[2] = {tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv};
+        const int n = max(nX[0], nX[1]);
+        for (int X = 0; X < 2 && ok; ++X) {
+          if (nX[X] == 0) continue;
+          // buffer X is free once the previous item's last S_X MMA has completed
+          if (q_use[X] >= 1 &&
+              !mbar_wait(bar + kBQEmpty + 8 * X, (q_use[X] - 1) & 1, p.wait, abort_flag, kSitePrefillQEmpty)) {
+            ok = false;
+            break;
+          }
+          const int row0 = (2 * pair + X) * 128;  // the tile's first row of Q' [b, hkv, T*G, d]
+          mbar_arrive_expect_tx(bar + kBQFull + 8 * X, kPfTile);
+          tma_load_4d(sb + kPfQ + X * kPfTile, &tmQ, bar + kBQFull + 8 * X, 0, row0, hkv, b);
+          tma_load_4d(sb + kPfQ + X * kPfTile + kPfBox, &tmQ, bar + kBQFull + 8 * X, 64, row0, hkv, b);
+          q_last[X] = static_cast<int>(q_use[X]++);
+        }
+        for (int j = 0; j < n && ok; ++j, ++it) {
           const int st = it & 1;
           const uint32_t ph = (it >> 1) & 1;
           if (it >= 2 && !mbar_wait(bar + kBKEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillKEmpty)) {
@@ -192,6 +209,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       }
       // Every issued copy must land before this CTA's shared memory is released.
       for (int s = 0; s < 2; ++s) {
+        if (q_last[s] >= 0) mbar_wait(bar + kBQFull + 8 * s, q_last[s] & 1, p.wait, nullptr, kSitePrefillDrain);
         if (k_last[s] >= 0) mbar_wait(bar + kBKFull + 8 * s, (k_last[s] >> 1) & 1, p.wait, nullptr, kSitePrefillDrain);
         if (v_last[s] >= 0) mbar_wait(bar + kBVFull + 8 * s, (v_last[s] >> 1) & 1, p.wait, nullptr, kSitePrefillDrain);
       }
@@ -210,7 +228,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X)
           if (nX[X] > 0) {
-            ok = mbar_wait(bar + kBQReady + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQReady);
+            ok = mbar_wait(bar + kBQFull + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQFull);
             ++q_cnt[X];
           }
         if (!ok) break;
@@ -227,6 +245,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         smem_desc_sw128(sK + (it & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
             }
             tc_commit(bar + kBSFull + 8 * X);
+            if (nX[X] == 1) tc_commit(bar + kBQEmpty + 8 * X);  // the item's last S_X
           }
         tc_commit(bar + kBKEmpty + 8 * (it & 1));
         // j >= 1: PV_X(j-1) then S_X(j), for X = A, B
@@ -259,6 +278,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                           smem_desc_sw128(sK + (cur & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
               }
               tc_commit(bar + kBSFull + 8 * X);
+              if (j == nX[X] - 1) tc_commit(bar + kBQEmpty + 8 * X);  // the item's last S_X
             }
           }
           if (!ok) break;
@@ -276,82 +296,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int X = (warp - 2) >> 2;     // 0: tile A, 1: tile B
     const int wq = warp & 3;           // TMEM lane quadrant this warp may access
     const int row = wq * 32 + lane;    // query-tile row owned by this thread
-    const uint32_t sQ = sb + kPfQ + X * kPfTile;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + tm_s(X), tO = tmem + lane_off + tm_o(X);
     const float sl2 = p.scale_log2;
     const int G = 1 << p.log2G;
-    // Q prologue of the query tile at (b, hkv, t0) into Q'_X, then signal qready_X.
-    auto q_prologue = [&](int b, int hkv, int t0) {
-      // Q prologue, one thread per row: QK-Norm of the raw row (a register-local sum of
-      // squares), gain, and rotate-half RoPE with the (cos, sin) of the row's position that
-      // the K-prologue kernel left in rope_tab; then the row goes to swizzled smem as 16
-      // chunks of 16 bytes (row r, chunk c at c ^ (r % 8): conflict-free across a warp).
-      const int t = t0 + (row >> p.log2G);
-      uint32_t w[64];  // bf16 pairs: w[i] = dims (2i, 2i+1)
-      if (t < p.T) {   // rows past T get Q' = 0
-        const uint4* qs = reinterpret_cast<const uint4*>(p.q) +
-                          (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint4 u = __ldg(qs + i);
-          w[4 * i] = u.x;
-          w[4 * i + 1] = u.y;
-          w[4 * i + 2] = u.z;
-          w[4 * i + 3] = u.w;
-        }
-        float ss4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float x0 = bf16lo(w[i]), x1 = bf16hi(w[i]);
-          ss4[i & 3] = fmaf(x0, x0, fmaf(x1, x1, ss4[i & 3]));
-        }
-        const float r = rsqrtf(fmaf((ss4[0] + ss4[1]) + (ss4[2] + ss4[3]), 1.0f / kD, p.eps));
-        griddep_wait();  // rope_tab is written by the K-prologue kernel (a no-op after the first)
-        const float4* tab = p.rope_tab + static_cast<size_t>(b * p.T + t) * 32;
-        const float2* g2 = reinterpret_cast<const float2*>(p.q_norm_w);
-        // The row's 32 (cos, sin) pairs come in four batches of eight loads each, all in
-        // flight together: one memory latency per batch, not one per frequency.
-#pragma unroll
-        for (int i0 = 0; i0 < 32; i0 += 8) {
-          float4 cs[8];  // (cos f0, sin f0, cos f1, sin f1) of frequencies 2i, 2i+1
-#pragma unroll
-          for (int u = 0; u < 8; ++u) cs[u] = ld_global_v4f(tab + i0 + u);
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {  // frequencies 2i, 2i+1 rotate dims (2i, 64+2i), (2i+1, 65+2i)
-            const int i = i0 + u;
-            const float2 ga = __ldg(g2 + i), gb = __ldg(g2 + 32 + i);
-            const float a0 = ga.x * (bf16lo(w[i]) * r), a1 = ga.y * (bf16hi(w[i]) * r);
-            const float b0 = gb.x * (bf16lo(w[32 + i]) * r), b1 = gb.y * (bf16hi(w[32 + i]) * r);
-            w[i] = pack_bf16x2(a0 * cs[u].x - b0 * cs[u].y, a1 * cs[u].z - b1 * cs[u].w);
-            w[32 + i] = pack_bf16x2(b0 * cs[u].x + a0 * cs[u].y, b1 * cs[u].z + a1 * cs[u].w);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) w[i] = 0u;
-      }
-#pragma unroll
-      for (int cb = 0; cb < 16; ++cb)
-        st_shared_v4(sQ + (cb >> 3) * kPfBox + sw128_offset(row, cb & 7), w[4 * cb], w[4 * cb + 1], w[4 * cb + 2],
-                     w[4 * cb + 3]);
-      fence_proxy_async_smem();
-      mbar_arrive(bar + kBQReady + 8 * X);
-    };
-    // Pull a tile's raw query rows and its rows' angles toward L2 ahead of its prologue.
-    auto prefetch_tile = [&](int b, int hkv, int t0) {
-      const int t = t0 + (row >> p.log2G);
-      if (t >= p.T) return;
-      const char* qrow = reinterpret_cast<const char*>(
-          p.q + (static_cast<long long>(b * p.T + t) * p.Hq + hkv * G + (row & (G - 1))) * (kD / 2));
-      const char* trow = reinterpret_cast<const char*>(p.rope_tab + static_cast<size_t>(b * p.T + t) * 32);
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow));
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + 128));
-      if ((row & (G - 1)) == 0) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) asm volatile("prefetch.global.L2 [%0];" ::"l"(trow + 128 * i));
-      }
-    };
     // Reference for the exponentials.  QK-Norm bounds every logit: by Cauchy-Schwarz on the
     // normalised, rotated (norm-preserving) vectors, |q'.k'|/sqrt(d) <= sqrt(d) max|g_q|
     // max|g_k| (times 1 + 2^-7 for their bf16 rounding).  With that bound bnd (in log2
@@ -380,33 +328,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const bool fast = bnd <= 60.0f;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
-    // The Q prologue of the next item runs as soon as this item's last S_X has been read
-    // (Q'_X is then free), before the epilogue: the tensor core can start the next item
-    // while this one's outputs are stored.  O_X stays safe: the next item's first PV_X
+    // The tensor core may start the next item (its Q' tiles arrive by TMA) while this
+    // group stores the current item's outputs.  O_X stays safe: the next item's first PV_X
     // waits for a P that is only written after this epilogue.
-    int k = 0, item = round_item(0);
-    if (item < p.n_items) {
+    for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
       int pair, b, hkv;
       item_coords(p, item, pair, b, hkv);
       const TileInfo ti = tile_info(p, 2 * pair + X);
-      if (ti.nkv > 0) q_prologue(b, hkv, ti.t0);
-    }
-    for (; item < p.n_items && ok; item = round_item(++k)) {
-      int pair, b, hkv;
-      item_coords(p, item, pair, b, hkv);
-      const TileInfo ti = tile_info(p, 2 * pair + X);
-      const int next = round_item(k + 1);
-      int npair = 0, nb = 0, nhkv = 0;
-      TileInfo tn{0, 0};
-      if (next < p.n_items) {
-        item_coords(p, next, npair, nb, nhkv);
-        tn = tile_info(p, 2 * npair + X);
-      }
-      if (ti.nkv == 0) {  // this item has no tile X (its prologue was skipped too)
-        if (tn.nkv > 0) q_prologue(nb, nhkv, tn.t0);
-        continue;
-      }
-      if (tn.nkv > 0) prefetch_tile(nb, nhkv, tn.t0);
+      if (ti.nkv == 0) continue;  // this item has no tile X
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
@@ -539,7 +468,6 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         mbar_arrive(bar + kBPReady + 8 * X);
       }
       if (!ok) break;
-      if (tn.nkv > 0) q_prologue(nb, nhkv, tn.t0);  // every S_X of this item has been read
       ok = mbar_wait(bar + kBOFull + 8 * X, o_cnt & 1, p.wait, abort_flag, kSitePrefillOFull);
       ++o_cnt;
       ok = __all_sync(0xffffffffu, ok);

@@ -19,8 +19,14 @@ struct PrologueParams {
   uint32_t* dst;       // [B, H, Tcap, d] bf16 pairs
   const uint2* v_src;  // optional [B, T, H, d], 4 bf16 per lane
   uint2* v_dst;        // optional [B, H, Tcap, d]
-  float4* rope_tab;    // optional [B*T][32]: (cos, sin) of frequencies 2i, 2i+1 at pos[b,t]
+  // Optional queries of the same tokens (the prefill): raw xq [B, T, Hq, d] with gain wq,
+  // written as Q' [B, H, T*G, d] with G = Hq / H: row t*G + g of KV head h holds query
+  // head h*G + g, the row order of the attention kernel's GQA-packed query tiles.
+  const uint32_t* xq;
+  const float* wq;
+  uint32_t* dstq;
   int B, T, H, Tcap, write_at_pos;
+  int Hq, log2G;
   float eps;
   RopeTable rope;
 };
@@ -28,8 +34,8 @@ struct PrologueParams {
 constexpr int kPrologueHeads = 8;  // head vectors of one token in flight per warp
 
 // One warp per token (b, t): its position and the sin/cos of its 64 angles are computed
-// once and shared by the token's H head vectors, whose loads are all issued first.  The
-// prefill also keeps the angles (rope_tab) for the query tiles of the attention kernel.
+// once and shared by the token's H key heads (and, for the prefill, its Hq query heads),
+// whose loads are issued a batch at a time before any arithmetic.
 __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant__ PrologueParams p) {
   // The RoPE constants go through shared memory once per block: read from parameter space
   // with a lane-dependent index they would serialise.
@@ -59,7 +65,6 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     float s0, c0, s1, c1;
     rope_sincos(ps, hi0, lo0, s0, c0);
     rope_sincos(ps, hi1, lo1, s1, c1);
-    if (p.rope_tab != nullptr) p.rope_tab[static_cast<size_t>(bt) * 32 + lane] = make_float4(c0, s0, c1, s1);
     for (int h0 = 0; h0 < p.H; h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
       uint2 vv[kPrologueHeads];
@@ -85,6 +90,34 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
         ds[lane] = pack_bf16x2(ya.x, ya.y);
         ds[32 + lane] = pack_bf16x2(yb.x, yb.y);
         if (p.v_src != nullptr) p.v_dst[drow * (kD / 4) + lane] = vv[u];
+      }
+    }
+    if (p.xq == nullptr) continue;
+    const float2 qa = reinterpret_cast<const float2*>(p.wq)[lane];
+    const float2 qb = reinterpret_cast<const float2*>(p.wq)[32 + lane];
+    const int G = 1 << p.log2G;
+    for (int h0 = 0; h0 < p.Hq; h0 += kPrologueHeads) {
+      uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
+#pragma unroll
+      for (int u = 0; u < kPrologueHeads; ++u) {
+        ua[u] = ub[u] = 0u;
+        if (h0 + u < p.Hq) {
+          const size_t v = static_cast<size_t>(bt) * p.Hq + h0 + u;
+          ua[u] = p.xq[v * (kD / 2) + lane];
+          ub[u] = p.xq[v * (kD / 2) + 32 + lane];
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kPrologueHeads; ++u) {
+        const int h = h0 + u;
+        if (h >= p.Hq) break;  // uniform across the warp
+        float2 ya, yb;
+        norm_rope_pairs(make_float2(bf16lo(ua[u]), bf16hi(ua[u])), make_float2(bf16lo(ub[u]), bf16hi(ub[u])), qa,
+                        qb, s0, c0, s1, c1, p.eps, ya, yb);
+        const size_t drow = ((static_cast<size_t>(b) * p.H + (h >> p.log2G)) * p.T + t) * G + (h & (G - 1));
+        uint32_t* ds = p.dstq + drow * (kD / 2);
+        ds[lane] = pack_bf16x2(ya.x, ya.y);
+        ds[32 + lane] = pack_bf16x2(yb.x, yb.y);
       }
     }
   }

@@ -130,9 +130,17 @@ int check_common(int Hq, int Hkv, int d) {
   return QWEN3_OK;
 }
 
+// Q (optional, the prefill): raw xq [B, T, Hq, d] with gain wq to Q' [B, H, T*Hq/H, d].
+struct PrologueQ {
+  const void* xq = nullptr;
+  const float* wq = nullptr;
+  void* dstq = nullptr;
+  int Hq = 0;
+};
+
 int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
                     int B, int T, int H, int Tcap, int write_at_pos, float theta, float eps, cudaStream_t stream,
-                    void* rope_tab = nullptr) {
+                    const PrologueQ& q = PrologueQ()) {
   q3::PrologueParams p;
   p.x = static_cast<const uint32_t*>(x);
   p.w = w;
@@ -140,7 +148,11 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.dst = static_cast<uint32_t*>(dst);
   p.v_src = static_cast<const uint2*>(v_src);
   p.v_dst = static_cast<uint2*>(v_dst);
-  p.rope_tab = static_cast<float4*>(rope_tab);
+  p.xq = static_cast<const uint32_t*>(q.xq);
+  p.wq = q.wq;
+  p.dstq = static_cast<uint32_t*>(q.dstq);
+  p.Hq = q.Hq;
+  p.log2G = q.xq != nullptr ? ilog2(q.Hq / H) : 0;
   p.B = B;
   p.T = T;
   p.H = H;
@@ -200,10 +212,10 @@ int qwen3_attn_device_status(qwen3_stream_t stream, int clear, int* site) {
   return h[0];
 }
 
-size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hkv, int d) {
-  if (B <= 0 || T <= 0 || Hkv <= 0 || d <= 0) return 0;
-  // K' [B, Hkv, T, d] bf16, then the per-token cos/sin table [B*T][64] float2
-  return kspace_bytes(B, T, Hkv, d) + static_cast<size_t>(B) * T * 64 * 8 + 256;
+size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d) {
+  if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return 0;
+  // K' [B, Hkv, T, d] bf16, then Q' [B, Hkv, T*G, d] bf16 (as many elements as q)
+  return kspace_bytes(B, T, Hkv, d) + kspace_bytes(B, T, Hq, d) + 256;
 }
 
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax) {
@@ -256,29 +268,42 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
   if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
-  if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hkv, d))
+  if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
     return QWEN3_ERR_WORKSPACE;
   if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
     return QWEN3_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
 
-  // 1. K prologue, written in cache layout [B, Hkv, Tc, d] from slot `start` on (and V copied
-  //    when filling a cache); it also leaves every new token's RoPE cos/sin in the workspace
-  //    for the query tiles.  Shifting the base by start rows puts token t at slot start + t.
+  // 1. QK prologue.  K' in cache layout [B, Hkv, Tc, d] from slot `start` on (and V copied
+  //    when filling a cache; shifting the base by start rows puts token t at slot start + t),
+  //    and Q' in the query tiles' row order [B, Hkv, T*G, d], both in one pass per token.
   const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
   qwen3_bf16* kdst = use_cache ? k_cache : reinterpret_cast<qwen3_bf16*>(w0);
-  void* rope_tab = reinterpret_cast<void*>(w0 + kspace_bytes(B, T, Hkv, d));
+  qwen3_bf16* qdst = reinterpret_cast<qwen3_bf16*>(w0 + kspace_bytes(B, T, Hkv, d));
   const int Tc = use_cache ? Tcap : T;
   const size_t shift = static_cast<size_t>(start) * kD;
+  PrologueQ pq;
+  pq.xq = q;
+  pq.wq = q_norm_w;
+  pq.dstq = qdst;
+  pq.Hq = Hq;
   st = launch_prologue(k, k_norm_w, pos, kdst + shift, use_cache ? v : nullptr, use_cache ? v_cache + shift : nullptr,
-                       B, T, Hkv, Tc, 0, theta, eps, s, rope_tab);
+                       B, T, Hkv, Tc, 0, theta, eps, s, pq);
   if (st != QWEN3_OK) return st;
 
   // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
   //    read as zeros.
-  CUtensorMap mk, mv;
+  CUtensorMap mq, mk, mv;
   const cuuint32_t box[4] = {64, 128, 1, 1};
+  {
+    // Q' rows past T*G read as zeros (their outputs are never stored)
+    const cuuint64_t TG = static_cast<cuuint64_t>(T) * (Hq / Hkv);
+    const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(kD), TG, static_cast<cuuint64_t>(Hkv),
+                                 static_cast<cuuint64_t>(B)};
+    const cuuint64_t qstr[3] = {kD * 2ull, TG * kD * 2ull, static_cast<cuuint64_t>(Hkv) * TG * kD * 2ull};
+    if (!make_map(&mq, qdst, 4, qdims, qstr, box)) return QWEN3_ERR_CUDA;
+  }
   {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(start) + T,
                                 static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(B)};
@@ -296,10 +321,8 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
 
   // 3. Attention.
   q3::PrefillParams p;
-  p.q = reinterpret_cast<const uint32_t*>(q);
   p.q_norm_w = q_norm_w;
   p.k_norm_w = k_norm_w;
-  p.rope_tab = static_cast<const float4*>(rope_tab);
   p.out = reinterpret_cast<uint4*>(out);
   p.lse = lse;
   p.B = B;
@@ -322,9 +345,9 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     p.fault = g_fault;
   }
   const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
-  // Programmatic dependent launch: the attention CTAs may be scheduled while the K prologue
-  // finishes; they set up, load their raw query rows, and wait (griddepcontrol.wait) before
-  // reading K', the cache or the RoPE table.
+  // Programmatic dependent launch: the attention CTAs may be scheduled while the prologue
+  // finishes; they set up (barriers, TMEM, tensor maps, the logit bound) and wait
+  // (griddepcontrol.wait) before their first load of Q', K' or the cache.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(q3::kPrefillThreads);
@@ -335,7 +358,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mk, mv, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mq, mk, mv, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return QWEN3_ERR_CUDA;
   }
@@ -371,7 +394,7 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
   const int st0 = check_common(Hq, Hkv, d);
   if (st0 != QWEN3_OK) return st0;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t bytes = qwen3_attn_prefill_workspace_size(B, T, Hkv, d);
+  const size_t bytes = qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d);
   void* ws = nullptr;
   if (cudaMallocAsync(&ws, bytes, s) != cudaSuccess) return QWEN3_ERR_CUDA;
   const int st = qwen3_attn_prefill_ex(q, k, v, q_norm_w, k_norm_w, pos, out, nullptr, nullptr, nullptr, 0, ws,

@@ -38,8 +38,9 @@ def test_version_and_status_strings():
 
 
 def test_workspace_and_cache_sizes():
-    assert qa.prefill_workspace_size(2, 2048, 8) >= 2 * 8 * 2048 * 128 * 2
-    assert qa.prefill_workspace_size(0, 10, 8) == 0
+    # K' [B, Hkv, T, d] and Q' (as many elements as q) in bf16
+    assert qa.prefill_workspace_size(2, 2048, 16, 8) >= 2 * 2048 * (16 + 8) * 128 * 2
+    assert qa.prefill_workspace_size(0, 10, 16, 8) == 0
     ns = -(-32769 // 1024)
     assert qa.decode_workspace_size(64, 32, 32769) >= 64 * 32 * ns * (128 + 1) * 4
     # 2*Hkv*d values per token per layer; 1024 for the wide-GQA block of the worked example
