@@ -44,7 +44,6 @@ namespace q3 {
 struct PrefillParams {
   const float* q_norm_w;  // the gains: only their max |g| is used here (the logit bound)
   const float* k_norm_w;
-  uint4* out;      // [B, T, Hq, d] bf16, 16-byte chunks
   float* lse;      // [B, Hq, T] or nullptr
   int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
   int start;  // cached keys before the first query row: query t is key index start + t
@@ -59,12 +58,15 @@ constexpr uint32_t kPfQ = 0;         // Q'_A, Q'_B
 constexpr uint32_t kPfK = 2 * kPfTile;  // 2 stages
 constexpr uint32_t kPfV = 4 * kPfTile;  // 2 stages
 constexpr uint32_t kPfBar = 6 * kPfTile;
+// Output staging, one 128-row x 64-dim box (16 KB, 128B-swizzled) per softmax group: the
+// epilogue writes half of O/l there and one thread stores it to `out` with a tiled bulk copy.
+constexpr uint32_t kPfStage = kPfBar + 1024;
 // barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage
 constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
                    kBOFull = 96, kBQFull = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
                    kBRed = 144,     // 2 groups x 4 warps x (max|g_q|, max|g_k|): 64 bytes
                    kBQEmpty = 208;  // [X]: the last S_X MMA of an item has read Q'_X
-constexpr uint32_t kPrefillSmemBytes = kPfBar + 256 + 1024;  // + slack to align the base to 1024
+constexpr uint32_t kPrefillSmemBytes = kPfStage + 2 * kPfBox + 1024;  // + slack to align the base to 1024
 constexpr int kPrefillThreads = 320;
 constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
 constexpr float kLn2 = 0.693147180559945309f;
@@ -119,7 +121,8 @@ __device__ __forceinline__ void item_coords(const PrefillParams& p, int item, in
 
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ PrefillParams p) {
+                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                        const __grid_constant__ PrefillParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -467,35 +470,49 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_before();
         mbar_arrive(bar + kBPReady + 8 * X);
       }
-      if (!ok) break;
-      ok = mbar_wait(bar + kBOFull + 8 * X, o_cnt & 1, p.wait, abort_flag, kSitePrefillOFull);
+      if (ok) ok = mbar_wait(bar + kBOFull + 8 * X, o_cnt & 1, p.wait, abort_flag, kSitePrefillOFull);
       ++o_cnt;
-      ok = __all_sync(0xffffffffu, ok);
+      // Every warp of the group gets here, from a finished or an abandoned key loop, and the
+      // four agree before the epilogue's group barriers: all go on or all stop.
+      ok = group_all(1 + X, ok);
       if (!ok) break;
       tc_fence_after();
       const int h = hkv * G + (row & (G - 1));
       const bool valid = t_row < p.T;
       const float inv_l = 1.0f / l;
-      uint4* dst = p.out + (static_cast<long long>(b * p.T + (valid ? t_row : 0)) * p.Hq + h) * (kD / 8);
+      // O/l in two 64-dim halves through this group's staging box.  Row r of the tile is row r
+      // of the box [P positions][G heads][64 dims], so one tiled store writes the half to
+      // out[b, t0 .. t0+P-1, hkv*G .. hkv*G+G-1, half*64 ..]; rows past T are clipped by the
+      // copy.  The storing thread waits until the previous store has read the buffer.
+      const uint32_t stg = sb + kPfStage + X * kPfBox;
+      const bool storer = row == 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + c * 32, r);
-        if (valid) {
+      for (int half = 0; half < 2; ++half) {
+        if (storer) bulk_wait_read_all();
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + X) : "memory");
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(r[8 * u + 0]) * inv_l, __uint_as_float(r[8 * u + 1]) * inv_l);
-            w.y = pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv_l, __uint_as_float(r[8 * u + 3]) * inv_l);
-            w.z = pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv_l, __uint_as_float(r[8 * u + 5]) * inv_l);
-            w.w = pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv_l, __uint_as_float(r[8 * u + 7]) * inv_l);
-            dst[c * 4 + u] = w;
-          }
+        for (int c = 0; c < 2; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + half * 64 + c * 32, r);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            st_shared_v4(stg + sw128_offset(row, c * 4 + u),
+                         pack_bf16x2(__uint_as_float(r[8 * u + 0]) * inv_l, __uint_as_float(r[8 * u + 1]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv_l, __uint_as_float(r[8 * u + 3]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv_l, __uint_as_float(r[8 * u + 5]) * inv_l),
+                         pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv_l, __uint_as_float(r[8 * u + 7]) * inv_l));
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + X) : "memory");
+        if (storer) {
+          tma_store_4d(&tmO, stg, half * 64, hkv * G, t0, b);
+          bulk_commit_group();
         }
       }
       if (p.lse != nullptr && valid)
         p.lse[(static_cast<long long>(b) * p.Hq + h) * p.T + t_row] = (m + log2f(l)) * kLn2;
     }
+    if (row == 0) bulk_wait_all();  // this group's output stores have completed
   }
 
   tc_fence_before();

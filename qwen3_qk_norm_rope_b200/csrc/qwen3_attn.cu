@@ -294,8 +294,18 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
 
   // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
   //    read as zeros.
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   const cuuint32_t box[4] = {64, 128, 1, 1};
+  {
+    // out [B, T, Hq, d] as boxes of [P positions][G heads][64 dims]: one query tile's half
+    const int G = Hq / Hkv;
+    const cuuint64_t odims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(Hq),
+                                 static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
+    const cuuint64_t ostr[3] = {kD * 2ull, static_cast<cuuint64_t>(Hq) * kD * 2ull,
+                                static_cast<cuuint64_t>(T) * Hq * kD * 2ull};
+    const cuuint32_t obox[4] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G), 1};
+    if (!make_map(&mo, out, 4, odims, ostr, obox)) return QWEN3_ERR_CUDA;
+  }
   {
     // Q' rows past T*G read as zeros (their outputs are never stored)
     const cuuint64_t TG = static_cast<cuuint64_t>(T) * (Hq / Hkv);
@@ -323,7 +333,6 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   q3::PrefillParams p;
   p.q_norm_w = q_norm_w;
   p.k_norm_w = k_norm_w;
-  p.out = reinterpret_cast<uint4*>(out);
   p.lse = lse;
   p.B = B;
   p.T = T;
@@ -358,7 +367,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mq, mk, mv, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mq, mk, mv, mo, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return QWEN3_ERR_CUDA;
   }
