@@ -37,6 +37,12 @@ What it computes, and where each step is defined:
      attends to all L+1 keys ("Assembling a large model", KVCache.update and
      Transformer.forward, start = cache.length).
 
+  7. Variants ("Qwen3 Architecture Layer-by-Layer", Per-layer attention type
+     and Qwen3RotaryEmbedding; "Qwen 3 From Scratch", long context with rotary
+     scaling): a sliding-window layer lets query i see only the last W keys,
+     i - W < j <= i; another rope type brings its own inv_freq and an
+     attention_scaling that multiplies cos and sin.
+
 Readings where the pages leave a step open:
   * No intermediate rounding: the pages' HF path casts to bf16 between the
     norm and the gain; the oracle keeps everything in fp64.  `staged=True`
@@ -47,6 +53,10 @@ Readings where the pages leave a step open:
     with its x.float(), hold q' and k' before the cast): fp64 -> fp32 -> bf16.
   * Rotate-half with theta from the argument (the page prose that speaks of
     adjacent pairs and base 10000 contradicts every code block on the pages).
+  * The sliding window counts the query's own key: W keys, i - W < j <= i (the
+    pages name the windowed mask but print no formula; this is the usual
+    reading of a window of W tokens).  YaRN's frequency formula is not on the
+    pages, so the variant takes any inv_freq table as an input.
 """
 from __future__ import annotations
 
@@ -78,29 +88,37 @@ def rope_inv_freq(d: int, theta: float) -> np.ndarray:
     return np.power(np.float64(theta), -2.0 * i / d)
 
 
-def rope(x: np.ndarray, pos: np.ndarray, theta: float) -> np.ndarray:
-    """Rotate-half RoPE.  x [..., T, H, d]; pos broadcastable to [..., T]."""
+def rope(x: np.ndarray, pos: np.ndarray, theta: float, inv_freq=None, scaling: float = 1.0) -> np.ndarray:
+    """Rotate-half RoPE.  x [..., T, H, d]; pos broadcastable to [..., T].
+
+    inv_freq: optional d/2 rotary frequencies (any rope type's initialisation) in place of
+    theta^(-2i/d); scaling: the attention_scaling that multiplies cos and sin
+    ("Qwen3 Architecture Layer-by-Layer", Qwen3RotaryEmbedding; 1 for the default type)."""
     x = np.asarray(x, dtype=np.float64)
     d = x.shape[-1]
     half = d // 2
-    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_inv_freq(d, theta)  # [..., T, d/2]
-    c = np.cos(ang)[..., None, :]  # broadcast over heads
-    s = np.sin(ang)[..., None, :]
+    inv = rope_inv_freq(d, theta) if inv_freq is None else np.asarray(inv_freq, dtype=np.float64)
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * inv  # [..., T, d/2]
+    c = (np.cos(ang) * scaling)[..., None, :]  # broadcast over heads
+    s = (np.sin(ang) * scaling)[..., None, :]
     x1, x2 = x[..., :half], x[..., half:]
     return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
 
 
 def qk_prologue(x: np.ndarray, g: np.ndarray, pos: np.ndarray, theta: float, eps: float,
-                staged: bool = False) -> np.ndarray:
+                staged: bool = False, inv_freq=None, scaling: float = 1.0) -> np.ndarray:
     """QK-Norm then RoPE of raw head vectors x [..., T, H, d] at positions pos [..., T].
 
     staged=True returns the bf16 value the result rounds to when held in float32."""
-    y = rope(rms_norm(x, g, eps), pos, theta)
+    y = rope(rms_norm(x, g, eps), pos, theta, inv_freq, scaling)
     return bf16_round(y.astype(np.float32).astype(np.float64)) if staged else y
 
 
-def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray):
-    """Softmax attention of query rows over keys 0..limit[r] (inclusive).
+def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray, window: int = 0):
+    """Softmax attention of query rows over keys 0..limit[r] (inclusive); with a sliding
+    window W > 0 only keys limit[r]-W < j <= limit[r] (the last W, the query's own key
+    included: the sliding-window causal mask of "Qwen3 Architecture Layer-by-Layer",
+    Per-layer attention type).
 
     qg [R, d] already-normed/rotated queries; kk, vv [S, d]; limit [R] int.
     Returns out [R, d] and lse [R] (natural log, scaled logits).
@@ -108,7 +126,10 @@ def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray):
     d = qg.shape[-1]
     s = (qg @ kk.T) / np.sqrt(np.float64(d))  # [R, S]
     j = np.arange(kk.shape[0])
-    s = np.where(j[None, :] <= limit[:, None], s, -np.inf)
+    visible = j[None, :] <= limit[:, None]
+    if window > 0:
+        visible &= j[None, :] > limit[:, None] - window
+    s = np.where(visible, s, -np.inf)
     m = np.max(s, axis=1, keepdims=True)
     e = np.exp(s - m)
     z = np.sum(e, axis=1, keepdims=True)
@@ -118,7 +139,8 @@ def _attend(qg: np.ndarray, kk: np.ndarray, vv: np.ndarray, limit: np.ndarray):
 
 
 def prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, theta: float, eps: float,
-                rows=None, staged: bool = False, block: int = 256):
+                rows=None, staged: bool = False, block: int = 256, window: int = 0, inv_freq=None,
+                scaling: float = 1.0):
     """Causal GQA prefill with the QK-Norm + RoPE prologue, in fp64.
 
     q [B,T,Hq,d], k and v [B,T,Hkv,d], gains [d], pos [B,T] (any real arrays;
@@ -126,7 +148,9 @@ def prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, theta: float, eps: float,
     [B,Hq,T].  With `rows` (a sorted int array of query indices) only those
     rows are computed and the returned arrays are [B,len(rows),Hq,d] and
     [B,Hq,len(rows)]; keys still run over every position the mask admits.
-    Query rows are processed in blocks so no T x T matrix is ever held.
+    Query rows are processed in blocks so no T x T matrix is ever held.  window, inv_freq
+    and scaling select the variants (a sliding window; another rope type's frequencies and
+    attention_scaling); the defaults are Qwen3's full causal attention and default RoPE.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -138,21 +162,22 @@ def prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, theta: float, eps: float,
     out = np.zeros((B, rows.size, Hq, d))
     lse = np.zeros((B, Hq, rows.size))
     for b in range(B):
-        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged)  # [T, Hkv, d]
-        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged)
+        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged, inv_freq, scaling)  # [T, Hkv, d]
+        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged, inv_freq, scaling)
         for h in range(Hq):
             hk = h // G
             for r0 in range(0, rows.size, block):
                 rr = rows[r0:r0 + block]
                 top = int(rr.max()) + 1
-                o, l = _attend(qp[r0:r0 + block, h], kp[:top, hk], v[b, :top, hk], rr)
+                o, l = _attend(qp[r0:r0 + block, h], kp[:top, hk], v[b, :top, hk], rr, window)
                 out[b, r0:r0 + block, h] = o
                 lse[b, h, r0:r0 + block] = l
     return out, lse
 
 
 def chunk_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int,
-                      theta: float, eps: float, rows=None, staged: bool = False, block: int = 256):
+                      theta: float, eps: float, rows=None, staged: bool = False, block: int = 256,
+                      window: int = 0, inv_freq=None, scaling: float = 1.0):
     """T new tokens per batch row over a cache that already holds `start` tokens, in fp64.
 
     "Assembling a large model from scratch", Attention.forward and the notes below
@@ -175,8 +200,8 @@ def chunk_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start:
     out = np.zeros((B, rows.size, Hq, d))
     lse = np.zeros((B, Hq, rows.size))
     for b in range(B):
-        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged)  # [T, Hkv, d]
-        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged)
+        kp = qk_prologue(k[b], k_norm_w, pos[b], theta, eps, staged, inv_freq, scaling)  # [T, Hkv, d]
+        qp = qk_prologue(q[b, rows], q_norm_w, np.asarray(pos[b])[rows], theta, eps, staged, inv_freq, scaling)
         kc = np.asarray(k_cache[b], dtype=np.float64)[:, :start]     # [Hkv, start, d]
         vc = np.asarray(v_cache[b], dtype=np.float64)[:, :start]
         for h in range(Hq):
@@ -186,21 +211,22 @@ def chunk_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start:
             for r0 in range(0, rows.size, block):
                 rr = rows[r0:r0 + block]
                 top = start + int(rr.max()) + 1
-                o, l = _attend(qp[r0:r0 + block, h], keys[:top], vals[:top], rr + start)
+                o, l = _attend(qp[r0:r0 + block, h], keys[:top], vals[:top], rr + start, window)
                 out[b, r0:r0 + block, h] = o
                 lse[b, h, r0:r0 + block] = l
     return out, lse
 
 
-def build_cache_k(k_hist, k_norm_w, theta: float, eps: float) -> np.ndarray:
+def build_cache_k(k_hist, k_norm_w, theta: float, eps: float, inv_freq=None, scaling: float = 1.0) -> np.ndarray:
     """Cache contents for a raw key history k_hist [L,Hkv,d]: QK-Norm and RoPE at
     positions 0..L-1, rounded to bf16 (the cache's storage type), as float64."""
     L = np.asarray(k_hist).shape[0]
-    return bf16_round(qk_prologue(k_hist, k_norm_w, np.arange(L), theta, eps))
+    return bf16_round(qk_prologue(k_hist, k_norm_w, np.arange(L), theta, eps, inv_freq=inv_freq, scaling=scaling))
 
 
 def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens,
-               theta: float, eps: float, seqs=None, staged: bool = False):
+               theta: float, eps: float, seqs=None, staged: bool = False, window: int = 0, inv_freq=None,
+               scaling: float = 1.0):
     """One decode step over a KV cache, in fp64.
 
     q [N,Hq,d], k_new and v_new [N,Hkv,d] raw; k_cache/v_cache indexable as
@@ -216,9 +242,9 @@ def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens
     outs, lses = [], []
     for n in seqs:
         L = int(cache_lens[n])
-        qp = qk_prologue(q[n][None], q_norm_w, np.array([L]), theta, eps, staged)[0]     # [Hq, d]
+        qp = qk_prologue(q[n][None], q_norm_w, np.array([L]), theta, eps, staged, inv_freq, scaling)[0]  # [Hq, d]
         kn = qk_prologue(np.asarray(k_new[n], dtype=np.float64)[None], k_norm_w, np.array([L]),
-                         theta, eps, staged)[0]                                            # [Hkv, d]
+                         theta, eps, staged, inv_freq, scaling)[0]                                    # [Hkv, d]
         kc = np.asarray(k_cache[n], dtype=np.float64)
         vc = np.asarray(v_cache[n], dtype=np.float64)
         o = np.zeros((Hq, d))
@@ -227,7 +253,7 @@ def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens
             hk = h // G
             keys = np.concatenate([kc[hk, :L], kn[hk][None]], axis=0)
             vals = np.concatenate([vc[hk, :L], np.asarray(v_new[n], dtype=np.float64)[hk][None]], axis=0)
-            oo, ll = _attend(qp[h][None], keys, vals, np.array([L]))
+            oo, ll = _attend(qp[h][None], keys, vals, np.array([L]), window)
             o[h], ls[h] = oo[0], ll[0]
         outs.append(o)
         lses.append(ls)

@@ -13,7 +13,7 @@ from __future__ import annotations
 import math
 
 
-def _norm_rope(vec, gain, pos, theta, eps):
+def _norm_rope(vec, gain, pos, theta, eps, inv_freq=None, scaling=1.0):
     d = len(vec)
     ms = sum(x * x for x in vec) / d
     r = 1.0 / math.sqrt(ms + eps)
@@ -21,37 +21,40 @@ def _norm_rope(vec, gain, pos, theta, eps):
     half = d // 2
     out = [0.0] * d
     for i in range(half):
-        a = pos * theta ** (-2.0 * i / d)
-        c, s = math.cos(a), math.sin(a)
+        a = pos * (theta ** (-2.0 * i / d) if inv_freq is None else float(inv_freq[i]))
+        c, s = math.cos(a) * scaling, math.sin(a) * scaling
         out[i] = y[i] * c - y[i + half] * s
         out[i + half] = y[i + half] * c + y[i] * s
     return out
 
 
-def prefill_loops(q, k, v, gq, gk, pos, theta, eps, S_minus_T=0):
+def prefill_loops(q, k, v, gq, gk, pos, theta, eps, S_minus_T=0, window=0, inv_freq=None, scaling=1.0):
     """q[b][t][h][i], k/v[b][t][hk][i] nested lists (or arrays); returns
-    out[b][t][h][i] and lse[b][h][t] as nested lists."""
+    out[b][t][h][i] and lse[b][h][t] as nested lists.  window > 0: query t sees only keys
+    j with t - window < j <= t; inv_freq / scaling: another rope type's frequencies and
+    the attention_scaling on cos and sin."""
     B, T, Hq, d = len(q), len(q[0]), len(q[0][0]), len(q[0][0][0])
     Hkv = len(k[0][0])
     G = Hq // Hkv
     out = [[[[0.0] * d for _ in range(Hq)] for _ in range(T)] for _ in range(B)]
     lse = [[[0.0] * T for _ in range(Hq)] for _ in range(B)]
     for b in range(B):
-        kk = [[_norm_rope([float(x) for x in k[b][t][h]], gk, float(pos[b][t]), theta, eps)
+        kk = [[_norm_rope([float(x) for x in k[b][t][h]], gk, float(pos[b][t]), theta, eps, inv_freq, scaling)
                for h in range(Hkv)] for t in range(T)]
         for t in range(T):
             for h in range(Hq):
-                qq = _norm_rope([float(x) for x in q[b][t][h]], gq, float(pos[b][t]), theta, eps)
+                qq = _norm_rope([float(x) for x in q[b][t][h]], gq, float(pos[b][t]), theta, eps, inv_freq, scaling)
                 hk = h // G
-                scores = []
+                scores, seen = [], []
                 for j in range(T):
-                    if j <= t + S_minus_T:
+                    if j <= t + S_minus_T and (window == 0 or j > t + S_minus_T - window):
                         scores.append(sum(qq[i] * kk[j][hk][i] for i in range(d)) / math.sqrt(d))
+                        seen.append(j)
                 m = max(scores)
                 w = [math.exp(s - m) for s in scores]
                 z = sum(w)
                 for i in range(d):
-                    out[b][t][h][i] = sum(w[j] * float(v[b][j][hk][i]) for j in range(len(w))) / z
+                    out[b][t][h][i] = sum(w[n] * float(v[b][seen[n]][hk][i]) for n in range(len(w))) / z
                 lse[b][h][t] = m + math.log(z)
     return out, lse
 

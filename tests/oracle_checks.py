@@ -290,6 +290,93 @@ def check_chunk_over_empty_cache_is_prefill():
     assert np.allclose(out, ref_o, rtol=0, atol=1e-14) and np.allclose(lse, ref_l, rtol=0, atol=1e-14)
 
 
+# ---------------------------------------------------------------- variants
+def check_brute_force_variants():
+    """Sliding window, another rope type's frequencies and attention_scaling against the
+    scalar loops."""
+    inv = 1.0 / (1.0 + np.arange(D // 2)) ** 1.3  # any decreasing table of frequencies
+    for (T, Hq, Hkv, seed, window, inv_freq, scaling) in [(9, 4, 2, 80, 3, None, 1.0), (7, 2, 1, 81, 1, inv, 1.0),
+                                                          (8, 4, 1, 82, 0, inv, 1.25), (10, 4, 2, 83, 4, None, 0.8)]:
+        q, k, v, gq, gk, pos = _inputs(1, T, Hq, Hkv, seed=seed)
+        out, lse = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, block=3, window=window, inv_freq=inv_freq,
+                                 scaling=scaling)
+        out_l, lse_l = Lp.prefill_loops(q.tolist(), k.tolist(), v.tolist(), gq.tolist(), gk.tolist(), pos.tolist(),
+                                        THETA, EPS, window=window, inv_freq=inv_freq, scaling=scaling)
+        assert np.allclose(out, np.array(out_l), rtol=0, atol=1e-12)
+        assert np.allclose(lse, np.array(lse_l), rtol=0, atol=1e-12)
+
+
+def check_window_special_cases():
+    """W >= T is full causal attention; W = 1 leaves each query its own key, so out_i is
+    v_i of its KV head and lse_i is s_ii; a window of W over a long prompt gives row i the
+    result of a causal prefill over just tokens i-W+1..i (positions kept)."""
+    q, k, v, gq, gk, pos = _inputs(2, 40, 8, 2, seed=84)
+    full_o, full_l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    o, l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, window=40)
+    assert np.array_equal(o, full_o) and np.array_equal(l, full_l)
+    o1, l1 = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, window=1)
+    G = 4
+    for h in range(8):
+        assert np.allclose(o1[:, :, h], v[:, :, h // G], rtol=0, atol=1e-14)
+    qp = A.qk_prologue(q, gq, pos, THETA, EPS)
+    kp = A.qk_prologue(k, gk, pos, THETA, EPS)
+    for b in range(2):
+        for h in range(8):
+            s = np.sum(qp[b, :, h] * kp[b, :, h // G], axis=-1) / np.sqrt(D)
+            assert np.allclose(l1[b, h], s, rtol=0, atol=1e-12)
+    W = 7
+    ow, lw = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, window=W)
+    for i in (0, 3, 6, 7, 20, 39):
+        lo = max(0, i - W + 1)
+        os_, ls_ = A.prefill_ref(q[:, lo:i + 1], k[:, lo:i + 1], v[:, lo:i + 1], gq, gk, pos[:, lo:i + 1], THETA, EPS)
+        assert np.allclose(ow[:, i], os_[:, -1], rtol=0, atol=1e-13)
+        assert np.allclose(lw[:, :, i], ls_[:, :, -1], rtol=0, atol=1e-13)
+
+
+def check_window_chunk_and_decode_agree_with_prefill():
+    """With a window, a chunk over a cached prefix reproduces the windowed prefill's tail
+    rows, and a decode step reproduces its last row."""
+    start, T, W = 30, 21, 9
+    q, k, v, gq, gk, pos = _inputs(1, start + T, 8, 2, seed=85)
+    full_o, full_l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, window=W)
+    qn, kn, vn, pn, kc, vc = _chunk_split(q, k, v, gk, pos, start)
+    o, l = A.chunk_prefill_ref(qn, kn, vn, gq, gk, pn, kc, vc, start, THETA, EPS, window=W)
+    assert np.allclose(o, full_o[:, start:], rtol=0, atol=1e-13) and np.allclose(l, full_l[:, :, start:], atol=1e-13)
+    L = start + T - 1
+    od, ld = A.decode_ref(q[:, L], k[:, L], v[:, L], gq, gk,
+                          A.qk_prologue(k[:, :L], gk, pos[:, :L], THETA, EPS).transpose(0, 2, 1, 3),
+                          v[:, :L].transpose(0, 2, 1, 3), np.array([L]), THETA, EPS, window=W)
+    assert np.allclose(od[0], full_o[0, L], rtol=0, atol=1e-13) and np.allclose(ld[0], full_l[0, :, L], atol=1e-13)
+
+
+def check_rope_variant_closed_forms():
+    """inv_freq = theta^(-2i/d) is the default; attention_scaling s multiplies the rotated
+    vector by s; a constant table c rotates every pair by pos*c (a plane rotation)."""
+    x = _rand((3, 5, 2, D), 86)
+    pos = np.array([[0, 1, 7, 100, 32768]] * 3)
+    assert np.array_equal(A.rope(x, pos, THETA, inv_freq=A.rope_inv_freq(D, THETA)), A.rope(x, pos, THETA))
+    assert np.allclose(A.rope(x, pos, THETA, scaling=1.7), 1.7 * A.rope(x, pos, THETA), rtol=1e-14, atol=1e-15)
+    c = 0.37
+    y = A.rope(x, pos, THETA, inv_freq=np.full(D // 2, c))
+    ang = pos[..., None, None] * c
+    assert np.allclose(y[..., :64], x[..., :64] * np.cos(ang) - x[..., 64:] * np.sin(ang), rtol=0, atol=1e-12)
+    assert np.allclose(y[..., 64:], x[..., 64:] * np.cos(ang) + x[..., :64] * np.sin(ang), rtol=0, atol=1e-12)
+
+
+def check_attention_scaling_against_torch_sdpa():
+    """attention_scaling s scales q' and k' by s, so the logits scale by s^2: torch fp64
+    SDPA with scale s^2/sqrt(d) on the default q', k' gives the same rows."""
+    q, k, v, gq, gk, pos = _inputs(1, 24, 4, 2, seed=87)
+    sc = 1.3
+    o, _ = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS, scaling=sc)
+    qp = torch.from_numpy(A.qk_prologue(q, gq, pos, THETA, EPS)).permute(0, 2, 1, 3)
+    kp = torch.from_numpy(A.qk_prologue(k, gk, pos, THETA, EPS)).permute(0, 2, 1, 3)
+    vt = torch.from_numpy(v).permute(0, 2, 1, 3)
+    ref = torch.nn.functional.scaled_dot_product_attention(qp, kp, vt, is_causal=True, enable_gqa=True,
+                                                           scale=sc * sc / np.sqrt(D))
+    assert np.allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
+
+
 def check_position_shift_invariance():
     """Shifting every position by a constant leaves outputs unchanged (RoPE is relative)."""
     q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=50)

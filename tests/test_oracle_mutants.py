@@ -1,8 +1,10 @@
 """Plant plausible mistakes in the oracle (on the CPU) and confirm the pins catch
 each one: a wrong RoPE sign, adjacent-pair RoPE, a missing eps, mean-centering,
 h mod Hkv head mapping, an off-by-one causal mask, a missing 1/sqrt(d) scale,
-a base-2 logsumexp, and in the chunked prefill a mask without the cached-prefix
-offset or cached keys rotated a second time."""
+a base-2 logsumexp, in the chunked prefill a mask without the cached-prefix
+offset or cached keys rotated a second time, and in the variants a sliding window
+one key too wide, attention_scaling applied to cos only, and a caller's inv_freq
+ignored."""
 import numpy as np
 import pytest
 
@@ -10,19 +12,23 @@ import oracle.attention as A
 from tests import oracle_checks as C
 
 
-def _rope_wrong_sign(x, pos, theta):
+def _inv(x, theta, inv_freq):
+    return A.rope_inv_freq(x.shape[-1], theta) if inv_freq is None else np.asarray(inv_freq, dtype=np.float64)
+
+
+def _rope_wrong_sign(x, pos, theta, inv_freq=None, scaling=1.0):
     x = np.asarray(x, dtype=np.float64)
     half = x.shape[-1] // 2
-    ang = np.asarray(pos, dtype=np.float64)[..., None] * A.rope_inv_freq(x.shape[-1], theta)
-    c, s = np.cos(ang)[..., None, :], np.sin(ang)[..., None, :]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * _inv(x, theta, inv_freq)
+    c, s = scaling * np.cos(ang)[..., None, :], scaling * np.sin(ang)[..., None, :]
     x1, x2 = x[..., :half], x[..., half:]
     return np.concatenate([x1 * c + x2 * s, x2 * c - x1 * s], axis=-1)
 
 
-def _rope_adjacent_pairs(x, pos, theta):
+def _rope_adjacent_pairs(x, pos, theta, inv_freq=None, scaling=1.0):
     x = np.asarray(x, dtype=np.float64)
-    ang = np.asarray(pos, dtype=np.float64)[..., None] * A.rope_inv_freq(x.shape[-1], theta)
-    c, s = np.cos(ang)[..., None, :], np.sin(ang)[..., None, :]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * _inv(x, theta, inv_freq)
+    c, s = scaling * np.cos(ang)[..., None, :], scaling * np.sin(ang)[..., None, :]
     xe, xo = x[..., 0::2], x[..., 1::2]
     y = np.empty_like(x)
     y[..., 0::2] = xe * c - xo * s
@@ -41,23 +47,42 @@ def _norm_centered(x, g, eps):
     return g * x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
 
 
-def _attend_off_by_one(qg, kk, vv, limit):
-    return _ORIG_ATTEND(qg, kk, vv, limit - 1 + (limit == 0))
+def _attend_off_by_one(qg, kk, vv, limit, window=0):
+    return _ORIG_ATTEND(qg, kk, vv, limit - 1 + (limit == 0), window)
 
 
-def _attend_no_scale(qg, kk, vv, limit):
-    return _ORIG_ATTEND(qg * np.sqrt(qg.shape[-1]), kk, vv, limit)
+def _attend_no_scale(qg, kk, vv, limit, window=0):
+    return _ORIG_ATTEND(qg * np.sqrt(qg.shape[-1]), kk, vv, limit, window)
 
 
-def _attend_log2(qg, kk, vv, limit):
-    o, l = _ORIG_ATTEND(qg, kk, vv, limit)
+def _attend_log2(qg, kk, vv, limit, window=0):
+    o, l = _ORIG_ATTEND(qg, kk, vv, limit, window)
     return o, l / np.log(2.0)
 
 
+def _attend_window_one_wider(qg, kk, vv, limit, window=0):
+    # the window lets in one key too many (i - W <= j instead of i - W < j)
+    return _ORIG_ATTEND(qg, kk, vv, limit, window + 1 if window > 0 else 0)
+
+
+def _rope_scaling_on_cos_only(x, pos, theta, inv_freq=None, scaling=1.0):
+    x = np.asarray(x, dtype=np.float64)
+    half = x.shape[-1] // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * _inv(x, theta, inv_freq)
+    c, s = scaling * np.cos(ang)[..., None, :], np.sin(ang)[..., None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def _rope_ignores_inv_freq(x, pos, theta, inv_freq=None, scaling=1.0):
+    return _ORIG_ROPE(x, pos, theta, None, scaling)
+
+
 _ORIG_ATTEND = A._attend
+_ORIG_ROPE = A.rope
 
 
-def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=False, block=256):
+def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=False, block=256, **kw):
     # h -> h % Hkv instead of h // G: permute the query heads so the oracle's
     # h // G lookup lands on h % Hkv, then undo the permutation on the output.
     q = np.asarray(q, dtype=np.float64)
@@ -66,14 +91,15 @@ def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=Fal
     perm = np.array([(h % Hkv) * G + h // Hkv for h in range(Hq)])
     qq = np.empty_like(q)
     qq[:, :, perm] = q
-    o, l = _ORIG_PREFILL(qq, k, v, gq, gk, pos, theta, eps, rows=rows, staged=staged, block=block)
+    o, l = _ORIG_PREFILL(qq, k, v, gq, gk, pos, theta, eps, rows=rows, staged=staged, block=block, **kw)
     return o[:, :, perm], l[:, perm]
 
 
 _ORIG_CHUNK = A.chunk_prefill_ref
 
 
-def _chunk_no_offset(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps, rows=None, staged=False, block=256):
+def _chunk_no_offset(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps, rows=None, staged=False, block=256,
+                     window=0, inv_freq=None, scaling=1.0):
     # the mask forgets the cached prefix: new row i sees keys 0..i of the concatenation
     q, k, v = (np.asarray(a, dtype=np.float64) for a in (q, k, v))
     B, T, Hq, d = q.shape
@@ -81,12 +107,12 @@ def _chunk_no_offset(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, eps, 
     rows = np.arange(T) if rows is None else np.asarray(rows)
     out, lse = np.zeros((B, rows.size, Hq, d)), np.zeros((B, Hq, rows.size))
     for b in range(B):
-        kp = A.qk_prologue(k[b], gk, pos[b], theta, eps, staged)
-        qp = A.qk_prologue(q[b, rows], gq, np.asarray(pos[b])[rows], theta, eps, staged)
+        kp = A.qk_prologue(k[b], gk, pos[b], theta, eps, staged, inv_freq, scaling)
+        qp = A.qk_prologue(q[b, rows], gq, np.asarray(pos[b])[rows], theta, eps, staged, inv_freq, scaling)
         for h in range(Hq):
             keys = np.concatenate([np.asarray(k_cache[b])[h // G, :start], kp[:, h // G]])
             vals = np.concatenate([np.asarray(v_cache[b])[h // G, :start], v[b, :, h // G]])
-            o, l = A._attend(qp[:, h], keys, vals, rows)
+            o, l = A._attend(qp[:, h], keys, vals, rows, window)
             out[b, :, h], lse[b, h] = o, l
     return out, lse
 
@@ -108,6 +134,9 @@ MUTANTS = [
     ("_attend", _attend_off_by_one),
     ("_attend", _attend_no_scale),
     ("_attend", _attend_log2),
+    ("_attend", _attend_window_one_wider),
+    ("rope", _rope_scaling_on_cos_only),
+    ("rope", _rope_ignores_inv_freq),
     ("prefill_ref", _prefill_mod_mapping),
     ("chunk_prefill_ref", _chunk_no_offset),
     ("chunk_prefill_ref", _chunk_rerotates_cache),
