@@ -53,6 +53,30 @@ typedef enum {
 } qwen3_status;
 
 /*
+ * qwen3_attn_variant - the variants of the core that a Qwen3 configuration can select.
+ * "Qwen3 Architecture Layer-by-Layer", Per-layer attention type: a layer is full or
+ * sliding-window attention.  Qwen3RotaryEmbedding: the rope type fixes inv_freq (its
+ * initialisation function) and an attention_scaling that multiplies cos and sin.  "Qwen 3
+ * From Scratch": long context through rotary scaling (YaRN) in the config.
+ *   theta              RoPE base: inv_i = theta^(-2i/d), used when inv_freq is NULL (> 0).
+ *   inv_freq           optional HOST array of d/2 rotary frequencies, e.g. a YaRN or linear
+ *                      scaling initialisation computed by the caller; it replaces theta.
+ *                      Read during the call only.  Entries must be finite.
+ *   attention_scaling  multiplies cos and sin, so q' and k' (and the keys the call writes to
+ *                      a cache); 1 for the default rope type.  Finite, > 0.
+ *   window             sliding window W >= 1: query at key index i sees keys i-W < j <= i,
+ *                      its own key included; 0 = full causal attention.
+ * An invalid variant returns QWEN3_ERR_INVALID_ARG.  The plain entry points are the
+ * variant {theta, NULL, 1, 0}.
+ */
+typedef struct qwen3_attn_variant {
+  float theta;
+  const double* inv_freq;
+  float attention_scaling;
+  int window;
+} qwen3_attn_variant;
+
+/*
  * qwen3_qk_norm_rope - QK-Norm then RoPE of raw head vectors, written in cache layout.
  * Defined by steps 1-2 above ("Hand-Writing ... Part 1": q_norm/k_norm run right after the
  * projection and before RoPE).
@@ -71,6 +95,13 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos,
                        qwen3_bf16* dst, const qwen3_bf16* v_src, qwen3_bf16* v_dst,
                        int B, int T, int H, int d, int Tcap, int write_at_pos,
                        float theta, float eps, qwen3_stream_t stream);
+
+/* qwen3_qk_norm_rope with a rope variant (inv_freq, attention_scaling; window unused). */
+int qwen3_qk_norm_rope_variant(const qwen3_bf16* x, const float* w, const int32_t* pos,
+                               qwen3_bf16* dst, const qwen3_bf16* v_src, qwen3_bf16* v_dst,
+                               int B, int T, int H, int d, int Tcap, int write_at_pos,
+                               const qwen3_attn_variant* variant, float eps,
+                               qwen3_stream_t stream);
 
 /*
  * qwen3_attn_prefill - causal GQA self-attention over T new tokens with the QK-Norm+RoPE
@@ -198,6 +229,33 @@ int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
                               qwen3_bf16* out, float* lse,
                               int N, int Hq, int Hkv, int d, int Lmax,
                               float theta, float eps, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_prefill_variant - the general prefill: qwen3_attn_prefill_ex (k_cache,
+ * v_cache NULL and start 0) or qwen3_attn_prefill_chunk (caches given, `start` cached
+ * tokens), with a qwen3_attn_variant in place of theta.  A sliding window keeps the last
+ * `window` keys of each query; the key tiles wholly before every row's window are not read.
+ */
+int qwen3_attn_prefill_variant(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                               const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                               qwen3_bf16* out, float* lse,
+                               qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap,
+                               void* workspace, size_t ws_bytes,
+                               int B, int T, int Hq, int Hkv, int d,
+                               const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_decode_variant - qwen3_attn_decode with a qwen3_attn_variant in place of theta.
+ * With a window the new token at position L attends to keys max(0, L-window+1)..L; the
+ * splits wholly before the window are not read.
+ */
+int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                              const float* q_norm_w, const float* k_norm_w,
+                              qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                              qwen3_bf16* out, float* lse,
+                              int N, int Hq, int Hkv, int d, int Lmax,
+                              const qwen3_attn_variant* variant, float eps,
+                              void* workspace, size_t ws_bytes, qwen3_stream_t stream);
 
 /* Scratch bytes qwen3_attn_prefill_ex and qwen3_attn_prefill_chunk need: B*T*Hkv*d*2
  * (normed, rotated keys) + B*T*Hq*d*2 (normed, rotated queries), plus alignment slack;

@@ -20,8 +20,16 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_WORKSPAC
 
 HEAD_DIM = 128
 
+class Variant(ctypes.Structure):
+    """qwen3_attn_variant: RoPE base, an optional host table of d/2 rotary frequencies,
+    the attention_scaling on cos/sin, and the sliding window (0 = full causal)."""
+    _fields_ = [("theta", ctypes.c_float), ("inv_freq", ctypes.POINTER(ctypes.c_double)),
+                ("attention_scaling", ctypes.c_float), ("window", ctypes.c_int)]
+
+
 # Every symbol include/qwen3_attn.h declares: (name, restype, argtypes)
 _P, _I, _F, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
+_V = ctypes.POINTER(Variant)
 SIGNATURES = {
     "qwen3_qk_norm_rope": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_prefill": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
@@ -31,6 +39,11 @@ SIGNATURES = {
                                       _I, _I, _I, _I, _I, _F, _F, _P]),
     "qwen3_attn_decode": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P, _Z, _P]),
     "qwen3_attn_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _F, _P]),
+    "qwen3_qk_norm_rope_variant": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _V, _F, _P]),
+    "qwen3_attn_prefill_variant": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _Z,
+                                        _I, _I, _I, _I, _I, _V, _F, _P]),
+    "qwen3_attn_decode_variant": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _V, _F, _P, _Z,
+                                       _P]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
@@ -64,6 +77,21 @@ class Qwen3AttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+def make_variant(theta: float = 1.0e6, inv_freq=None, attention_scaling: float = 1.0, window: int = 0):
+    """A Variant plus the ctypes buffer its inv_freq points into (keep both alive for the call)."""
+    buf = None
+    if inv_freq is not None:
+        vals = [float(x) for x in inv_freq]
+        buf = (ctypes.c_double * len(vals))(*vals)
+    v = Variant(theta, ctypes.cast(buf, ctypes.POINTER(ctypes.c_double)) if buf is not None else None,
+                attention_scaling, int(window))
+    return v, buf
+
+
+def _is_default(inv_freq, attention_scaling, window) -> bool:
+    return inv_freq is None and attention_scaling == 1.0 and window == 0
 
 
 def status_string(status: int) -> str:
@@ -109,9 +137,11 @@ def kv_cache_bytes(N: int, Hkv: int, Lmax: int, d: int = HEAD_DIM) -> int:
 
 
 def qk_norm_rope(x, w, pos, dst, v_src=None, v_dst=None, *, write_at_pos: bool = False,
-                 theta: float = 1.0e6, eps: float = 1.0e-6) -> torch.Tensor:
+                 theta: float = 1.0e6, eps: float = 1.0e-6, inv_freq=None,
+                 attention_scaling: float = 1.0) -> torch.Tensor:
     """QK-Norm + RoPE of x [B,T,H,d] into dst [B,H,Tcap,d] (row t, or row pos[b,t] when
-    write_at_pos); optionally copies v_src [B,T,H,d] to v_dst at the same slots."""
+    write_at_pos); optionally copies v_src [B,T,H,d] to v_dst at the same slots.  inv_freq
+    (d/2 values) and attention_scaling select another rope type."""
     dev = x.device
     B, T, H, d = x.shape
     Tcap = dst.shape[2]
@@ -122,14 +152,22 @@ def qk_norm_rope(x, w, pos, dst, v_src=None, v_dst=None, *, write_at_pos: bool =
     if v_src is not None:
         _need(v_src, "v_src", torch.bfloat16, (B, T, H, d), dev)
         _need(v_dst, "v_dst", torch.bfloat16, (B, H, Tcap, d), dev)
-    _check(lib().qwen3_qk_norm_rope(_ptr(x), _ptr(w), _ptr(pos), _ptr(dst), _ptr(v_src), _ptr(v_dst),
-                                    B, T, H, d, Tcap, int(write_at_pos), theta, eps, _stream(dev)),
-           "qwen3_qk_norm_rope")
+    if _is_default(inv_freq, attention_scaling, 0):
+        _check(lib().qwen3_qk_norm_rope(_ptr(x), _ptr(w), _ptr(pos), _ptr(dst), _ptr(v_src), _ptr(v_dst),
+                                        B, T, H, d, Tcap, int(write_at_pos), theta, eps, _stream(dev)),
+               "qwen3_qk_norm_rope")
+    else:
+        var, _keep = make_variant(theta, inv_freq, attention_scaling, 0)
+        _check(lib().qwen3_qk_norm_rope_variant(_ptr(x), _ptr(w), _ptr(pos), _ptr(dst), _ptr(v_src), _ptr(v_dst),
+                                                B, T, H, d, Tcap, int(write_at_pos), ctypes.byref(var), eps,
+                                                _stream(dev)),
+               "qwen3_qk_norm_rope_variant")
     return dst
 
 
 def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: float = 1.0e-6,
-            out=None, lse=None, k_cache=None, v_cache=None, workspace=None):
+            out=None, lse=None, k_cache=None, v_cache=None, workspace=None, window: int = 0, inv_freq=None,
+            attention_scaling: float = 1.0):
     """Causal GQA prefill with the QK-Norm+RoPE prologue.  q [B,T,Hq,d], k/v [B,T,Hkv,d] bf16,
     gains [d] fp32, pos [B,T] int32.  Returns out [B,T,Hq,d] bf16 (and writes lse [B,Hq,T]
     fp32 and the caches [B,Hkv,Tcap,d] when given)."""
@@ -155,15 +193,24 @@ def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: floa
     if workspace is None:
         workspace = torch.empty(prefill_workspace_size(B, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().qwen3_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
-                                       _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
-                                       _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
-           "qwen3_attn_prefill_ex")
+    if _is_default(inv_freq, attention_scaling, window):
+        _check(lib().qwen3_attn_prefill_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                           _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), Tcap,
+                                           _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
+               "qwen3_attn_prefill_ex")
+    else:
+        var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+        _check(lib().qwen3_attn_prefill_variant(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w),
+                                                _ptr(pos), _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), 0,
+                                                Tcap, _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d,
+                                                ctypes.byref(var), eps, _stream(dev)),
+               "qwen3_attn_prefill_variant")
     return out
 
 
 def prefill_chunk(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int, *, theta: float = 1.0e6,
-                  eps: float = 1.0e-6, out=None, lse=None, workspace=None):
+                  eps: float = 1.0e-6, out=None, lse=None, workspace=None, window: int = 0, inv_freq=None,
+                  attention_scaling: float = 1.0):
     """Chunked prefill: T new tokens per batch row over caches [B,Hkv,Tcap,d] that already
     hold `start` tokens.  The new keys (normed, rotated) and values are written to slots
     start..start+T-1, and new token i attends to keys 0..start+i.  Returns out [B,T,Hq,d]."""
@@ -187,10 +234,19 @@ def prefill_chunk(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int
     if workspace is None:
         workspace = torch.empty(prefill_workspace_size(B, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().qwen3_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
-                                          _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache), int(start), Tcap,
-                                          _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta, eps, _stream(dev)),
-           "qwen3_attn_prefill_chunk")
+    if _is_default(inv_freq, attention_scaling, window):
+        _check(lib().qwen3_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w),
+                                              _ptr(pos), _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache),
+                                              int(start), Tcap, _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d, theta,
+                                              eps, _stream(dev)),
+               "qwen3_attn_prefill_chunk")
+    else:
+        var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+        _check(lib().qwen3_attn_prefill_variant(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w),
+                                                _ptr(pos), _ptr(out), _ptr(lse), _ptr(k_cache), _ptr(v_cache),
+                                                int(start), Tcap, _ptr(workspace), ws_bytes, B, T, Hq, Hkv, d,
+                                                ctypes.byref(var), eps, _stream(dev)),
+               "qwen3_attn_prefill_variant")
     return out
 
 
@@ -209,7 +265,8 @@ def prefill_simple(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, ep
 
 
 def decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *, theta: float = 1.0e6,
-           eps: float = 1.0e-6, out=None, lse=None, workspace=None):
+           eps: float = 1.0e-6, out=None, lse=None, workspace=None, window: int = 0, inv_freq=None,
+           attention_scaling: float = 1.0):
     """One decode step.  q [N,Hq,d], k_new/v_new [N,Hkv,d] bf16 raw; caches [N,Hkv,Lmax,d]
     bf16 (slot L = cache_lens[n] is written); cache_lens [N] int32 (not advanced).
     Returns out [N,Hq,d] bf16."""
@@ -233,10 +290,18 @@ def decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *,
     if workspace is None:
         workspace = torch.empty(decode_workspace_size(N, Hq, Lmax, d), dtype=torch.uint8, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
-    _check(lib().qwen3_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
-                                   _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
-                                   N, Hq, Hkv, d, Lmax, theta, eps, _ptr(workspace), ws_bytes, _stream(dev)),
-           "qwen3_attn_decode")
+    if _is_default(inv_freq, attention_scaling, window):
+        _check(lib().qwen3_attn_decode(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
+                                       _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
+                                       N, Hq, Hkv, d, Lmax, theta, eps, _ptr(workspace), ws_bytes, _stream(dev)),
+               "qwen3_attn_decode")
+    else:
+        var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+        _check(lib().qwen3_attn_decode_variant(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
+                                               _ptr(k_cache), _ptr(v_cache), _ptr(cache_lens), _ptr(out), _ptr(lse),
+                                               N, Hq, Hkv, d, Lmax, ctypes.byref(var), eps, _ptr(workspace),
+                                               ws_bytes, _stream(dev)),
+               "qwen3_attn_decode_variant")
     return out
 
 

@@ -30,7 +30,9 @@ struct DecodeParams {
   float* part_o;          // [N, Hq, n_split_max, d]
   float* part_lse;        // [N, Hq, n_split_max]
   int N, Hq, Hkv, log2G, Lmax, split, n_split_max;
+  int window;        // sliding window W: the query sees keys L-W < j <= L; 0 = all
   float eps, scale_log2;
+  float rope_scale;  // attention_scaling on cos and sin
   WaitCfg wait;
   RopeTable rope;
 };
@@ -80,7 +82,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int tok0 = s_idx * p.split;
   const int ntok = min(p.split, L + 1 - tok0);  // keys of this split (slot L = new token)
   if (ntok <= 0) return;
+  const int wlo = p.window > 0 ? max(0, L - p.window + 1) : 0;  // first visible key
+  if (tok0 + ntok <= wlo) return;  // the whole split lies before the window
   const int nchunk = (ntok + 63) >> 6;
+  const int cbeg = max(0, wlo - tok0) >> 6;  // chunks wholly before the window are skipped
   const int G = 1 << p.log2G;
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -109,10 +114,11 @@ __global__ void __launch_bounds__(kDecodeThreads)
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
       int last[kDcStages] = {-1, -1, -1};
-      for (int c = 0; c < nchunk; ++c) {
-        const int st = c % kDcStages;
-        const uint32_t ph = (c / kDcStages) & 1;
-        if (c >= kDcStages && !mbar_wait(bar + kDcBEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSiteDecodeEmpty))
+      for (int c = cbeg; c < nchunk; ++c) {
+        const int u = c - cbeg;  // ring use
+        const int st = u % kDcStages;
+        const uint32_t ph = (u / kDcStages) & 1;
+        if (u >= kDcStages && !mbar_wait(bar + kDcBEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSiteDecodeEmpty))
           break;
         const uint32_t dst = sb + st * kDcStage;
         const uint32_t fb = bar + kDcBFull + 8 * st;
@@ -122,7 +128,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
         tma_load_2d(dst + kDcBox, &tmK, fb, 64, r);
         tma_load_2d(dst + kDcChunk, &tmV, fb, 0, r);
         tma_load_2d(dst + kDcChunk + kDcBox, &tmV, fb, 64, r);
-        last[st] = c;
+        last[st] = u;
       }
       for (int s = 0; s < kDcStages; ++s)
         if (last[s] >= 0)
@@ -138,6 +144,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
     float s0, c0, s1, c1;
     rope_sincos(L, p.rope.hi[2 * lane], p.rope.lo[2 * lane], s0, c0);
     rope_sincos(L, p.rope.hi[2 * lane + 1], p.rope.lo[2 * lane + 1], s1, c1);
+    s0 *= p.rope_scale;
+    c0 *= p.rope_scale;
+    s1 *= p.rope_scale;
+    c1 *= p.rope_scale;
     for (int g = warp; g < 16; g += 4) {
       uint32_t wa = 0u, wb = 0u;
       if (g < G) {
@@ -176,14 +186,15 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const float sl2 = p.scale_log2;
   const int tw = warp * 16;  // this warp's keys inside every chunk
   bool ok = true;
-  for (int c = 0; c < nchunk; ++c) {
-    const int st = c % kDcStages;
-    ok = mbar_wait(bar + kDcBFull + 8 * st, (c / kDcStages) & 1, p.wait, abort_flag, kSiteDecodeFull);
+  for (int c = cbeg; c < nchunk; ++c) {
+    const int st = (c - cbeg) % kDcStages;
+    ok = mbar_wait(bar + kDcBFull + 8 * st, ((c - cbeg) / kDcStages) & 1, p.wait, abort_flag, kSiteDecodeFull);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     const uint32_t sKc = sb + st * kDcStage, sVc = sKc + kDcChunk;
-    const int valid = ntok - c * 64 - tw;  // keys of this warp's 16 that exist
-    if (valid > 0) {
+    const int valid = ntok - c * 64 - tw;          // keys of this warp's 16 that exist
+    const int below = wlo - (tok0 + c * 64 + tw);  // keys of this warp's 16 before the window
+    if (valid > 0 && below < 16) {
       if (valid < 16) {
         // Slots past the sequence hold stale cache contents: zero their V rows so that
         // P = 0 never meets a non-finite value in P.V.
@@ -215,6 +226,12 @@ __global__ void __launch_bounds__(kDecodeThreads)
         if (kc + 1 >= valid) x[1] = x[3] = -INFINITY;
         if (8 + kc >= valid) x[4] = x[6] = -INFINITY;
         if (9 + kc >= valid) x[5] = x[7] = -INFINITY;
+      }
+      if (below > 0) {  // keys before the window (at least one of the 16 is inside it)
+        if (kc < below) x[0] = x[2] = -INFINITY;
+        if (kc + 1 < below) x[1] = x[3] = -INFINITY;
+        if (8 + kc < below) x[4] = x[6] = -INFINITY;
+        if (9 + kc < below) x[5] = x[7] = -INFINITY;
       }
       float mx0 = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[4], x[5]));
       float mx1 = fmaxf(fmaxf(x[2], x[3]), fmaxf(x[6], x[7]));
@@ -307,6 +324,7 @@ struct CombineParams {
   uint4* out;  // [N, Hq, d] bf16
   float* lse;  // [N, Hq] or nullptr
   int Hq, Lmax, split, n_split_max;
+  int window;  // as in DecodeParams: splits wholly before the window wrote nothing
 };
 
 // One CTA of 128 threads per (sequence, query head); thread i owns output dim i.
@@ -316,13 +334,14 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   const int L = p.cache_lens[n];
   if (L < 0 || L >= p.Lmax) return;
   const int ns = L / p.split + 1;  // splits covering keys 0..L
+  const int s0 = p.window > 0 ? max(0, L - p.window + 1) / p.split : 0;  // the first one in the window
   const float* lse_s = p.part_lse + static_cast<long long>(hq) * p.n_split_max;
   float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
+  for (int s = s0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
   const float kLog2e = 1.44269504088896341f;
   float z = 0.f, acc = 0.f;
   const float* po = p.part_o + static_cast<long long>(hq) * p.n_split_max * kD + threadIdx.x;
-  for (int s = 0; s < ns; ++s) {
+  for (int s = s0; s < ns; ++s) {
     const float w = ex2d((lse_s[s] - M) * kLog2e);
     z += w;
     acc += w * po[s * kD];

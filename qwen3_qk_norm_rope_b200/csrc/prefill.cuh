@@ -46,8 +46,10 @@ struct PrefillParams {
   const float* k_norm_w;
   float* lse;      // [B, Hq, T] or nullptr
   int B, T, Hq, Hkv, log2G, P, n_qt, n_pairs, n_items;
-  int start;  // cached keys before the first query row: query t is key index start + t
+  int start;   // cached keys before the first query row: query t is key index start + t
+  int window;  // sliding window W: query key index i sees keys i-W < j <= i; 0 = all
   float eps, scale_log2;
+  float rope_scale;  // attention_scaling that scaled q' and k' (enters the logit bound squared)
   WaitCfg wait;
   int fault;
 };
@@ -92,13 +94,19 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 }
 
 struct TileInfo {
-  int t0, nkv;  // first query row; key tiles it reads (0 = the tile lies past T)
+  int t0, nkv;  // first query row; key tiles it reads from the item's first (0 = past T)
 };
 
-__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt) {
+// First key tile of a pair item: 0, or with a sliding window the tile holding the first key
+// that tile A's first row may see (tile B's rows start later, so they mask one tile at most).
+__device__ __forceinline__ int item_lo(const PrefillParams& p, int pair) {
+  return p.window > 0 ? max(0, p.start + 2 * pair * p.P - p.window + 1) >> 7 : 0;
+}
+
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt, int lo) {
   TileInfo ti;
   ti.t0 = qt * p.P;
-  ti.nkv = (ti.t0 < p.T) ? (p.start + min(ti.t0 + p.P, p.T) - 1) / 128 + 1 : 0;
+  ti.nkv = (ti.t0 < p.T) ? (p.start + min(ti.t0 + p.P, p.T) - 1) / 128 + 1 - lo : 0;
   return ti;
 }
 
@@ -171,7 +179,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
-        const int nX[2] = {tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv};
+        const int lo = item_lo(p, pair);
+        const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X) {
           if (nX[X] == 0) continue;
@@ -196,8 +205,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           if (!(p.fault != 0 && it == 0)) {
             mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
-            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, j * 128, hkv, b);
-            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, j * 128, hkv, b);
+            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, (lo + j) * 128, hkv, b);
+            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, (lo + j) * 128, hkv, b);
             k_last[st] = static_cast<int>(it);
           }
           if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
@@ -205,8 +214,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
-          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, j * 128, hkv, b);
-          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, j * 128, hkv, b);
+          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, (lo + j) * 128, hkv, b);
+          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, (lo + j) * 128, hkv, b);
           v_last[st] = static_cast<int>(it);
         }
       }
@@ -227,7 +236,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
-        const int nX[2] = {tile_info(p, 2 * pair).nkv, tile_info(p, 2 * pair + 1).nkv};
+        const int lo = item_lo(p, pair);
+        const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X)
           if (nX[X] > 0) {
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       asm volatile("bar.sync %0, 128;" ::"r"(1 + X) : "memory");
       gq = fmaxf(fmaxf(red[0], red[2]), fmaxf(red[4], red[6]));
       gk = fmaxf(fmaxf(red[1], red[3]), fmaxf(red[5], red[7]));
-      bnd = gq * gk * (11.3137085f * (1.0f + 0.0078125f) * 1.44269504f);
+      bnd = gq * gk * p.rope_scale * p.rope_scale * (11.3137085f * (1.0f + 0.0078125f) * 1.44269504f);
     }
     const bool fast = bnd <= 60.0f;
     uint32_t s_cnt = 0, o_cnt = 0;
@@ -337,12 +347,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
       int pair, b, hkv;
       item_coords(p, item, pair, b, hkv);
-      const TileInfo ti = tile_info(p, 2 * pair + X);
+      const int lo = item_lo(p, pair);
+      const TileInfo ti = tile_info(p, 2 * pair + X, lo);
       if (ti.nkv == 0) continue;  // this item has no tile X
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
       const int lim = p.start + min(t_row, p.T - 1);  // last key index this row may see
+      const int wfirst = p.window > 0 ? lim - p.window + 1 : 0;  // first one, with a window
       float m = fast ? bnd : -INFINITY, l = 0.f;
       for (int j = 0; j < ti.nkv; ++j) {
         ok = mbar_wait(bar + kBSFull + 8 * X, s_cnt & 1, p.wait, abort_flag, kSitePrefillSFull);
@@ -350,8 +362,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int kv0 = j * 128;
-        const bool diag = kv0 + 127 > p.start + t0;  // some key of this tile lies past some row's limit
+        const int kv0 = (lo + j) * 128;
+        // some key of this tile lies past some row's limit, or before some row's window
+        const bool diag = kv0 + 127 > p.start + t0 || (p.window > 0 && kv0 < p.start + t0 + p.P - p.window);
         if (fast) {
           // One pass in four 32-column chunks, the next chunk's TMEM load in flight while the
           // current one is processed.  bf16 P goes to S columns [0,64): chunk c of P
@@ -366,7 +379,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             if (c < 3) tmem_ld32_nowait(tS + 32 * (c + 1), nxt);
             if (diag) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) cur[i] = (kv0 + 32 * c + i <= lim) ? cur[i] : 0xff800000u;  // -inf
+              for (int i = 0; i < 32; ++i) {
+                const int key = kv0 + 32 * c + i;
+                cur[i] = (key <= lim && key >= wfirst) ? cur[i] : 0xff800000u;  // -inf
+              }
             }
             uint32_t pk[16];
 #pragma unroll
@@ -403,7 +419,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_ld64(tS + 64 * hh, sr);
           if (diag) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) sr[c] = (kv0 + 64 * hh + c <= lim) ? sr[c] : 0xff800000u;  // -inf
+            for (int c = 0; c < 64; ++c) {
+              const int key = kv0 + 64 * hh + c;
+              sr[c] = (key <= lim && key >= wfirst) ? sr[c] : 0xff800000u;  // -inf
+            }
           }
 #pragma unroll
           for (int c = 0; c < 64; c += 2)
@@ -419,7 +438,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // Pass 2: p = 2^(s*scale*log2(e) - m) on pairs; bf16 pairs go straight to P's TMEM
         // columns.  P occupies S columns [0,64): chunk c of P (columns [16c,16c+16)) only
         // overwrites S columns that chunks 0..c have already read.
-        const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(-m_new, -m_new);
+        // a row whose keys so far all lie outside its window has no max yet: p = 0 for it
+        const float mref = m_new == -INFINITY ? 0.0f : m_new;
+        const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(-mref, -mref);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -427,7 +448,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           tmem_ld32(tS + 32 * c, sr);
           if (diag) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sr[i] = (kv0 + 32 * c + i <= lim) ? sr[i] : 0xff800000u;
+            for (int i = 0; i < 32; ++i) {
+              const int key = kv0 + 32 * c + i;
+              sr[i] = (key <= lim && key >= wfirst) ? sr[i] : 0xff800000u;
+            }
           }
           uint32_t pk[16];
 #pragma unroll

@@ -28,6 +28,7 @@ struct PrologueParams {
   int B, T, H, Tcap, write_at_pos;
   int Hq, log2G;
   float eps;
+  float rope_scale;  // attention_scaling: multiplies cos and sin (1 for the default rope type)
   RopeTable rope;
 };
 
@@ -65,6 +66,10 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     float s0, c0, s1, c1;
     rope_sincos(ps, hi0, lo0, s0, c0);
     rope_sincos(ps, hi1, lo1, s1, c1);
+    s0 *= p.rope_scale;
+    c0 *= p.rope_scale;
+    s1 *= p.rope_scale;
+    c1 *= p.rope_scale;
     for (int h0 = 0; h0 < p.H; h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
       uint2 vv[kPrologueHeads];

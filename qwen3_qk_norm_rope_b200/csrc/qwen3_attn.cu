@@ -48,15 +48,47 @@ int ilog2(int x) {
   return r;
 }
 
-// inv_i = theta^(-2i/d) in double, split into a float and the float of its remainder.
-q3::RopeTable make_rope_table(float theta) {
+// Rotary frequencies in double (inv_i = theta^(-2i/d), or a caller's table), each split
+// into a float and the float of its remainder.
+q3::RopeTable make_rope_table(float theta, const double* inv_freq = nullptr) {
   q3::RopeTable t;
   for (int i = 0; i < q3::kHalf; ++i) {
-    const double inv = std::pow(static_cast<double>(theta), -2.0 * i / kD);
+    const double inv = inv_freq != nullptr ? inv_freq[i] : std::pow(static_cast<double>(theta), -2.0 * i / kD);
     t.hi[i] = static_cast<float>(inv);
     t.lo[i] = static_cast<float>(inv - static_cast<double>(t.hi[i]));
   }
   return t;
+}
+
+// A checked qwen3_attn_variant: the rotary table, the scale on cos/sin, the window.
+struct Variant {
+  q3::RopeTable rope;
+  float scale = 1.0f;
+  int window = 0;
+};
+
+int make_variant(const qwen3_attn_variant* v, Variant& out) {
+  if (v == nullptr) return QWEN3_ERR_INVALID_ARG;
+  if (v->inv_freq == nullptr && !(v->theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (!(v->attention_scaling > 0.f) || !std::isfinite(v->attention_scaling)) return QWEN3_ERR_INVALID_ARG;
+  if (v->window < 0) return QWEN3_ERR_INVALID_ARG;
+  if (v->inv_freq != nullptr)
+    for (int i = 0; i < q3::kHalf; ++i)
+      if (!std::isfinite(v->inv_freq[i]) || std::fabs(v->inv_freq[i]) >= 1e30) return QWEN3_ERR_INVALID_ARG;
+  out.rope = make_rope_table(v->theta, v->inv_freq);
+  out.scale = v->attention_scaling;
+  out.window = v->window;
+  return QWEN3_OK;
+}
+
+// The default rope type with base theta, full causal attention.
+int theta_variant(float theta, Variant& out) {
+  qwen3_attn_variant v;
+  v.theta = theta;
+  v.inv_freq = nullptr;
+  v.attention_scaling = 1.0f;
+  v.window = 0;
+  return make_variant(&v, out);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -139,8 +171,8 @@ struct PrologueQ {
 };
 
 int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
-                    int B, int T, int H, int Tcap, int write_at_pos, float theta, float eps, cudaStream_t stream,
-                    const PrologueQ& q = PrologueQ()) {
+                    int B, int T, int H, int Tcap, int write_at_pos, const Variant& var, float eps,
+                    cudaStream_t stream, const PrologueQ& q = PrologueQ()) {
   q3::PrologueParams p;
   p.x = static_cast<const uint32_t*>(x);
   p.w = w;
@@ -159,7 +191,8 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.Tcap = Tcap;
   p.write_at_pos = write_at_pos;
   p.eps = eps;
-  p.rope = make_rope_table(theta);
+  p.rope_scale = var.scale;
+  p.rope = var.rope;
   const long long ntok = static_cast<long long>(B) * T;
   if (ntok > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   const int warps = 8;
@@ -230,9 +263,13 @@ size_t qwen3_attn_kv_cache_bytes(int N, int Hkv, int Lmax, int d) {
   return static_cast<size_t>(2) * N * Hkv * Lmax * d * sizeof(qwen3_bf16);
 }
 
-int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, qwen3_bf16* dst,
-                       const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
-                       int write_at_pos, float theta, float eps, qwen3_stream_t stream) {
+int qwen3_qk_norm_rope_variant(const qwen3_bf16* x, const float* w, const int32_t* pos, qwen3_bf16* dst,
+                               const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
+                               int write_at_pos, const qwen3_attn_variant* variant, float eps,
+                               qwen3_stream_t stream) {
+  Variant var;
+  const int sv = make_variant(variant, var);
+  if (sv != QWEN3_OK) return sv;
   if (x == nullptr || w == nullptr || pos == nullptr || dst == nullptr) return QWEN3_ERR_INVALID_ARG;
   if ((v_src == nullptr) != (v_dst == nullptr)) return QWEN3_ERR_INVALID_ARG;
   if (B <= 0 || T <= 0 || H <= 0 || Tcap <= 0) return QWEN3_ERR_INVALID_ARG;
@@ -240,9 +277,16 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, 
   if (!write_at_pos && Tcap < T) return QWEN3_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(dst, 16) || !aligned(w, 8) || !aligned(pos, 4)) return QWEN3_ERR_INVALID_ARG;
   if (v_src != nullptr && (!aligned(v_src, 16) || !aligned(v_dst, 16))) return QWEN3_ERR_INVALID_ARG;
-  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
-  return launch_prologue(x, w, pos, dst, v_src, v_dst, B, T, H, Tcap, write_at_pos, theta, eps,
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
+  return launch_prologue(x, w, pos, dst, v_src, v_dst, B, T, H, Tcap, write_at_pos, var, eps,
                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, qwen3_bf16* dst,
+                       const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
+                       int write_at_pos, float theta, float eps, qwen3_stream_t stream) {
+  const qwen3_attn_variant v = {theta, nullptr, 1.0f, 0};
+  return qwen3_qk_norm_rope_variant(x, w, pos, dst, v_src, v_dst, B, T, H, d, Tcap, write_at_pos, &v, eps, stream);
 }
 
 namespace {
@@ -251,7 +295,7 @@ namespace {
 int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
                  const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse, qwen3_bf16* k_cache,
                  qwen3_bf16* v_cache, int start, int Tcap, void* workspace, size_t ws_bytes, int B, int T, int Hq,
-                 int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+                 int Hkv, int d, const Variant& var, float eps, qwen3_stream_t stream) {
   if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       pos == nullptr || out == nullptr)
     return QWEN3_ERR_INVALID_ARG;
@@ -267,7 +311,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
       !aligned(k_norm_w, 8) || !aligned(pos, 4) || (lse != nullptr && !aligned(lse, 4)))
     return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
-  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
   if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
     return QWEN3_ERR_WORKSPACE;
   if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
@@ -289,7 +333,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   pq.dstq = qdst;
   pq.Hq = Hq;
   st = launch_prologue(k, k_norm_w, pos, kdst + shift, use_cache ? v : nullptr, use_cache ? v_cache + shift : nullptr,
-                       B, T, Hkv, Tc, 0, theta, eps, s, pq);
+                       B, T, Hkv, Tc, 0, var, eps, s, pq);
   if (st != QWEN3_OK) return st;
 
   // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
@@ -346,6 +390,8 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   if (n_items > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   p.n_items = static_cast<int>(n_items);
   p.start = start;
+  p.window = var.window;
+  p.rope_scale = var.scale;
   p.eps = eps;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
   p.wait = next_wait_cfg();
@@ -380,8 +426,23 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
                           const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
                           qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap, void* workspace, size_t ws_bytes,
                           int B, int T, int Hq, int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+  Variant var;
+  const int sv = theta_variant(theta, var);
+  if (sv != QWEN3_OK) return sv;
   return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, k_cache, v_cache, 0, Tcap, workspace, ws_bytes,
-                      B, T, Hq, Hkv, d, theta, eps, stream);
+                      B, T, Hq, Hkv, d, var, eps, stream);
+}
+
+int qwen3_attn_prefill_variant(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                               const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
+                               qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap, void* workspace,
+                               size_t ws_bytes, int B, int T, int Hq, int Hkv, int d,
+                               const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream) {
+  Variant var;
+  const int sv = make_variant(variant, var);
+  if (sv != QWEN3_OK) return sv;
+  return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, k_cache, v_cache, start, Tcap, workspace,
+                      ws_bytes, B, T, Hq, Hkv, d, var, eps, stream);
 }
 
 int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
@@ -390,8 +451,11 @@ int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
                              size_t ws_bytes, int B, int T, int Hq, int Hkv, int d, float theta, float eps,
                              qwen3_stream_t stream) {
   if (k_cache == nullptr || v_cache == nullptr) return QWEN3_ERR_INVALID_ARG;
+  Variant var;
+  const int sv = theta_variant(theta, var);
+  if (sv != QWEN3_OK) return sv;
   return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, k_cache, v_cache, start, Tcap, workspace,
-                      ws_bytes, B, T, Hq, Hkv, d, theta, eps, stream);
+                      ws_bytes, B, T, Hq, Hkv, d, var, eps, stream);
 }
 
 int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
@@ -413,10 +477,14 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
   return freed ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
-int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
-                      const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
-                      qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta, float eps,
-                      void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
+                const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, const Variant& var, float eps,
+                void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
   if (q == nullptr || k_new == nullptr || v_new == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       k_cache == nullptr || v_cache == nullptr || cache_lens == nullptr || out == nullptr)
     return QWEN3_ERR_INVALID_ARG;
@@ -429,13 +497,13 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
       !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) ||
       !aligned(cache_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
     return QWEN3_ERR_INVALID_ARG;
-  if (!(eps >= 0.f) || !(theta > 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
   if (workspace == nullptr || ws_bytes < qwen3_attn_decode_workspace_size(N, Hq, d, Lmax)) return QWEN3_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
 
   // 1. Append: normed+rotated k_new and raw v_new into slot L = cache_lens[n].
-  st = launch_prologue(k_new, k_norm_w, cache_lens, k_cache, v_new, v_cache, N, 1, Hkv, Lmax, 1, theta, eps, s);
+  st = launch_prologue(k_new, k_norm_w, cache_lens, k_cache, v_new, v_cache, N, 1, Hkv, Lmax, 1, var, eps, s);
   if (st != QWEN3_OK) return st;
 
   // 2. Split-KV attention.
@@ -465,7 +533,9 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
   p.eps = eps;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
   p.wait = next_wait_cfg();
-  p.rope = make_rope_table(theta);
+  p.window = var.window;
+  p.rope_scale = var.scale;
+  p.rope = var.rope;
   q3::decode_split_kernel<<<dim3(ns, Hkv, N), q3::kDecodeThreads, q3::kDecodeSmemBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
 
@@ -480,8 +550,36 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
   c.Lmax = Lmax;
   c.split = kDecodeSplit;
   c.n_split_max = ns;
+  c.window = var.window;
   q3::decode_combine_kernel<<<N * Hq, 128, 0, s>>>(c);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
+                      const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
+                      qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta, float eps,
+                      void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
+  Variant var;
+  const int sv = theta_variant(theta, var);
+  if (sv != QWEN3_OK) return sv;
+  return decode_impl(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq, Hkv, d,
+                     Lmax, var, eps, workspace, ws_bytes, stream);
+}
+
+int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                              const float* q_norm_w, const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache,
+                              const int32_t* cache_lens, qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d,
+                              int Lmax, const qwen3_attn_variant* variant, float eps, void* workspace,
+                              size_t ws_bytes, qwen3_stream_t stream) {
+  Variant var;
+  const int sv = make_variant(variant, var);
+  if (sv != QWEN3_OK) return sv;
+  return decode_impl(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq, Hkv, d,
+                     Lmax, var, eps, workspace, ws_bytes, stream);
 }
 
 }  // extern "C"

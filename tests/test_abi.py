@@ -103,6 +103,31 @@ def test_chunked_prefill_argument_checks():
     assert _prefill_ex(kc=FAKE, vc=FAKE, Tcap=128) == qa.ERR_WORKSPACE
 
 
+def test_variant_argument_checks():
+    lib = qa.lib()
+    good, _ = qa.make_variant(1e6, None, 1.0, 0)
+
+    def pre(var):
+        return lib.qwen3_attn_prefill_variant(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 0, 0, None,
+                                              0, 1, 128, 16, 8, 128, var, 1e-6, None)
+
+    def dec(var):
+        return lib.qwen3_attn_decode_variant(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4, 32, 8,
+                                             128, 1000, var, 1e-6, None, 0, None)
+
+    assert pre(ctypes.byref(good)) == qa.ERR_WORKSPACE  # a valid variant gets as far as the workspace check
+    assert dec(ctypes.byref(good)) == qa.ERR_WORKSPACE
+    assert pre(None) == qa.ERR_INVALID_ARG
+    for theta, inv, sc, win in [(0.0, None, 1.0, 0), (1e6, None, 0.0, 0), (1e6, None, float("nan"), 0),
+                                (1e6, None, 1.0, -1), (1e6, [float("inf")] + [1.0] * 63, 1.0, 0)]:
+        bad, _keep = qa.make_variant(theta, inv, sc, win)
+        assert pre(ctypes.byref(bad)) == qa.ERR_INVALID_ARG, (theta, sc, win)
+        assert dec(ctypes.byref(bad)) == qa.ERR_INVALID_ARG, (theta, sc, win)
+    # a caller's table stands in for theta
+    tab, _keep = qa.make_variant(0.0, [0.5 ** i for i in range(64)], 1.0, 64)
+    assert pre(ctypes.byref(tab)) == qa.ERR_WORKSPACE
+
+
 def test_decode_and_prologue_argument_checks():
     lib = qa.lib()
 
