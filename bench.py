@@ -65,8 +65,8 @@ def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
 # DRAM traffic of the decode split-KV kernel per cached token (dram__bytes_read.sum +
 # dram__bytes_write.sum of one ncu capture of a smaller case, divided by its cached tokens),
 # valid only for the kernel source it was measured on.  Refreshed with each new capture.
-DECODE_TRAFFIC = {"src_sha256": "bd2c84e9ee529b80e5f1797279784c54abfecf2b695386d38f6a4e4de3731d07",
-                  "bytes_per_cached_token": (630.624512e6 + 6.021376e6) / 153639}
+DECODE_TRAFFIC = {"src_sha256": "f9d0ff22d1b944a29783c29346ec878f23d53bdc66c476d421fb02983b9a3ff2",
+                  "bytes_per_cached_token": (630.630656e6 + 5.910528e6) / 153639}
 
 
 def decode_src_sha256() -> str:
