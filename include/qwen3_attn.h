@@ -257,6 +257,65 @@ int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
                               const qwen3_attn_variant* variant, float eps,
                               void* workspace, size_t ws_bytes, qwen3_stream_t stream);
 
+/*
+ * qwen3_paged_kv - a KV cache in pages, as paged serving engines keep it ("LLM Internals -
+ * Assembling a large model from scratch", the notes below the code: real systems replace the
+ * grow-by-concatenation cache with preallocated paged memory).
+ *   k_pages, v_pages  [num_pages, Hkv, page_size, d] bf16 device pools (16-byte aligned).
+ *   block_table       [rows, max_blocks] int32 device array: key index j of batch row (or
+ *                     sequence) b lives in page block_table[b, j / page_size] at offset
+ *                     j % page_size.  Only the blocks that hold keys the call reads or writes
+ *                     are read; an entry outside [0, num_pages) is recorded as
+ *                     QWEN3_ERR_INVALID_ARG in the device status word and its keys skipped.
+ *   page_size         a power of two in [16, 1024].
+ * The caller owns the pools and the table.
+ */
+typedef struct qwen3_paged_kv {
+  qwen3_bf16* k_pages;
+  qwen3_bf16* v_pages;
+  const int32_t* block_table;
+  int num_pages;
+  int page_size;
+  int max_blocks;
+} qwen3_paged_kv;
+
+/*
+ * qwen3_attn_decode_paged - qwen3_attn_decode_variant over a paged cache: the new key and
+ * value go to key index L = cache_lens[n] of sequence n (its page must be in the table), and
+ * the split-KV kernel reads each 64-key chunk page by page with TMA.  L + 1 <=
+ * max_blocks * page_size.  Workspace: qwen3_attn_decode_workspace_size(N, Hq, d,
+ * max_blocks * page_size) bytes.
+ */
+int qwen3_attn_decode_paged(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                            const float* q_norm_w, const float* k_norm_w,
+                            const qwen3_paged_kv* kv, const int32_t* cache_lens,
+                            qwen3_bf16* out, float* lse,
+                            int N, int Hq, int Hkv, int d,
+                            const qwen3_attn_variant* variant, float eps,
+                            void* workspace, size_t ws_bytes, qwen3_stream_t stream);
+
+/*
+ * qwen3_attn_prefill_paged - chunked prefill over a paged cache: T new tokens per batch row
+ * after `start` cached ones (start = 0: a fresh prompt).  The new keys (normed, rotated) and
+ * values are written into their pages at key indices start..start+T-1.  The row's first
+ * start + T keys are then gathered from the pages into the workspace, where the attention
+ * kernel reads them, as for qwen3_attn_prefill_chunk.  The gather costs a read and a write
+ * of those keys, small next to the attention's arithmetic.  start + T <=
+ * max_blocks * page_size.  Workspace:
+ * qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d) bytes.
+ */
+int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                             const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                             qwen3_bf16* out, float* lse,
+                             const qwen3_paged_kv* kv, int start,
+                             void* workspace, size_t ws_bytes,
+                             int B, int T, int Hq, int Hkv, int d,
+                             const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream);
+
+/* Scratch bytes qwen3_attn_prefill_paged needs: K and V of start + T keys per row, Q', and
+ * alignment slack; 0 when a size is not positive (start may be 0). */
+size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d);
+
 /* Scratch bytes qwen3_attn_prefill_ex and qwen3_attn_prefill_chunk need: B*T*Hkv*d*2
  * (normed, rotated keys) + B*T*Hq*d*2 (normed, rotated queries), plus alignment slack;
  * 0 when a size is not positive. */

@@ -11,6 +11,7 @@ from .attention import (  # noqa: F401
     chunk_prefill_ref,
     decode_ref,
     kv_cache_values_per_token,
+    paged_gather,
     prefill_ref,
     qk_prologue,
     rms_norm,

@@ -260,6 +260,19 @@ def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens
     return np.stack(outs), np.stack(lses)
 
 
+def paged_gather(pages, block_table_row, n: int, page_size: int) -> np.ndarray:
+    """The first n keys of one sequence out of a paged pool, as [Hkv, n, d].
+
+    pages [num_pages, Hkv, page_size, d]; key j lives in page block_table_row[j // page_size]
+    at offset j % page_size (the block-table layout of paged KV caches, which "Assembling a
+    large model from scratch" names as what real systems use instead of concatenation)."""
+    pages = np.asarray(pages)
+    out = np.empty((pages.shape[1], n, pages.shape[3]), dtype=np.float64)
+    for j in range(n):
+        out[:, j] = pages[int(block_table_row[j // page_size]), :, j % page_size]
+    return out
+
+
 def kv_cache_values_per_token(Hkv: int, d: int) -> int:
     """Values one layer's cache holds per token: a key and a value per KV head
     ("Qwen 3 From Scratch", Worked example: 2 x Hkv x d_head)."""

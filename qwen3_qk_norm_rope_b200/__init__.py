@@ -27,6 +27,13 @@ class Variant(ctypes.Structure):
                 ("attention_scaling", ctypes.c_float), ("window", ctypes.c_int)]
 
 
+class PagedKV(ctypes.Structure):
+    """qwen3_paged_kv: page pools [num_pages, Hkv, page_size, d] bf16 and the block table
+    [rows, max_blocks] int32 (device pointers)."""
+    _fields_ = [("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int), ("page_size", ctypes.c_int), ("max_blocks", ctypes.c_int)]
+
+
 # Every symbol include/qwen3_attn.h declares: (name, restype, argtypes)
 _P, _I, _F, _Z, _U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.c_uint64
 _V = ctypes.POINTER(Variant)
@@ -44,6 +51,11 @@ SIGNATURES = {
                                         _I, _I, _I, _I, _I, _V, _F, _P]),
     "qwen3_attn_decode_variant": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _V, _F, _P, _Z,
                                        _P]),
+    "qwen3_attn_decode_paged": (_I, [_P, _P, _P, _P, _P, ctypes.POINTER(PagedKV), _P, _P, _P, _I, _I, _I, _I, _V, _F,
+                                     _P, _Z, _P]),
+    "qwen3_attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(PagedKV), _I, _P, _Z,
+                                      _I, _I, _I, _I, _I, _V, _F, _P]),
+    "qwen3_attn_prefill_paged_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
@@ -126,6 +138,20 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device: 
 
 def prefill_workspace_size(B: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
     return int(lib().qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
+
+
+def prefill_paged_workspace_size(B: int, start: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d))
+
+
+def _paged(k_pages, v_pages, block_table, dev, Hkv, d):
+    num_pages, _, page_size, _ = k_pages.shape
+    _need(k_pages, "k_pages", torch.bfloat16, (num_pages, Hkv, page_size, d), dev)
+    _need(v_pages, "v_pages", torch.bfloat16, (num_pages, Hkv, page_size, d), dev)
+    _need(block_table, "block_table", torch.int32, tuple(block_table.shape), dev)
+    if block_table.dim() != 2 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous [rows, max_blocks] int32 tensor")
+    return PagedKV(_ptr(k_pages), _ptr(v_pages), _ptr(block_table), num_pages, page_size, block_table.shape[1])
 
 
 def decode_workspace_size(N: int, Hq: int, Lmax: int, d: int = HEAD_DIM) -> int:
@@ -302,6 +328,69 @@ def decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, *,
                                                N, Hq, Hkv, d, Lmax, ctypes.byref(var), eps, _ptr(workspace),
                                                ws_bytes, _stream(dev)),
                "qwen3_attn_decode_variant")
+    return out
+
+
+def decode_paged(q, k_new, v_new, q_norm_w, k_norm_w, k_pages, v_pages, block_table, cache_lens, *,
+                 theta: float = 1.0e6, eps: float = 1.0e-6, out=None, lse=None, workspace=None, window: int = 0,
+                 inv_freq=None, attention_scaling: float = 1.0):
+    """One decode step over a paged cache: pools [num_pages, Hkv, page_size, d] bf16 and the
+    block table [N, max_blocks] int32.  The new key and value go to key index cache_lens[n]."""
+    dev = q.device
+    N, Hq, d = q.shape
+    Hkv = k_new.shape[1]
+    _need(q, "q", torch.bfloat16, (N, Hq, d), dev)
+    _need(k_new, "k_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(v_new, "v_new", torch.bfloat16, (N, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(cache_lens, "cache_lens", torch.int32, (N,), dev)
+    kv = _paged(k_pages, v_pages, block_table, dev, Hkv, d)
+    if out is None:
+        out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (N, Hq), dev)
+    if workspace is None:
+        workspace = torch.empty(decode_workspace_size(N, Hq, kv.max_blocks * kv.page_size, d), dtype=torch.uint8,
+                                device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+    _check(lib().qwen3_attn_decode_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(q_norm_w), _ptr(k_norm_w),
+                                         ctypes.byref(kv), _ptr(cache_lens), _ptr(out), _ptr(lse), N, Hq, Hkv, d,
+                                         ctypes.byref(var), eps, _ptr(workspace), ws_bytes, _stream(dev)),
+           "qwen3_attn_decode_paged")
+    return out
+
+
+def prefill_paged(q, k, v, q_norm_w, k_norm_w, pos, k_pages, v_pages, block_table, start: int, *,
+                  theta: float = 1.0e6, eps: float = 1.0e-6, out=None, lse=None, workspace=None, window: int = 0,
+                  inv_freq=None, attention_scaling: float = 1.0):
+    """Chunked prefill over a paged cache (start = 0 for a fresh prompt): the new keys and
+    values are written into their pages; returns out [B,T,Hq,d]."""
+    dev = q.device
+    B, T, Hq, d = q.shape
+    Hkv = k.shape[2]
+    _need(q, "q", torch.bfloat16, (B, T, Hq, d), dev)
+    _need(k, "k", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(v, "v", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (B, T), dev)
+    kv = _paged(k_pages, v_pages, block_table, dev, Hkv, d)
+    if out is None:
+        out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, T, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (B, Hq, T), dev)
+    if workspace is None:
+        workspace = torch.empty(prefill_paged_workspace_size(B, start, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+    _check(lib().qwen3_attn_prefill_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                          _ptr(out), _ptr(lse), ctypes.byref(kv), int(start), _ptr(workspace),
+                                          ws_bytes, B, T, Hq, Hkv, d, ctypes.byref(var), eps, _stream(dev)),
+           "qwen3_attn_prefill_paged")
     return out
 
 

@@ -31,6 +31,7 @@ enum Site : int {
   kSiteDecodeFull = 40,
   kSiteDecodeEmpty = 41,
   kSiteDecodeLen = 42,
+  kSitePagedTable = 50,
 };
 
 // Device status word: [0] = first qwen3_status recorded, [1] = its site.

@@ -31,6 +31,11 @@ struct DecodeParams {
   float* part_lse;        // [N, Hq, n_split_max]
   int N, Hq, Hkv, log2G, Lmax, split, n_split_max;
   int window;        // sliding window W: the query sees keys L-W < j <= L; 0 = all
+  // Paged cache (block_table != nullptr): the tensor maps cover the page pools as rows of d,
+  // [num_pages * Hkv * page, d], with boxes of min(page, 64) rows; key j of sequence n is in
+  // page block_table[n, j / page] at offset j % page.  page = 1 << log2_page, >= 16.
+  const int* block_table;
+  int max_blocks, log2_page, num_pages;
   float eps, scale_log2;
   float rope_scale;  // attention_scaling on cos and sin
   WaitCfg wait;
@@ -122,12 +127,43 @@ __global__ void __launch_bounds__(kDecodeThreads)
           break;
         const uint32_t dst = sb + st * kDcStage;
         const uint32_t fb = bar + kDcBFull + 8 * st;
-        const int r = static_cast<int>(row0 + c * 64);
-        mbar_arrive_expect_tx(fb, kDcStage);
-        tma_load_2d(dst, &tmK, fb, 0, r);
-        tma_load_2d(dst + kDcBox, &tmK, fb, 64, r);
-        tma_load_2d(dst + kDcChunk, &tmV, fb, 0, r);
-        tma_load_2d(dst + kDcChunk + kDcBox, &tmV, fb, 64, r);
+        if (p.block_table == nullptr) {
+          const int r = static_cast<int>(row0 + c * 64);
+          mbar_arrive_expect_tx(fb, kDcStage);
+          tma_load_2d(dst, &tmK, fb, 0, r);
+          tma_load_2d(dst + kDcBox, &tmK, fb, 64, r);
+          tma_load_2d(dst + kDcChunk, &tmV, fb, 0, r);
+          tma_load_2d(dst + kDcChunk + kDcBox, &tmV, fb, 64, r);
+        } else {
+          // Boxes of br keys, each inside one page; boxes wholly past key L are not loaded
+          // (the consumers mask those keys and zero their V rows).
+          const int br = min(1 << p.log2_page, 64);
+          int rows[4], nb = 0;
+          for (int r0 = 0; r0 < 64 && nb < 4; r0 += br) {
+            const int key = tok0 + c * 64 + r0;
+            if (key > L) break;
+            const int blk = key >> p.log2_page;
+            const int page = blk < p.max_blocks ? p.block_table[static_cast<long long>(n) * p.max_blocks + blk] : -1;
+            if (page < 0 || page >= p.num_pages) {
+              record_error(QWEN3_ERR_INVALID_ARG, kSitePagedTable);
+              rows[nb++] = -1;
+              continue;
+            }
+            rows[nb++] = ((page * p.Hkv + h) << p.log2_page) + (key & ((1 << p.log2_page) - 1));
+          }
+          uint32_t bytes = 0;
+          for (int i = 0; i < nb; ++i)
+            if (rows[i] >= 0) bytes += 4u * br * 128u;
+          mbar_arrive_expect_tx(fb, bytes);
+          for (int i = 0; i < nb; ++i) {
+            if (rows[i] < 0) continue;
+            const uint32_t off = static_cast<uint32_t>(i * br) * 128u;
+            tma_load_2d(dst + off, &tmK, fb, 0, rows[i]);
+            tma_load_2d(dst + kDcBox + off, &tmK, fb, 64, rows[i]);
+            tma_load_2d(dst + kDcChunk + off, &tmV, fb, 0, rows[i]);
+            tma_load_2d(dst + kDcChunk + kDcBox + off, &tmV, fb, 64, rows[i]);
+          }
+        }
         last[st] = u;
       }
       for (int s = 0; s < kDcStages; ++s)

@@ -27,6 +27,11 @@ struct PrologueParams {
   uint32_t* dstq;
   int B, T, H, Tcap, write_at_pos;
   int Hq, log2G;
+  // Optional paged destination: dst and v_dst are page pools [num_pages, H, page, d]; key
+  // index kk of batch row b (pos[b,t] when write_at_pos, else key0 + t) lives in page
+  // block_table[b, kk / page] at offset kk % page.  page = 1 << log2_page.
+  const int* block_table;
+  int max_blocks, log2_page, num_pages, key0;
   float eps;
   float rope_scale;  // attention_scaling: multiplies cos and sin (1 for the default rope type)
   RopeTable rope;
@@ -58,10 +63,26 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     const int b = bt / p.T;
     const int t = bt - b * p.T;
     const int ps = p.pos[bt];
-    const int row = p.write_at_pos ? ps : t;
-    if (row < 0 || row >= p.Tcap) {
-      if (lane == 0) record_error(QWEN3_ERR_INVALID_ARG, kSitePrologueRow);
-      continue;
+    // destination of head 0 and the distance between heads, in rows of d
+    size_t row0, hstride;
+    if (p.block_table == nullptr) {
+      const int row = p.write_at_pos ? ps : t;
+      if (row < 0 || row >= p.Tcap) {
+        if (lane == 0) record_error(QWEN3_ERR_INVALID_ARG, kSitePrologueRow);
+        continue;
+      }
+      row0 = static_cast<size_t>(b) * p.H * p.Tcap + row;
+      hstride = p.Tcap;
+    } else {
+      const int kk = p.write_at_pos ? ps : p.key0 + t;
+      const int blk = kk >> p.log2_page;
+      const int page = (kk >= 0 && blk < p.max_blocks) ? p.block_table[static_cast<size_t>(b) * p.max_blocks + blk] : -1;
+      if (page < 0 || page >= p.num_pages) {
+        if (lane == 0) record_error(QWEN3_ERR_INVALID_ARG, kSitePrologueRow);
+        continue;
+      }
+      row0 = (static_cast<size_t>(page) * p.H << p.log2_page) + (kk & ((1 << p.log2_page) - 1));
+      hstride = static_cast<size_t>(1) << p.log2_page;
     }
     float s0, c0, s1, c1;
     rope_sincos(ps, hi0, lo0, s0, c0);
@@ -90,7 +111,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
         float2 ya, yb;
         norm_rope_pairs(make_float2(bf16lo(ua[u]), bf16hi(ua[u])), make_float2(bf16lo(ub[u]), bf16hi(ub[u])), ga,
                         gb, s0, c0, s1, c1, p.eps, ya, yb);
-        const size_t drow = (static_cast<size_t>(b) * p.H + h0 + u) * p.Tcap + row;
+        const size_t drow = row0 + static_cast<size_t>(h0 + u) * hstride;
         uint32_t* ds = p.dst + drow * (kD / 2);
         ds[lane] = pack_bf16x2(ya.x, ya.y);
         ds[32 + lane] = pack_bf16x2(yb.x, yb.y);

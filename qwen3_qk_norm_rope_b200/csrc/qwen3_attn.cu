@@ -1,6 +1,7 @@
 // qwen3_attn.cu - the C ABI of libqwen3attn.so: argument checks, RoPE constants, TMA
 // tensor maps and kernel launches.  All device work lives in the kernels included below;
 // this file does no arithmetic on tensor data.
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -10,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "paged.cuh"
 #include "prologue.cuh"
 
 namespace {
@@ -78,6 +80,35 @@ int make_variant(const qwen3_attn_variant* v, Variant& out) {
   out.rope = make_rope_table(v->theta, v->inv_freq);
   out.scale = v->attention_scaling;
   out.window = v->window;
+  return QWEN3_OK;
+}
+
+// A checked qwen3_paged_kv.
+struct PagedKV {
+  qwen3_bf16* k = nullptr;
+  qwen3_bf16* v = nullptr;
+  const int32_t* table = nullptr;
+  int num_pages = 0, page = 0, max_blocks = 0, log2_page = 0;
+};
+
+int make_paged(const qwen3_paged_kv* kv, int Hkv, PagedKV& out) {
+  if (kv == nullptr || kv->k_pages == nullptr || kv->v_pages == nullptr || kv->block_table == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (kv->num_pages <= 0 || kv->max_blocks <= 0 || kv->page_size < 16 || kv->page_size > 1024 ||
+      (kv->page_size & (kv->page_size - 1)) != 0)
+    return QWEN3_ERR_INVALID_ARG;
+  if (!aligned(kv->k_pages, 16) || !aligned(kv->v_pages, 16) || !aligned(kv->block_table, 4))
+    return QWEN3_ERR_INVALID_ARG;
+  // rows of d in a pool must index as int32 (TMA row coordinates)
+  if (static_cast<long long>(kv->num_pages) * Hkv * kv->page_size > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  if (static_cast<long long>(kv->max_blocks) * kv->page_size > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  out.k = kv->k_pages;
+  out.v = kv->v_pages;
+  out.table = kv->block_table;
+  out.num_pages = kv->num_pages;
+  out.page = kv->page_size;
+  out.max_blocks = kv->max_blocks;
+  out.log2_page = ilog2(kv->page_size);
   return QWEN3_OK;
 }
 
@@ -172,7 +203,8 @@ struct PrologueQ {
 
 int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
                     int B, int T, int H, int Tcap, int write_at_pos, const Variant& var, float eps,
-                    cudaStream_t stream, const PrologueQ& q = PrologueQ()) {
+                    cudaStream_t stream, const PrologueQ& q = PrologueQ(), const PagedKV* pg = nullptr,
+                    int key0 = 0) {
   q3::PrologueParams p;
   p.x = static_cast<const uint32_t*>(x);
   p.w = w;
@@ -193,6 +225,11 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.eps = eps;
   p.rope_scale = var.scale;
   p.rope = var.rope;
+  p.block_table = pg != nullptr ? pg->table : nullptr;
+  p.max_blocks = pg != nullptr ? pg->max_blocks : 0;
+  p.log2_page = pg != nullptr ? pg->log2_page : 0;
+  p.num_pages = pg != nullptr ? pg->num_pages : 0;
+  p.key0 = key0;
   const long long ntok = static_cast<long long>(B) * T;
   if (ntok > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   const int warps = 8;
@@ -251,6 +288,12 @@ size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d) {
   return kspace_bytes(B, T, Hkv, d) + kspace_bytes(B, T, Hq, d) + 256;
 }
 
+size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d) {
+  if (B <= 0 || start < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return 0;
+  // K and V of the row's first start + T keys gathered out of the pages, then Q'
+  return 2 * kspace_bytes(B, start + T, Hkv, d) + kspace_bytes(B, T, Hq, d) + 256;
+}
+
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax) {
   if (N <= 0 || Hq <= 0 || d <= 0 || Lmax <= 0) return 0;
   const size_t ns = (static_cast<size_t>(Lmax) + kDecodeSplit - 1) / kDecodeSplit;
@@ -292,10 +335,13 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, 
 namespace {
 
 // Prefill of T new tokens per batch row after `start` cached ones (start > 0 needs the caches).
+// With `pg`, the cache is paged: the new keys and values go into the pages, and the row's
+// first start + T keys are gathered from the pages into the workspace for the attention.
 int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
                  const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse, qwen3_bf16* k_cache,
                  qwen3_bf16* v_cache, int start, int Tcap, void* workspace, size_t ws_bytes, int B, int T, int Hq,
-                 int Hkv, int d, const Variant& var, float eps, qwen3_stream_t stream) {
+                 int Hkv, int d, const Variant& var, float eps, qwen3_stream_t stream,
+                 const PagedKV* pg = nullptr) {
   if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       pos == nullptr || out == nullptr)
     return QWEN3_ERR_INVALID_ARG;
@@ -304,17 +350,23 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   if (st != QWEN3_OK) return st;
   if (Hq / Hkv > 128) return QWEN3_ERR_UNSUPPORTED;
   if ((k_cache == nullptr) != (v_cache == nullptr)) return QWEN3_ERR_INVALID_ARG;
+  if (pg != nullptr && k_cache != nullptr) return QWEN3_ERR_INVALID_ARG;
   const bool use_cache = k_cache != nullptr;
-  if (start < 0 || (start > 0 && !use_cache)) return QWEN3_ERR_INVALID_ARG;
+  if (start < 0 || (start > 0 && !use_cache && pg == nullptr)) return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (Tcap <= 0 || static_cast<long long>(start) + T > Tcap)) return QWEN3_ERR_INVALID_ARG;
+  if (pg != nullptr && static_cast<long long>(start) + T > static_cast<long long>(pg->max_blocks) * pg->page)
+    return QWEN3_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) ||
       !aligned(k_norm_w, 8) || !aligned(pos, 4) || (lse != nullptr && !aligned(lse, 4)))
     return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
   if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
-  if (workspace == nullptr || ws_bytes < qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
-    return QWEN3_ERR_WORKSPACE;
+  const size_t need = pg != nullptr ? qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d)
+                                    : qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d);
+  if (workspace == nullptr || need == 0 || ws_bytes < need) return QWEN3_ERR_WORKSPACE;
   if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
+    return QWEN3_ERR_UNSUPPORTED;
+  if (pg != nullptr && static_cast<long long>(B) * Hkv * (static_cast<long long>(start) + T) > (1LL << 31) / kD)
     return QWEN3_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
@@ -324,17 +376,49 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   //    and Q' in the query tiles' row order [B, Hkv, T*G, d], both in one pass per token.
   const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
   qwen3_bf16* kdst = use_cache ? k_cache : reinterpret_cast<qwen3_bf16*>(w0);
+  qwen3_bf16* vsrc = use_cache ? v_cache : nullptr;  // V in cache layout, when not read raw
   qwen3_bf16* qdst = reinterpret_cast<qwen3_bf16*>(w0 + kspace_bytes(B, T, Hkv, d));
-  const int Tc = use_cache ? Tcap : T;
+  int Tc = use_cache ? Tcap : T;
   const size_t shift = static_cast<size_t>(start) * kD;
   PrologueQ pq;
   pq.xq = q;
   pq.wq = q_norm_w;
   pq.dstq = qdst;
   pq.Hq = Hq;
-  st = launch_prologue(k, k_norm_w, pos, kdst + shift, use_cache ? v : nullptr, use_cache ? v_cache + shift : nullptr,
-                       B, T, Hkv, Tc, 0, var, eps, s, pq);
-  if (st != QWEN3_OK) return st;
+  if (pg == nullptr) {
+    st = launch_prologue(k, k_norm_w, pos, kdst + shift, use_cache ? v : nullptr,
+                         use_cache ? v_cache + shift : nullptr, B, T, Hkv, Tc, 0, var, eps, s, pq);
+    if (st != QWEN3_OK) return st;
+  } else {
+    // Paged: K' and V of the new tokens into their pages (keys start..start+T-1), Q' into the
+    // workspace; then the row's first start + T keys and values out of the pages into the
+    // workspace, [B, Hkv, start + T, d] each, where the attention reads them.
+    const int n = start + T;
+    qdst = reinterpret_cast<qwen3_bf16*>(w0 + 2 * kspace_bytes(B, n, Hkv, d));
+    pq.dstq = qdst;
+    st = launch_prologue(k, k_norm_w, pos, pg->k, v, pg->v, B, T, Hkv, 1, 0, var, eps, s, pq, pg, start);
+    if (st != QWEN3_OK) return st;
+    kdst = reinterpret_cast<qwen3_bf16*>(w0);
+    vsrc = reinterpret_cast<qwen3_bf16*>(w0 + kspace_bytes(B, n, Hkv, d));
+    Tc = n;
+    q3::GatherParams gp;
+    gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
+    gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
+    gp.block_table = pg->table;
+    gp.k_out = reinterpret_cast<uint4*>(kdst);
+    gp.v_out = reinterpret_cast<uint4*>(vsrc);
+    gp.B = B;
+    gp.Hkv = Hkv;
+    gp.n = n;
+    gp.max_blocks = pg->max_blocks;
+    gp.log2_page = pg->log2_page;
+    gp.num_pages = pg->num_pages;
+    const long long chunks = static_cast<long long>(B) * n * Hkv * 16;
+    long long blocks = (chunks + 255) / 256;
+    if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
+    q3::paged_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
+    if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+  }
 
   // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
   //    read as zeros.
@@ -364,8 +448,8 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     const cuuint64_t str[3] = {kD * 2ull, static_cast<cuuint64_t>(Tc) * kD * 2ull,
                                static_cast<cuuint64_t>(Hkv) * Tc * kD * 2ull};
     if (!make_map(&mk, kdst, 4, dims, str, box)) return QWEN3_ERR_CUDA;
-    if (use_cache) {
-      if (!make_map(&mv, v_cache, 4, dims, str, box)) return QWEN3_ERR_CUDA;
+    if (vsrc != nullptr) {
+      if (!make_map(&mv, vsrc, 4, dims, str, box)) return QWEN3_ERR_CUDA;
     } else {
       const cuuint64_t vstr[3] = {static_cast<cuuint64_t>(Hkv) * kD * 2ull, kD * 2ull,
                                   static_cast<cuuint64_t>(T) * Hkv * kD * 2ull};
@@ -481,10 +565,16 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
 
 namespace {
 
+// With `pg`, the cache is paged (k_cache, v_cache unused; Lmax = max_blocks * page).
 int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
                 const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
                 qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, const Variant& var, float eps,
-                void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
+                void* workspace, size_t ws_bytes, qwen3_stream_t stream, const PagedKV* pg = nullptr) {
+  if (pg != nullptr) {
+    k_cache = pg->k;
+    v_cache = pg->v;
+    Lmax = pg->max_blocks * pg->page;
+  }
   if (q == nullptr || k_new == nullptr || v_new == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       k_cache == nullptr || v_cache == nullptr || cache_lens == nullptr || out == nullptr)
     return QWEN3_ERR_INVALID_ARG;
@@ -492,7 +582,7 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   int st = check_common(Hq, Hkv, d);
   if (st != QWEN3_OK) return st;
   if (Hq / Hkv > 16 || N > 65535 || Hkv > 65535) return QWEN3_ERR_UNSUPPORTED;
-  if (static_cast<long long>(N) * Hkv * Lmax > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  if (pg == nullptr && static_cast<long long>(N) * Hkv * Lmax > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
       !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) ||
       !aligned(cache_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
@@ -503,7 +593,8 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
 
   // 1. Append: normed+rotated k_new and raw v_new into slot L = cache_lens[n].
-  st = launch_prologue(k_new, k_norm_w, cache_lens, k_cache, v_new, v_cache, N, 1, Hkv, Lmax, 1, var, eps, s);
+  st = launch_prologue(k_new, k_norm_w, cache_lens, k_cache, v_new, v_cache, N, 1, Hkv, Lmax, 1, var, eps, s,
+                       PrologueQ(), pg, 0);
   if (st != QWEN3_OK) return st;
 
   // 2. Split-KV attention.
@@ -513,9 +604,11 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   float* part_o = reinterpret_cast<float*>(w0);
   float* part_lse = reinterpret_cast<float*>((w0 + o_bytes + 255) & ~static_cast<uintptr_t>(255));
   CUtensorMap mk, mv;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(N) * Hkv * Lmax};
+  const cuuint64_t rows = pg != nullptr ? static_cast<cuuint64_t>(pg->num_pages) * Hkv * pg->page
+                                        : static_cast<cuuint64_t>(N) * Hkv * Lmax;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
   const cuuint64_t str[1] = {kD * 2ull};
-  const cuuint32_t box[2] = {64, 64};
+  const cuuint32_t box[2] = {64, pg != nullptr ? static_cast<cuuint32_t>(std::min(pg->page, 64)) : 64u};
   if (!make_map(&mk, k_cache, 2, dims, str, box) || !make_map(&mv, v_cache, 2, dims, str, box)) return QWEN3_ERR_CUDA;
   q3::DecodeParams p;
   p.q = reinterpret_cast<const uint32_t*>(q);
@@ -536,6 +629,10 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   p.window = var.window;
   p.rope_scale = var.scale;
   p.rope = var.rope;
+  p.block_table = pg != nullptr ? pg->table : nullptr;
+  p.max_blocks = pg != nullptr ? pg->max_blocks : 0;
+  p.log2_page = pg != nullptr ? pg->log2_page : 0;
+  p.num_pages = pg != nullptr ? pg->num_pages : 0;
   q3::decode_split_kernel<<<dim3(ns, Hkv, N), q3::kDecodeThreads, q3::kDecodeSmemBytes, s>>>(mk, mv, p);
   if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
 
@@ -568,6 +665,36 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
   if (sv != QWEN3_OK) return sv;
   return decode_impl(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq, Hkv, d,
                      Lmax, var, eps, workspace, ws_bytes, stream);
+}
+
+int qwen3_attn_decode_paged(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,
+                            const float* q_norm_w, const float* k_norm_w, const qwen3_paged_kv* kv,
+                            const int32_t* cache_lens, qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d,
+                            const qwen3_attn_variant* variant, float eps, void* workspace, size_t ws_bytes,
+                            qwen3_stream_t stream) {
+  Variant var;
+  int st = make_variant(variant, var);
+  if (st != QWEN3_OK) return st;
+  if (Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
+  PagedKV pg;
+  if ((st = make_paged(kv, Hkv, pg)) != QWEN3_OK) return st;
+  return decode_impl(q, k_new, v_new, q_norm_w, k_norm_w, nullptr, nullptr, cache_lens, out, lse, N, Hq, Hkv, d, 0,
+                     var, eps, workspace, ws_bytes, stream, &pg);
+}
+
+int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                             const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
+                             const qwen3_paged_kv* kv, int start, void* workspace, size_t ws_bytes, int B, int T,
+                             int Hq, int Hkv, int d, const qwen3_attn_variant* variant, float eps,
+                             qwen3_stream_t stream) {
+  Variant var;
+  int st = make_variant(variant, var);
+  if (st != QWEN3_OK) return st;
+  if (Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
+  PagedKV pg;
+  if ((st = make_paged(kv, Hkv, pg)) != QWEN3_OK) return st;
+  return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, nullptr, nullptr, start, 0, workspace, ws_bytes, B,
+                      T, Hq, Hkv, d, var, eps, stream, &pg);
 }
 
 int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,

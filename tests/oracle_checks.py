@@ -377,6 +377,21 @@ def check_attention_scaling_against_torch_sdpa():
     assert np.allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
 
 
+def check_paged_gather_addressing():
+    """A pool whose every slot holds 1000*page + offset (per head and dim) gathers, for a
+    hand-written block table, to 1000*table[j // size] + j % size at key j."""
+    num_pages, Hkv, size, d = 7, 2, 4, 3
+    pages = np.zeros((num_pages, Hkv, size, d))
+    for pg in range(num_pages):
+        for off in range(size):
+            pages[pg, :, off] = 1000 * pg + off
+    table = [5, 0, 3, 6]
+    got = A.paged_gather(pages, table, 14, size)
+    want = np.array([1000 * table[j // size] + j % size for j in range(14)], dtype=np.float64)
+    assert got.shape == (Hkv, 14, d)
+    assert np.array_equal(got, np.broadcast_to(want[None, :, None], (Hkv, 14, d)))
+
+
 def check_position_shift_invariance():
     """Shifting every position by a constant leaves outputs unchanged (RoPE is relative)."""
     q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=50)

@@ -128,6 +128,36 @@ def test_variant_argument_checks():
     assert pre(ctypes.byref(tab)) == qa.ERR_WORKSPACE
 
 
+def test_paged_argument_checks():
+    lib = qa.lib()
+    var, _ = qa.make_variant()
+
+    def dec(kv):
+        return lib.qwen3_attn_decode_paged(FAKE, FAKE, FAKE, FAKE, FAKE, kv, FAKE, FAKE, None, 4, 32, 8, 128,
+                                           ctypes.byref(var), 1e-6, None, 0, None)
+
+    def pre(kv, start=0, T=128):
+        return lib.qwen3_attn_prefill_paged(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, kv, start, None, 0, 1, T,
+                                            16, 8, 128, ctypes.byref(var), 1e-6, None)
+
+    good = qa.PagedKV(1 << 20, 1 << 20, 1 << 20, 100, 64, 40)
+    assert dec(ctypes.byref(good)) == qa.ERR_WORKSPACE
+    assert pre(ctypes.byref(good)) == qa.ERR_WORKSPACE
+    assert pre(ctypes.byref(good), start=40 * 64 - 128) == qa.ERR_WORKSPACE  # start + T == capacity
+    assert pre(ctypes.byref(good), start=40 * 64 - 127) == qa.ERR_INVALID_ARG  # past the table's capacity
+    assert dec(None) == qa.ERR_INVALID_ARG
+    for bad in (qa.PagedKV(0, 1 << 20, 1 << 20, 100, 64, 40),        # no pool
+                qa.PagedKV(1 << 20, 1 << 20, 0, 100, 64, 40),        # no table
+                qa.PagedKV(1 << 20, 1 << 20, 1 << 20, 100, 48, 40),  # page not a power of two
+                qa.PagedKV(1 << 20, 1 << 20, 1 << 20, 100, 8, 40),   # page under 16
+                qa.PagedKV(1 << 20, 1 << 20, 1 << 20, 0, 64, 40),    # no pages
+                qa.PagedKV((1 << 20) + 2, 1 << 20, 1 << 20, 100, 64, 40)):  # misaligned pool
+        assert dec(ctypes.byref(bad)) == qa.ERR_INVALID_ARG
+        assert pre(ctypes.byref(bad)) == qa.ERR_INVALID_ARG
+    assert qa.prefill_paged_workspace_size(2, 100, 300, 16, 8) >= 2 * 2 * 8 * 400 * 256 + 2 * 300 * 16 * 256
+    assert qa.prefill_paged_workspace_size(2, -1, 300, 16, 8) == 0
+
+
 def test_decode_and_prologue_argument_checks():
     lib = qa.lib()
 
