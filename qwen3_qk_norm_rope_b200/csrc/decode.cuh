@@ -49,7 +49,8 @@ constexpr uint32_t kDcStage = 2 * kDcChunk;   // K chunk + V chunk
 constexpr uint32_t kDcQ = kDcStages * kDcStage;  // q' [16][128] bf16 = 4096 B
 constexpr uint32_t kDcBar = kDcQ + 4096;
 constexpr uint32_t kDcBFull = 0, kDcBEmpty = 32, kDcBAbort = 64;
-constexpr uint32_t kDecodeSmemBytes = kDcBar + 128 + 1024;
+constexpr uint32_t kDcTab = kDcBar + 128;  // a paged split's page indices: <= 1024 / 16 of them
+constexpr uint32_t kDecodeSmemBytes = kDcTab + 256 + 1024;
 constexpr int kDecodeThreads = 160;
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -115,6 +116,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const long long row0 = (static_cast<long long>(n) * p.Hkv + h) * p.Lmax + tok0;
   if (warp == 4) {
     // ------------------------------------------------------------------ TMA producer
+    // A paged split first stages its page indices in shared memory, one coalesced load by
+    // the warp, so the chunk loop never waits on the block table.
+    int* s_tab = reinterpret_cast<int*>(sgen + kDcTab);
+    const int blk0 = tok0 >> p.log2_page;
+    if (p.block_table != nullptr) {
+      const int nblk = min(((tok0 + ntok - 1) >> p.log2_page) - blk0 + 1, 64);
+      for (int i = lane; i < nblk; i += 32)
+        s_tab[i] = blk0 + i < p.max_blocks ? p.block_table[static_cast<long long>(n) * p.max_blocks + blk0 + i] : -1;
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
@@ -142,8 +153,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
           for (int r0 = 0; r0 < 64 && nb < 4; r0 += br) {
             const int key = tok0 + c * 64 + r0;
             if (key > L) break;
-            const int blk = key >> p.log2_page;
-            const int page = blk < p.max_blocks ? p.block_table[static_cast<long long>(n) * p.max_blocks + blk] : -1;
+            const int page = s_tab[(key >> p.log2_page) - blk0];
             if (page < 0 || page >= p.num_pages) {
               record_error(QWEN3_ERR_INVALID_ARG, kSitePagedTable);
               rows[nb++] = -1;
