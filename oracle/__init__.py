@@ -14,8 +14,9 @@ from .attention import (  # noqa: F401
     paged_gather,
     prefill_ref,
     qk_prologue,
+    qkv_proj_norm_rope_ref,
     rms_norm,
     rope,
     rope_inv_freq,
 )
-from .loops import chunk_prefill_loops, decode_loops, prefill_loops  # noqa: F401
+from .loops import chunk_prefill_loops, decode_loops, prefill_loops, qkv_proj_norm_rope_loops  # noqa: F401

@@ -260,6 +260,31 @@ def decode_ref(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens
     return np.stack(outs), np.stack(lses)
 
 
+def qkv_proj_norm_rope_ref(x, w_qkv, q_norm_w, k_norm_w, pos, Hq: int, Hkv: int, theta: float, eps: float,
+                           staged: bool = False, inv_freq=None, scaling: float = 1.0):
+    """The merged qkv projection followed by QK-Norm and RoPE, in fp64.
+
+    x [M, hidden] token hidden states; w_qkv [(Hq + 2 Hkv) d, hidden], the q, k and v
+    projection weights stacked in that order (one GEMM for the three: "Assembling a large
+    model from scratch", the comparison with inference engines, qkv_proj); pos [M].
+    y = x w_qkv^T splits into q [M, Hq, d], k [M, Hkv, d], v [M, Hkv, d]; q and k get
+    QK-Norm then RoPE at pos ("Hand-Writing ... Part 1", order of operations), v is
+    returned as projected.  Returns (q', k', v).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    w = np.asarray(w_qkv, dtype=np.float64)
+    d = w.shape[0] // (Hq + 2 * Hkv)
+    y = x @ w.T
+    M = x.shape[0]
+    q = y[:, :Hq * d].reshape(M, Hq, d)
+    k = y[:, Hq * d:(Hq + Hkv) * d].reshape(M, Hkv, d)
+    v = y[:, (Hq + Hkv) * d:].reshape(M, Hkv, d)
+    pos = np.asarray(pos)
+    qp = qk_prologue(q, q_norm_w, pos, theta, eps, staged, inv_freq, scaling)
+    kp = qk_prologue(k, k_norm_w, pos, theta, eps, staged, inv_freq, scaling)
+    return qp, kp, v
+
+
 def paged_gather(pages, block_table_row, n: int, page_size: int) -> np.ndarray:
     """The first n keys of one sequence out of a paged pool, as [Hkv, n, d].
 

@@ -113,3 +113,17 @@ def chunk_prefill_loops(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, ep
                     out[b][t][h][i] = sum(w[j] * vals[j][i] for j in range(len(w))) / z
                 lse[b][h][t] = m + math.log(z)
     return out, lse
+
+
+def qkv_proj_norm_rope_loops(x, w_qkv, gq, gk, pos, Hq, Hkv, theta, eps):
+    """The merged projection element by element, then QK-Norm and RoPE per head vector.
+    x[m][i], w_qkv[o][i]; returns q'[m][h][i], k'[m][h][i], v[m][h][i]."""
+    M, hidden = len(x), len(x[0])
+    n_out = len(w_qkv)
+    d = n_out // (Hq + 2 * Hkv)
+    y = [[sum(float(x[m][i]) * float(w_qkv[o][i]) for i in range(hidden)) for o in range(n_out)] for m in range(M)]
+    q = [[_norm_rope(y[m][h * d:(h + 1) * d], gq, float(pos[m]), theta, eps) for h in range(Hq)] for m in range(M)]
+    k = [[_norm_rope(y[m][(Hq + h) * d:(Hq + h + 1) * d], gk, float(pos[m]), theta, eps) for h in range(Hkv)]
+         for m in range(M)]
+    v = [[y[m][(Hq + Hkv + h) * d:(Hq + Hkv + h + 1) * d] for h in range(Hkv)] for m in range(M)]
+    return q, k, v

@@ -392,6 +392,43 @@ def check_paged_gather_addressing():
     assert np.array_equal(got, np.broadcast_to(want[None, :, None], (Hkv, 14, d)))
 
 
+# ---------------------------------------------------------------- merged qkv projection
+def check_qkv_projection_brute_force_and_identity():
+    """The merged projection against scalar loops; with w_qkv = the identity on each head's
+    block it reduces to QK-Norm + RoPE of x itself (the prologue pinned above)."""
+    rng = np.random.default_rng(90)
+    Hq, Hkv, hidden, M = 2, 1, 16, 3
+    d = D
+    x = rng.standard_normal((M, hidden))
+    w = rng.standard_normal(((Hq + 2 * Hkv) * d, hidden)) / 4
+    gq, gk = _gain(91), _gain(92)
+    pos = np.array([0, 5, 300])
+    q, k, v = A.qkv_proj_norm_rope_ref(x, w, gq, gk, pos, Hq, Hkv, THETA, EPS)
+    ql, kl, vl = Lp.qkv_proj_norm_rope_loops(x.tolist(), w.tolist(), gq.tolist(), gk.tolist(), pos.tolist(), Hq, Hkv,
+                                             THETA, EPS)
+    assert np.allclose(q, np.array(ql), rtol=0, atol=1e-12)
+    assert np.allclose(k, np.array(kl), rtol=0, atol=1e-12)
+    assert np.allclose(v, np.array(vl), rtol=0, atol=1e-12)
+    xh = rng.standard_normal((M, d))
+    eye = np.concatenate([np.eye(d)] * (Hq + 2 * Hkv), axis=0)  # every head projects x itself
+    q2, k2, v2 = A.qkv_proj_norm_rope_ref(xh, eye, gq, gk, pos, Hq, Hkv, THETA, EPS)
+    want_q = A.qk_prologue(np.repeat(xh[:, None], Hq, axis=1), gq, pos, THETA, EPS)
+    assert np.allclose(q2, want_q, rtol=0, atol=1e-13) and np.allclose(v2[:, 0], xh, rtol=0, atol=0)
+
+
+def check_qkv_projection_scale_invariance():
+    """Scaling the hidden states scales v and leaves q', k' unchanged up to the eps term."""
+    rng = np.random.default_rng(93)
+    x = rng.standard_normal((5, 64))
+    w = rng.standard_normal(((4 + 4) * D, 64)) / 8
+    gq, gk = _gain(94), _gain(95)
+    pos = np.arange(5) * 7
+    q1, k1, v1 = A.qkv_proj_norm_rope_ref(x, w, gq, gk, pos, 4, 2, THETA, 0.0)
+    q2, k2, v2 = A.qkv_proj_norm_rope_ref(3.0 * x, w, gq, gk, pos, 4, 2, THETA, 0.0)
+    assert np.allclose(q1, q2, rtol=0, atol=1e-12) and np.allclose(k1, k2, rtol=0, atol=1e-12)
+    assert np.allclose(3.0 * v1, v2, rtol=1e-12, atol=1e-13)
+
+
 def check_position_shift_invariance():
     """Shifting every position by a constant leaves outputs unchanged (RoPE is relative)."""
     q, k, v, gq, gk, pos = _inputs(1, 20, 4, 2, seed=50)

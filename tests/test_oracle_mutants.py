@@ -78,8 +78,17 @@ def _rope_ignores_inv_freq(x, pos, theta, inv_freq=None, scaling=1.0):
     return _ORIG_ROPE(x, pos, theta, None, scaling)
 
 
+def _qkv_swapped_kv(x, w_qkv, gq, gk, pos, Hq, Hkv, theta, eps, **kw):
+    # the k and v blocks of the merged weight taken in the wrong order
+    w = np.asarray(w_qkv, dtype=np.float64)
+    d = w.shape[0] // (Hq + 2 * Hkv)
+    w2 = np.concatenate([w[:Hq * d], w[(Hq + Hkv) * d:], w[Hq * d:(Hq + Hkv) * d]], axis=0)
+    return _ORIG_QKV(x, w2, gq, gk, pos, Hq, Hkv, theta, eps, **kw)
+
+
 _ORIG_ATTEND = A._attend
 _ORIG_ROPE = A.rope
+_ORIG_QKV = A.qkv_proj_norm_rope_ref
 
 
 def _prefill_mod_mapping(q, k, v, gq, gk, pos, theta, eps, rows=None, staged=False, block=256, **kw):
@@ -137,6 +146,7 @@ MUTANTS = [
     ("_attend", _attend_window_one_wider),
     ("rope", _rope_scaling_on_cos_only),
     ("rope", _rope_ignores_inv_freq),
+    ("qkv_proj_norm_rope_ref", _qkv_swapped_kv),
     ("prefill_ref", _prefill_mod_mapping),
     ("chunk_prefill_ref", _chunk_no_offset),
     ("chunk_prefill_ref", _chunk_rerotates_cache),
