@@ -316,6 +316,33 @@ int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
  * alignment slack; 0 when a size is not positive (start may be 0). */
 size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d);
 
+/*
+ * qwen3_qkv_proj_norm_rope - the merged q/k/v projection with QK-Norm and RoPE in the GEMM
+ * epilogue.  y = x w_qkv^T ("LLM Internals - Assembling a large model from scratch": one
+ * qkv_proj GEMM for the three projections), split into q [M, Hq, d], k [M, Hkv, d],
+ * v [M, Hkv, d]; q and k get QK-Norm (fp32 statistics of the fp32 accumulator) and RoPE at
+ * pos, then one bf16 rounding; v is stored as projected.
+ *   x         [M, hidden] bf16 token hidden states (hidden a multiple of 8).
+ *   w_qkv     [(Hq + 2 Hkv) d, hidden] bf16: q's Hq*d rows, then k's, then v's (the layout of
+ *             a PyTorch Linear weight, out x in).
+ *   pos       [M] int32 positions.
+ *   q_out, k_out, v_out  [M, Hq, d], [M, Hkv, d], [M, Hkv, d] bf16.
+ *   variant   the rope type (theta or a frequency table, attention_scaling); window unused.
+ *   workspace at least qwen3_qkv_proj_workspace_size(M) bytes (the RoPE table of the
+ *             tokens), else QWEN3_ERR_WORKSPACE.
+ * q_out and k_out are the normed, rotated vectors the attention entry points compute
+ * themselves from raw q and k.
+ */
+int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv,
+                             const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                             qwen3_bf16* q_out, qwen3_bf16* k_out, qwen3_bf16* v_out,
+                             int M, int hidden, int Hq, int Hkv, int d,
+                             const qwen3_attn_variant* variant, float eps,
+                             void* workspace, size_t ws_bytes, qwen3_stream_t stream);
+
+/* Scratch bytes qwen3_qkv_proj_norm_rope needs: ceil(M/128) * 64 KB; 0 when M <= 0. */
+size_t qwen3_qkv_proj_workspace_size(int M);
+
 /* Scratch bytes qwen3_attn_prefill_ex and qwen3_attn_prefill_chunk need: B*T*Hkv*d*2
  * (normed, rotated keys) + B*T*Hq*d*2 (normed, rotated queries), plus alignment slack;
  * 0 when a size is not positive. */

@@ -56,6 +56,8 @@ SIGNATURES = {
     "qwen3_attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(PagedKV), _I, _P, _Z,
                                       _I, _I, _I, _I, _I, _V, _F, _P]),
     "qwen3_attn_prefill_paged_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "qwen3_qkv_proj_norm_rope": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _V, _F, _P, _Z, _P]),
+    "qwen3_qkv_proj_workspace_size": (_Z, [_I]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
@@ -392,6 +394,44 @@ def prefill_paged(q, k, v, q_norm_w, k_norm_w, pos, k_pages, v_pages, block_tabl
                                           ws_bytes, B, T, Hq, Hkv, d, ctypes.byref(var), eps, _stream(dev)),
            "qwen3_attn_prefill_paged")
     return out
+
+
+def qkv_proj_workspace_size(M: int) -> int:
+    return int(lib().qwen3_qkv_proj_workspace_size(M))
+
+
+def qkv_proj_norm_rope(x, w_qkv, q_norm_w, k_norm_w, pos, Hq: int, Hkv: int, *, theta: float = 1.0e6,
+                       eps: float = 1.0e-6, inv_freq=None, attention_scaling: float = 1.0, q_out=None, k_out=None,
+                       v_out=None, workspace=None):
+    """The merged qkv projection with QK-Norm + RoPE in its epilogue: x [M, hidden] bf16,
+    w_qkv [(Hq + 2 Hkv) d, hidden] bf16, pos [M] int32.  Returns (q' [M,Hq,d], k' [M,Hkv,d],
+    v [M,Hkv,d]) bf16."""
+    dev = x.device
+    M, hidden = x.shape
+    d = HEAD_DIM
+    _need(x, "x", torch.bfloat16, (M, hidden), dev)
+    _need(w_qkv, "w_qkv", torch.bfloat16, ((Hq + 2 * Hkv) * d, hidden), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (M,), dev)
+    if q_out is None:
+        q_out = torch.empty((M, Hq, d), dtype=torch.bfloat16, device=dev)
+    if k_out is None:
+        k_out = torch.empty((M, Hkv, d), dtype=torch.bfloat16, device=dev)
+    if v_out is None:
+        v_out = torch.empty((M, Hkv, d), dtype=torch.bfloat16, device=dev)
+    _need(q_out, "q_out", torch.bfloat16, (M, Hq, d), dev)
+    _need(k_out, "k_out", torch.bfloat16, (M, Hkv, d), dev)
+    _need(v_out, "v_out", torch.bfloat16, (M, Hkv, d), dev)
+    if workspace is None:
+        workspace = torch.empty(qkv_proj_workspace_size(M), dtype=torch.uint8, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    var, _keep = make_variant(theta, inv_freq, attention_scaling, 0)
+    _check(lib().qwen3_qkv_proj_norm_rope(_ptr(x), _ptr(w_qkv), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos), _ptr(q_out),
+                                          _ptr(k_out), _ptr(v_out), M, hidden, Hq, Hkv, d, ctypes.byref(var), eps,
+                                          _ptr(workspace), ws_bytes, _stream(dev)),
+           "qwen3_qkv_proj_norm_rope")
+    return q_out, k_out, v_out
 
 
 NOALLOC_SCRATCH_BYTES = 48 << 20

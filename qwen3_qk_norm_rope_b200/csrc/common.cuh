@@ -32,6 +32,11 @@ enum Site : int {
   kSiteDecodeEmpty = 41,
   kSiteDecodeLen = 42,
   kSitePagedTable = 50,
+  kSiteQkvFull = 60,
+  kSiteQkvEmpty = 61,
+  kSiteQkvAcc = 62,
+  kSiteQkvRope = 63,
+  kSiteQkvDrain = 64,
 };
 
 // Device status word: [0] = first qwen3_status recorded, [1] = its site.

@@ -1,0 +1,300 @@
+// qkv_proj.cuh - the merged q/k/v projection with QK-Norm and RoPE in the GEMM epilogue.
+//
+// What it computes: y = x w_qkv^T for token hidden states x [M, hidden] and the stacked
+// projection weights w_qkv [(Hq + 2 Hkv) d, hidden] (q, k and v in one GEMM: "LLM Internals -
+// Assembling a large model from scratch", the comparison with inference engines: qkv_proj);
+// the q and k heads of y then get QK-Norm and rotate-half RoPE at their token's position
+// ("Hand-Writing a Vision-Language Model, Part 1", order of operations; "Qwen3 Architecture
+// Layer-by-Layer", Qwen3RMSNorm and apply_rotary_pos_emb), v is stored as projected.
+//
+// A head is 128 columns of y, so the accumulator of an N tile holds whole head vectors and
+// the norm needs no reduction across CTAs: the epilogue thread that owns a token row has its
+// head's 128 values in registers.  Normalising the fp32 accumulator directly also skips the
+// bf16 rounding the pages' path takes between the projection and q_norm.
+//
+// Tiles: 128 tokens x 256 columns (two heads), K in chunks of 64 (one 128B-swizzled row per
+// token).  Persistent CTAs take contiguous runs of tiles in token-tile-major order, so a run
+// mostly stays on one token tile and reuses its RoPE table.  Six warps:
+//   warp 0     TMA producer: x and w_qkv chunks into a 3-stage ring; the token tile's RoPE
+//              table (cos, sin per position and frequency, [64][128] float2, 64 KB) by one
+//              bulk copy when the run moves to a new token tile; owns TMEM.
+//   warp 1     MMA issuer (one thread): tcgen05.mma M=128 N=256 K=16, 4 per chunk, into one
+//              of two TMEM accumulators (256 columns each), so the epilogue of a tile
+//              overlaps the next tile's MMAs.
+//   warps 2-5  epilogue, one thread per token row (TMEM lane quadrant = warp % 4): per head,
+//              tcgen05.ld of 128 fp32, then for q and k heads the sum of squares, 1/rms,
+//              gain and the rotation from the table; bf16 rows to q_out / k_out / v_out.
+#pragma once
+#include "common.cuh"
+
+namespace q3 {
+
+struct QkvParams {
+  const float* q_norm_w;  // [d]
+  const float* k_norm_w;  // [d]
+  const float2* rope;     // [ceil(M/128)][64][128]: (cos, sin) x attention_scaling
+  uint4* q_out;           // [M, Hq, d] bf16
+  uint4* k_out;           // [M, Hkv, d]
+  uint4* v_out;           // [M, Hkv, d]
+  int M, hidden, Hq, Hkv, n_heads, n_mt, n_nt, n_tiles, n_k;
+  float eps;
+  WaitCfg wait;
+};
+
+constexpr int kQkvThreads = 192;
+constexpr int kQkvStages = 3;
+constexpr uint32_t kQkA = 16384;                  // 128 tokens x 64 bf16
+constexpr uint32_t kQkB = 32768;                  // 256 columns x 64 bf16
+constexpr uint32_t kQkStage = kQkA + kQkB;
+constexpr uint32_t kQkRope = kQkvStages * kQkStage;  // 64 KB table
+constexpr uint32_t kQkGain = kQkRope + 65536;        // q gain, k gain: 2 x 512 B
+constexpr uint32_t kQkBar = kQkGain + 1024;
+// barrier block: full[3], empty[3], acc_full[2], acc_empty[2], rope_full, rope_empty, done, tmem slot
+constexpr uint32_t kQbFull = 0, kQbEmpty = 24, kQbAccFull = 48, kQbAccEmpty = 64, kQbRopeFull = 80,
+                   kQbRopeEmpty = 88, kQbDone = 96, kQbTmem = 104, kQbAbort = 108;
+constexpr uint32_t kQkvSmemBytes = kQkBar + 128 + 1024;
+
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+// The RoPE table of every token tile: entry [mt][i][r] = (cos, sin)(pos[mt*128 + r] * inv_i)
+// times attention_scaling; rows past M use position 0.
+struct QkvRopeParams {
+  const int* pos;
+  float2* rope;
+  int M, n_mt;
+  float scale;
+  RopeTable tab;
+};
+
+__global__ void __launch_bounds__(256) qkv_rope_table_kernel(const __grid_constant__ QkvRopeParams p) {
+  const long long total = static_cast<long long>(p.n_mt) * 64 * 128;
+  for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(e & 127);
+    const int i = static_cast<int>((e >> 7) & 63);
+    const long long m = (e >> 13) * 128 + r;
+    const int ps = m < p.M ? p.pos[m] : 0;
+    float s, c;
+    rope_sincos(ps, p.tab.hi[i], p.tab.lo[i], s, c);
+    p.rope[e] = make_float2(c * p.scale, s * p.scale);
+  }
+}
+
+__device__ __forceinline__ void qkv_tile_coords(const QkvParams& p, int tile, int& mt, int& nt) {
+  mt = tile / p.n_nt;
+  nt = tile - mt * p.n_nt;
+}
+
+__global__ void __launch_bounds__(kQkvThreads, 1)
+    qkv_proj_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                    const __grid_constant__ QkvParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sgen = smem_raw + (sb - raw);
+  const uint32_t bar = sb + kQkBar;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kQkBar + kQbAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + kQkBar + kQbTmem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // this CTA's run of tiles
+  const int per = (p.n_tiles + gridDim.x - 1) / gridDim.x;
+  const int t_begin = blockIdx.x * per;
+  const int t_end = min(p.n_tiles, t_begin + per);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kQkvStages; ++s) {
+      mbar_init(bar + kQbFull + 8 * s, 1);
+      mbar_init(bar + kQbEmpty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar + kQbAccFull + 8 * b, 1);
+      mbar_init(bar + kQbAccEmpty + 8 * b, 128);
+    }
+    mbar_init(bar + kQbRopeFull, 1);
+    mbar_init(bar + kQbRopeEmpty, 128);
+    mbar_init(bar + kQbDone, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+    fence_proxy_async_smem();
+  }
+  if (threadIdx.x < 128) {  // gains into shared memory
+    float* sg = reinterpret_cast<float*>(sgen + kQkGain);
+    sg[threadIdx.x] = p.q_norm_w[threadIdx.x];
+    sg[128 + threadIdx.x] = p.k_norm_w[threadIdx.x];
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_map(&tmX);
+      tma_prefetch_map(&tmW);
+      int last[kQkvStages] = {-1, -1, -1};
+      uint32_t it = 0, rope_uses = 0;
+      int cur_mt = -1;
+      bool ok = true;
+      for (int tile = t_begin; tile < t_end && ok; ++tile) {
+        int mt, nt;
+        qkv_tile_coords(p, tile, mt, nt);
+        if (mt != cur_mt) {  // the run reaches a new token tile: its RoPE table
+          if (rope_uses >= 1 &&
+              !mbar_wait(bar + kQbRopeEmpty, (rope_uses - 1) & 1, p.wait, abort_flag, kSiteQkvRope)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar + kQbRopeFull, 65536);
+          bulk_copy_g2s(sb + kQkRope, p.rope + static_cast<size_t>(mt) * 64 * 128, 65536, bar + kQbRopeFull);
+          ++rope_uses;
+          cur_mt = mt;
+        }
+        for (int kc = 0; kc < p.n_k; ++kc, ++it) {
+          const int st = static_cast<int>(it % kQkvStages);
+          const uint32_t ph = (it / kQkvStages) & 1;
+          if (it >= kQkvStages &&
+              !mbar_wait(bar + kQbEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSiteQkvEmpty)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sb + st * kQkStage;
+          mbar_arrive_expect_tx(bar + kQbFull + 8 * st, kQkStage);
+          tma_load_2d(dst, &tmX, bar + kQbFull + 8 * st, kc * 64, mt * 128);
+          tma_load_2d(dst + kQkA, &tmW, bar + kQbFull + 8 * st, kc * 64, nt * 256);
+          last[st] = static_cast<int>(it);
+        }
+      }
+      for (int s = 0; s < kQkvStages; ++s)
+        if (last[s] >= 0)
+          mbar_wait(bar + kQbFull + 8 * s, (last[s] / kQkvStages) & 1, p.wait, nullptr, kSiteQkvDrain);
+      if (rope_uses >= 1) mbar_wait(bar + kQbRopeFull, (rope_uses - 1) & 1, p.wait, nullptr, kSiteQkvDrain);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kId = idesc_bf16(128, 256, false);  // A = x rows, B = w rows, both K-major
+      uint32_t it = 0;
+      bool ok = true;
+      int n = 0;
+      for (int tile = t_begin; tile < t_end && ok; ++tile, ++n) {
+        const int buf = n & 1;
+        if (n >= 2 && !mbar_wait(bar + kQbAccEmpty + 8 * buf, ((n >> 1) - 1) & 1, p.wait, abort_flag, kSiteQkvAcc)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(buf * 256);
+        for (int kc = 0; kc < p.n_k; ++kc, ++it) {
+          const int st = static_cast<int>(it % kQkvStages);
+          if (!mbar_wait(bar + kQbFull + 8 * st, (it / kQkvStages) & 1, p.wait, abort_flag, kSiteQkvFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sb + st * kQkStage, sbw = sa + kQkA;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_ss(acc, smem_desc_sw128(sa + kk * 32, 16, 1024), smem_desc_sw128(sbw + kk * 32, 16, 1024), kId,
+                      (kc > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(bar + kQbEmpty + 8 * st);
+        }
+        if (!ok) break;
+        tc_commit(bar + kQbAccFull + 8 * buf);
+      }
+      tc_commit(bar + kQbDone);
+      mbar_wait(bar + kQbDone, 0, p.wait, nullptr, kSiteQkvDrain);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;  // token row of the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float* sg = reinterpret_cast<const float*>(sgen + kQkGain);
+    const float2* srope = reinterpret_cast<const float2*>(sgen + kQkRope);
+    uint32_t rope_uses = 0;
+    int cur_mt = -1;
+    bool ok = true;
+    int n = 0;
+    for (int tile = t_begin; tile < t_end && ok; ++tile, ++n) {
+      int mt, nt;
+      qkv_tile_coords(p, tile, mt, nt);
+      if (mt != cur_mt) {
+        if (rope_uses >= 1) mbar_arrive(bar + kQbRopeEmpty);  // done with the previous token tile's table
+        ok = mbar_wait(bar + kQbRopeFull, rope_uses & 1, p.wait, abort_flag, kSiteQkvRope);
+        ++rope_uses;
+        cur_mt = mt;
+        if (!ok) break;
+      }
+      const int buf = n & 1;
+      ok = mbar_wait(bar + kQbAccFull + 8 * buf, (n >> 1) & 1, p.wait, abort_flag, kSiteQkvAcc);
+      if (!ok) break;
+      tc_fence_after();
+      const long long m = static_cast<long long>(mt) * 128 + row;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int h = nt * 2 + hh;  // head index in [q heads | k heads | v heads]
+        uint32_t y[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_off + static_cast<uint32_t>(buf * 256 + hh * 128 + c * 32), r);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[c * 32 + i] = r[i];
+        }
+        if (hh == 1) {  // both heads are in registers or stored: the accumulator is free
+          tc_fence_before();
+          mbar_arrive(bar + kQbAccEmpty + 8 * buf);
+        }
+        if (h >= p.n_heads || m >= p.M) continue;
+        uint4* dst;
+        if (h < p.Hq + p.Hkv) {
+          // QK-Norm: 1/rms of the fp32 row, then gain and rotate-half RoPE, pairs (i, i+64)
+          const bool is_q = h < p.Hq;
+          const float* g = sg + (is_q ? 0 : 128);
+          float ss = 0.f;
+#pragma unroll
+          for (int i = 0; i < 128; ++i) ss = fmaf(__uint_as_float(y[i]), __uint_as_float(y[i]), ss);
+          const float rn = rsqrtf(fmaf(ss, 1.0f / kD, p.eps));
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const float2 cs = srope[i * 128 + row];
+            const float a = g[i] * (__uint_as_float(y[i]) * rn);
+            const float b = g[64 + i] * (__uint_as_float(y[64 + i]) * rn);
+            y[i] = __float_as_uint(a * cs.x - b * cs.y);
+            y[64 + i] = __float_as_uint(b * cs.x + a * cs.y);
+          }
+          dst = is_q ? p.q_out + (m * p.Hq + h) * (kD / 8) : p.k_out + (m * p.Hkv + (h - p.Hq)) * (kD / 8);
+        } else {
+          dst = p.v_out + (m * p.Hkv + (h - p.Hq - p.Hkv)) * (kD / 8);
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(y[8 * c + 0]), __uint_as_float(y[8 * c + 1]));
+          w.y = pack_bf16x2(__uint_as_float(y[8 * c + 2]), __uint_as_float(y[8 * c + 3]));
+          w.z = pack_bf16x2(__uint_as_float(y[8 * c + 4]), __uint_as_float(y[8 * c + 5]));
+          w.w = pack_bf16x2(__uint_as_float(y[8 * c + 6]), __uint_as_float(y[8 * c + 7]));
+          dst[c] = w;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace q3

@@ -13,6 +13,7 @@
 #include "prefill.cuh"
 #include "paged.cuh"
 #include "prologue.cuh"
+#include "qkv_proj.cuh"
 
 namespace {
 
@@ -163,6 +164,9 @@ int ensure_kernel_attrs() {
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kDecodeSmemBytes) != cudaSuccess)
+    return QWEN3_ERR_CUDA;
+  if (cudaFuncSetAttribute(q3::qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kQkvSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   done[dev] = true;
   return QWEN3_OK;
@@ -695,6 +699,85 @@ int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
   if ((st = make_paged(kv, Hkv, pg)) != QWEN3_OK) return st;
   return prefill_impl(q, k, v, q_norm_w, k_norm_w, pos, out, lse, nullptr, nullptr, start, 0, workspace, ws_bytes, B,
                       T, Hq, Hkv, d, var, eps, stream, &pg);
+}
+
+size_t qwen3_qkv_proj_workspace_size(int M) {
+  if (M <= 0) return 0;
+  return static_cast<size_t>((M + 127) / 128) * 64 * 128 * sizeof(float2) + 256;  // the RoPE table
+}
+
+int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const float* q_norm_w,
+                             const float* k_norm_w, const int32_t* pos, qwen3_bf16* q_out, qwen3_bf16* k_out,
+                             qwen3_bf16* v_out, int M, int hidden, int Hq, int Hkv, int d,
+                             const qwen3_attn_variant* variant, float eps, void* workspace, size_t ws_bytes,
+                             qwen3_stream_t stream) {
+  Variant var;
+  int st = make_variant(variant, var);
+  if (st != QWEN3_OK) return st;
+  if (x == nullptr || w_qkv == nullptr || q_norm_w == nullptr || k_norm_w == nullptr || pos == nullptr ||
+      q_out == nullptr || k_out == nullptr || v_out == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (M <= 0 || hidden <= 0 || Hq <= 0 || Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
+  if (d != kD) return QWEN3_ERR_UNSUPPORTED;
+  if (hidden % 8 != 0) return QWEN3_ERR_UNSUPPORTED;  // 16-byte rows for TMA
+  if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(q_out, 16) || !aligned(k_out, 16) || !aligned(v_out, 16) ||
+      !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) || !aligned(pos, 4))
+    return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < qwen3_qkv_proj_workspace_size(M)) return QWEN3_ERR_WORKSPACE;
+  const int n_heads = Hq + 2 * Hkv;
+  if (static_cast<long long>(n_heads) * kD > 0x7fffffffLL || static_cast<long long>(M) * n_heads > 0x7fffffffLL)
+    return QWEN3_ERR_UNSUPPORTED;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
+  const int n_mt = (M + 127) / 128;
+  float2* rope = reinterpret_cast<float2*>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255));
+  {
+    q3::QkvRopeParams rp;
+    rp.pos = pos;
+    rp.rope = rope;
+    rp.M = M;
+    rp.n_mt = n_mt;
+    rp.scale = var.scale;
+    rp.tab = var.rope;
+    const long long total = static_cast<long long>(n_mt) * 64 * 128;
+    long long blocks = (total + 255) / 256;
+    if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
+    q3::qkv_rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(rp);
+    if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+  }
+  CUtensorMap mx, mw;
+  {
+    const cuuint64_t xd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(M)};
+    const cuuint64_t xs[1] = {static_cast<cuuint64_t>(hidden) * 2ull};
+    const cuuint32_t xb[2] = {64, 128};
+    const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(n_heads) * kD};
+    const cuuint32_t wb[2] = {64, 256};
+    if (!make_map(&mx, x, 2, xd, xs, xb) || !make_map(&mw, w_qkv, 2, wd, xs, wb)) return QWEN3_ERR_CUDA;
+  }
+  q3::QkvParams p;
+  p.q_norm_w = q_norm_w;
+  p.k_norm_w = k_norm_w;
+  p.rope = rope;
+  p.q_out = reinterpret_cast<uint4*>(q_out);
+  p.k_out = reinterpret_cast<uint4*>(k_out);
+  p.v_out = reinterpret_cast<uint4*>(v_out);
+  p.M = M;
+  p.hidden = hidden;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.n_heads = n_heads;
+  p.n_mt = n_mt;
+  p.n_nt = (n_heads + 1) / 2;
+  const long long n_tiles = static_cast<long long>(p.n_mt) * p.n_nt;
+  if (n_tiles > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  p.n_tiles = static_cast<int>(n_tiles);
+  p.n_k = (hidden + 63) / 64;
+  p.eps = eps;
+  p.wait = next_wait_cfg();
+  const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
+  q3::qkv_proj_kernel<<<grid, q3::kQkvThreads, q3::kQkvSmemBytes, s>>>(mx, mw, p);
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
 int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new,

@@ -166,6 +166,47 @@ def chunk_inputs(shape: ChunkShape, seed: int = 0) -> dict:
     }
 
 
+@dataclass(frozen=True)
+class QkvShape:
+    """A merged qkv projection: M tokens of `hidden` features to Hq + 2 Hkv heads of d."""
+    name: str
+    M: int
+    hidden: int
+    Hq: int
+    Hkv: int
+    d: int = HEAD_DIM
+    theta: float = ROPE_THETA
+    eps: float = RMS_EPS
+
+    def flops(self) -> float:
+        return 2.0 * self.M * self.hidden * (self.Hq + 2 * self.Hkv) * self.d
+
+
+QKV_SHAPES = {
+    "qwen3-0.6b-qkv": QkvShape("Qwen3-0.6B-shaped qkv projection M=4096 hidden=1024 Hq=16 Hkv=8", 4096, 1024, 16, 8),
+    "qwen3-4b-qkv": QkvShape("Qwen3-4B-shaped qkv projection M=8192 hidden=2560 Hq=32 Hkv=8", 8192, 2560, 32, 8),
+}
+
+
+def qkv_proj_inputs(shape: QkvShape, seed: int = 0) -> dict:
+    """Hidden states x ~ N(0,1) [M, hidden] and stacked weights w_qkv ~ N(0, 1/hidden)
+    [(Hq + 2 Hkv) d, hidden], the q and k rows multiplied per output channel by scale
+    vectors s_q, s_k (log-uniform in [0.5, 4], as the prefill recipe scales q and k), all
+    bf16; gains 1 + 0.1 N(0,1) fp32; positions 0..M-1 int32."""
+    rng = np.random.default_rng(seed)
+    d = shape.d
+    x = rng.standard_normal((shape.M, shape.hidden), dtype=np.float32)
+    w = rng.standard_normal(((shape.Hq + 2 * shape.Hkv) * d, shape.hidden), dtype=np.float32)
+    w *= np.float32(1.0 / np.sqrt(shape.hidden))
+    s_q, s_k = _scales(rng, d), _scales(rng, d)
+    g_q, g_k = _gains(rng, d), _gains(rng, d)
+    nq, nk = shape.Hq * d, shape.Hkv * d
+    w[:nq] *= np.tile(s_q, shape.Hq)[:, None]
+    w[nq:nq + nk] *= np.tile(s_k, shape.Hkv)[:, None]
+    return {"x": _bf16(x), "w_qkv": _bf16(w), "q_norm_w": torch.from_numpy(g_q), "k_norm_w": torch.from_numpy(g_k),
+            "pos": torch.arange(shape.M, dtype=torch.int32)}
+
+
 def decode_step_inputs(shape: DecodeShape, seed: int = 0) -> dict:
     """The new token of every sequence plus the cached lengths.
 

@@ -1,0 +1,86 @@
+"""The merged qkv projection with QK-Norm + RoPE in the GEMM epilogue, through the C ABI,
+against the fp64 oracle (oracle.qkv_proj_norm_rope_ref) on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qwen3_qk_norm_rope_b200 as qa
+from synthetic import QKV_SHAPES, QkvShape, as_f64, qkv_proj_inputs
+from tests.gpu_common import assert_status_ok, dev, to_np
+
+pytestmark = pytest.mark.gpu
+THETA, EPS = 1.0e6, 1.0e-6
+
+
+def _run(shape: QkvShape, seed: int, inv_freq=None, scaling=1.0, pos=None):
+    inp = qkv_proj_inputs(shape, seed=seed)
+    if pos is not None:
+        inp["pos"] = pos
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items()}
+    q, k, v = qa.qkv_proj_norm_rope(t["x"], t["w_qkv"], t["q_norm_w"], t["k_norm_w"], t["pos"], shape.Hq, shape.Hkv,
+                                    inv_freq=inv_freq, attention_scaling=scaling)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    ref = oracle.qkv_proj_norm_rope_ref(as_f64(inp["x"]), as_f64(inp["w_qkv"]), as_f64(inp["q_norm_w"]),
+                                        as_f64(inp["k_norm_w"]), inp["pos"].numpy(), shape.Hq, shape.Hkv, THETA, EPS,
+                                        inv_freq=inv_freq, scaling=scaling)
+    return (to_np(q), to_np(k), to_np(v)), ref
+
+
+def _check(got, ref, what):
+    # fp32 accumulation of exact bf16 products (relative error ~ hidden * 2^-24), the norm and
+    # rotation in fp32, then one bf16 rounding (2^-9 relative): 2^-8 |ref| plus a small
+    # absolute term for entries near zero, scaled to the tensor's RMS.
+    for name, g, r in zip("qkv", got, ref):
+        assert np.isfinite(g).all(), f"{what} {name}: non-finite"
+        rms = np.sqrt(np.mean(r * r))
+        err = np.abs(g - r)
+        bound = np.abs(r) * 2.0 ** -8 + 2e-3 * rms
+        assert np.all(err <= bound), f"{what} {name}: worst excess {(err - bound).max():.3e} (rms {rms:.3f})"
+        assert err.mean() <= 2.0 ** -9 * np.mean(np.abs(r)) + 1e-4 * rms, f"{what} {name}: mean {err.mean():.3e}"
+
+
+@pytest.mark.parametrize("M,hidden,Hq,Hkv", [
+    (300, 256, 4, 2),    # M off the 128-row tile, hidden a few chunks
+    (128, 200, 3, 3),    # an odd head count (the last tile holds one head), hidden off the 64-chunk
+    (1000, 512, 16, 8),  # several token tiles per CTA run
+])
+def test_qkv_proj_small(M, hidden, Hq, Hkv):
+    shape = QkvShape("qkv small", M, hidden, Hq, Hkv)
+    got, ref = _run(shape, seed=M + hidden)
+    _check(got, ref, f"M{M} hidden{hidden} Hq{Hq} Hkv{Hkv}")
+
+
+def test_qkv_proj_full_size():
+    shape = QKV_SHAPES["qwen3-0.6b-qkv"]
+    got, ref = _run(shape, seed=0)
+    _check(got, ref, shape.name)
+
+
+def test_qkv_proj_rope_variant_and_positions():
+    shape = QkvShape("qkv variant", 384, 256, 8, 4)
+    i = np.arange(64, dtype=np.float64)
+    inv = (1e6 ** (-2.0 * i / 128)) / np.where(i > 40, 4.0, 1.0)  # a rescaled table
+    pos = torch.from_numpy(np.random.default_rng(5).integers(0, 40000, size=384).astype(np.int32))
+    got, ref = _run(shape, seed=7, inv_freq=inv, scaling=1.1, pos=pos)
+    _check(got, ref, "table + scaling, gapped positions")
+
+
+def test_qkv_proj_feeds_the_prologue_definition():
+    """Its q', k' are the normed, rotated vectors the attention entry points build from raw q
+    and k: applying the standalone prologue kernel to the projection's raw output (taken
+    from the oracle's fp64 product, rounded to bf16) agrees within the two bf16 roundings."""
+    shape = QkvShape("qkv vs prologue", 256, 256, 4, 2)
+    inp = qkv_proj_inputs(shape, seed=11)
+    (q, k, v), _ = _run(shape, seed=11)
+    y = as_f64(inp["x"]) @ as_f64(inp["w_qkv"]).T
+    d = dev()
+    qraw = torch.from_numpy(y[:, :4 * 128].reshape(1, 256, 4, 128).astype(np.float32)).to(torch.bfloat16).to(d)
+    dst = torch.empty((1, 4, 256, 128), dtype=torch.bfloat16, device=d)
+    qa.qk_norm_rope(qraw, inp["q_norm_w"].to(d), inp["pos"][None].to(d), dst)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    via_prologue = to_np(dst[0].permute(1, 0, 2))
+    assert np.allclose(q, via_prologue, rtol=2.0 ** -6, atol=2e-2)
