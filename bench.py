@@ -12,6 +12,7 @@ prologue is counted as free work); the decode throughput in GB/s rides along und
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --workload chunked-prefill    # the chunked-prefill call alone
+    python bench.py --workload qkv-proj           # the merged qkv projection + QK-Norm/RoPE
 
 The chunked-prefill workload times qwen3_attn_prefill_chunk on the Qwen3-4B-shaped
 second chunk (B=1, 4096 new tokens over 4096 cached, Hq=32, Hkv=8) and prints its own
@@ -36,8 +37,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, chunk_inputs, decode_step_inputs, \
-    prefill_inputs  # noqa: E402
+from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, QKV_SHAPES, chunk_inputs, decode_step_inputs, \
+    prefill_inputs, qkv_proj_inputs  # noqa: E402
 
 METRIC = "causal GQA attn TFLOP/s (+QK-Norm/RoPE) % bf16 peak; decode HBM GB/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -478,6 +479,134 @@ def run_chunk(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------ qkv projection
+QKV_METRIC = "merged qkv projection GEMM TFLOP/s (QK-Norm + RoPE epilogue) % bf16 peak"
+
+
+def cpu_oracle_qkv_sample(name: str, rows: int = 256, seed: int = 0):
+    """The oracle's projection + QK-Norm + RoPE on the first `rows` tokens of the workload."""
+    import oracle
+    from synthetic import as_f64
+
+    sh = QKV_SHAPES[name]
+    inp = qkv_proj_inputs(sh, seed=seed)
+    t0 = time.perf_counter()
+    oracle.qkv_proj_norm_rope_ref(as_f64(inp["x"][:rows]), as_f64(inp["w_qkv"]), as_f64(inp["q_norm_w"]),
+                                  as_f64(inp["k_norm_w"]), inp["pos"][:rows].numpy(), sh.Hq, sh.Hkv, sh.theta, sh.eps)
+    secs = time.perf_counter() - t0
+    flops = 2.0 * rows * sh.hidden * (sh.Hq + 2 * sh.Hkv) * sh.d
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "flops": flops,
+            "sample": f"first {rows} of {sh.M} tokens of the {sh.name} ({flops:.3g} flops)"}
+
+
+def run_qkv(args, world, rank, local):
+    name = args.qkv
+    sh = QKV_SHAPES[name]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        secs = flops = 0.0
+        res = None
+        for _ in range(args.steps):
+            res = cpu_oracle_qkv_sample(name, rows=256)
+            secs += res["seconds"]
+            flops += res["flops"]
+        value = flops / secs / 1e12
+        line = {"impl": "reference", "metric": QKV_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": sh.name},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
+                                 "sample": "per step, " + res["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    import qwen3_qk_norm_rope_b200 as qa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    host = qkv_proj_inputs(sh, seed=0)
+    t = {k: v.to(dev) for k, v in host.items()}
+    outs = (torch.empty((sh.M, sh.Hq, sh.d), dtype=torch.bfloat16, device=dev),
+            torch.empty((sh.M, sh.Hkv, sh.d), dtype=torch.bfloat16, device=dev),
+            torch.empty((sh.M, sh.Hkv, sh.d), dtype=torch.bfloat16, device=dev))
+    ws = torch.empty(qa.qkv_proj_workspace_size(sh.M), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        qa.qkv_proj_norm_rope(t["x"], t["w_qkv"], t["q_norm_w"], t["k_norm_w"], t["pos"], sh.Hq, sh.Hkv,
+                              q_out=outs[0], k_out=outs[1], v_out=outs[2], workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.fill_(1.0)
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+    st, site = qa.device_status(clear=True, device=dev)
+    if st != qa.OK:
+        raise RuntimeError(f"device status {qa.status_string(st)} at site {site}")
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    ph = {k: v.pin_memory() for k, v in host.items()}
+    oh = [torch.empty(o.shape, dtype=torch.bfloat16).pin_memory() for o in outs]
+    h2d = sum(v.numel() * v.element_size() for v in ph.values())
+    d2h = sum(o.numel() * 2 for o in oh)
+    e_steps = max(1, min(K, 100))
+    e_ms = 0.0
+    for _ in range(e_steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k, v in ph.items():
+            t[k].copy_(v, non_blocking=True)
+        step()
+        for o, h in zip(outs, oh):
+            h.copy_(o, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        e_ms += e0.elapsed_time(e1)
+    ms, e_ms = max_over_ranks(world, [ms, e_ms], dev)
+    if rank != 0:
+        return
+    flops = sh.flops()
+    achieved = flops / (ms * 1e-3 / K) / 1e12
+    line = {"metric": QKV_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": sh.name, "M": sh.M, "hidden": sh.hidden, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+                       "l2": "flushed before every step (256 MiB write, outside the timed windows)",
+                       "parallelism": "replicas (one independent workload per GPU)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "qkv projection call (RoPE table + GEMM with the norm/rope epilogue)",
+                         "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
+            "gpu_launches": 2 * K, "clocks": clk.summary(),
+            "e2e": {"value": world * flops * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "ms_per_step": e_ms / e_steps}}
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_qkv_sample(name, rows=sh.M)
+        line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
+                                "sample": cb["sample"], "seconds": cb["seconds"]}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------------------ main
 def dist_setup(backend: str = "nccl"):
     """One process per GPU (torchrun env).  The process group only carries the timing
@@ -569,13 +698,16 @@ def main():
                     help="prefill workload of the step (profiling of the other shapes)")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="decode the first n of the 64 sequences (small cases for ncu captures)")
-    ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill"],
-                    help="step: 0.6B prefill + batched decode (default); chunked-prefill: the chunk call alone")
+    ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill", "qkv-proj"],
+                    help="step: 0.6B prefill + batched decode (default); chunked-prefill: the chunk call alone; "
+                         "qkv-proj: the merged projection with the QK-Norm/RoPE epilogue")
+    ap.add_argument("--qkv", default="qwen3-0.6b-qkv", choices=sorted(QKV_SHAPES),
+                    help="the qkv-proj workload's shape")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup("nccl")
-    if args.workload == "chunked-prefill":
-        run_chunk(args, world, rank, local)
+    if args.workload in ("chunked-prefill", "qkv-proj"):
+        (run_chunk if args.workload == "chunked-prefill" else run_qkv)(args, world, rank, local)
         if world > 1:
             import torch.distributed as dist
 
