@@ -66,8 +66,8 @@ def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
 # DRAM traffic of the decode split-KV kernel per cached token (dram__bytes_read.sum +
 # dram__bytes_write.sum of one ncu capture of a smaller case, divided by its cached tokens),
 # valid only for the kernel source it was measured on.  Refreshed with each new capture.
-DECODE_TRAFFIC = {"src_sha256": "f9d0ff22d1b944a29783c29346ec878f23d53bdc66c476d421fb02983b9a3ff2",
-                  "bytes_per_cached_token": (630.630656e6 + 5.910528e6) / 153639}
+DECODE_TRAFFIC = {"src_sha256": "65820a30e1e2921678f67e2648cdf0c555a6a54bee07c421d033d25db85efed8",
+                  "bytes_per_cached_token": (630.653696e6 + 6.289664e6) / 153639}
 
 
 def decode_src_sha256() -> str:

@@ -99,8 +99,10 @@ struct TileInfo {
 
 // First key tile of a pair item: 0, or with a sliding window the tile holding the first key
 // that tile A's first row may see (tile B's rows start later, so they mask one tile at most).
+template <bool kWin>
 __device__ __forceinline__ int item_lo(const PrefillParams& p, int pair) {
-  return p.window > 0 ? max(0, p.start + 2 * pair * p.P - p.window + 1) >> 7 : 0;
+  if constexpr (!kWin) return 0;
+  return max(0, p.start + 2 * pair * p.P - p.window + 1) >> 7;
 }
 
 __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt, int lo) {
@@ -127,6 +129,9 @@ __device__ __forceinline__ void item_coords(const PrefillParams& p, int item, in
   hkv = bh % p.Hkv;
 }
 
+// kWin: a sliding window is set (p.window > 0); the full-causal instance carries none of its
+// masks or bookkeeping.
+template <bool kWin>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -179,7 +184,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
-        const int lo = item_lo(p, pair);
+        const int lo = item_lo<kWin>(p, pair);
         const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X) {
@@ -236,7 +241,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
         item_coords(p, item, pair, b, hkv);
-        const int lo = item_lo(p, pair);
+        const int lo = item_lo<kWin>(p, pair);
         const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X)
@@ -347,14 +352,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
       int pair, b, hkv;
       item_coords(p, item, pair, b, hkv);
-      const int lo = item_lo(p, pair);
+      const int lo = item_lo<kWin>(p, pair);
       const TileInfo ti = tile_info(p, 2 * pair + X, lo);
       if (ti.nkv == 0) continue;  // this item has no tile X
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
       const int lim = p.start + min(t_row, p.T - 1);  // last key index this row may see
-      const int wfirst = p.window > 0 ? lim - p.window + 1 : 0;  // first one, with a window
+      const int wfirst = kWin ? lim - p.window + 1 : 0;  // first one, with a window
       float m = fast ? bnd : -INFINITY, l = 0.f;
       for (int j = 0; j < ti.nkv; ++j) {
         ok = mbar_wait(bar + kBSFull + 8 * X, s_cnt & 1, p.wait, abort_flag, kSitePrefillSFull);
@@ -364,7 +369,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         const int kv0 = (lo + j) * 128;
         // some key of this tile lies past some row's limit, or before some row's window
-        const bool diag = kv0 + 127 > p.start + t0 || (p.window > 0 && kv0 < p.start + t0 + p.P - p.window);
+        const bool diag = kv0 + 127 > p.start + t0 || (kWin && kv0 < p.start + t0 + p.P - p.window);
         if (fast) {
           // One pass in four 32-column chunks, the next chunk's TMEM load in flight while the
           // current one is processed.  bf16 P goes to S columns [0,64): chunk c of P
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
               for (int i = 0; i < 32; ++i) {
                 const int key = kv0 + 32 * c + i;
-                cur[i] = (key <= lim && key >= wfirst) ? cur[i] : 0xff800000u;  // -inf
+                cur[i] = (key <= lim && (!kWin || key >= wfirst)) ? cur[i] : 0xff800000u;  // -inf
               }
             }
             uint32_t pk[16];
@@ -421,7 +426,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
               const int key = kv0 + 64 * hh + c;
-              sr[c] = (key <= lim && key >= wfirst) ? sr[c] : 0xff800000u;  // -inf
+              sr[c] = (key <= lim && (!kWin || key >= wfirst)) ? sr[c] : 0xff800000u;  // -inf
             }
           }
 #pragma unroll
@@ -439,7 +444,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // columns.  P occupies S columns [0,64): chunk c of P (columns [16c,16c+16)) only
         // overwrites S columns that chunks 0..c have already read.
         // a row whose keys so far all lie outside its window has no max yet: p = 0 for it
-        const float mref = m_new == -INFINITY ? 0.0f : m_new;
+        const float mref = (kWin && m_new == -INFINITY) ? 0.0f : m_new;
         const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(-mref, -mref);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -450,7 +455,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int key = kv0 + 32 * c + i;
-              sr[i] = (key <= lim && key >= wfirst) ? sr[i] : 0xff800000u;
+              sr[i] = (key <= lim && (!kWin || key >= wfirst)) ? sr[i] : 0xff800000u;
             }
           }
           uint32_t pk[16];

@@ -159,7 +159,9 @@ int ensure_kernel_attrs() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QWEN3_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   if (done[dev]) return QWEN3_OK;
-  if (cudaFuncSetAttribute(q3::fmha_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(q3::fmha_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kPrefillSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::fmha_prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -501,7 +503,9 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel, mq, mk, mv, mo, p) != cudaSuccess) {
+  const cudaError_t le = var.window > 0 ? cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<true>, mq, mk, mv, mo, p)
+                                        : cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false>, mq, mk, mv, mo, p);
+  if (le != cudaSuccess) {
     (void)cudaGetLastError();
     return QWEN3_ERR_CUDA;
   }
