@@ -13,8 +13,13 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "qwen3_attn.cu")
 LIB = os.path.join(PKG, "libqwen3attn.so")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("qwen3_attn.cu", "common.cuh", "prologue.cuh", "prefill.cuh",
-                                                "decode.cuh")] + [os.path.join(ROOT, "include", "qwen3_attn.h")]
+
+
+def deps() -> list[str]:
+    """Every source the library is built from: the .cu, its headers and the C ABI header."""
+    csrc = os.path.join(PKG, "csrc")
+    return sorted(os.path.join(csrc, f) for f in os.listdir(csrc) if f.endswith((".cu", ".cuh"))) + \
+        [os.path.join(ROOT, "include", "qwen3_attn.h")]
 
 
 def nvcc_path() -> str:
@@ -36,7 +41,7 @@ def up_to_date() -> bool:
     if not os.path.exists(LIB):
         return False
     t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(d) <= t for d in DEPS)
+    return all(os.path.getmtime(d) <= t for d in deps())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

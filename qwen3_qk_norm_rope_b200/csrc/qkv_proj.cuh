@@ -14,16 +14,18 @@
 //
 // Tiles: 128 tokens x 256 columns (two heads), K in chunks of 64 (one 128B-swizzled row per
 // token).  Persistent CTAs take contiguous runs of tiles in token-tile-major order, so a run
-// mostly stays on one token tile and reuses its RoPE table.  Six warps:
-//   warp 0     TMA producer: x and w_qkv chunks into a 3-stage ring; the token tile's RoPE
-//              table (cos, sin per position and frequency, [64][128] float2, 64 KB) by one
-//              bulk copy when the run moves to a new token tile; owns TMEM.
+// mostly stays on one token tile.  Six warps:
+//   warp 0     TMA producer: x and w_qkv chunks into a 4-stage ring; owns TMEM.
 //   warp 1     MMA issuer (one thread): tcgen05.mma M=128 N=256 K=16, 4 per chunk, into one
 //              of two TMEM accumulators (256 columns each), so the epilogue of a tile
 //              overlaps the next tile's MMAs.
 //   warps 2-5  epilogue, one thread per token row (TMEM lane quadrant = warp % 4): per head,
 //              tcgen05.ld of 128 fp32, then for q and k heads the sum of squares, 1/rms,
-//              gain and the rotation from the table; bf16 rows to q_out / k_out / v_out.
+//              gain and the rotation; bf16 rows to q_out / k_out / v_out.  The rotation's
+//              (cos, sin) come from the token tile's RoPE table ([64][128] float2, 64 KB,
+//              built by qkv_rope_table_kernel): for one frequency the 32 rows of a warp are
+//              one coalesced 256-byte read, and the table stays in L2 for all the tile's
+//              column tiles.  Left out of shared memory, it leaves room for a fourth stage.
 #pragma once
 #include "common.cuh"
 
@@ -42,23 +44,18 @@ struct QkvParams {
 };
 
 constexpr int kQkvThreads = 192;
-constexpr int kQkvStages = 3;
+constexpr int kQkvStages = 4;
 constexpr uint32_t kQkA = 16384;                  // 128 tokens x 64 bf16
 constexpr uint32_t kQkB = 32768;                  // 256 columns x 64 bf16
 constexpr uint32_t kQkStage = kQkA + kQkB;
-constexpr uint32_t kQkRope = kQkvStages * kQkStage;  // 64 KB table
-constexpr uint32_t kQkGain = kQkRope + 65536;        // q gain, k gain: 2 x 512 B
+constexpr uint32_t kQkGain = kQkvStages * kQkStage;  // q gain, k gain: 2 x 512 B
 constexpr uint32_t kQkBar = kQkGain + 1024;
-// barrier block: full[3], empty[3], acc_full[2], acc_empty[2], rope_full, rope_empty, done, tmem slot
-constexpr uint32_t kQbFull = 0, kQbEmpty = 24, kQbAccFull = 48, kQbAccEmpty = 64, kQbRopeFull = 80,
-                   kQbRopeEmpty = 88, kQbDone = 96, kQbTmem = 104, kQbAbort = 108;
+// barrier block: full[stages], empty[stages], acc_full[2], acc_empty[2], done, tmem slot, abort flag
+constexpr uint32_t kQbFull = 0, kQbEmpty = kQbFull + 8 * kQkvStages, kQbAccFull = kQbEmpty + 8 * kQkvStages,
+                   kQbAccEmpty = kQbAccFull + 16, kQbDone = kQbAccEmpty + 16, kQbTmem = kQbDone + 8,
+                   kQbAbort = kQbTmem + 4;
+static_assert(kQbAbort + 4 <= 128, "the qkv barrier block is 128 bytes");
 constexpr uint32_t kQkvSmemBytes = kQkBar + 128 + 1024;
-
-__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
-}
 
 // The RoPE table of every token tile: entry [mt][i][r] = (cos, sin)(pos[mt*128 + r] * inv_i)
 // times attention_scaling; rows past M use position 0.
@@ -115,8 +112,6 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       mbar_init(bar + kQbAccFull + 8 * b, 1);
       mbar_init(bar + kQbAccEmpty + 8 * b, 128);
     }
-    mbar_init(bar + kQbRopeFull, 1);
-    mbar_init(bar + kQbRopeEmpty, 128);
     mbar_init(bar + kQbDone, 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -141,24 +136,13 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     if (lane == 0) {
       tma_prefetch_map(&tmX);
       tma_prefetch_map(&tmW);
-      int last[kQkvStages] = {-1, -1, -1};
-      uint32_t it = 0, rope_uses = 0;
-      int cur_mt = -1;
+      int last[kQkvStages];
+      for (int s = 0; s < kQkvStages; ++s) last[s] = -1;
+      uint32_t it = 0;
       bool ok = true;
       for (int tile = t_begin; tile < t_end && ok; ++tile) {
         int mt, nt;
         qkv_tile_coords(p, tile, mt, nt);
-        if (mt != cur_mt) {  // the run reaches a new token tile: its RoPE table
-          if (rope_uses >= 1 &&
-              !mbar_wait(bar + kQbRopeEmpty, (rope_uses - 1) & 1, p.wait, abort_flag, kSiteQkvRope)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar + kQbRopeFull, 65536);
-          bulk_copy_g2s(sb + kQkRope, p.rope + static_cast<size_t>(mt) * 64 * 128, 65536, bar + kQbRopeFull);
-          ++rope_uses;
-          cur_mt = mt;
-        }
         for (int kc = 0; kc < p.n_k; ++kc, ++it) {
           const int st = static_cast<int>(it % kQkvStages);
           const uint32_t ph = (it / kQkvStages) & 1;
@@ -177,7 +161,6 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       for (int s = 0; s < kQkvStages; ++s)
         if (last[s] >= 0)
           mbar_wait(bar + kQbFull + 8 * s, (last[s] / kQkvStages) & 1, p.wait, nullptr, kSiteQkvDrain);
-      if (rope_uses >= 1) mbar_wait(bar + kQbRopeFull, (rope_uses - 1) & 1, p.wait, nullptr, kSiteQkvDrain);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -220,21 +203,11 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     const int row = wq * 32 + lane;  // token row of the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float* sg = reinterpret_cast<const float*>(sgen + kQkGain);
-    const float2* srope = reinterpret_cast<const float2*>(sgen + kQkRope);
-    uint32_t rope_uses = 0;
-    int cur_mt = -1;
     bool ok = true;
     int n = 0;
     for (int tile = t_begin; tile < t_end && ok; ++tile, ++n) {
       int mt, nt;
       qkv_tile_coords(p, tile, mt, nt);
-      if (mt != cur_mt) {
-        if (rope_uses >= 1) mbar_arrive(bar + kQbRopeEmpty);  // done with the previous token tile's table
-        ok = mbar_wait(bar + kQbRopeFull, rope_uses & 1, p.wait, abort_flag, kSiteQkvRope);
-        ++rope_uses;
-        cur_mt = mt;
-        if (!ok) break;
-      }
       const int buf = n & 1;
       ok = mbar_wait(bar + kQbAccFull + 8 * buf, (n >> 1) & 1, p.wait, abort_flag, kSiteQkvAcc);
       if (!ok) break;
@@ -264,9 +237,10 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
 #pragma unroll
           for (int i = 0; i < 128; ++i) ss = fmaf(__uint_as_float(y[i]), __uint_as_float(y[i]), ss);
           const float rn = rsqrtf(fmaf(ss, 1.0f / kD, p.eps));
+          const float2* rope = p.rope + static_cast<size_t>(mt) * 64 * 128;  // this token tile's table
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            const float2 cs = srope[i * 128 + row];
+            const float2 cs = rope[i * 128 + row];
             const float a = g[i] * (__uint_as_float(y[i]) * rn);
             const float b = g[64 + i] * (__uint_as_float(y[64 + i]) * rn);
             y[i] = __float_as_uint(a * cs.x - b * cs.y);
