@@ -18,5 +18,12 @@ from .attention import (  # noqa: F401
     rms_norm,
     rope,
     rope_inv_freq,
+    varlen_prefill_ref,
 )
-from .loops import chunk_prefill_loops, decode_loops, prefill_loops, qkv_proj_norm_rope_loops  # noqa: F401
+from .loops import (  # noqa: F401
+    chunk_prefill_loops,
+    decode_loops,
+    prefill_loops,
+    qkv_proj_norm_rope_loops,
+    varlen_prefill_loops,
+)

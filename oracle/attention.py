@@ -42,6 +42,10 @@ What it computes, and where each step is defined:
      scaling): a sliding-window layer lets query i see only the last W keys,
      i - W < j <= i; another rope type brings its own inv_freq and an
      attention_scaling that multiplies cos and sin.
+  8. Varlen batches: several sequences packed on one token axis with offsets
+     cu_seqlens, each an independent (chunked) causal prefill ("Assembling a large
+     model", the comparison with inference engines and the review question on
+     vLLM: flattened tokens plus batching metadata, attention per request).
 
 Readings where the pages leave a step open:
   * No intermediate rounding: the pages' HF path casts to bf16 between the
@@ -214,6 +218,51 @@ def chunk_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start:
                 o, l = _attend(qp[r0:r0 + block, h], keys[:top], vals[:top], rr + start, window)
                 out[b, r0:r0 + block, h] = o
                 lse[b, h, r0:r0 + block] = l
+    return out, lse
+
+
+def varlen_prefill_ref(q, k, v, q_norm_w, k_norm_w, pos, cu_seqlens, theta: float, eps: float,
+                       k_prefix=None, v_prefix=None, staged: bool = False, window: int = 0, inv_freq=None,
+                       scaling: float = 1.0):
+    """Prefill of several sequences packed on one token axis, in fp64.
+
+    The batching of serving engines ("Assembling a large model from scratch", the
+    comparison with inference engines: the tokens of many requests form one batch and
+    attention is computed per request; and the review question on vLLM: one forward pass
+    over a variable-length batch, flattened tokens plus batching metadata): q [N,Hq,d], k
+    and v [N,Hkv,d] and pos [N] hold the tokens of all sequences back to back, and sequence
+    b owns tokens cu_seqlens[b] .. cu_seqlens[b+1]-1.
+    Each sequence is an independent causal prefill: its tokens see only keys of their own
+    sequence.  With k_prefix and v_prefix (per sequence [Hkv, ctx_b, d]: cached keys as
+    stored, values raw) sequence b's new tokens follow its ctx_b cached ones, as in the
+    chunked prefill; without them every sequence is a fresh prompt.
+
+    Returns out [N,Hq,d] and lse [Hq,N]; rows of tokens that belong to no sequence are NaN.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    cu = np.asarray(cu_seqlens, dtype=np.int64)
+    pos = np.asarray(pos)
+    out = np.full((N, Hq, d), np.nan)
+    lse = np.full((Hq, N), np.nan)
+    for b in range(cu.size - 1):
+        lo, hi = int(cu[b]), int(cu[b + 1])
+        if hi == lo:
+            continue
+        if k_prefix is None:
+            kc = np.zeros((1, Hkv, 0, d))
+            vc = np.zeros((1, Hkv, 0, d))
+        else:
+            kc = np.asarray(k_prefix[b], dtype=np.float64)[None]
+            vc = np.asarray(v_prefix[b], dtype=np.float64)[None]
+        o, l = chunk_prefill_ref(q[None, lo:hi], k[None, lo:hi], v[None, lo:hi], q_norm_w, k_norm_w,
+                                 pos[None, lo:hi], kc, vc, kc.shape[2], theta, eps, staged=staged, window=window,
+                                 inv_freq=inv_freq, scaling=scaling)
+        out[lo:hi] = o[0]
+        lse[:, lo:hi] = l[0]
     return out, lse
 
 

@@ -115,6 +115,43 @@ def chunk_prefill_loops(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta, ep
     return out, lse
 
 
+def varlen_prefill_loops(q, k, v, gq, gk, pos, cu_seqlens, theta, eps, k_prefix=None, v_prefix=None):
+    """Packed sequences, token by token.  Token n belongs to the sequence b with
+    cu_seqlens[b] <= n < cu_seqlens[b+1]; its keys are that sequence's ctx_b cached keys
+    (k_prefix[b][hk][j], already normed and rotated; values v_prefix[b][hk][j] raw) followed
+    by the sequence's own new tokens up to n.  Tokens in no sequence get None."""
+    N, Hq, d = len(q), len(q[0]), len(q[0][0])
+    Hkv = len(k[0])
+    G = Hq // Hkv
+    out = [None] * N
+    lse = [[None] * N for _ in range(Hq)]
+    for n in range(N):
+        owner = [b for b in range(len(cu_seqlens) - 1) if cu_seqlens[b] <= n < cu_seqlens[b + 1]]
+        if not owner:
+            continue
+        b = owner[0]
+        first = int(cu_seqlens[b])
+        ctx = 0 if k_prefix is None else len(k_prefix[b][0])
+        row = [[0.0] * d for _ in range(Hq)]
+        for h in range(Hq):
+            hk = h // G
+            keys = [[float(x) for x in k_prefix[b][hk][j]] for j in range(ctx)]
+            vals = [[float(x) for x in v_prefix[b][hk][j]] for j in range(ctx)]
+            for m in range(first, n + 1):
+                keys.append(_norm_rope([float(x) for x in k[m][hk]], gk, float(pos[m]), theta, eps))
+                vals.append([float(x) for x in v[m][hk]])
+            qq = _norm_rope([float(x) for x in q[n][h]], gq, float(pos[n]), theta, eps)
+            scores = [sum(qq[i] * key[i] for i in range(d)) / math.sqrt(d) for key in keys]
+            mx = max(scores)
+            w = [math.exp(x - mx) for x in scores]
+            z = sum(w)
+            for i in range(d):
+                row[h][i] = sum(w[j] * vals[j][i] for j in range(len(w))) / z
+            lse[h][n] = mx + math.log(z)
+        out[n] = row
+    return out, lse
+
+
 def qkv_proj_norm_rope_loops(x, w_qkv, gq, gk, pos, Hq, Hkv, theta, eps):
     """The merged projection element by element, then QK-Norm and RoPE per head vector.
     x[m][i], w_qkv[o][i]; returns q'[m][h][i], k'[m][h][i], v[m][h][i]."""

@@ -290,6 +290,80 @@ def check_chunk_over_empty_cache_is_prefill():
     assert np.allclose(out, ref_o, rtol=0, atol=1e-14) and np.allclose(lse, ref_l, rtol=0, atol=1e-14)
 
 
+# ---------------------------------------------------------------- varlen batches
+def _packed(lens, Hq, Hkv, seed, lead=0, tail=0, ctx=None):
+    """Sequences of the given lengths packed back to back after `lead` unowned tokens and
+    before `tail` more; positions run from ctx_b (0 without a prefix) within each sequence.
+    With ctx, also the cached prefixes: keys normed and rotated at 0..ctx_b-1, values raw."""
+    cu = np.concatenate([[lead], lead + np.cumsum(lens)]).astype(np.int64)
+    N = int(cu[-1]) + tail
+    c = [0] * len(lens) if ctx is None else list(ctx)
+    pos = np.zeros(N, dtype=np.int64)
+    for b, L in enumerate(lens):
+        pos[cu[b]:cu[b + 1]] = c[b] + np.arange(L)
+    q, k, v = _rand((N, Hq, D), seed), _rand((N, Hkv, D), seed + 1), _rand((N, Hkv, D), seed + 2)
+    gq, gk = _gain(seed + 3), _gain(seed + 4)
+    kp = vp = None
+    if ctx is not None:
+        kp = [A.qk_prologue(_rand((n, Hkv, D), seed + 10 + b), gk, np.arange(n), THETA, EPS).transpose(1, 0, 2)
+              for b, n in enumerate(ctx)]
+        vp = [_rand((Hkv, n, D), seed + 40 + b) for b, n in enumerate(ctx)]
+    return q, k, v, gq, gk, pos, cu, kp, vp
+
+
+def check_brute_force_varlen_prefill():
+    """Ragged sequences (an empty one, a single token, unowned tokens before and after),
+    fresh and over cached prefixes, against the token-by-token loops."""
+    for (lens, Hq, Hkv, seed, lead, tail, ctx) in [((3, 0, 1, 5), 4, 2, 90, 0, 0, None),
+                                                   ((4, 2), 2, 1, 91, 2, 1, (3, 0)),
+                                                   ((1, 6, 2), 4, 1, 92, 0, 3, (2, 5, 1))]:
+        q, k, v, gq, gk, pos, cu, kp, vp = _packed(lens, Hq, Hkv, seed, lead, tail, ctx)
+        out, lse = A.varlen_prefill_ref(q, k, v, gq, gk, pos, cu, THETA, EPS, k_prefix=kp, v_prefix=vp)
+        lp = None if kp is None else [x.tolist() for x in kp]
+        lv = None if vp is None else [x.tolist() for x in vp]
+        out_l, lse_l = Lp.varlen_prefill_loops(q.tolist(), k.tolist(), v.tolist(), gq.tolist(), gk.tolist(),
+                                               pos.tolist(), cu.tolist(), THETA, EPS, k_prefix=lp, v_prefix=lv)
+        for n in range(q.shape[0]):
+            if out_l[n] is None:
+                assert np.isnan(out[n]).all() and np.isnan(lse[:, n]).all()
+            else:
+                assert np.allclose(out[n], np.array(out_l[n]), rtol=0, atol=1e-12)
+                assert np.allclose(lse[:, n], [lse_l[h][n] for h in range(Hq)], rtol=0, atol=1e-12)
+
+
+def check_varlen_of_equal_lengths_is_the_batch():
+    """Packing B sequences of equal length T on one token axis gives the batched prefill
+    [B, T] row for row (the token axis is the batch axis flattened)."""
+    B, T, Hq, Hkv = 3, 37, 8, 2
+    q, k, v, gq, gk, pos = _inputs(B, T, Hq, Hkv, seed=93)
+    ref_o, ref_l = A.prefill_ref(q, k, v, gq, gk, pos, THETA, EPS)
+    cu = np.arange(B + 1) * T
+    out, lse = A.varlen_prefill_ref(q.reshape(B * T, Hq, D), k.reshape(B * T, Hkv, D), v.reshape(B * T, Hkv, D), gq,
+                                    gk, pos.reshape(-1), cu, THETA, EPS)
+    assert np.allclose(out, ref_o.reshape(B * T, Hq, D), rtol=0, atol=1e-14)
+    assert np.allclose(lse, ref_l.transpose(1, 0, 2).reshape(Hq, B * T), rtol=0, atol=1e-14)
+
+
+def check_varlen_sequences_are_independent():
+    """Attention stays inside each sequence: reversing the order of the packed sequences
+    moves their outputs with them and changes nothing else; a prefixed sequence equals the
+    chunked prefill over its prefix."""
+    lens, ctx = (5, 9, 1, 4), (0, 6, 3, 2)
+    q, k, v, gq, gk, pos, cu, kp, vp = _packed(lens, 4, 2, 94, ctx=ctx)
+    out, lse = A.varlen_prefill_ref(q, k, v, gq, gk, pos, cu, THETA, EPS, k_prefix=kp, v_prefix=vp)
+    order = list(range(len(lens)))[::-1]
+    idx = np.concatenate([np.arange(cu[b], cu[b + 1]) for b in order])
+    cu_r = np.concatenate([[0], np.cumsum([lens[b] for b in order])])
+    out_r, lse_r = A.varlen_prefill_ref(q[idx], k[idx], v[idx], gq, gk, pos[idx], cu_r, THETA, EPS,
+                                        k_prefix=[kp[b] for b in order], v_prefix=[vp[b] for b in order])
+    assert np.array_equal(out_r, out[idx]) and np.array_equal(lse_r, lse[:, idx])
+    b = 1
+    sl = slice(cu[b], cu[b + 1])
+    o1, l1 = A.chunk_prefill_ref(q[None, sl], k[None, sl], v[None, sl], gq, gk, pos[None, sl], kp[b][None],
+                                 vp[b][None], ctx[b], THETA, EPS)
+    assert np.array_equal(o1[0], out[sl]) and np.array_equal(l1[0], lse[:, sl])
+
+
 # ---------------------------------------------------------------- variants
 def check_brute_force_variants():
     """Sliding window, another rope type's frequencies and attention_scaling against the

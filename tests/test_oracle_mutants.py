@@ -4,7 +4,7 @@ h mod Hkv head mapping, an off-by-one causal mask, a missing 1/sqrt(d) scale,
 a base-2 logsumexp, in the chunked prefill a mask without the cached-prefix
 offset or cached keys rotated a second time, and in the variants a sliding window
 one key too wide, attention_scaling applied to cos only, and a caller's inv_freq
-ignored."""
+ignored, and in the varlen batch one causal mask over the whole packed token axis."""
 import numpy as np
 import pytest
 
@@ -133,6 +133,19 @@ def _chunk_rerotates_cache(q, k, v, gq, gk, pos, k_cache, v_cache, start, theta,
     return _ORIG_CHUNK(q, k, v, gq, gk, pos, kc, v_cache, start, theta, eps, **kw)
 
 
+_ORIG_VARLEN = A.varlen_prefill_ref
+
+
+def _varlen_one_causal_axis(q, k, v, gq, gk, pos, cu_seqlens, theta, eps, k_prefix=None, v_prefix=None, **kw):
+    # attention runs causally over the whole packed axis: a token also sees the tokens of
+    # the sequences packed before it
+    cu = np.asarray(cu_seqlens)
+    whole = np.array([cu[0], cu[-1]])
+    return _ORIG_VARLEN(q, k, v, gq, gk, pos, whole, theta, eps,
+                        k_prefix=None if k_prefix is None else k_prefix[:1],
+                        v_prefix=None if v_prefix is None else v_prefix[:1], **kw)
+
+
 _ORIG_PREFILL = A.prefill_ref
 
 MUTANTS = [
@@ -150,6 +163,7 @@ MUTANTS = [
     ("prefill_ref", _prefill_mod_mapping),
     ("chunk_prefill_ref", _chunk_no_offset),
     ("chunk_prefill_ref", _chunk_rerotates_cache),
+    ("varlen_prefill_ref", _varlen_one_causal_axis),
 ]
 
 
