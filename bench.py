@@ -13,6 +13,7 @@ prologue is counted as free work); the decode throughput in GB/s rides along und
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
     python bench.py --workload chunked-prefill    # the chunked-prefill call alone
     python bench.py --workload qkv-proj           # the merged qkv projection + QK-Norm/RoPE
+    python bench.py --workload varlen-prefill     # a ragged batch of prompts on one token axis
 
 The chunked-prefill workload times qwen3_attn_prefill_chunk on the Qwen3-4B-shaped
 second chunk (B=1, 4096 new tokens over 4096 cached, Hq=32, Hkv=8) and prints its own
@@ -37,8 +38,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, QKV_SHAPES, chunk_inputs, decode_step_inputs, \
-    prefill_inputs, qkv_proj_inputs  # noqa: E402
+from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, QKV_SHAPES, VARLEN_SHAPES, chunk_inputs, \
+    decode_step_inputs, prefill_inputs, qkv_proj_inputs, varlen_inputs  # noqa: E402
 
 METRIC = "causal GQA attn TFLOP/s (+QK-Norm/RoPE) % bf16 peak; decode HBM GB/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -607,6 +608,157 @@ def run_qkv(args, world, rank, local):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------------------------ varlen prefill
+VARLEN_METRIC = "varlen batched causal GQA prefill TFLOP/s (+QK-Norm/RoPE) % bf16 peak"
+
+
+def cpu_oracle_varlen_sample(name: str, rows: int = 256, seed: int = 0):
+    """The oracle's prefill of the last `rows` query rows (every head) of the batch's longest
+    sequence, keys over the whole sequence."""
+    import oracle
+    from synthetic import as_f64
+
+    sh = VARLEN_SHAPES[name]
+    inp = varlen_inputs(sh, seed=seed)
+    b = int(np.argmax(sh.lens))
+    cu = inp["cu_seqlens"].numpy()
+    sl = slice(int(cu[b]), int(cu[b + 1]))
+    T = sh.lens[b]
+    rows = min(rows, T)
+    sel = np.arange(T - rows, T)
+    empty = np.zeros((1, sh.Hkv, 0, sh.d))
+    t0 = time.perf_counter()
+    oracle.chunk_prefill_ref(as_f64(inp["q"][sl])[None], as_f64(inp["k"][sl])[None], as_f64(inp["v"][sl])[None],
+                             as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][sl].numpy()[None], empty,
+                             empty, 0, sh.theta, sh.eps, rows=sel)
+    secs = time.perf_counter() - t0
+    flops = 4.0 * sh.Hq * sh.d * float((sel + 1).sum())
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        threads = os.cpu_count()
+    sample = (f"last {rows} of {T} query rows x {sh.Hq} heads of the longest sequence of the {sh.name} "
+              f"({flops:.3g} causal flops)")
+    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "sample": sample, "flops": flops}
+
+
+def time_call(step, flush, host: dict, dev_inputs: dict, outputs: list, K: int, warmup: int, world, local, dev,
+              e2e_steps: int):
+    """Time K calls of `step` (L2 flushed before each, outside the event windows) and the same
+    call end to end: pinned host inputs in, the call, its outputs back, inside one window."""
+    import qwen3_qk_norm_rope_b200 as qa
+
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.fill_(1.0)
+            ev[i][0].record()
+            step()
+            ev[i][1].record()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+    st, site = qa.device_status(clear=True, device=dev)
+    if st != qa.OK:
+        raise RuntimeError(f"device status {qa.status_string(st)} at site {site}")
+    ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    ph = {k: v.pin_memory() for k, v in host.items()}
+    oh = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outputs]
+    h2d = sum(v.numel() * v.element_size() for v in ph.values())
+    d2h = sum(o.numel() * o.element_size() for o in oh)
+    e_ms = 0.0
+    for _ in range(e2e_steps):
+        flush.fill_(1.0)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for k, v in ph.items():
+            dev_inputs[k].copy_(v, non_blocking=True)
+        step()
+        for o, h in zip(outputs, oh):
+            h.copy_(o, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        e_ms += e0.elapsed_time(e1)
+    ms, e_ms = max_over_ranks(world, [ms, e_ms], dev)
+    return ms, e_ms, h2d, d2h, clk
+
+
+def run_varlen(args, world, rank, local):
+    name = args.varlen
+    sh = VARLEN_SHAPES[name]
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cal = cpu_oracle_varlen_sample(name, rows=16)
+        rows = int(max(4, min(max(sh.lens), (120.0 / max(args.steps, 1)) / max(cal["seconds"] / 16, 1e-6))))
+        secs = flops = 0.0
+        res = None
+        for _ in range(args.steps):
+            res = cpu_oracle_varlen_sample(name, rows=rows)
+            secs += res["seconds"]
+            flops += res["flops"]
+        value = flops / secs / 1e12
+        line = {"impl": "reference", "metric": VARLEN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": {"workload": sh.name},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
+                                 "sample": "per step, " + res["sample"]},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    import qwen3_qk_norm_rope_b200 as qa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    inp = varlen_inputs(sh, seed=0)
+    host = {k: inp[k] for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos", "cu_seqlens")}
+    t = {k: v.to(dev) for k, v in host.items()}
+    out = torch.empty((sh.N, sh.Hq, sh.d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(qa.prefill_varlen_workspace_size(sh.B, sh.N, sh.Hq, sh.Hkv), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"], out=out,
+                          workspace=ws, theta=sh.theta, eps=sh.eps)
+
+    K = args.steps
+    ms, e_ms, h2d, d2h, clk = time_call(step, flush, host, t, [out], K, args.warmup, world, local, dev,
+                                        max(1, min(K, 100)))
+    if rank != 0:
+        return
+    flops = sh.causal_flops()
+    achieved = flops / (ms * 1e-3 / K) / 1e12
+    line = {"metric": VARLEN_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": sh.name, "lens": list(sh.lens), "N": sh.N, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+                       "rope_theta": sh.theta, "rms_eps": sh.eps, "seed": 0,
+                       "l2": "flushed before every step (256 MiB write, outside the timed windows)",
+                       "parallelism": "replicas (one independent workload per GPU)"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                         "kernel": "varlen prefill call (metadata + QK prologue + attention)",
+                         "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
+            "gpu_launches": 3 * K, "clocks": clk.summary(),
+            "e2e": {"value": world * flops * max(1, min(K, 100)) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                    "ms_per_step": e_ms / max(1, min(K, 100))}}
+    if world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_varlen_sample(name, rows=512)
+        line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
+                                "sample": cb["sample"], "seconds": cb["seconds"]}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------------------ main
 def dist_setup(backend: str = "nccl"):
     """One process per GPU (torchrun env).  The process group only carries the timing
@@ -698,16 +850,20 @@ def main():
                     help="prefill workload of the step (profiling of the other shapes)")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="decode the first n of the 64 sequences (small cases for ncu captures)")
-    ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill", "qkv-proj"],
+    ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill", "qkv-proj", "varlen-prefill"],
                     help="step: 0.6B prefill + batched decode (default); chunked-prefill: the chunk call alone; "
-                         "qkv-proj: the merged projection with the QK-Norm/RoPE epilogue")
+                         "qkv-proj: the merged projection with the QK-Norm/RoPE epilogue; varlen-prefill: a "
+                         "ragged batch of prompts packed on one token axis")
     ap.add_argument("--qkv", default="qwen3-0.6b-qkv", choices=sorted(QKV_SHAPES),
                     help="the qkv-proj workload's shape")
+    ap.add_argument("--varlen", default="qwen3-4b-varlen", choices=sorted(VARLEN_SHAPES),
+                    help="the varlen-prefill workload's shape")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup("nccl")
-    if args.workload in ("chunked-prefill", "qkv-proj"):
-        (run_chunk if args.workload == "chunked-prefill" else run_qkv)(args, world, rank, local)
+    legs = {"chunked-prefill": run_chunk, "qkv-proj": run_qkv, "varlen-prefill": run_varlen}
+    if args.workload in legs:
+        legs[args.workload](args, world, rank, local)
         if world > 1:
             import torch.distributed as dist
 

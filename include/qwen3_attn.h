@@ -317,6 +317,47 @@ int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
 size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d);
 
 /*
+ * qwen3_attn_prefill_varlen - prefill of B sequences packed on one token axis, the batching
+ * of serving engines ("LLM Internals - Assembling a large model from scratch", the
+ * comparison with inference engines: the tokens of many requests form one batch and
+ * attention is computed per request; the review question on vLLM: flattened tokens plus
+ * batching metadata).  Each sequence is an independent causal prefill, as
+ * qwen3_attn_prefill_chunk computes it for one batch row.
+ *   q          [N, Hq, d] bf16; k, v [N, Hkv, d]: the raw tokens of all sequences.
+ *   pos        [N] int32 rotary positions (usually ctx_lens[b] + t for token t of b).
+ *   cu_seqlens [B + 1] int32 device array: sequence b owns tokens cu_seqlens[b] ..
+ *              cu_seqlens[b+1] - 1, with 0 <= cu_seqlens[b] <= cu_seqlens[b+1] <= N.
+ *              Tokens before cu_seqlens[0] or from cu_seqlens[B] on belong to no
+ *              sequence (padding); their rows of out and lse are not written.  An empty
+ *              sequence is allowed.
+ *   out        [N, Hq, d] bf16; lse [Hq, N] float (natural log) or NULL.
+ *   kv         NULL: fresh prompts; the keys of a sequence are its own tokens, and ctx_lens
+ *              must be NULL and key_cap 0.  Otherwise a paged cache (row b of the block
+ *              table is sequence b): the sequence's new keys (normed, rotated) and values go
+ *              to its key indices ctx_lens[b] .. ctx_lens[b] + T_b - 1, and its queries see
+ *              its ctx_lens[b] cached keys first, as in qwen3_attn_prefill_paged.
+ *   ctx_lens   [B] int32 device array of cached keys per sequence, or NULL (all 0).
+ *   key_cap    with kv: a bound on the sum over sequences of ctx_lens[b] + T_b (the
+ *              workspace holds that many gathered keys and values).
+ * The lengths stay on the device: the host reads none of them.  A sequence whose metadata
+ * is out of range (offsets outside [0, N] or decreasing, a negative ctx_lens, keys past
+ * max_blocks * page_size, or keys past key_cap) is recorded as QWEN3_ERR_INVALID_ARG in
+ * the device status word and skipped.  Workspace:
+ * qwen3_attn_prefill_varlen_workspace_size(B, N, key_cap, Hq, Hkv, d) bytes.
+ */
+int qwen3_attn_prefill_varlen(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
+                              const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
+                              const int32_t* cu_seqlens, qwen3_bf16* out, float* lse,
+                              const qwen3_paged_kv* kv, const int32_t* ctx_lens, long long key_cap,
+                              void* workspace, size_t ws_bytes,
+                              int B, int N, int Hq, int Hkv, int d,
+                              const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream);
+
+/* Scratch bytes qwen3_attn_prefill_varlen needs: the sequence metadata and work list, Q',
+ * and K' and V for N rows (key_cap = 0) or key_cap rows; 0 for an unsupported shape. */
+size_t qwen3_attn_prefill_varlen_workspace_size(int B, int N, long long key_cap, int Hq, int Hkv, int d);
+
+/*
  * qwen3_qkv_proj_norm_rope - the merged q/k/v projection with QK-Norm and RoPE in the GEMM
  * epilogue.  y = x w_qkv^T ("LLM Internals - Assembling a large model from scratch": one
  * qkv_proj GEMM for the three projections), split into q [M, Hq, d], k [M, Hkv, d],

@@ -56,6 +56,9 @@ SIGNATURES = {
     "qwen3_attn_prefill_paged": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(PagedKV), _I, _P, _Z,
                                       _I, _I, _I, _I, _I, _V, _F, _P]),
     "qwen3_attn_prefill_paged_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "qwen3_attn_prefill_varlen": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.POINTER(PagedKV), _P,
+                                       ctypes.c_longlong, _P, _Z, _I, _I, _I, _I, _I, _V, _F, _P]),
+    "qwen3_attn_prefill_varlen_workspace_size": (_Z, [_I, _I, ctypes.c_longlong, _I, _I, _I]),
     "qwen3_qkv_proj_norm_rope": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _V, _F, _P, _Z, _P]),
     "qwen3_qkv_proj_workspace_size": (_Z, [_I]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
@@ -393,6 +396,56 @@ def prefill_paged(q, k, v, q_norm_w, k_norm_w, pos, k_pages, v_pages, block_tabl
                                           _ptr(out), _ptr(lse), ctypes.byref(kv), int(start), _ptr(workspace),
                                           ws_bytes, B, T, Hq, Hkv, d, ctypes.byref(var), eps, _stream(dev)),
            "qwen3_attn_prefill_paged")
+    return out
+
+
+def prefill_varlen_workspace_size(B: int, N: int, Hq: int, Hkv: int, key_cap: int = 0, d: int = HEAD_DIM) -> int:
+    return int(lib().qwen3_attn_prefill_varlen_workspace_size(B, N, key_cap, Hq, Hkv, d))
+
+
+def prefill_varlen(q, k, v, q_norm_w, k_norm_w, pos, cu_seqlens, *, k_pages=None, v_pages=None, block_table=None,
+                   ctx_lens=None, key_cap: int = 0, theta: float = 1.0e6, eps: float = 1.0e-6, out=None, lse=None,
+                   workspace=None, window: int = 0, inv_freq=None, attention_scaling: float = 1.0):
+    """Prefill of B sequences packed on one token axis: q [N,Hq,d], k/v [N,Hkv,d], pos [N],
+    cu_seqlens [B+1] int32 (sequence b owns tokens cu_seqlens[b] .. cu_seqlens[b+1]-1).
+    With k_pages/v_pages/block_table, a paged cache: sequence b has ctx_lens[b] cached keys
+    (ctx_lens [B] int32, None = all 0), its new keys and values go to its pages, and key_cap
+    must bound the sum of ctx_lens[b] + T_b.  Returns out [N,Hq,d] (rows of tokens outside
+    every sequence untouched) and writes lse [Hq,N] when given."""
+    dev = q.device
+    N, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.shape[0] - 1
+    _need(q, "q", torch.bfloat16, (N, Hq, d), dev)
+    _need(k, "k", torch.bfloat16, (N, Hkv, d), dev)
+    _need(v, "v", torch.bfloat16, (N, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (N,), dev)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, (B + 1,), dev)
+    kv = None
+    if k_pages is not None:
+        kv = _paged(k_pages, v_pages, block_table, dev, Hkv, d)
+        if block_table.shape[0] < B:
+            raise ValueError(f"block_table has {block_table.shape[0]} rows for {B} sequences")
+        if ctx_lens is not None:
+            _need(ctx_lens, "ctx_lens", torch.int32, (B,), dev)
+    if out is None:
+        out = torch.empty((N, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (N, Hq, d), dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, (Hq, N), dev)
+    if workspace is None:
+        workspace = torch.empty(prefill_varlen_workspace_size(B, N, Hq, Hkv, key_cap, d), dtype=torch.uint8,
+                                device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    var, _keep = make_variant(theta, inv_freq, attention_scaling, window)
+    _check(lib().qwen3_attn_prefill_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
+                                           _ptr(cu_seqlens), _ptr(out), _ptr(lse),
+                                           ctypes.byref(kv) if kv is not None else None, _ptr(ctx_lens),
+                                           int(key_cap), _ptr(workspace), ws_bytes, B, N, Hq, Hkv, d,
+                                           ctypes.byref(var), eps, _stream(dev)),
+           "qwen3_attn_prefill_varlen")
     return out
 
 

@@ -52,6 +52,13 @@ struct PrefillParams {
   float rope_scale;  // attention_scaling that scaled q' and k' (enters the logit bound squared)
   WaitCfg wait;
   int fault;
+  // Varlen batches (the kVar instance): the entry list {qoff, T, start, koff}, {pair, b}
+  // and its item count, both written on the device; B is then the sequence count, T the
+  // packed token count N, and `out` [N, Hq, d] takes the rows of tiles that end past their
+  // sequence (a tiled store of those would write into the next sequence's rows).
+  const int4* vl_ent;
+  const int* vl_n_items;
+  uint4* out;
 };
 
 constexpr uint32_t kPfTile = 32768;  // 128 rows x 128 bf16
@@ -97,18 +104,25 @@ struct TileInfo {
   int t0, nkv;  // first query row; key tiles it reads from the item's first (0 = past T)
 };
 
+// The sequence an item belongs to: its first token on the query axis, its new tokens, its
+// cached keys before them, and its first key row.  One batch row of a uniform batch is
+// {0, T, start, 0} (its rows are addressed through the batch coordinate instead).
+struct ItemSeq {
+  int qoff, T, start, koff;
+};
+
 // First key tile of a pair item: 0, or with a sliding window the tile holding the first key
 // that tile A's first row may see (tile B's rows start later, so they mask one tile at most).
 template <bool kWin>
-__device__ __forceinline__ int item_lo(const PrefillParams& p, int pair) {
+__device__ __forceinline__ int item_lo(const PrefillParams& p, const ItemSeq& sq, int pair) {
   if constexpr (!kWin) return 0;
-  return max(0, p.start + 2 * pair * p.P - p.window + 1) >> 7;
+  return max(0, sq.start + 2 * pair * p.P - p.window + 1) >> 7;
 }
 
-__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, int qt, int lo) {
+__device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, const ItemSeq& sq, int qt, int lo) {
   TileInfo ti;
   ti.t0 = qt * p.P;
-  ti.nkv = (ti.t0 < p.T) ? (p.start + min(ti.t0 + p.P, p.T) - 1) / 128 + 1 - lo : 0;
+  ti.nkv = (ti.t0 < sq.T) ? (sq.start + min(ti.t0 + p.P, sq.T) - 1) / 128 + 1 - lo : 0;
   return ti;
 }
 
@@ -129,9 +143,35 @@ __device__ __forceinline__ void item_coords(const PrefillParams& p, int item, in
   hkv = bh % p.Hkv;
 }
 
+// Items of a launch: from the parameters, or for a varlen batch from the device's entry list.
+template <bool kVar>
+__device__ __forceinline__ int item_count(const PrefillParams& p) {
+  if constexpr (kVar) return __ldcg(p.vl_n_items);
+  return p.n_items;
+}
+
+// Work item -> (pair, batch coordinate, KV head, sequence).  A varlen item reads its entry
+// (two independent 16-byte loads); its batch coordinate is 0 (the packed axis is one row).
+template <bool kVar>
+__device__ __forceinline__ void item_fetch(const PrefillParams& p, int item, int& pair, int& b, int& hkv,
+                                           ItemSeq& sq) {
+  if constexpr (kVar) {
+    const int e = item / p.Hkv;
+    hkv = item - e * p.Hkv;
+    const int4 a = __ldcg(p.vl_ent + 2 * e);
+    const int4 c = __ldcg(p.vl_ent + 2 * e + 1);
+    sq = ItemSeq{a.x, a.y, a.z, a.w};
+    pair = c.x;
+    b = 0;
+  } else {
+    item_coords(p, item, pair, b, hkv);
+    sq = ItemSeq{0, p.T, p.start, 0};
+  }
+}
+
 // kWin: a sliding window is set (p.window > 0); the full-causal instance carries none of its
-// masks or bookkeeping.
-template <bool kWin>
+// masks or bookkeeping.  kVar: a varlen batch (items from the device's entry list).
+template <bool kWin, bool kVar>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -181,11 +221,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last[2] = {-1, -1};
       uint32_t it = 0, q_use[2] = {0, 0};
       bool ok = true;
-      for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
+      const int n_items = item_count<kVar>(p);
+      for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
-        item_coords(p, item, pair, b, hkv);
-        const int lo = item_lo<kWin>(p, pair);
-        const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
+        ItemSeq sq;
+        item_fetch<kVar>(p, item, pair, b, hkv, sq);
+        const int lo = item_lo<kWin>(p, sq, pair);
+        const int nX[2] = {tile_info(p, sq, 2 * pair, lo).nkv, tile_info(p, sq, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
         for (int X = 0; X < 2 && ok; ++X) {
           if (nX[X] == 0) continue;
@@ -195,7 +237,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ok = false;
             break;
           }
-          const int row0 = (2 * pair + X) * 128;  // the tile's first row of Q' [b, hkv, T*G, d]
+          // the tile's first row of Q' [b, hkv, T*G, d] (a varlen batch: [0, hkv, N*G, d])
+          const int row0 = (sq.qoff << p.log2G) + (2 * pair + X) * 128;
           mbar_arrive_expect_tx(bar + kBQFull + 8 * X, kPfTile);
           tma_load_4d(sb + kPfQ + X * kPfTile, &tmQ, bar + kBQFull + 8 * X, 0, row0, hkv, b);
           tma_load_4d(sb + kPfQ + X * kPfTile + kPfBox, &tmQ, bar + kBQFull + 8 * X, 64, row0, hkv, b);
@@ -210,8 +253,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           }
           if (!(p.fault != 0 && it == 0)) {
             mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
-            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, (lo + j) * 128, hkv, b);
-            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, (lo + j) * 128, hkv, b);
+            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, sq.koff + (lo + j) * 128, hkv, b);
+            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, sq.koff + (lo + j) * 128, hkv,
+                        b);
             k_last[st] = static_cast<int>(it);
           }
           if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
@@ -219,8 +263,9 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
-          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, (lo + j) * 128, hkv, b);
-          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, (lo + j) * 128, hkv, b);
+          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, sq.koff + (lo + j) * 128, hkv, b);
+          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, sq.koff + (lo + j) * 128, hkv,
+                      b);
           v_last[st] = static_cast<int>(it);
         }
       }
@@ -238,12 +283,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t kIdPV = idesc_bf16(128, 128, true);   // B = V, dims contiguous (MN-major)
       uint32_t it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
       bool ok = true;
-      for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
+      const int n_items = item_count<kVar>(p);
+      for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
         int pair, b, hkv;
-        item_coords(p, item, pair, b, hkv);
-        const int lo = item_lo<kWin>(p, pair);
-        const int nX[2] = {tile_info(p, 2 * pair, lo).nkv, tile_info(p, 2 * pair + 1, lo).nkv};
+        ItemSeq sq;
+        item_fetch<kVar>(p, item, pair, b, hkv, sq);
+        const int lo = item_lo<kWin>(p, sq, pair);
+        const int nX[2] = {tile_info(p, sq, 2 * pair, lo).nkv, tile_info(p, sq, 2 * pair + 1, lo).nkv};
         const int n = max(nX[0], nX[1]);
+        if (kVar && n == 0) continue;  // an empty entry (none is built; the producer skips it too)
         for (int X = 0; X < 2 && ok; ++X)
           if (nX[X] > 0) {
             ok = mbar_wait(bar + kBQFull + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQFull);
@@ -349,16 +397,18 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // The tensor core may start the next item (its Q' tiles arrive by TMA) while this
     // group stores the current item's outputs.  O_X stays safe: the next item's first PV_X
     // waits for a P that is only written after this epilogue.
-    for (int k = 0, item = round_item(0); item < p.n_items && ok; item = round_item(++k)) {
+    const int n_items = item_count<kVar>(p);
+    for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
       int pair, b, hkv;
-      item_coords(p, item, pair, b, hkv);
-      const int lo = item_lo<kWin>(p, pair);
-      const TileInfo ti = tile_info(p, 2 * pair + X, lo);
+      ItemSeq sq;
+      item_fetch<kVar>(p, item, pair, b, hkv, sq);
+      const int lo = item_lo<kWin>(p, sq, pair);
+      const TileInfo ti = tile_info(p, sq, 2 * pair + X, lo);
       if (ti.nkv == 0) continue;  // this item has no tile X
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
-      const int lim = p.start + min(t_row, p.T - 1);  // last key index this row may see
+      const int lim = sq.start + min(t_row, sq.T - 1);  // last key index this row may see
       const int wfirst = kWin ? lim - p.window + 1 : 0;  // first one, with a window
       float m = fast ? bnd : -INFINITY, l = 0.f;
       for (int j = 0; j < ti.nkv; ++j) {
@@ -369,7 +419,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         tc_fence_after();
         const int kv0 = (lo + j) * 128;
         // some key of this tile lies past some row's limit, or before some row's window
-        const bool diag = kv0 + 127 > p.start + t0 || (kWin && kv0 < p.start + t0 + p.P - p.window);
+        const bool diag = kv0 + 127 > sq.start + t0 || (kWin && kv0 < sq.start + t0 + p.P - p.window);
         if (fast) {
           // One pass in four 32-column chunks, the next chunk's TMEM load in flight while the
           // current one is processed.  bf16 P goes to S columns [0,64): chunk c of P
@@ -507,14 +557,35 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const int h = hkv * G + (row & (G - 1));
-      const bool valid = t_row < p.T;
+      const bool valid = t_row < sq.T;
       const float inv_l = 1.0f / l;
       // O/l in two 64-dim halves through this group's staging box.  Row r of the tile is row r
       // of the box [P positions][G heads][64 dims], so one tiled store writes the half to
       // out[b, t0 .. t0+P-1, hkv*G .. hkv*G+G-1, half*64 ..]; rows past T are clipped by the
-      // copy.  The storing thread waits until the previous store has read the buffer.
+      // copy (a varlen batch: out[qoff + t0 ..], with rows past the sequence stored below).
+      // The storing thread waits until the previous store has read the buffer.
       const uint32_t stg = sb + kPfStage + X * kPfBox;
       const bool storer = row == 0;
+      if (kVar && t0 + p.P > sq.T) {
+        // A varlen tile that ends past its sequence: the rows after it on the packed axis
+        // belong to the next sequence, so each thread stores its own row, if it has one,
+        // straight from TMEM (eight 16-byte stores per 64 dims).
+        uint4* dst = p.out + (static_cast<long long>(sq.qoff + t_row) * p.Hq + h) * (kD / 8);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          if (valid) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[c * 4 + u] =
+                  make_uint4(pack_bf16x2(__uint_as_float(r[8 * u + 0]) * inv_l, __uint_as_float(r[8 * u + 1]) * inv_l),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 2]) * inv_l, __uint_as_float(r[8 * u + 3]) * inv_l),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 4]) * inv_l, __uint_as_float(r[8 * u + 5]) * inv_l),
+                             pack_bf16x2(__uint_as_float(r[8 * u + 6]) * inv_l, __uint_as_float(r[8 * u + 7]) * inv_l));
+          }
+        }
+      } else {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         if (storer) bulk_wait_read_all();
@@ -534,12 +605,13 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         fence_proxy_async_smem();
         asm volatile("bar.sync %0, 128;" ::"r"(1 + X) : "memory");
         if (storer) {
-          tma_store_4d(&tmO, stg, half * 64, hkv * G, t0, b);
+          tma_store_4d(&tmO, stg, half * 64, hkv * G, sq.qoff + t0, b);
           bulk_commit_group();
         }
       }
+      }
       if (p.lse != nullptr && valid)
-        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.T + t_row] = (m + log2f(l)) * kLn2;
+        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.T + sq.qoff + t_row] = (m + log2f(l)) * kLn2;
     }
     if (row == 0) bulk_wait_all();  // this group's output stores have completed
   }

@@ -32,6 +32,15 @@ struct PrologueParams {
   // block_table[b, kk / page] at offset kk % page.  page = 1 << log2_page.
   const int* block_table;
   int max_blocks, log2_page, num_pages, key0;
+  // Optional varlen batch (B = 1, T = N packed tokens; sequence b owns tokens cu[b] ..
+  // cu[b+1]-1).  Without pages, tokens before cu[0] or from cu[B] on belong to no sequence
+  // and get zero keys and values (a sequence's last key tile reads past its end, and the
+  // values there still enter P.V as 0 x value).  With pages, a token's keys go to its own
+  // sequence's pages (seq[b] = {qoff, T, start, koff}: key index start + token - qoff), and
+  // tokens of no valid sequence write no key or value.
+  const int* vl_cu;
+  const int4* vl_seq;
+  int vl_B;
   float eps;
   float rope_scale;  // attention_scaling: multiplies cos and sin (1 for the default rope type)
   RopeTable rope;
@@ -64,7 +73,8 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     const int t = bt - b * p.T;
     const int ps = p.pos[bt];
     // destination of head 0 and the distance between heads, in rows of d
-    size_t row0, hstride;
+    size_t row0 = 0, hstride = 0;
+    bool kv_write = true, kv_zero = false;
     if (p.block_table == nullptr) {
       const int row = p.write_at_pos ? ps : t;
       if (row < 0 || row >= p.Tcap) {
@@ -73,16 +83,37 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
       }
       row0 = static_cast<size_t>(b) * p.H * p.Tcap + row;
       hstride = p.Tcap;
+      if (p.vl_cu != nullptr) kv_zero = bt < __ldg(p.vl_cu) || bt >= __ldg(p.vl_cu + p.vl_B);
     } else {
-      const int kk = p.write_at_pos ? ps : p.key0 + t;
-      const int blk = kk >> p.log2_page;
-      const int page = (kk >= 0 && blk < p.max_blocks) ? p.block_table[static_cast<size_t>(b) * p.max_blocks + blk] : -1;
-      if (page < 0 || page >= p.num_pages) {
-        if (lane == 0) record_error(QWEN3_ERR_INVALID_ARG, kSitePrologueRow);
-        continue;
+      int bs = b, kk = p.write_at_pos ? ps : p.key0 + t;
+      if (p.vl_seq != nullptr) {
+        // the token's sequence: the last b with cu[b] <= bt, checked against its metadata
+        int lo = 0, hi = p.vl_B - 1;
+        bs = -1;
+        while (lo <= hi) {
+          const int mid = (lo + hi) >> 1;
+          if (__ldg(p.vl_cu + mid) <= bt) {
+            bs = mid;
+            lo = mid + 1;
+          } else {
+            hi = mid - 1;
+          }
+        }
+        const int4 sq = bs >= 0 ? p.vl_seq[bs] : make_int4(0, 0, 0, 0);
+        kv_write = bs >= 0 && bt >= sq.x && bt < sq.x + sq.y;
+        kk = sq.z + (bt - sq.x);
       }
-      row0 = (static_cast<size_t>(page) * p.H << p.log2_page) + (kk & ((1 << p.log2_page) - 1));
-      hstride = static_cast<size_t>(1) << p.log2_page;
+      if (kv_write) {
+        const int blk = kk >> p.log2_page;
+        const int page =
+            (kk >= 0 && blk < p.max_blocks) ? p.block_table[static_cast<size_t>(bs) * p.max_blocks + blk] : -1;
+        if (page < 0 || page >= p.num_pages) {
+          if (lane == 0) record_error(QWEN3_ERR_INVALID_ARG, kSitePrologueRow);
+          continue;
+        }
+        row0 = (static_cast<size_t>(page) * p.H << p.log2_page) + (kk & ((1 << p.log2_page) - 1));
+        hstride = static_cast<size_t>(1) << p.log2_page;
+      }
     }
     float s0, c0, s1, c1;
     rope_sincos(ps, hi0, lo0, s0, c0);
@@ -91,7 +122,7 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
     c0 *= p.rope_scale;
     s1 *= p.rope_scale;
     c1 *= p.rope_scale;
-    for (int h0 = 0; h0 < p.H; h0 += kPrologueHeads) {
+    for (int h0 = 0; kv_write && h0 < p.H; h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
       uint2 vv[kPrologueHeads];
 #pragma unroll
@@ -111,6 +142,10 @@ __global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant
         float2 ya, yb;
         norm_rope_pairs(make_float2(bf16lo(ua[u]), bf16hi(ua[u])), make_float2(bf16lo(ub[u]), bf16hi(ub[u])), ga,
                         gb, s0, c0, s1, c1, p.eps, ya, yb);
+        if (kv_zero) {
+          ya = yb = make_float2(0.f, 0.f);
+          vv[u] = make_uint2(0u, 0u);
+        }
         const size_t drow = row0 + static_cast<size_t>(h0 + u) * hstride;
         uint32_t* ds = p.dst + drow * (kD / 2);
         ds[lane] = pack_bf16x2(ya.x, ya.y);

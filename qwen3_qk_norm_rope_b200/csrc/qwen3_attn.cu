@@ -14,6 +14,7 @@
 #include "paged.cuh"
 #include "prologue.cuh"
 #include "qkv_proj.cuh"
+#include "varlen.cuh"
 
 namespace {
 
@@ -159,9 +160,13 @@ int ensure_kernel_attrs() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QWEN3_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   if (done[dev]) return QWEN3_OK;
-  if (cudaFuncSetAttribute(q3::fmha_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(q3::fmha_prefill_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(q3::fmha_prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(q3::fmha_prefill_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kPrefillSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::fmha_prefill_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kPrefillSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::fmha_prefill_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -207,10 +212,17 @@ struct PrologueQ {
   int Hq = 0;
 };
 
+// A varlen batch (optional): token offsets [B + 1] and, with pages, the checked metadata.
+struct PrologueVarlen {
+  const int32_t* cu = nullptr;
+  const int4* seq = nullptr;
+  int B = 0;
+};
+
 int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst, const void* v_src, void* v_dst,
                     int B, int T, int H, int Tcap, int write_at_pos, const Variant& var, float eps,
                     cudaStream_t stream, const PrologueQ& q = PrologueQ(), const PagedKV* pg = nullptr,
-                    int key0 = 0) {
+                    int key0 = 0, const PrologueVarlen& vl = PrologueVarlen()) {
   q3::PrologueParams p;
   p.x = static_cast<const uint32_t*>(x);
   p.w = w;
@@ -236,6 +248,9 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   p.log2_page = pg != nullptr ? pg->log2_page : 0;
   p.num_pages = pg != nullptr ? pg->num_pages : 0;
   p.key0 = key0;
+  p.vl_cu = vl.cu;
+  p.vl_seq = vl.seq;
+  p.vl_B = vl.B;
   const long long ntok = static_cast<long long>(B) * T;
   if (ntok > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   const int warps = 8;
@@ -343,6 +358,37 @@ namespace {
 // Prefill of T new tokens per batch row after `start` cached ones (start > 0 needs the caches).
 // With `pg`, the cache is paged: the new keys and values go into the pages, and the row's
 // first start + T keys are gathered from the pages into the workspace for the attention.
+// The attention kernel, persistent (one CTA per SM, fewer for fewer items), as a
+// programmatic dependent launch: its CTAs may be scheduled while the kernel before it
+// finishes; they set up (barriers, TMEM, tensor maps, the logit bound) and wait
+// (griddepcontrol.wait) before their first load of Q', K' or the cache.
+int launch_fmha(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                const q3::PrefillParams& p, int max_items, bool window, bool varlen, cudaStream_t s) {
+  const int grid = max_items < num_sms() ? max_items : num_sms();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(q3::kPrefillThreads);
+  cfg.dynamicSmemBytes = q3::kPrefillSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t le;
+  if (varlen)
+    le = window ? cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<true, true>, mq, mk, mv, mo, p)
+                : cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false, true>, mq, mk, mv, mo, p);
+  else
+    le = window ? cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<true, false>, mq, mk, mv, mo, p)
+                : cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false, false>, mq, mk, mv, mo, p);
+  if (le != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+}
+
 int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
                  const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse, qwen3_bf16* k_cache,
                  qwen3_bf16* v_cache, int start, int Tcap, void* workspace, size_t ws_bytes, int B, int T, int Hq,
@@ -464,7 +510,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   }
 
   // 3. Attention.
-  q3::PrefillParams p;
+  q3::PrefillParams p{};
   p.q_norm_w = q_norm_w;
   p.k_norm_w = k_norm_w;
   p.lse = lse;
@@ -489,27 +535,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     std::lock_guard<std::mutex> lk(g_mu);
     p.fault = g_fault;
   }
-  const int grid = static_cast<int>(n_items < num_sms() ? n_items : num_sms());  // persistent: one CTA per SM
-  // Programmatic dependent launch: the attention CTAs may be scheduled while the prologue
-  // finishes; they set up (barriers, TMEM, tensor maps, the logit bound) and wait
-  // (griddepcontrol.wait) before their first load of Q', K' or the cache.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(q3::kPrefillThreads);
-  cfg.dynamicSmemBytes = q3::kPrefillSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t le = var.window > 0 ? cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<true>, mq, mk, mv, mo, p)
-                                        : cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false>, mq, mk, mv, mo, p);
-  if (le != cudaSuccess) {
-    (void)cudaGetLastError();
-    return QWEN3_ERR_CUDA;
-  }
-  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
+  return launch_fmha(mq, mk, mv, mo, p, static_cast<int>(n_items), var.window > 0, false, s);
 }
 
 }  // namespace
@@ -838,3 +864,225 @@ extern "C" int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* 
   return qwen3_attn_decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq,
                            Hkv, d, Lmax, theta, eps, scratch, QWEN3_ATTN_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// ---------------------------------------------------------------------------------------
+// Varlen batches: sequences packed on one token axis, optionally over a paged cache.
+namespace {
+
+// Workspace regions of a varlen prefill, each 256-byte aligned: the checked metadata
+// (seq [B], the entry list, the item count, level scratch), Q' [Hkv, N*G, d], and K' and V
+// [Hkv, rows, d] with rows = N (fresh prompts: the tokens' own keys) or key_cap (a cache:
+// every sequence's cached and new keys, gathered out of the pages).
+struct VarlenLayout {
+  size_t seq = 0, ent = 0, n_items = 0, lvl = 0, qp = 0, kp = 0, vp = 0, total = 0;
+  int two_p = 0, n_lvl = 0, max_entries = 0;
+  long long rows = 0;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool varlen_layout(int B, int N, long long key_cap, int Hq, int Hkv, VarlenLayout& L) {
+  if (B <= 0 || N <= 0 || key_cap < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !is_pow2(Hq / Hkv) ||
+      Hq / Hkv > 128)
+    return false;
+  const int G = Hq / Hkv;
+  L.two_p = 2 * (128 / G);
+  L.n_lvl = (N + L.two_p - 1) / L.two_p;
+  const long long max_entries = static_cast<long long>(L.n_lvl) + B;
+  if (max_entries * Hkv > 0x7fffffffLL) return false;
+  L.max_entries = static_cast<int>(max_entries);
+  L.rows = key_cap > 0 ? key_cap : N;
+  size_t o = 0;
+  L.seq = o;
+  o = align256(o + static_cast<size_t>(B) * 16);
+  L.ent = o;
+  o = align256(o + static_cast<size_t>(L.max_entries) * 32);
+  L.n_items = o;
+  o = align256(o + 4);
+  L.lvl = o;
+  o = align256(o + static_cast<size_t>(3) * (L.n_lvl + 1) * 4);
+  L.qp = o;
+  o = align256(o + static_cast<size_t>(N) * Hq * kD * 2);
+  L.kp = o;
+  o = align256(o + static_cast<size_t>(L.rows) * Hkv * kD * 2);
+  L.vp = o;
+  o = align256(o + static_cast<size_t>(L.rows) * Hkv * kD * 2);
+  L.total = o + 256;  // + slack to align the base
+  return true;
+}
+
+int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                const float* k_norm_w, const int32_t* pos, const int32_t* cu, qwen3_bf16* out, float* lse,
+                const PagedKV* pg, const int32_t* ctx, long long key_cap, void* workspace, size_t ws_bytes, int B,
+                int N, int Hq, int Hkv, int d, const Variant& var, float eps, qwen3_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr || pos == nullptr ||
+      cu == nullptr || out == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (B <= 0 || N <= 0) return QWEN3_ERR_INVALID_ARG;
+  int st = check_common(Hq, Hkv, d);
+  if (st != QWEN3_OK) return st;
+  if (Hq / Hkv > 128) return QWEN3_ERR_UNSUPPORTED;
+  if (pg == nullptr && (ctx != nullptr || key_cap != 0)) return QWEN3_ERR_INVALID_ARG;  // cached keys need a cache
+  if (pg != nullptr && key_cap <= 0) return QWEN3_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) ||
+      !aligned(k_norm_w, 8) || !aligned(pos, 4) || !aligned(cu, 4) || (ctx != nullptr && !aligned(ctx, 4)) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
+  // TMA row coordinates and element offsets stay within int32
+  if (static_cast<long long>(N) * Hq > (1LL << 31) / kD || key_cap > (1LL << 31) / kD / Hkv ||
+      static_cast<long long>(N) * Hkv > (1LL << 31) / kD)
+    return QWEN3_ERR_UNSUPPORTED;
+  VarlenLayout L;
+  if (!varlen_layout(B, N, key_cap, Hq, Hkv, L)) return QWEN3_ERR_UNSUPPORTED;
+  if (workspace == nullptr || ws_bytes < L.total) return QWEN3_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
+  const uintptr_t w0 = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~static_cast<uintptr_t>(255);
+  int4* seq = reinterpret_cast<int4*>(w0 + L.seq);
+  int4* ent = reinterpret_cast<int4*>(w0 + L.ent);
+  int* n_items = reinterpret_cast<int*>(w0 + L.n_items);
+  qwen3_bf16* qp = reinterpret_cast<qwen3_bf16*>(w0 + L.qp);
+  qwen3_bf16* kp = reinterpret_cast<qwen3_bf16*>(w0 + L.kp);
+  qwen3_bf16* vp = reinterpret_cast<qwen3_bf16*>(w0 + L.vp);
+
+  // 1. Metadata: checked sequences and the item list, on the device.
+  q3::VarlenParams vp_{};
+  vp_.cu = cu;
+  vp_.ctx = ctx;
+  vp_.seq = seq;
+  vp_.ent = ent;
+  vp_.n_items = n_items;
+  vp_.lvl = reinterpret_cast<int*>(w0 + L.lvl);
+  vp_.key_cap = pg != nullptr ? key_cap : 0;
+  vp_.B = B;
+  vp_.N = N;
+  vp_.two_p = L.two_p;
+  vp_.Hkv = Hkv;
+  vp_.n_lvl = L.n_lvl;
+  vp_.max_entries = L.max_entries;
+  vp_.max_keys = pg != nullptr ? pg->max_blocks * pg->page : 0x7fffffff;
+  q3::varlen_setup_kernel<<<1, q3::kVarlenThreads, 0, s>>>(vp_);
+  if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+
+  // 2. QK prologue over the packed axis (one batch row of N tokens): Q' in the query tiles'
+  //    row order; K' and a copy of V into the workspace (fresh prompts) or into each
+  //    sequence's pages (a cache).
+  PrologueQ pq;
+  pq.xq = q;
+  pq.wq = q_norm_w;
+  pq.dstq = qp;
+  pq.Hq = Hq;
+  PrologueVarlen vl;
+  vl.cu = cu;
+  vl.B = B;
+  if (pg == nullptr) {
+    st = launch_prologue(k, k_norm_w, pos, kp, v, vp, 1, N, Hkv, N, 0, var, eps, s, pq, nullptr, 0, vl);
+    if (st != QWEN3_OK) return st;
+  } else {
+    vl.seq = seq;
+    st = launch_prologue(k, k_norm_w, pos, pg->k, v, pg->v, 1, N, Hkv, 1, 0, var, eps, s, pq, pg, 0, vl);
+    if (st != QWEN3_OK) return st;
+    // 3. Every sequence's keys and values, cached and new, out of the pages.
+    q3::VarlenGatherParams gp{};
+    gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
+    gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
+    gp.block_table = pg->table;
+    gp.seq = seq;
+    gp.k_out = reinterpret_cast<uint4*>(kp);
+    gp.v_out = reinterpret_cast<uint4*>(vp);
+    gp.key_cap = key_cap;
+    gp.B = B;
+    gp.Hkv = Hkv;
+    gp.max_blocks = pg->max_blocks;
+    gp.log2_page = pg->log2_page;
+    gp.num_pages = pg->num_pages;
+    const long long chunks = key_cap * Hkv * 16;
+    long long blocks = (chunks + 255) / 256;
+    if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
+    q3::varlen_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
+    if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+  }
+
+  // 4. Tensor maps over the packed layouts (batch coordinate 0).
+  const int G = Hq / Hkv;
+  CUtensorMap mq, mk, mv, mo;
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  {
+    const cuuint64_t odims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(Hq),
+                                 static_cast<cuuint64_t>(N), 1};
+    const cuuint64_t ostr[3] = {kD * 2ull, static_cast<cuuint64_t>(Hq) * kD * 2ull,
+                                static_cast<cuuint64_t>(N) * Hq * kD * 2ull};
+    const cuuint32_t obox[4] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G), 1};
+    if (!make_map(&mo, out, 4, odims, ostr, obox)) return QWEN3_ERR_CUDA;
+  }
+  {
+    const cuuint64_t NG = static_cast<cuuint64_t>(N) * G;
+    const cuuint64_t qdims[4] = {static_cast<cuuint64_t>(kD), NG, static_cast<cuuint64_t>(Hkv), 1};
+    const cuuint64_t qstr[3] = {kD * 2ull, NG * kD * 2ull, static_cast<cuuint64_t>(Hkv) * NG * kD * 2ull};
+    if (!make_map(&mq, qp, 4, qdims, qstr, box)) return QWEN3_ERR_CUDA;
+  }
+  {
+    const cuuint64_t R = static_cast<cuuint64_t>(L.rows);
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), R, static_cast<cuuint64_t>(Hkv), 1};
+    const cuuint64_t str[3] = {kD * 2ull, R * kD * 2ull, static_cast<cuuint64_t>(Hkv) * R * kD * 2ull};
+    if (!make_map(&mk, kp, 4, dims, str, box) || !make_map(&mv, vp, 4, dims, str, box)) return QWEN3_ERR_CUDA;
+  }
+
+  // 5. Attention over the device's item list.
+  q3::PrefillParams p{};
+  p.q_norm_w = q_norm_w;
+  p.k_norm_w = k_norm_w;
+  p.lse = lse;
+  p.B = B;
+  p.T = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.log2G = ilog2(G);
+  p.P = 128 >> p.log2G;
+  p.n_items = L.max_entries * Hkv;
+  p.start = 0;
+  p.window = var.window;
+  p.rope_scale = var.scale;
+  p.eps = eps;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(kD)));
+  p.wait = next_wait_cfg();
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    p.fault = g_fault;
+  }
+  p.vl_ent = ent;
+  p.vl_n_items = n_items;
+  p.out = reinterpret_cast<uint4*>(out);
+  return launch_fmha(mq, mk, mv, mo, p, p.n_items, var.window > 0, true, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t qwen3_attn_prefill_varlen_workspace_size(int B, int N, long long key_cap, int Hq, int Hkv, int d) {
+  VarlenLayout L;
+  if (d != kD || !varlen_layout(B, N, key_cap, Hq, Hkv, L)) return 0;
+  return L.total;
+}
+
+int qwen3_attn_prefill_varlen(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
+                              const float* k_norm_w, const int32_t* pos, const int32_t* cu_seqlens, qwen3_bf16* out,
+                              float* lse, const qwen3_paged_kv* kv, const int32_t* ctx_lens, long long key_cap,
+                              void* workspace, size_t ws_bytes, int B, int N, int Hq, int Hkv, int d,
+                              const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream) {
+  Variant var;
+  int st = make_variant(variant, var);
+  if (st != QWEN3_OK) return st;
+  if (kv == nullptr)
+    return varlen_impl(q, k, v, q_norm_w, k_norm_w, pos, cu_seqlens, out, lse, nullptr, ctx_lens, key_cap, workspace,
+                       ws_bytes, B, N, Hq, Hkv, d, var, eps, stream);
+  if (Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
+  PagedKV pg;
+  if ((st = make_paged(kv, Hkv, pg)) != QWEN3_OK) return st;
+  return varlen_impl(q, k, v, q_norm_w, k_norm_w, pos, cu_seqlens, out, lse, &pg, ctx_lens, key_cap, workspace,
+                     ws_bytes, B, N, Hq, Hkv, d, var, eps, stream);
+}
+
+}  // extern "C"

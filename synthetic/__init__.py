@@ -116,6 +116,50 @@ CHUNK_SHAPES = {
 }
 
 
+@dataclass(frozen=True)
+class VarlenShape:
+    """B sequences packed on one token axis: new lengths `lens`, cached prefix lengths `ctx`
+    (empty: fresh prompts), and `lead` / `tail` padding tokens that belong to no sequence."""
+    name: str
+    lens: tuple
+    Hq: int
+    Hkv: int
+    ctx: tuple = ()
+    lead: int = 0
+    tail: int = 0
+    d: int = HEAD_DIM
+    theta: float = ROPE_THETA
+    eps: float = RMS_EPS
+
+    @property
+    def B(self) -> int:
+        return len(self.lens)
+
+    @property
+    def N(self) -> int:
+        return self.lead + sum(self.lens) + self.tail
+
+    @property
+    def contexts(self) -> tuple:
+        return self.ctx if self.ctx else (0,) * self.B
+
+    def causal_flops(self) -> float:
+        """QK^T and PV over each sequence's visible keys (new row i sees ctx + i + 1)."""
+        return sum(4.0 * self.Hq * self.d * (T * c + T * (T + 1) / 2.0) for T, c in zip(self.lens, self.contexts))
+
+
+def ragged_lengths(B: int, lo: int, hi: int, seed: int) -> tuple:
+    """B lengths log-uniform in [lo, hi] (a serving batch's mix of short and long prompts)."""
+    rng = np.random.default_rng(seed)
+    return tuple(int(x) for x in np.exp(rng.uniform(np.log(lo), np.log(hi), size=B)).round())
+
+
+VARLEN_SHAPES = {
+    "qwen3-4b-varlen": VarlenShape("Qwen3-4B-shaped varlen prefill, 16 prompts of log-uniform length in "
+                                   "[128, 8192], Hq=32 Hkv=8", ragged_lengths(16, 128, 8192, 2024), 32, 8),
+}
+
+
 def _bf16(x: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16)
 
@@ -248,3 +292,37 @@ def decode_history(shape: DecodeShape, n: int, length: int, s_k: torch.Tensor, s
 def as_f64(t: torch.Tensor) -> np.ndarray:
     """Exact widening of a bf16/fp32/int tensor to a float64 numpy array."""
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def varlen_inputs(shape: VarlenShape, seed: int = 0) -> dict:
+    """Packed inputs as CPU tensors: q [N,Hq,d], k and v [N,Hkv,d] drawn as one prompt of N
+    tokens by the recipe above; cu_seqlens [B+1] int32 (the first sequence starts after the
+    lead padding); pos [N] int32, ctx_b + t for token t of sequence b and 0 for padding;
+    ctx_lens [B] int32; and per sequence the raw history k_hist[b], v_hist[b] [ctx_b,Hkv,d]
+    (drawn after the gains, N(0,1), k scaled by s_k), which a cache holds after QK-Norm and
+    RoPE at positions 0..ctx_b-1."""
+    N, Hq, Hkv, d = shape.N, shape.Hq, shape.Hkv, shape.d
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((N, Hq, d), dtype=np.float32)
+    k = rng.standard_normal((N, Hkv, d), dtype=np.float32)
+    v = rng.standard_normal((N, Hkv, d), dtype=np.float32)
+    s_q, s_k = _scales(rng, d), _scales(rng, d)
+    g_q, g_k = _gains(rng, d), _gains(rng, d)
+    q *= s_q
+    k *= s_k
+    cu = np.concatenate([[shape.lead], shape.lead + np.cumsum(shape.lens, dtype=np.int64)]).astype(np.int32)
+    pos = np.zeros(N, dtype=np.int32)
+    k_hist, v_hist = [], []
+    for b, (T, c) in enumerate(zip(shape.lens, shape.contexts)):
+        pos[cu[b]:cu[b + 1]] = c + np.arange(T, dtype=np.int32)
+        kh = rng.standard_normal((c, Hkv, d), dtype=np.float32) * s_k
+        vh = rng.standard_normal((c, Hkv, d), dtype=np.float32)
+        k_hist.append(_bf16(kh))
+        v_hist.append(_bf16(vh))
+    return {
+        "q": _bf16(q), "k": _bf16(k), "v": _bf16(v),
+        "q_norm_w": torch.from_numpy(g_q), "k_norm_w": torch.from_numpy(g_k),
+        "pos": torch.from_numpy(pos), "cu_seqlens": torch.from_numpy(cu),
+        "ctx_lens": torch.from_numpy(np.asarray(shape.contexts, dtype=np.int32)),
+        "k_hist": k_hist, "v_hist": v_hist,
+    }

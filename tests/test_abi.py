@@ -158,6 +158,38 @@ def test_paged_argument_checks():
     assert qa.prefill_paged_workspace_size(2, -1, 300, 16, 8) == 0
 
 
+def test_varlen_argument_checks():
+    lib = qa.lib()
+    var, _ = qa.make_variant()
+
+    def pre(kv=None, ctx=None, key_cap=0, ws=None, ws_bytes=0, B=4, N=1000, Hq=16, Hkv=8, d=128, cu=FAKE, q=FAKE,
+            out=FAKE):
+        return lib.qwen3_attn_prefill_varlen(q, FAKE, FAKE, FAKE, FAKE, FAKE, cu, out, None, kv, ctx, key_cap, ws,
+                                             ws_bytes, B, N, Hq, Hkv, d, ctypes.byref(var), 1e-6, None)
+
+    good = qa.PagedKV(1 << 20, 1 << 20, 1 << 20, 100, 64, 40)
+    assert pre() == qa.ERR_WORKSPACE
+    assert pre(kv=ctypes.byref(good), key_cap=5000) == qa.ERR_WORKSPACE
+    assert pre(kv=ctypes.byref(good), ctx=FAKE, key_cap=5000) == qa.ERR_WORKSPACE
+    assert pre(ctx=FAKE) == qa.ERR_INVALID_ARG            # cached keys without a cache
+    assert pre(key_cap=10) == qa.ERR_INVALID_ARG          # a key capacity without a cache
+    assert pre(kv=ctypes.byref(good)) == qa.ERR_INVALID_ARG  # a cache without a key capacity
+    assert pre(cu=None) == qa.ERR_INVALID_ARG
+    assert pre(q=None) == qa.ERR_INVALID_ARG
+    assert pre(cu=ctypes.c_void_p((1 << 20) + 2)) == qa.ERR_INVALID_ARG  # misaligned offsets
+    assert pre(B=0) == qa.ERR_INVALID_ARG and pre(N=0) == qa.ERR_INVALID_ARG
+    assert pre(Hq=12) == qa.ERR_UNSUPPORTED and pre(d=64) == qa.ERR_UNSUPPORTED
+    # metadata, entry list and level scratch, Q' [N, Hq, d], K' and V [N, Hkv, d] (or key_cap rows)
+    n = qa.prefill_varlen_workspace_size(4, 1000, 16, 8)
+    assert n >= 1000 * (16 + 2 * 8) * 128 * 2 + 4 * 16
+    m = qa.prefill_varlen_workspace_size(4, 1000, 16, 8, key_cap=5000)
+    assert m - n >= 2 * (5000 - 1000) * 8 * 128 * 2
+    assert qa.prefill_varlen_workspace_size(0, 1000, 16, 8) == 0
+    assert qa.prefill_varlen_workspace_size(4, 1000, 16, 8, key_cap=-1) == 0
+    assert qa.prefill_varlen_workspace_size(4, 1000, 16, 8, d=64) == 0
+    assert pre(ws=FAKE, ws_bytes=n - 1) == qa.ERR_WORKSPACE
+
+
 def test_decode_and_prologue_argument_checks():
     lib = qa.lib()
 

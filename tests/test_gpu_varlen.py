@@ -1,0 +1,289 @@
+"""Varlen batched prefill through the C ABI: sequences packed on one token axis, fresh or
+over a paged cache, against the fp64 oracle (oracle.varlen_prefill_ref) on the same seeded
+inputs, and bit for bit against the uniform-batch entry points run one sequence at a time.
+Padding tokens (before the first sequence and after the last) hold NaN inputs: they must
+neither leak into any sequence nor have their output rows written."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import qwen3_qk_norm_rope_b200 as qa
+from synthetic import VarlenShape, as_f64, varlen_inputs
+from tests.gpu_common import LSE_TOL, assert_status_ok, compare, dev, to_np
+
+pytestmark = pytest.mark.gpu
+NAN16 = 0x7FC1
+THETA, EPS = 1.0e6, 1.0e-6
+
+
+def _poison_padding(inp, shape):
+    """NaN raw q/k/v for the padding tokens (no sequence owns them)."""
+    for name in ("q", "k", "v"):
+        t = inp[name]
+        t[:shape.lead] = float("nan")
+        if shape.tail:
+            t[shape.N - shape.tail:] = float("nan")
+
+
+def _prefix(inp, b, gk):
+    """Sequence b's cache contents in key order: keys normed and rotated at 0..ctx-1, raw values."""
+    kc = oracle.build_cache_k(as_f64(inp["k_hist"][b]), gk, THETA, EPS).transpose(1, 0, 2)  # [Hkv, ctx, d]
+    vc = as_f64(inp["v_hist"][b]).transpose(1, 0, 2)
+    return kc, vc
+
+
+def _oracle(inp, shape, prefixes=None, window=0):
+    args = (as_f64(inp["q"]), as_f64(inp["k"]), as_f64(inp["v"]), as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]),
+            inp["pos"].numpy(), inp["cu_seqlens"].numpy(), THETA, EPS)
+    kw = dict(window=window)
+    if prefixes is not None:
+        kw.update(k_prefix=[p[0] for p in prefixes], v_prefix=[p[1] for p in prefixes])
+    ref, ref_lse = oracle.varlen_prefill_ref(*args, **kw)
+    _, st_lse = oracle.varlen_prefill_ref(*args, staged=True, **kw)
+    return ref, ref_lse, st_lse
+
+
+def _owned(shape):
+    return np.arange(shape.lead, shape.N - shape.tail)
+
+
+# The LSE checks.  Against the pure fp64 oracle each row is held to a rigorous bound: the
+# LSE is 1-Lipschitz in the largest change of any logit, and rounding q' and k' to bf16
+# (2^-9 relative each; fp32 accumulation adds 2^-17) changes logit j by at most
+# (2^-8 + 2^-17) sum_i |q'_i k'_ji| / sqrt(d); the fp32 softmax sum adds at most
+# keys x 2^-24 relative.  Against the staged oracle (q', k' rounded to bf16 as the kernels
+# round them) the kernel differs only where its fp32 q' or k' element lands on the other
+# side of a bf16 rounding boundary: rare, and at most 2^-8 |q'_i k'_i| / sqrt(d) (~3e-3 at
+# these inputs' sizes) in a row whose softmax is dominated by that key.  A varlen batch has
+# many rows that see few keys (each sequence's first rows), so the staged check allows
+# STRADDLE_TOL on at most 1 row-head in 10^4 and holds the rest to 1e-3.
+STRADDLE_TOL, STRADDLE_FRACTION = 4e-3, 1e-4
+
+
+def _rigorous_bound(inp, shape, prefixes=None):
+    """Per (head, token) bound on |LSE_kernel - LSE_pure| for the owned rows, NaN elsewhere."""
+    G = shape.Hq // shape.Hkv
+    gq, gk = as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"])
+    cu = inp["cu_seqlens"].numpy()
+    bound = np.full((shape.Hq, shape.N), np.nan)
+    for b, (T, c) in enumerate(zip(shape.lens, shape.contexts)):
+        if T == 0:
+            continue
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        qp = np.abs(oracle.qk_prologue(as_f64(inp["q"][sl]), gq, inp["pos"][sl].numpy(), THETA, EPS))  # [T, Hq, d]
+        kp = np.abs(oracle.qk_prologue(as_f64(inp["k"][sl]), gk, inp["pos"][sl].numpy(), THETA, EPS))  # [T, Hkv, d]
+        if c:
+            kp = np.concatenate([np.abs(prefixes[b][0]).transpose(1, 0, 2), kp], axis=0)  # cached keys first
+        visible = np.arange(c + T)[None, :] <= (c + np.arange(T))[:, None]  # [T, c + T]
+        for h in range(shape.Hq):
+            a = np.where(visible, qp[:, h] @ kp[:, h // G].T, 0.0)
+            bound[h, sl] = (2.0 ** -8 + 2.0 ** -17) * a.max(-1) / np.sqrt(128.0) + 1e-5 + \
+                (c + 1 + np.arange(T)) * 2.0 ** -24
+    return bound
+
+
+def _compare(out, lse, ref, ref_lse, st_lse, shape, what, inp, prefixes=None):
+    """Owned rows only: outputs by the usual bounds; the LSE by the rigorous bound against
+    the pure oracle and by the straddle rule against the staged one."""
+    own = _owned(shape)
+    compare(to_np(out[own]), None, ref[own], None, None, what)
+    got = to_np(lse)[:, own]
+    bound = _rigorous_bound(inp, shape, prefixes)[:, own]
+    e_pure = np.abs(got - ref_lse[:, own])
+    assert np.all(e_pure <= bound), f"{what}: lse vs pure oracle {(e_pure - bound).max():.3e} over the rigorous bound"
+    e_st = np.abs(got - st_lse[:, own])
+    assert e_st.max() <= STRADDLE_TOL, f"{what}: lse vs staged oracle {e_st.max():.3e}"
+    frac = float(np.mean(e_st > LSE_TOL))
+    assert frac <= STRADDLE_FRACTION, f"{what}: {frac:.2e} of row-heads over {LSE_TOL} against the staged oracle"
+
+
+def _run_fresh(inp, shape, window=0):
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    out = torch.empty((shape.N, shape.Hq, 128), dtype=torch.bfloat16, device=d)
+    out.view(torch.int16).fill_(NAN16)
+    lse = torch.full((shape.Hq, shape.N), float("nan"), dtype=torch.float32, device=d)
+    qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"], out=out,
+                      lse=lse, window=window)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    return out, lse
+
+
+@pytest.mark.parametrize("lens,Hq,Hkv,lead,tail", [
+    ((1, 129, 700, 0, 300, 64), 16, 8, 3, 5),   # G=2: a single token, an empty sequence, ragged tails
+    ((2053, 128, 5), 32, 8, 0, 0),             # G=4: one long sequence, a tile-aligned one
+    ((257, 1000, 31), 64, 4, 7, 0),            # G=16: P=8 positions per tile
+])
+def test_varlen_fresh(lens, Hq, Hkv, lead, tail):
+    shape = VarlenShape("varlen fresh", lens, Hq, Hkv, lead=lead, tail=tail)
+    inp = varlen_inputs(shape, seed=sum(lens) + Hq)
+    _poison_padding(inp, shape)
+    out, lse = _run_fresh(inp, shape)
+    ref, ref_lse, st_lse = _oracle(inp, shape)
+    _compare(out, lse, ref, ref_lse, st_lse, shape, f"varlen {lens} G{Hq // Hkv}", inp)
+    _check_padding_untouched(out, lse, shape)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (64, 4)])
+def test_varlen_equals_one_sequence_at_a_time(Hq, Hkv):
+    """Each packed sequence gives the same bits as the uniform prefill of that sequence alone
+    (the same tiles, keys and accumulation order; only the work list differs)."""
+    shape = VarlenShape("varlen vs uniform", (300, 1, 1500, 129, 640), Hq, Hkv, lead=2, tail=3)
+    inp = varlen_inputs(shape, seed=5)
+    out, lse = _run_fresh(inp, shape)
+    d = dev()
+    cu = inp["cu_seqlens"].numpy()
+    for b in range(shape.B):
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        one = {k: inp[k][sl][None].to(d) for k in ("q", "k", "v", "pos")}
+        l1 = torch.empty((1, shape.Hq, sl.stop - sl.start), dtype=torch.float32, device=d)
+        o1 = qa.prefill(one["q"], one["k"], one["v"], inp["q_norm_w"].to(d), inp["k_norm_w"].to(d), one["pos"], lse=l1)
+        torch.cuda.synchronize()
+        assert_status_ok()
+        assert torch.equal(o1[0], out[sl]), f"sequence {b}"
+        assert torch.equal(l1[0], lse[:, sl]), f"sequence {b} lse"
+
+
+def test_varlen_window():
+    shape = VarlenShape("varlen window", (900, 77, 400), 16, 8, tail=2)
+    inp = varlen_inputs(shape, seed=17)
+    out, lse = _run_fresh(inp, shape, window=256)
+    ref, ref_lse, st_lse = _oracle(inp, shape, window=256)
+    _compare(out, lse, ref, ref_lse, st_lse, shape, "varlen window 256", inp)
+
+
+def _tables(rows, blocks_needed, max_blocks, num_pages, seed):
+    rng = np.random.default_rng(seed)
+    perm = rng.permutation(num_pages)
+    table = np.full((rows, max_blocks), -1, dtype=np.int32)
+    k = 0
+    for r in range(rows):
+        for b in range(blocks_needed[r]):
+            table[r, b] = perm[k]
+            k += 1
+    return table
+
+
+def _scatter(pool, table_row, keys, page):
+    for j in range(keys.shape[1]):
+        pool[int(table_row[j // page]), :, j % page] = keys[:, j]
+
+
+@pytest.mark.parametrize("page", [16, 64, 256])
+def test_varlen_paged(page):
+    lens, ctx = (300, 1, 129, 500, 0), (0, 300, 1000, 17, 40)
+    shape = VarlenShape("varlen paged", lens, 16, 8, ctx=ctx, lead=1, tail=4)
+    inp = varlen_inputs(shape, seed=page)
+    _poison_padding(inp, shape)
+    gk = as_f64(inp["k_norm_w"])
+    need = [-(-(c + T) // page) for T, c in zip(lens, ctx)]
+    max_blocks = max(need) + 2
+    num_pages = sum(need) + 6
+    table = _tables(shape.B, need, max_blocks, num_pages, seed=page + 1)
+    kp = torch.empty((num_pages, 8, page, 128), dtype=torch.bfloat16)
+    kp.view(torch.int16).fill_(NAN16)
+    vp = kp.clone()
+    prefixes = []
+    for b in range(shape.B):
+        kc, vc = _prefix(inp, b, gk)
+        _scatter(kp, table[b], torch.from_numpy(kc.copy()).to(torch.bfloat16), page)
+        _scatter(vp, table[b], torch.from_numpy(vc.copy()).to(torch.bfloat16), page)
+        prefixes.append((kc, vc))
+    before_k, before_v = kp.clone(), vp.clone()
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    kpd, vpd = kp.to(d), vp.to(d)
+    out = torch.empty((shape.N, 16, 128), dtype=torch.bfloat16, device=d)
+    out.view(torch.int16).fill_(NAN16)
+    lse = torch.full((16, shape.N), float("nan"), dtype=torch.float32, device=d)
+    key_cap = sum(c + T for T, c in zip(lens, ctx)) + 3
+    qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"], k_pages=kpd,
+                      v_pages=vpd, block_table=torch.from_numpy(table).to(d), ctx_lens=t["ctx_lens"], key_cap=key_cap,
+                      out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    ref, ref_lse, st_lse = _oracle(inp, shape, prefixes)
+    _compare(out, lse, ref, ref_lse, st_lse, shape, f"varlen paged {page}", inp, prefixes)
+    _check_padding_untouched(out, lse, shape)
+    # the new keys and values sit in their sequences' pages after the cached ones; nothing
+    # else in the pools changed
+    ka, va = kpd.cpu(), vpd.cpu()
+    cu = inp["cu_seqlens"].numpy()
+    written = torch.zeros_like(ka, dtype=torch.bool)
+    for b, (T, c) in enumerate(zip(lens, ctx)):
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        kref = oracle.qk_prologue(as_f64(inp["k"][sl]), gk, inp["pos"][sl].numpy(), THETA, EPS).transpose(1, 0, 2)
+        got = oracle.paged_gather(to_np(ka), table[b], c + T, page)
+        assert np.array_equal(got[:, :c], prefixes[b][0])  # the cached keys are as they were
+        assert np.all(np.abs(got[:, c:] - kref) <= np.abs(kref) * 2.0 ** -8 + 2e-5)
+        gotv = oracle.paged_gather(to_np(va), table[b], c + T, page)[:, c:]
+        assert np.array_equal(gotv, as_f64(inp["v"][sl]).transpose(1, 0, 2))
+        for j in range(c, c + T):
+            written[int(table[b, j // page]), :, j % page] = True
+    keep = ~written
+    assert torch.equal(ka.view(torch.int16)[keep], before_k.view(torch.int16)[keep])
+    assert torch.equal(va.view(torch.int16)[keep], before_v.view(torch.int16)[keep])
+
+
+def test_varlen_paged_equals_prefill_paged():
+    """A paged varlen batch gives the same bits as qwen3_attn_prefill_paged run on each
+    sequence alone with start = its cached length."""
+    lens, ctx, page = (200, 640, 3), (500, 0, 129), 64
+    shape = VarlenShape("varlen paged vs chunk", lens, 32, 8, ctx=ctx)
+    inp = varlen_inputs(shape, seed=23)
+    gk = as_f64(inp["k_norm_w"])
+    need = [-(-(c + T) // page) for T, c in zip(lens, ctx)]
+    max_blocks = max(need)
+    table = _tables(shape.B, need, max_blocks, sum(need), seed=3)
+    kp = torch.zeros((sum(need), 8, page, 128), dtype=torch.bfloat16)
+    vp = torch.zeros_like(kp)
+    for b in range(shape.B):
+        kc, vc = _prefix(inp, b, gk)
+        _scatter(kp, table[b], torch.from_numpy(kc.copy()).to(torch.bfloat16), page)
+        _scatter(vp, table[b], torch.from_numpy(vc.copy()).to(torch.bfloat16), page)
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    tab = torch.from_numpy(table).to(d)
+    kv1, vv1 = kp.to(d), vp.to(d)
+    lse = torch.empty((32, shape.N), dtype=torch.float32, device=d)
+    out = qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"],
+                            k_pages=kv1, v_pages=vv1, block_table=tab, ctx_lens=t["ctx_lens"],
+                            key_cap=sum(lens) + sum(ctx), lse=lse)
+    kv2, vv2 = kp.to(d), vp.to(d)
+    cu = inp["cu_seqlens"].numpy()
+    for b in range(shape.B):
+        sl = slice(int(cu[b]), int(cu[b + 1]))
+        l1 = torch.empty((1, 32, lens[b]), dtype=torch.float32, device=d)
+        o1 = qa.prefill_paged(t["q"][sl][None], t["k"][sl][None], t["v"][sl][None], t["q_norm_w"], t["k_norm_w"],
+                              t["pos"][sl][None], kv2, vv2, tab[b:b + 1].contiguous(), ctx[b], lse=l1)
+        torch.cuda.synchronize()
+        assert_status_ok()
+        assert torch.equal(o1[0], out[sl]), f"sequence {b}"
+        assert torch.equal(l1[0], lse[:, sl]), f"sequence {b} lse"
+    assert torch.equal(kv1, kv2) and torch.equal(vv1, vv2)
+
+
+def test_varlen_invalid_sequence_is_skipped_and_reported():
+    """A sequence whose end lies past N is recorded as an invalid argument and skipped; the
+    others are computed as usual."""
+    shape = VarlenShape("varlen invalid", (200, 300, 100), 16, 8)
+    inp = varlen_inputs(shape, seed=31)
+    inp["cu_seqlens"] = torch.tensor([0, 200, 500, shape.N + 7], dtype=torch.int32)
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    out = torch.empty((shape.N, 16, 128), dtype=torch.bfloat16, device=d)
+    out.view(torch.int16).fill_(NAN16)
+    qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"], out=out)
+    torch.cuda.synchronize()
+    st, site = qa.device_status(clear=True)
+    assert st == qa.ERR_INVALID_ARG and site == 70
+    assert torch.all(out[500:].view(torch.int16) == NAN16)
+    good = dict(inp)
+    for k in ("q", "k", "v", "pos"):
+        good[k] = inp[k][:500]
+    good["cu_seqlens"] = torch.tensor([0, 200, 500], dtype=torch.int32)
+    ref, _, _ = _oracle(good, None)
+    err = np.abs(to_np(out[:500]) - ref)
+    assert err.max() <= 2e-2 and err.mean() <= 2e-3
