@@ -22,9 +22,14 @@
 //      the heaviest items go first (for fresh prompts an item's work grows with its pair
 //      index), and within one pair index by np_b descending: at pair index L the sequences
 //      with np_b > L are exactly the first count_L of that order.  A sequence's rank in it
-//      is (number of sequences with more pairs) + (a tie counter); its entry at pair index
-//      L sits at base_L + rank.  No sort is needed, only level histograms and two scans.
+//      is (number of sequences with more pairs) + (a tie counter), and order[rank] = b.
+//      Entry e then lies at the pair index L with base_L <= e < base_L + count_L (a binary
+//      search over base) and belongs to sequence order[e - base_L].  No sort is needed,
+//      only a level histogram and two scans, and every loop is spread over the CTA.
 //   4. n_items = Hkv x entries; item i is entry i / Hkv for KV head i % Hkv.
+// The three level arrays live in shared memory when they fit in 36 KB (up to 3071 pair
+// indices; with the 8 KB scan buffer the CTA stays within the default 48 KB), else in the
+// workspace.
 #pragma once
 #include "common.cuh"
 
@@ -32,6 +37,7 @@ namespace q3 {
 
 constexpr int kSiteVarlenMeta = 70;  // a sequence's metadata failed validation
 constexpr int kVarlenThreads = 1024;
+constexpr int kVarlenSmemLevels = 3072;  // level entries kept in shared memory: 3 arrays, 36 KB
 
 struct VarlenParams {
   const int* cu;    // [B + 1] token offsets
@@ -40,6 +46,8 @@ struct VarlenParams {
   int4* ent;        // [2 * max_entries] out: {qoff, T, start, koff}, {pair, b, 0, 0}
   int* n_items;     // [1] out
   int* lvl;         // scratch [3 * (n_lvl + 1)]: histogram, tie counters, then count_L / base_L
+  int* order;       // scratch [B]: the sequence at each rank
+  int lvl_in_smem;  // the level arrays are in dynamic shared memory instead of lvl
   long long key_cap;  // key rows of the gathered layout (cache), 0 without a cache
   int B, N, two_p, Hkv, n_lvl, max_entries;
   int max_keys;       // keys one sequence may address (cache: max_blocks * page_size)
@@ -65,11 +73,13 @@ __device__ __forceinline__ T cta_exclusive_scan(T v, T* s, T& total) {
 
 __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const __grid_constant__ VarlenParams p) {
   __shared__ long long s_scan[kVarlenThreads];
+  extern __shared__ int s_levels[];
   const int tid = threadIdx.x;
-  int* hist = p.lvl;                    // [n_lvl + 1]: sequences with np_b = v
-  int* tie = p.lvl + (p.n_lvl + 1);     // [n_lvl + 1]: ranks handed out among equal np_b
-  int* lvl = p.lvl + 2 * (p.n_lvl + 1); // [n_lvl + 1]: count_L, then base_L
-  for (int i = tid; i < 3 * (p.n_lvl + 1); i += kVarlenThreads) p.lvl[i] = 0;
+  int* const L3 = p.lvl_in_smem ? s_levels : p.lvl;
+  int* hist = L3;                    // [n_lvl + 1]: sequences with np_b = v
+  int* tie = L3 + (p.n_lvl + 1);     // [n_lvl + 1]: ranks handed out among equal np_b
+  int* lvl = L3 + 2 * (p.n_lvl + 1); // [n_lvl + 1]: count_L, then base_L
+  for (int i = tid; i < 3 * (p.n_lvl + 1); i += kVarlenThreads) L3[i] = 0;
 
   // 1-2. validate, then key offsets by a running sum over the sequences (each thread owns a
   //      contiguous run of them, so the order of koff is the order of b).
@@ -146,23 +156,33 @@ __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const _
   }
   __syncthreads();
 
-  // 4. entries.  base_{L-1} - base_L = count_L, so the number of sequences with more pairs
+  // 4. ranks.  base_{L-1} - base_L = count_L, so the number of sequences with more pairs
   //    than this one is base_{np_b - 1} - base_{np_b}.
   for (int b = b0; b < b1; ++b) {
-    const int4 s = p.seq[b];
-    const int np = min((s.y + p.two_p - 1) / p.two_p, p.n_lvl);
+    const int np = min((p.seq[b].y + p.two_p - 1) / p.two_p, p.n_lvl);
     if (np == 0) continue;
-    const int above = lvl[np - 1] - lvl[np];  // sequences with more pairs than this one
-    const int rank = above + atomicAdd(&tie[np], 1);
-    for (int L = 0; L < np; ++L) {
-      const int e = lvl[L] + rank;
-      if (e < p.max_entries) {
-        p.ent[2 * e] = s;
-        p.ent[2 * e + 1] = make_int4(L, b, 0, 0);
+    const int rank = (lvl[np - 1] - lvl[np]) + atomicAdd(&tie[np], 1);
+    p.order[rank] = b;
+  }
+  __syncthreads();
+  // 5. entries, one per thread and step: pair index L = the smallest with base_L <= e
+  //    (base_L does not increase with L), sequence order[e - base_L].
+  const int n_ent = min(total_entries, p.max_entries);
+  for (int e = tid; e < n_ent; e += kVarlenThreads) {
+    int lo = 0, hi = p.n_lvl - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (lvl[mid] <= e) {
+        hi = mid;
+      } else {
+        lo = mid + 1;
       }
     }
+    const int b = p.order[e - lvl[lo]];
+    p.ent[2 * e] = p.seq[b];
+    p.ent[2 * e + 1] = make_int4(lo, b, 0, 0);
   }
-  if (tid == 0) *p.n_items = min(total_entries, p.max_entries) * p.Hkv;
+  if (tid == 0) *p.n_items = n_ent * p.Hkv;
 }
 
 // Keys and values of every sequence (its ctx cached keys and its new ones) out of the pages

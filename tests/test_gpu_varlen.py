@@ -98,6 +98,13 @@ def _compare(out, lse, ref, ref_lse, st_lse, shape, what, inp, prefixes=None):
     assert frac <= STRADDLE_FRACTION, f"{what}: {frac:.2e} of row-heads over {LSE_TOL} against the staged oracle"
 
 
+def _check_padding_untouched(out, lse, shape):
+    pad = np.r_[0:shape.lead, shape.N - shape.tail:shape.N]
+    if pad.size:
+        assert torch.all(out[pad].view(torch.int16) == NAN16)
+        assert torch.isnan(lse[:, pad]).all()
+
+
 def _run_fresh(inp, shape, window=0):
     d = dev()
     t = {k: v.to(d) for k, v in inp.items() if isinstance(v, torch.Tensor)}
