@@ -324,16 +324,34 @@ def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seq
 CHUNK_METRIC = "chunked-prefill causal GQA attn TFLOP/s (+QK-Norm/RoPE, cache append) % bf16 peak"
 
 
+def paged_copy(caches, n: int, page: int, seed: int, dev):
+    """Page pools [num_pages, Hkv, page, d] holding the first n rows of each [B, Hkv, >=n, d]
+    cache, pages dealt in a seeded random order, and the [B, ceil(n/page)] block table."""
+    B, Hkv, _, d = caches[0].shape
+    nb = -(-n // page)
+    g = torch.Generator().manual_seed(seed + 77)
+    table = torch.randperm(B * nb, generator=g).to(torch.int32).view(B, nb)
+    pools = []
+    for c in caches:
+        pool = torch.zeros((B * nb, Hkv, page, d), dtype=c.dtype, device=dev)
+        src = torch.zeros((B, Hkv, nb * page, d), dtype=c.dtype, device=dev)
+        src[:, :, :n] = c[:, :, :n]
+        pool[table.view(-1).long().to(dev)] = src.view(B, Hkv, nb, page, d).permute(0, 2, 1, 3, 4).reshape(
+            B * nb, Hkv, page, d)
+        pools.append(pool)
+    return pools[0], pools[1], table.to(dev)
+
+
 class ChunkWorkload:
     """Device-resident inputs of the chunked-prefill call: the new tokens, and caches whose
     first `start` slots hold the prefix (normed and rotated by the library's prologue)."""
 
     LAUNCHES_PER_STEP = 2  # K prologue (cache append) + attention
 
-    def __init__(self, dev: torch.device, name: str = "qwen3-4b-second-chunk", seed: int = 0):
+    def __init__(self, dev: torch.device, name: str = "qwen3-4b-second-chunk", seed: int = 0, page: int = 0):
         import qwen3_qk_norm_rope_b200 as qa
 
-        self.qa, self.dev = qa, dev
+        self.qa, self.dev, self.page = qa, dev, page
         self.cs = cs = CHUNK_SHAPES[name]
         inp = chunk_inputs(cs, seed=seed)
         self.host = {k: inp[k] for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
@@ -346,6 +364,11 @@ class ChunkWorkload:
                         v_dst=self.vc, theta=cs.theta, eps=cs.eps)
         self.out = torch.empty_like(self.t["q"])
         self.ws = torch.empty(qa.prefill_workspace_size(cs.B, cs.T, cs.Hq, cs.Hkv), dtype=torch.uint8, device=dev)
+        if page:
+            # the same caches in pages of `page` tokens, dealt to the rows in a seeded random order
+            self.k_pages, self.v_pages, self.table = paged_copy([self.kc, self.vc], Tcap, page, seed, dev)
+            self.ws = torch.empty(qa.prefill_paged_workspace_size(cs.B, cs.start, cs.T, cs.Hq, cs.Hkv),
+                                  dtype=torch.uint8, device=dev)
         self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
         st, site = qa.device_status(clear=True, device=dev)
@@ -354,12 +377,18 @@ class ChunkWorkload:
 
     def step(self):
         t, cs = self.t, self.cs
+        if self.page:
+            self.qa.prefill_paged(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], self.k_pages,
+                                  self.v_pages, self.table, cs.start, out=self.out, workspace=self.ws,
+                                  theta=cs.theta, eps=cs.eps)
+            return
         self.qa.prefill_chunk(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], self.kc, self.vc,
                               cs.start, out=self.out, workspace=self.ws, theta=cs.theta, eps=cs.eps)
 
     def config(self):
         cs = self.cs
-        return {"workload": cs.name, "B": cs.B, "start": cs.start, "T": cs.T, "Hq": cs.Hq, "Hkv": cs.Hkv,
+        return {"workload": cs.name + (f", cache in pages of {self.page}" if self.page else ""), "B": cs.B,
+                "start": cs.start, "T": cs.T, "Hq": cs.Hq, "Hkv": cs.Hkv, "page": self.page or None,
                 "d": cs.d, "rope_theta": cs.theta, "rms_eps": cs.eps, "seed": 0,
                 "l2": "flushed before every step (256 MiB write, outside the timed windows)",
                 "parallelism": "replicas (one independent workload per GPU)"}
@@ -417,7 +446,7 @@ def run_chunk(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    w = ChunkWorkload(dev)
+    w = ChunkWorkload(dev, page=args.paged)
     for _ in range(args.warmup):
         w.flush.fill_(1.0)
         w.step()
@@ -467,9 +496,10 @@ def run_chunk(args, world, rank, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": w.config(),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                         "kernel": "chunked-prefill call (K prologue + cache append + attention)",
+                         "kernel": "chunked-prefill call (K prologue + cache append + attention)" if not w.page
+                         else "paged chunked-prefill call (K prologue into pages + gather + attention)",
                          "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
-            "gpu_launches": ChunkWorkload.LAUNCHES_PER_STEP * K, "clocks": clk.summary(),
+            "gpu_launches": (ChunkWorkload.LAUNCHES_PER_STEP + (1 if w.page else 0)) * K, "clocks": clk.summary(),
             "e2e": {"value": world * flops * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
                     "ms_per_step": e_ms / e_steps}}
@@ -623,23 +653,24 @@ def cpu_oracle_varlen_sample(name: str, rows: int = 256, seed: int = 0):
     b = int(np.argmax(sh.lens))
     cu = inp["cu_seqlens"].numpy()
     sl = slice(int(cu[b]), int(cu[b + 1]))
-    T = sh.lens[b]
+    T, c = sh.lens[b], sh.contexts[b]
     rows = min(rows, T)
     sel = np.arange(T - rows, T)
-    empty = np.zeros((1, sh.Hkv, 0, sh.d))
+    kc = oracle.build_cache_k(as_f64(inp["k_hist"][b]), as_f64(inp["k_norm_w"]), sh.theta, sh.eps).transpose(1, 0, 2)
+    vc = as_f64(inp["v_hist"][b]).transpose(1, 0, 2)
     t0 = time.perf_counter()
     oracle.chunk_prefill_ref(as_f64(inp["q"][sl])[None], as_f64(inp["k"][sl])[None], as_f64(inp["v"][sl])[None],
-                             as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][sl].numpy()[None], empty,
-                             empty, 0, sh.theta, sh.eps, rows=sel)
+                             as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][sl].numpy()[None], kc[None],
+                             vc[None], c, sh.theta, sh.eps, rows=sel)
     secs = time.perf_counter() - t0
-    flops = 4.0 * sh.Hq * sh.d * float((sel + 1).sum())
+    flops = 4.0 * sh.Hq * sh.d * float((c + sel + 1).sum())
     try:
         from threadpoolctl import threadpool_info
         threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:  # noqa: BLE001
         threads = os.cpu_count()
-    sample = (f"last {rows} of {T} query rows x {sh.Hq} heads of the longest sequence of the {sh.name} "
-              f"({flops:.3g} causal flops)")
+    sample = (f"last {rows} of {T} query rows x {sh.Hq} heads of the longest sequence of the {sh.name}"
+              + (f" (over its {c} cached keys)" if c else "") + f" ({flops:.3g} causal flops)")
     return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "sample": sample, "flops": flops}
 
 
@@ -723,12 +754,49 @@ def run_varlen(args, world, rank, local):
     host = {k: inp[k] for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos", "cu_seqlens")}
     t = {k: v.to(dev) for k, v in host.items()}
     out = torch.empty((sh.N, sh.Hq, sh.d), dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(qa.prefill_varlen_workspace_size(sh.B, sh.N, sh.Hq, sh.Hkv), dtype=torch.uint8, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    cached = any(sh.contexts)
+    page = (args.paged or 64) if cached else 0
+    kv = {}
+    key_cap = 0
+    if cached:
+        # each sequence's prefix, normed and rotated by the library's prologue, in pages of
+        # `page` tokens dealt in a seeded random order; the call appends the new keys after it
+        need = [-(-(c + T) // page) for T, c in zip(sh.lens, sh.contexts)]
+        g = torch.Generator().manual_seed(78)
+        perm = torch.randperm(sum(need), generator=g).to(torch.int32)
+        table = torch.full((sh.B, max(need)), -1, dtype=torch.int32)
+        off = 0
+        for b, nb in enumerate(need):
+            table[b, :nb] = perm[off:off + nb]
+            off += nb
+        k_pages = torch.zeros((sum(need), sh.Hkv, page, sh.d), dtype=torch.bfloat16, device=dev)
+        v_pages = torch.zeros_like(k_pages)
+        for b, c in enumerate(sh.contexts):
+            if c == 0:
+                continue
+            nb = -(-c // page)
+            kc = torch.zeros((1, sh.Hkv, nb * page, sh.d), dtype=torch.bfloat16, device=dev)
+            vc = torch.zeros_like(kc)
+            pos_b = torch.arange(c, dtype=torch.int32, device=dev)[None]
+            qa.qk_norm_rope(inp["k_hist"][b][None].to(dev), t["k_norm_w"], pos_b, kc,
+                            v_src=inp["v_hist"][b][None].to(dev), v_dst=vc, theta=sh.theta, eps=sh.eps)
+            rows = table[b, :nb].long().to(dev)
+            k_pages[rows] = kc[0].view(sh.Hkv, nb, page, sh.d).permute(1, 0, 2, 3)
+            v_pages[rows] = vc[0].view(sh.Hkv, nb, page, sh.d).permute(1, 0, 2, 3)
+        key_cap = sum(sh.lens) + sum(sh.contexts)
+        kv = dict(k_pages=k_pages, v_pages=v_pages, block_table=table.to(dev), ctx_lens=inp["ctx_lens"].to(dev),
+                  key_cap=key_cap)
+        torch.cuda.synchronize(dev)
+        st, site = qa.device_status(clear=True, device=dev)
+        if st != qa.OK:
+            raise RuntimeError(f"cache build failed: {qa.status_string(st)} at site {site}")
+    ws = torch.empty(qa.prefill_varlen_workspace_size(sh.B, sh.N, sh.Hq, sh.Hkv, key_cap=key_cap),
+                     dtype=torch.uint8, device=dev)
 
     def step():
         qa.prefill_varlen(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], t["cu_seqlens"], out=out,
-                          workspace=ws, theta=sh.theta, eps=sh.eps)
+                          workspace=ws, theta=sh.theta, eps=sh.eps, **kv)
 
     K = args.steps
     ms, e_ms, h2d, d2h, clk = time_call(step, flush, host, t, [out], K, args.warmup, world, local, dev,
@@ -740,15 +808,17 @@ def run_varlen(args, world, rank, local):
     line = {"metric": VARLEN_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": sh.name, "lens": list(sh.lens), "N": sh.N, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+            "config": {"workload": sh.name + (f", pages of {page}" if page else ""), "lens": list(sh.lens),
+                       "ctx": list(sh.contexts) if cached else None, "N": sh.N, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
                        "rope_theta": sh.theta, "rms_eps": sh.eps, "seed": 0,
                        "l2": "flushed before every step (256 MiB write, outside the timed windows)",
                        "parallelism": "replicas (one independent workload per GPU)"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                         "kernel": "varlen prefill call (metadata + QK prologue + attention)",
+                         "kernel": "varlen prefill call (metadata + QK prologue + attention)" if not cached
+                         else "paged varlen prefill call (metadata + QK prologue into pages + gather + attention)",
                          "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
-            "gpu_launches": 3 * K, "clocks": clk.summary(),
+            "gpu_launches": (4 if cached else 3) * K, "clocks": clk.summary(),
             "e2e": {"value": world * flops * max(1, min(K, 100)) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e_ms / max(1, min(K, 100))}}
@@ -858,6 +928,9 @@ def main():
                     help="the qkv-proj workload's shape")
     ap.add_argument("--varlen", default="qwen3-4b-varlen", choices=sorted(VARLEN_SHAPES),
                     help="the varlen-prefill workload's shape")
+    ap.add_argument("--paged", type=int, default=0,
+                    help="chunked-prefill: keep the cache in pages of this many tokens (0: contiguous); "
+                         "varlen-prefill: the page size of a shape with cached prefixes (default 64)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup("nccl")

@@ -870,11 +870,11 @@ extern "C" int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* 
 namespace {
 
 // Workspace regions of a varlen prefill, each 256-byte aligned: the checked metadata
-// (seq [B], the entry list, the item count, level scratch), Q' [Hkv, N*G, d], and K' and V
+// (seq [B], the entry list, the item count, rank scratch), Q' [Hkv, N*G, d], and K' and V
 // [Hkv, rows, d] with rows = N (fresh prompts: the tokens' own keys) or key_cap (a cache:
 // every sequence's cached and new keys, gathered out of the pages).
 struct VarlenLayout {
-  size_t seq = 0, ent = 0, n_items = 0, lvl = 0, order = 0, qp = 0, kp = 0, vp = 0, total = 0;
+  size_t seq = 0, ent = 0, n_items = 0, np = 0, sbase = 0, qp = 0, kp = 0, vp = 0, total = 0;
   int two_p = 0, n_lvl = 0, max_entries = 0;
   long long rows = 0;
 };
@@ -899,9 +899,9 @@ bool varlen_layout(int B, int N, long long key_cap, int Hq, int Hkv, VarlenLayou
   o = align256(o + static_cast<size_t>(L.max_entries) * 32);
   L.n_items = o;
   o = align256(o + 4);
-  L.lvl = o;
-  o = align256(o + static_cast<size_t>(3) * (L.n_lvl + 1) * 4);
-  L.order = o;
+  L.np = o;
+  o = align256(o + static_cast<size_t>(B) * 4);
+  L.sbase = o;
   o = align256(o + static_cast<size_t>(B) * 4);
   L.qp = o;
   o = align256(o + static_cast<size_t>(N) * Hq * kD * 2);
@@ -955,19 +955,16 @@ int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, c
   vp_.seq = seq;
   vp_.ent = ent;
   vp_.n_items = n_items;
-  vp_.lvl = reinterpret_cast<int*>(w0 + L.lvl);
-  vp_.order = reinterpret_cast<int*>(w0 + L.order);
-  vp_.lvl_in_smem = L.n_lvl + 1 <= q3::kVarlenSmemLevels;
+  vp_.np = reinterpret_cast<int*>(w0 + L.np);
+  vp_.sbase = reinterpret_cast<int*>(w0 + L.sbase);
   vp_.key_cap = pg != nullptr ? key_cap : 0;
   vp_.B = B;
   vp_.N = N;
   vp_.two_p = L.two_p;
   vp_.Hkv = Hkv;
-  vp_.n_lvl = L.n_lvl;
   vp_.max_entries = L.max_entries;
   vp_.max_keys = pg != nullptr ? pg->max_blocks * pg->page : 0x7fffffff;
-  const size_t lvl_smem = vp_.lvl_in_smem ? static_cast<size_t>(3) * (L.n_lvl + 1) * 4 : 0;
-  q3::varlen_setup_kernel<<<1, q3::kVarlenThreads, lvl_smem, s>>>(vp_);
+  q3::varlen_setup_kernel<<<1, q3::kVarlenThreads, 0, s>>>(vp_);
   if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
 
   // 2. QK prologue over the packed axis (one batch row of N tokens): Q' in the query tiles'

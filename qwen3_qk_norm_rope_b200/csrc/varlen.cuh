@@ -18,18 +18,20 @@
 //      row of the sequence's keys in the gathered key layout (a running sum of ctx + T;
 //      without a cache the keys are the tokens themselves, koff = qoff);
 //   3. the entry list: sequence b has np_b = ceil(T_b / 2P) pairs of query tiles (P token
-//      positions per 128-row tile).  Entries are ordered by pair index, highest first, so
-//      the heaviest items go first (for fresh prompts an item's work grows with its pair
-//      index), and within one pair index by np_b descending: at pair index L the sequences
-//      with np_b > L are exactly the first count_L of that order.  A sequence's rank in it
-//      is (number of sequences with more pairs) + (a tie counter), and order[rank] = b.
-//      Entry e then lies at the pair index L with base_L <= e < base_L + count_L (a binary
-//      search over base) and belongs to sequence order[e - base_L].  No sort is needed,
-//      only a level histogram and two scans, and every loop is spread over the CTA.
+//      positions per 128-row tile), and its pair p reads about c_b + (p + 1) 2P keys (its
+//      cached ones and the new ones up to the pair's diagonal).  Entries go by that count,
+//      largest first, ties by sequence: the heaviest items lead and the lightest fill the
+//      tail, as in the uniform kernel's order.  For fresh prompts that is pair index first;
+//      with long cached prefixes the prefix dominates the count, so the items of one
+//      sequence come together and the CTAs that take them at the same time share its keys
+//      and values in L2 (a batch's prefixes can exceed L2, and an order that visits every
+//      sequence at each pair index reads each prefix from DRAM once per pair).
+//      Entry e of sequence b (found by binary search over the running sum of np in b
+//      order) counts, over every sequence, the entries with a larger key count or an equal
+//      one and a smaller b: that is its position.  O(B) per entry, spread over the CTA;
+//      the pair counts and cached lengths sit in shared memory for up to kVarlenSmemSeqs
+//      sequences.  No sort is needed.
 //   4. n_items = Hkv x entries; item i is entry i / Hkv for KV head i % Hkv.
-// The three level arrays live in shared memory when they fit in 36 KB (up to 3071 pair
-// indices; with the 8 KB scan buffer the CTA stays within the default 48 KB), else in the
-// workspace.
 #pragma once
 #include "common.cuh"
 
@@ -37,7 +39,7 @@ namespace q3 {
 
 constexpr int kSiteVarlenMeta = 70;  // a sequence's metadata failed validation
 constexpr int kVarlenThreads = 1024;
-constexpr int kVarlenSmemLevels = 3072;  // level entries kept in shared memory: 3 arrays, 36 KB
+constexpr int kVarlenSmemSeqs = 2048;  // pair counts and cached lengths kept in shared memory (16 KB)
 
 struct VarlenParams {
   const int* cu;    // [B + 1] token offsets
@@ -45,11 +47,10 @@ struct VarlenParams {
   int4* seq;        // [B] out: {qoff, T, start, koff}
   int4* ent;        // [2 * max_entries] out: {qoff, T, start, koff}, {pair, b, 0, 0}
   int* n_items;     // [1] out
-  int* lvl;         // scratch [3 * (n_lvl + 1)]: histogram, tie counters, then count_L / base_L
-  int* order;       // scratch [B]: the sequence at each rank
-  int lvl_in_smem;  // the level arrays are in dynamic shared memory instead of lvl
+  int* np;          // scratch [B]: pairs of each sequence
+  int* sbase;       // scratch [B]: its first entry in sequence order
   long long key_cap;  // key rows of the gathered layout (cache), 0 without a cache
-  int B, N, two_p, Hkv, n_lvl, max_entries;
+  int B, N, two_p, Hkv, max_entries;
   int max_keys;       // keys one sequence may address (cache: max_blocks * page_size)
 };
 
@@ -73,13 +74,9 @@ __device__ __forceinline__ T cta_exclusive_scan(T v, T* s, T& total) {
 
 __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const __grid_constant__ VarlenParams p) {
   __shared__ long long s_scan[kVarlenThreads];
-  extern __shared__ int s_levels[];
+  __shared__ int s_np[kVarlenSmemSeqs], s_ctx[kVarlenSmemSeqs];
   const int tid = threadIdx.x;
-  int* const L3 = p.lvl_in_smem ? s_levels : p.lvl;
-  int* hist = L3;                    // [n_lvl + 1]: sequences with np_b = v
-  int* tie = L3 + (p.n_lvl + 1);     // [n_lvl + 1]: ranks handed out among equal np_b
-  int* lvl = L3 + 2 * (p.n_lvl + 1); // [n_lvl + 1]: count_L, then base_L
-  for (int i = tid; i < 3 * (p.n_lvl + 1); i += kVarlenThreads) L3[i] = 0;
+  const bool in_smem = p.B <= kVarlenSmemSeqs;
 
   // 1-2. validate, then key offsets by a running sum over the sequences (each thread owns a
   //      contiguous run of them, so the order of koff is the order of b).
@@ -95,7 +92,7 @@ __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const _
   long long total_keys;
   long long koff = cta_exclusive_scan(mine, s_scan, total_keys);
   (void)total_keys;
-  __syncthreads();  // the level scratch is cleared before the histogram below
+  long long n_mine = 0;  // entries of this thread's sequences
   for (int b = b0; b < b1; ++b) {
     int lo = p.cu[b], hi = p.cu[b + 1];
     int c = p.ctx != nullptr ? p.ctx[b] : 0;
@@ -117,70 +114,54 @@ __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const _
     const int T = hi - lo;
     p.seq[b] = make_int4(lo, T, c, static_cast<int>(kb));
     const int np = (T + p.two_p - 1) / p.two_p;
-    if (np > 0) atomicAdd(&hist[min(np, p.n_lvl)], 1);
-  }
-  __syncthreads();
-
-  // 3. count_L = #{b : np_b > L} = sum of hist[v] over v > L (a suffix sum), then
-  //    base_L = sum of count_L' over L' > L (another); both as CTA scans over level runs.
-  const int lper = (p.n_lvl + 1 + kVarlenThreads - 1) / kVarlenThreads;
-  const int l0 = min(p.n_lvl + 1, tid * lper), l1 = min(p.n_lvl + 1, l0 + lper);
-  {
-    // Suffix sums: the levels above a thread's run are the runs of the higher threads,
-    // whose sum is the total minus this thread's inclusive prefix.
-    long long run = 0;
-    for (int v = l0; v < l1; ++v) run += hist[v];
-    long long tot;
-    const long long before = cta_exclusive_scan(run, s_scan, tot);
-    long long after = tot - before - run;  // sequences counted at levels above this thread's run
-    for (int v = l1 - 1; v >= l0; --v) {
-      lvl[v] = static_cast<int>(after);  // count_v = #{np > v}
-      after += hist[v];
+    p.np[b] = np;
+    if (in_smem) {
+      s_np[b] = np;
+      s_ctx[b] = c;
     }
+    n_mine += np;
   }
-  __syncthreads();
-  int total_entries;
-  {
-    long long run = 0;
-    for (int v = l0; v < l1; ++v) run += lvl[v];
-    long long tot;
-    const long long before = cta_exclusive_scan(run, s_scan, tot);
-    long long after = tot - before - run;
-    __syncthreads();
-    for (int v = l1 - 1; v >= l0; --v) {
-      const int cnt = lvl[v];
-      lvl[v] = static_cast<int>(after);  // base_v: entries of all higher pair indices
-      after += cnt;
-    }
-    total_entries = static_cast<int>(tot);
-  }
-  __syncthreads();
-
-  // 4. ranks.  base_{L-1} - base_L = count_L, so the number of sequences with more pairs
-  //    than this one is base_{np_b - 1} - base_{np_b}.
+  // 3a. each sequence's first entry in sequence order
+  long long total;
+  long long e0 = cta_exclusive_scan(n_mine, s_scan, total);
   for (int b = b0; b < b1; ++b) {
-    const int np = min((p.seq[b].y + p.two_p - 1) / p.two_p, p.n_lvl);
-    if (np == 0) continue;
-    const int rank = (lvl[np - 1] - lvl[np]) + atomicAdd(&tie[np], 1);
-    p.order[rank] = b;
+    p.sbase[b] = static_cast<int>(min(e0, static_cast<long long>(p.max_entries)));
+    e0 += p.np[b];
   }
   __syncthreads();
-  // 5. entries, one per thread and step: pair index L = the smallest with base_L <= e
-  //    (base_L does not increase with L), sequence order[e - base_L].
-  const int n_ent = min(total_entries, p.max_entries);
+
+  // 3b. entries: entry e of sequence b (the last b whose first entry is <= e: sequences with
+  //     no pairs share the first entry of the next one) is pair p = e - sbase[b], reading
+  //     about kc = c_b + (p + 1) 2P keys; its position counts the entries with more keys,
+  //     and those with as many keys in a sequence before b.
+  const int* const NP = in_smem ? s_np : p.np;
+  const int n_ent = static_cast<int>(min(total, static_cast<long long>(p.max_entries)));
   for (int e = tid; e < n_ent; e += kVarlenThreads) {
-    int lo = 0, hi = p.n_lvl - 1;
+    int lo = 0, hi = p.B - 1;
     while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (lvl[mid] <= e) {
-        hi = mid;
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.sbase[mid] <= e) {
+        lo = mid;
       } else {
-        lo = mid + 1;
+        hi = mid - 1;
       }
     }
-    const int b = p.order[e - lvl[lo]];
-    p.ent[2 * e] = p.seq[b];
-    p.ent[2 * e + 1] = make_int4(lo, b, 0, 0);
+    const int b = lo;
+    const int pair = e - p.sbase[b];
+    const int4 sq = p.seq[b];
+    const long long kc = sq.z + static_cast<long long>(pair + 1) * p.two_p;
+    long long pos = 0;
+    for (int o = 0; o < p.B; ++o) {
+      const int npo = NP[o];
+      const long long k = kc - (in_smem ? s_ctx[o] : p.seq[o].z);  // pairs of o with more keys: (q + 1) 2P > k
+      const long long first = k < 0 ? 0 : min(static_cast<long long>(npo), k / p.two_p);
+      pos += npo - first;
+      if (o < b && k >= p.two_p && k % p.two_p == 0 && k / p.two_p <= npo) ++pos;  // as many keys, earlier b
+    }
+    if (pos < p.max_entries) {
+      p.ent[2 * pos] = sq;
+      p.ent[2 * pos + 1] = make_int4(pair, b, 0, 0);
+    }
   }
   if (tid == 0) *p.n_items = n_ent * p.Hkv;
 }

@@ -157,6 +157,12 @@ def ragged_lengths(B: int, lo: int, hi: int, seed: int) -> tuple:
 VARLEN_SHAPES = {
     "qwen3-4b-varlen": VarlenShape("Qwen3-4B-shaped varlen prefill, 16 prompts of log-uniform length in "
                                    "[128, 8192], Hq=32 Hkv=8", ragged_lengths(16, 128, 8192, 2024), 32, 8),
+    # continuous batching: new chunks of 64..2048 tokens over cached prefixes of 256..16384
+    "qwen3-4b-varlen-cached": VarlenShape("Qwen3-4B-shaped varlen prefill over a paged cache, 16 chunks of "
+                                          "log-uniform length in [64, 2048] after cached prefixes of log-uniform "
+                                          "length in [256, 16384], Hq=32 Hkv=8",
+                                          ragged_lengths(16, 64, 2048, 7), 32, 8,
+                                          ctx=ragged_lengths(16, 256, 16384, 8)),
 }
 
 
