@@ -50,8 +50,12 @@ constexpr int kPrologueHeads = 8;  // head vectors of one token in flight per wa
 
 // One warp per token (b, t): its position and the sin/cos of its 64 angles are computed
 // once and shared by the token's H key heads (and, for the prefill, its Hq query heads),
-// whose loads are issued a batch at a time before any arithmetic.
-__global__ void __launch_bounds__(256) qk_norm_rope_kernel(const __grid_constant__ PrologueParams p) {
+// whose loads are issued a batch at a time before any arithmetic.  Each warp's work is a
+// fixed chain of dependent loads, so the kernel takes as many chain times as it has waves:
+// at most 64 registers a thread keeps 4 blocks (32 warps) resident per SM, which holds the
+// 4096 tokens of a B=2, T=2048 prefill in one wave (at 80 registers only 3 blocks fit and
+// 68 blocks ran as a second wave).
+__global__ void __launch_bounds__(256, 4) qk_norm_rope_kernel(const __grid_constant__ PrologueParams p) {
   // The RoPE constants go through shared memory once per block: read from parameter space
   // with a lane-dependent index they would serialise.
   __shared__ float s_rope[2 * kHalf];
