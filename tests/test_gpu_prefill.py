@@ -1,6 +1,7 @@
 """Prefill parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
-seeded inputs.  Full parity on the small and Qwen3-0.6B-shaped workloads and on ragged
-shapes; sampled query rows on the 4B-shaped and long wide-GQA workloads at full size."""
+seeded inputs.  Full parity on the small, Qwen3-0.6B-shaped and Qwen3-4B-shaped workloads
+and on ragged shapes; on the long wide-GQA workload (T = 32768, 64 query heads) every head
+of the first 256 rows, 1024 seeded random rows and the last 256 rows, at full size."""
 import numpy as np
 import pytest
 import torch
@@ -8,12 +9,13 @@ import torch
 import oracle
 import qwen3_qk_norm_rope_b200 as qa
 from synthetic import PREFILL_SHAPES, PrefillShape, as_f64, prefill_inputs
-from tests.gpu_common import (assert_status_ok, compare, dev, prefill_gpu, prefill_oracle, to_np)
+from tests.gpu_common import (assert_status_ok, check_lse_straddle, compare, dev, prefill_gpu,
+                              prefill_lse_bound, prefill_oracle, to_np)
 
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("name", ["tiny", "qwen3-0.6b"])
+@pytest.mark.parametrize("name", ["tiny", "qwen3-0.6b", "qwen3-4b"])
 def test_prefill_full_parity(name):
     shape = PREFILL_SHAPES[name]
     inp = prefill_inputs(shape, seed=0)
@@ -55,8 +57,7 @@ def _sampled_rows(T, n_first, n_rand, n_last, seed):
     return np.unique(np.concatenate([np.arange(n_first), mid, np.arange(T - n_last, T)]))
 
 
-@pytest.mark.parametrize("name,n_first,n_rand,n_last", [("qwen3-4b", 256, 512, 256),
-                                                         ("long-wide-gqa", 128, 192, 128)])
+@pytest.mark.parametrize("name,n_first,n_rand,n_last", [("long-wide-gqa", 256, 1024, 256)])
 def test_prefill_full_size_sampled_rows(name, n_first, n_rand, n_last):
     shape = PREFILL_SHAPES[name]
     inp = prefill_inputs(shape, seed=0)
@@ -65,7 +66,10 @@ def test_prefill_full_size_sampled_rows(name, n_first, n_rand, n_last):
     ref, ref_lse, st_lse = prefill_oracle(inp, rows=rows)
     o = to_np(out[:, torch.from_numpy(rows).to(out.device)])
     l = to_np(lse[:, :, torch.from_numpy(rows).to(out.device)])
-    compare(o, l, ref, ref_lse, st_lse, name + " sampled rows")
+    compare(o, None, ref, None, None, name + " sampled rows")
+    # 98K row-heads of G = 16, a quarter of them in rows that see at most 256 keys: the LSE
+    # goes by the straddle rule (one straddle was measured at 2.05e-3 here).
+    check_lse_straddle(l, ref_lse, st_lse, prefill_lse_bound(inp, rows), name + " sampled rows")
     # every row, not only the sampled ones, must be finite
     assert torch.isfinite(out.float()).all()
 
