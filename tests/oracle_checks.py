@@ -123,6 +123,25 @@ def check_rope_relative_position():
         assert abs(val - base) < 1e-9 * max(1.0, abs(base))
 
 
+def check_rope_relative_position_printed_pairs():
+    """The pages' own example: token 5 attending to token 3 and token 50 attending to token
+    48 get the same score, for every query and key vector and every frequency."""
+    pairs = json.load(open(GOLDEN))["rope_relative_position"]["same_signal_pairs"]
+    q = _rand((8, 1, D), 16)
+    k = _rand((8, 1, D), 17)
+    vals = []
+    for m, n in pairs:
+        dq = A.rope(q, np.full(8, m), THETA)[:, 0]
+        dk = A.rope(k, np.full(8, n), THETA)[:, 0]
+        vals.append(np.sum(dq * dk, axis=-1))
+    assert np.allclose(vals[0], vals[1], rtol=1e-12, atol=1e-12)
+    # and the signal does change with the distance (the pin would pass for a RoPE that
+    # ignored positions altogether otherwise)
+    m, n = pairs[0]
+    far = np.sum(A.rope(q, np.full(8, m), THETA)[:, 0] * A.rope(k, np.full(8, n + 7), THETA)[:, 0], axis=-1)
+    assert np.max(np.abs(far - vals[0])) > 1e-3
+
+
 # ---------------------------------------------------------------- attention
 def check_row0_is_v0():
     """Prefill row 0 sees only key 0: out = v_0 of KV head h//G, lse = s_00."""
