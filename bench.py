@@ -272,52 +272,109 @@ def time_e2e(w: Workload, steps: int):
 
 
 # ------------------------------------------------------------------------------ CPU oracle
+def oracle_threads() -> int:
+    """BLAS threads the oracle's numpy runs on: the cores a CPU-baseline figure used."""
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        return os.cpu_count()
+
+
+def prefill_oracle(batch_rows: int = 2, seed: int = 0):
+    """The fp64 oracle on the Qwen3-0.6B-shaped prefill with its inputs built once: the
+    returned run(rows) times one oracle call on the last `rows` query rows (every head) of
+    the first `batch_rows` batch rows and returns its seconds, causal flops and a
+    description of the sample."""
+    import oracle
+    from synthetic import as_f64
+
+    ps = PREFILL_SHAPES["qwen3-0.6b"]
+    inp = prefill_inputs(ps, seed=seed)
+    args = (as_f64(inp["q"][:batch_rows]), as_f64(inp["k"][:batch_rows]), as_f64(inp["v"][:batch_rows]),
+            as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][:batch_rows].numpy(), ps.theta, ps.eps)
+
+    def run(rows: int) -> dict:
+        sel = np.arange(ps.T - rows, ps.T)
+        t0 = time.perf_counter()
+        oracle.prefill_ref(*args, rows=sel)
+        secs = time.perf_counter() - t0
+        flops = batch_rows * 4.0 * ps.Hq * ps.d * float((sel + 1).sum())
+        return {"seconds": secs, "flops": flops,
+                "sample": (f"prefill: last {rows} of {ps.T} query rows x {ps.Hq} heads of {batch_rows} of {ps.B} "
+                           f"batch rows of the Qwen3-0.6B-shaped workload ({flops:.3g} causal flops)")}
+
+    run.max_rows = ps.T
+    return run
+
+
+def decode_oracle_sample(decode_seqs: int = 16, seed: int = 0) -> dict:
+    """The oracle's decode of the first `decode_seqs` sequences of the batched decode; their
+    caches are built (normed and rotated keys) before the timed call."""
+    import oracle
+    from synthetic import as_f64, decode_history
+
+    ds = DECODE_SHAPES["batched-decode"]
+    step = decode_step_inputs(ds, seed=seed)
+    lens = step["cache_lens"].numpy()
+    sel = list(range(decode_seqs))
+    kh, vh = [], []
+    for n in sel:
+        h = decode_history(ds, n, int(lens[n]), step["s_k"], seed=seed)
+        kh.append(oracle.build_cache_k(as_f64(h["k_hist"]), as_f64(step["k_norm_w"]), ds.theta,
+                                       ds.eps).transpose(1, 0, 2))
+        vh.append(as_f64(h["v_hist"]).transpose(1, 0, 2))
+    t0 = time.perf_counter()
+    oracle.decode_ref(as_f64(step["q"])[sel], as_f64(step["k_new"])[sel], as_f64(step["v_new"])[sel],
+                      as_f64(step["q_norm_w"]), as_f64(step["k_norm_w"]), kh, vh, lens[sel], ds.theta, ds.eps)
+    secs = time.perf_counter() - t0
+    return {"seconds": secs, "gbs": decode_bytes(lens[sel], ds.Hq, ds.Hkv) / secs / 1e9,
+            "sample": f"decode: first {decode_seqs} of 64 sequences ({int(lens[sel].sum())} cached tokens)"}
+
+
 def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seqs: int = 16, seed: int = 0):
     """The fp64 oracle, as it stands, on a bounded sample of the same workload: the last
     `rows_per_head` query rows (every head) of the first `batch_rows` batch rows of the
     Qwen3-0.6B-shaped prefill (the defaults are the whole prefill), and the first
     `decode_seqs` sequences of the batched decode.  Returns TFLOP/s on the prefill sample,
     GB/s on the decode sample, the seconds each took and the BLAS thread count."""
-    import oracle
-    from synthetic import as_f64, decode_history
+    pre = prefill_oracle(batch_rows, seed)(rows_per_head)
+    dec = decode_oracle_sample(decode_seqs, seed) if decode_seqs > 0 else \
+        {"seconds": 0.0, "gbs": 0.0, "sample": "no decode"}
+    return {"tflops": pre["flops"] / pre["seconds"] / 1e12, "gbs": dec["gbs"], "t_prefill_s": pre["seconds"],
+            "t_decode_s": dec["seconds"], "threads": oracle_threads(), "sample": pre["sample"] + "; " + dec["sample"],
+            "flops": pre["flops"]}
 
-    ps = PREFILL_SHAPES["qwen3-0.6b"]
-    inp = prefill_inputs(ps, seed=seed)
-    rows = np.arange(ps.T - rows_per_head, ps.T)
-    args = (as_f64(inp["q"][:batch_rows]), as_f64(inp["k"][:batch_rows]), as_f64(inp["v"][:batch_rows]),
-            as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][:batch_rows].numpy(), ps.theta, ps.eps)
-    t0 = time.perf_counter()
-    oracle.prefill_ref(*args, rows=rows)
-    t_pre = time.perf_counter() - t0
-    flops = batch_rows * 4.0 * ps.Hq * ps.d * float((rows + 1).sum())
-    t_dec, gbs, lens_sel = 0.0, 0.0, []
-    if decode_seqs > 0:
-        ds = DECODE_SHAPES["batched-decode"]
-        step = decode_step_inputs(ds, seed=seed)
-        lens = step["cache_lens"].numpy()
-        sel = list(range(decode_seqs))
-        kh, vh = [], []
-        for n in sel:
-            h = decode_history(ds, n, int(lens[n]), step["s_k"], seed=seed)
-            kh.append(oracle.build_cache_k(as_f64(h["k_hist"]), as_f64(step["k_norm_w"]), ds.theta,
-                                           ds.eps).transpose(1, 0, 2))
-            vh.append(as_f64(h["v_hist"]).transpose(1, 0, 2))
-        t0 = time.perf_counter()
-        oracle.decode_ref(as_f64(step["q"])[sel], as_f64(step["k_new"])[sel], as_f64(step["v_new"])[sel],
-                          as_f64(step["q_norm_w"]), as_f64(step["k_norm_w"]), kh, vh, lens[sel], ds.theta, ds.eps)
-        t_dec = time.perf_counter() - t0
-        gbs = decode_bytes(lens[sel], ds.Hq, ds.Hkv) / t_dec / 1e9
-        lens_sel = [int(lens[n]) for n in sel]
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count()
-    sample = (f"prefill: last {rows_per_head} of {ps.T} query rows x {ps.Hq} heads of {batch_rows} of {ps.B} "
-              f"batch rows of the Qwen3-0.6B-shaped workload ({flops:.3g} causal flops); decode: first "
-              f"{decode_seqs} of 64 sequences ({sum(lens_sel)} cached tokens)")
-    return {"tflops": flops / t_pre / 1e12, "gbs": gbs, "t_prefill_s": t_pre, "t_decode_s": t_dec,
-            "threads": threads, "sample": sample, "flops": flops}
+
+# The reference arm times the oracle for about this many seconds in all (warm-up and timed
+# steps together), whatever --steps and --warmup ask for: each step's sample is sized to fit.
+REFERENCE_BUDGET_S = 120.0
+
+
+def reference_steps(run, steps: int, warmup: int):
+    """The reference arm's loop over an oracle whose inputs are already built: calibrate its
+    cost per query row from two sample sizes (so a fixed per-call cost is not taken for a
+    per-row one), size each step's sample so that `warmup` + `steps` calls take about
+    REFERENCE_BUDGET_S seconds (one row at least), then run the untimed warm-up calls and
+    the timed steps.  Only the oracle calls themselves are timed.  Returns the timed
+    seconds, the flops, the rows per step and the last step's sample description."""
+    lo, hi = min(8, run.max_rows), min(264, run.max_rows)
+    t_lo = min(run(lo)["seconds"] for _ in range(2))  # the better of two calls: the first is a warm-up too
+    t_hi = min(run(hi)["seconds"] for _ in range(2))
+    per_row = max((t_hi - t_lo) / max(hi - lo, 1), 1e-7)
+    fixed = max(t_lo - lo * per_row, 0.0)
+    per_step = REFERENCE_BUDGET_S / max(steps + warmup, 1)
+    rows = int(max(1, min(run.max_rows, (per_step - fixed) / per_row)))
+    for _ in range(warmup):
+        run(rows)
+    secs = flops = 0.0
+    res = None
+    for _ in range(steps):
+        res = run(rows)
+        secs += res["seconds"]
+        flops += res["flops"]
+    return secs, flops, rows, res["sample"]
 
 
 # ------------------------------------------------------------------------------ chunked prefill
@@ -394,8 +451,9 @@ class ChunkWorkload:
                 "parallelism": "replicas (one independent workload per GPU)"}
 
 
-def cpu_oracle_chunk_sample(name: str = "qwen3-4b-second-chunk", rows: int = 512, seed: int = 0):
-    """The oracle's chunked prefill on the last `rows` new rows (every head) of the chunk."""
+def chunk_oracle(name: str = "qwen3-4b-second-chunk", seed: int = 0):
+    """The oracle's chunked prefill with its inputs and cached prefix built once: run(rows)
+    times one call on the last `rows` new rows (every head) of the chunk."""
     import oracle
     from synthetic import as_f64
 
@@ -404,42 +462,41 @@ def cpu_oracle_chunk_sample(name: str = "qwen3-4b-second-chunk", rows: int = 512
     kc = np.stack([oracle.build_cache_k(as_f64(inp["k_hist"][b]), as_f64(inp["k_norm_w"]), cs.theta, cs.eps)
                    .transpose(1, 0, 2) for b in range(cs.B)])
     vc = as_f64(inp["v_hist"]).transpose(0, 2, 1, 3)
-    sel = np.arange(cs.T - rows, cs.T)
-    t0 = time.perf_counter()
-    oracle.chunk_prefill_ref(as_f64(inp["q"]), as_f64(inp["k"]), as_f64(inp["v"]), as_f64(inp["q_norm_w"]),
-                             as_f64(inp["k_norm_w"]), inp["pos"].numpy(), kc, vc, cs.start, cs.theta, cs.eps,
-                             rows=sel)
-    secs = time.perf_counter() - t0
-    flops = cs.B * 4.0 * cs.Hq * cs.d * float((cs.start + sel + 1).sum())
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count()
-    sample = (f"last {rows} of {cs.T} new rows x {cs.Hq} heads of the {cs.name} ({flops:.3g} causal flops)")
-    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "sample": sample, "flops": flops}
+    args = (as_f64(inp["q"]), as_f64(inp["k"]), as_f64(inp["v"]), as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]),
+            inp["pos"].numpy(), kc, vc, cs.start, cs.theta, cs.eps)
+
+    def run(rows: int) -> dict:
+        sel = np.arange(cs.T - rows, cs.T)
+        t0 = time.perf_counter()
+        oracle.chunk_prefill_ref(*args, rows=sel)
+        secs = time.perf_counter() - t0
+        flops = cs.B * 4.0 * cs.Hq * cs.d * float((cs.start + sel + 1).sum())
+        return {"seconds": secs, "flops": flops,
+                "sample": f"last {rows} of {cs.T} new rows x {cs.Hq} heads of the {cs.name} ({flops:.3g} causal flops)"}
+
+    run.max_rows = cs.T
+    return run
+
+
+def cpu_oracle_chunk_sample(name: str = "qwen3-4b-second-chunk", rows: int = 512, seed: int = 0):
+    """The oracle's chunked prefill on the last `rows` new rows (every head) of the chunk."""
+    res = chunk_oracle(name, seed)(rows)
+    return dict(res, tflops=res["flops"] / res["seconds"] / 1e12, threads=oracle_threads())
 
 
 def run_chunk(args, world, rank, local):
     if args.impl == "reference":
         if rank != 0:
             return
-        cal = cpu_oracle_chunk_sample(rows=16)
-        rows = int(max(4, min(4096, (120.0 / max(args.steps, 1)) / max(cal["seconds"] / 16, 1e-6))))
-        secs = flops = 0.0
-        res = None
-        for _ in range(args.steps):
-            res = cpu_oracle_chunk_sample(rows=rows)
-            secs += res["seconds"]
-            flops += res["flops"]
+        secs, flops, _, sample = reference_steps(chunk_oracle(), args.steps, args.warmup)
         value = flops / secs / 1e12
         cs = CHUNK_SHAPES["qwen3-4b-second-chunk"]
         line = {"impl": "reference", "metric": CHUNK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": cs.name},
-                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
-                                 "sample": "per step, " + res["sample"]},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": "per step, " + sample},
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -514,25 +571,33 @@ def run_chunk(args, world, rank, local):
 QKV_METRIC = "merged qkv projection GEMM TFLOP/s (QK-Norm + RoPE epilogue) % bf16 peak"
 
 
-def cpu_oracle_qkv_sample(name: str, rows: int = 256, seed: int = 0):
-    """The oracle's projection + QK-Norm + RoPE on the first `rows` tokens of the workload."""
+def qkv_oracle(name: str, seed: int = 0):
+    """The oracle's projection + QK-Norm + RoPE with its inputs built once: run(rows) times
+    one call on the first `rows` tokens of the workload."""
     import oracle
     from synthetic import as_f64
 
     sh = QKV_SHAPES[name]
     inp = qkv_proj_inputs(sh, seed=seed)
-    t0 = time.perf_counter()
-    oracle.qkv_proj_norm_rope_ref(as_f64(inp["x"][:rows]), as_f64(inp["w_qkv"]), as_f64(inp["q_norm_w"]),
-                                  as_f64(inp["k_norm_w"]), inp["pos"][:rows].numpy(), sh.Hq, sh.Hkv, sh.theta, sh.eps)
-    secs = time.perf_counter() - t0
-    flops = 2.0 * rows * sh.hidden * (sh.Hq + 2 * sh.Hkv) * sh.d
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count()
-    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "flops": flops,
-            "sample": f"first {rows} of {sh.M} tokens of the {sh.name} ({flops:.3g} flops)"}
+    x, w = as_f64(inp["x"]), as_f64(inp["w_qkv"])
+    gq, gk, pos = as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"].numpy()
+
+    def run(rows: int) -> dict:
+        t0 = time.perf_counter()
+        oracle.qkv_proj_norm_rope_ref(x[:rows], w, gq, gk, pos[:rows], sh.Hq, sh.Hkv, sh.theta, sh.eps)
+        secs = time.perf_counter() - t0
+        flops = 2.0 * rows * sh.hidden * (sh.Hq + 2 * sh.Hkv) * sh.d
+        return {"seconds": secs, "flops": flops,
+                "sample": f"first {rows} of {sh.M} tokens of the {sh.name} ({flops:.3g} flops)"}
+
+    run.max_rows = sh.M
+    return run
+
+
+def cpu_oracle_qkv_sample(name: str, rows: int = 256, seed: int = 0):
+    """The oracle's projection + QK-Norm + RoPE on the first `rows` tokens of the workload."""
+    res = qkv_oracle(name, seed)(rows)
+    return dict(res, tflops=res["flops"] / res["seconds"] / 1e12, threads=oracle_threads())
 
 
 def run_qkv(args, world, rank, local):
@@ -541,19 +606,14 @@ def run_qkv(args, world, rank, local):
     if args.impl == "reference":
         if rank != 0:
             return
-        secs = flops = 0.0
-        res = None
-        for _ in range(args.steps):
-            res = cpu_oracle_qkv_sample(name, rows=256)
-            secs += res["seconds"]
-            flops += res["flops"]
+        secs, flops, _, sample = reference_steps(qkv_oracle(name), args.steps, args.warmup)
         value = flops / secs / 1e12
         line = {"impl": "reference", "metric": QKV_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": sh.name},
-                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
-                                 "sample": "per step, " + res["sample"]},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": "per step, " + sample},
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -642,9 +702,10 @@ def run_qkv(args, world, rank, local):
 VARLEN_METRIC = "varlen batched causal GQA prefill TFLOP/s (+QK-Norm/RoPE) % bf16 peak"
 
 
-def cpu_oracle_varlen_sample(name: str, rows: int = 256, seed: int = 0):
-    """The oracle's prefill of the last `rows` query rows (every head) of the batch's longest
-    sequence, keys over the whole sequence."""
+def varlen_oracle(name: str, seed: int = 0):
+    """The oracle's prefill of the batch's longest sequence (over its cached keys, if any)
+    with its inputs built once: run(rows) times one call on the last `rows` query rows
+    (every head), keys over the whole sequence."""
     import oracle
     from synthetic import as_f64
 
@@ -654,24 +715,32 @@ def cpu_oracle_varlen_sample(name: str, rows: int = 256, seed: int = 0):
     cu = inp["cu_seqlens"].numpy()
     sl = slice(int(cu[b]), int(cu[b + 1]))
     T, c = sh.lens[b], sh.contexts[b]
-    rows = min(rows, T)
-    sel = np.arange(T - rows, T)
     kc = oracle.build_cache_k(as_f64(inp["k_hist"][b]), as_f64(inp["k_norm_w"]), sh.theta, sh.eps).transpose(1, 0, 2)
     vc = as_f64(inp["v_hist"][b]).transpose(1, 0, 2)
-    t0 = time.perf_counter()
-    oracle.chunk_prefill_ref(as_f64(inp["q"][sl])[None], as_f64(inp["k"][sl])[None], as_f64(inp["v"][sl])[None],
-                             as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][sl].numpy()[None], kc[None],
-                             vc[None], c, sh.theta, sh.eps, rows=sel)
-    secs = time.perf_counter() - t0
-    flops = 4.0 * sh.Hq * sh.d * float((c + sel + 1).sum())
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count()
-    sample = (f"last {rows} of {T} query rows x {sh.Hq} heads of the longest sequence of the {sh.name}"
-              + (f" (over its {c} cached keys)" if c else "") + f" ({flops:.3g} causal flops)")
-    return {"tflops": flops / secs / 1e12, "seconds": secs, "threads": threads, "sample": sample, "flops": flops}
+    args = (as_f64(inp["q"][sl])[None], as_f64(inp["k"][sl])[None], as_f64(inp["v"][sl])[None],
+            as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][sl].numpy()[None], kc[None], vc[None], c,
+            sh.theta, sh.eps)
+
+    def run(rows: int) -> dict:
+        rows = min(rows, T)
+        sel = np.arange(T - rows, T)
+        t0 = time.perf_counter()
+        oracle.chunk_prefill_ref(*args, rows=sel)
+        secs = time.perf_counter() - t0
+        flops = 4.0 * sh.Hq * sh.d * float((c + sel + 1).sum())
+        sample = (f"last {rows} of {T} query rows x {sh.Hq} heads of the longest sequence of the {sh.name}"
+                  + (f" (over its {c} cached keys)" if c else "") + f" ({flops:.3g} causal flops)")
+        return {"seconds": secs, "flops": flops, "sample": sample}
+
+    run.max_rows = T
+    return run
+
+
+def cpu_oracle_varlen_sample(name: str, rows: int = 256, seed: int = 0):
+    """The oracle's prefill of the last `rows` query rows (every head) of the batch's longest
+    sequence, keys over the whole sequence."""
+    res = varlen_oracle(name, seed)(rows)
+    return dict(res, tflops=res["flops"] / res["seconds"] / 1e12, threads=oracle_threads())
 
 
 def time_call(step, flush, host: dict, dev_inputs: dict, outputs: list, K: int, warmup: int, world, local, dev,
@@ -727,21 +796,14 @@ def run_varlen(args, world, rank, local):
     if args.impl == "reference":
         if rank != 0:
             return
-        cal = cpu_oracle_varlen_sample(name, rows=16)
-        rows = int(max(4, min(max(sh.lens), (120.0 / max(args.steps, 1)) / max(cal["seconds"] / 16, 1e-6))))
-        secs = flops = 0.0
-        res = None
-        for _ in range(args.steps):
-            res = cpu_oracle_varlen_sample(name, rows=rows)
-            secs += res["seconds"]
-            flops += res["flops"]
+        secs, flops, _, sample = reference_steps(varlen_oracle(name), args.steps, args.warmup)
         value = flops / secs / 1e12
         line = {"impl": "reference", "metric": VARLEN_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": sh.name},
-                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
-                                 "sample": "per step, " + res["sample"]},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                                 "sample": "per step, " + sample},
                 "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -868,31 +930,24 @@ def max_over_ranks(world, vals, dev):
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the fp64 oracle on the host cores, as it stands.  Each step is a
-    bounded sample of the workload (the last rows of one prefill batch row and one decode
-    sequence), sized from a calibration run so all K steps take about two minutes."""
+    """The reference arm: the fp64 oracle on the host cores, as it stands.  Its inputs are
+    built once; each step is the oracle's prefill of the last rows (every head) of one batch
+    row of the Qwen3-0.6B-shaped workload, sized so that the warm-up and the K steps take
+    about two minutes of oracle time.  The oracle's decode of one sequence takes longer
+    than such a step, so its GB/s comes from one separate call."""
     if rank != 0:
         return
-    cal = cpu_oracle_sample(rows_per_head=64, batch_rows=1, decode_seqs=1)  # warm-up + calibration
-    per_row = cal["t_prefill_s"] / 64
-    budget = 120.0 / max(args.steps, 1) - cal["t_decode_s"]
-    rows = int(max(4, min(2048, budget / max(per_row, 1e-6))))
-    t_pre = t_tot = flops = 0.0
-    res = None
-    for _ in range(args.steps):
-        res = cpu_oracle_sample(rows_per_head=rows, batch_rows=1, decode_seqs=1)
-        t_pre += res["t_prefill_s"]
-        t_tot += res["t_prefill_s"] + res["t_decode_s"]
-        flops += res["flops"]
-    value = flops / t_pre / 1e12
+    secs, flops, rows, sample = reference_steps(prefill_oracle(batch_rows=1), args.steps, args.warmup)
+    dec = decode_oracle_sample(decode_seqs=1)
+    value = flops / secs / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_tot / args.steps,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": config_dict(),
-            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": res["threads"], "kind": "oracle",
-                             "sample": "per step, " + res["sample"]},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                             "sample": f"per step, {sample}; {dec['sample']} once, outside the steps"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "decode": {"value": res["gbs"], "unit": "GB/s"}}
+            "decode": {"value": dec["gbs"], "unit": "GB/s"}}
     print(json.dumps(line), flush=True)
 
 
