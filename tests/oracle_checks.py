@@ -470,6 +470,22 @@ def check_attention_scaling_against_torch_sdpa():
     assert np.allclose(o, ref.permute(0, 2, 1, 3).numpy(), rtol=0, atol=1e-12)
 
 
+def check_build_cache_k_stores_bf16():
+    """The cache holds bf16 values: each key element is exactly representable in bf16 (a
+    float32 whose low 16 bits are zero) and lies within half a bf16 ulp (at most 2^-8 of its
+    magnitude: bf16 keeps 8 significant bits) of
+    the normed, rotated fp64 key."""
+    k = _rand((40, 2, D), 95, 3.0)
+    g = _gain(96)
+    c = A.build_cache_k(k, g, THETA, EPS)
+    f32 = c.astype(np.float32)
+    assert np.array_equal(f32.astype(np.float64), c)
+    assert np.all((f32.view(np.uint32) & 0xFFFF) == 0)
+    exact = A.qk_prologue(k, g, np.arange(40), THETA, EPS)
+    assert np.all(np.abs(c - exact) <= np.abs(exact) * 2.0 ** -8)
+    assert np.any(c != exact)
+
+
 def check_paged_gather_addressing():
     """A pool whose every slot holds 1000*page + offset (per head and dim) gathers, for a
     hand-written block table, to 1000*table[j // size] + j % size at key j."""

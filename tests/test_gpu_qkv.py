@@ -31,8 +31,9 @@ def _run(shape: QkvShape, seed: int, inv_freq=None, scaling=1.0, pos=None):
 
 def _check(got, ref, what):
     # fp32 accumulation of exact bf16 products (relative error ~ hidden * 2^-24), the norm and
-    # rotation in fp32, then one bf16 rounding (2^-9 relative): 2^-8 |ref| plus a small
-    # absolute term for entries near zero, scaled to the tensor's RMS.
+    # rotation in fp32, then one bf16 rounding (unit roundoff 2^-8): 2^-8 |ref| plus a small
+    # absolute term for entries near zero, scaled to the tensor's RMS.  Round-to-nearest errors
+    # average about a quarter ulp, under 2^-9 of the magnitude: the bound on the mean.
     for name, g, r in zip("qkv", got, ref):
         assert np.isfinite(g).all(), f"{what} {name}: non-finite"
         rms = np.sqrt(np.mean(r * r))

@@ -64,8 +64,9 @@ WINDOWS = [
 # maximum over many keys.  With a window of one key every row's LSE IS one logit, and rows
 # under a short window with large gains are nearly so: a single bf16 rounding-boundary
 # straddle of one q' or k' element (the kernel's fp32 value a few ulp from the correctly
-# rounded one) then moves the LSE by up to 2^-8 |q'_i k'_i| / sqrt(d), ~3e-3 at the element
-# sizes of these inputs, with nothing to average it out.  Those cases are held to 4e-3
+# rounded one) moves that element by one bf16 ulp, at most 2^-7 of it, and the LSE by up to
+# 2^-7 |q'_i k'_i| / sqrt(d), with nothing to average it out.  The straddles measured at the
+# element sizes of these inputs stayed near 3e-3 at most.  Those cases are held to 4e-3
 # (times the gain product squared where the gains are scaled).
 SINGLE_LOGIT_LSE_TOL = 4e-3
 
@@ -78,20 +79,22 @@ def test_prefill_sliding_window(B, T, Hq, Hkv, window):
         compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, what)
         return
     # Every row sees only its own key.  out = v of its KV head (up to the bf16 P); the LSE is
-    # the logit s = q'.k'/sqrt(d) itself, which the bf16 rounding of q' and k' (relative
-    # error <= 2^-9 each) moves by at most 2^-8 sum_i |q'_i k'_i| / sqrt(d): that per-row
-    # bound holds against the pure oracle, and one straddle's worth against the staged one.
+    # the logit s = q'.k'/sqrt(d) itself, which the bf16 rounding of q' and k' (unit roundoff
+    # u = 2^-8 each) and the fp32 accumulation move by less than
+    # (2^-7 + 2^-15) sum_i |q'_i k'_i| / sqrt(d) (prefill_lse_bound in gpu_common): that
+    # per-row bound holds against the pure oracle, one straddle's worth against the staged one.
     compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, what, lse_tol=SINGLE_LOGIT_LSE_TOL,
             lse_pure_tol=float("inf"))
     inp = prefill_inputs(PrefillShape("variant", B, T, Hq, Hkv), seed=T + window)
     G = Hq // Hkv
     v = inp["v"].float().numpy()
-    # P is bf16(p) against the fp32 l, and out is rounded to bf16: two roundings of 2^-9
+    # P is bf16(p) against the fp32 l, and out is rounded to bf16: two roundings of at most
+    # 2^-8 each (with one visible key p = l = 1 and out is v exactly)
     assert np.allclose(to_np(out), np.repeat(v, G, axis=2), rtol=2.0 ** -7, atol=1e-6)
     qp = oracle.qk_prologue(as_f64(inp["q"]), as_f64(inp["q_norm_w"]), inp["pos"].numpy(), THETA, EPS)
     kp = np.repeat(oracle.qk_prologue(as_f64(inp["k"]), as_f64(inp["k_norm_w"]), inp["pos"].numpy(), THETA, EPS),
                    G, axis=2)
-    bound = (2.0 ** -8 + 2.0 ** -17) * np.abs(qp * kp).sum(-1) / np.sqrt(128.0) + 1e-5  # [B, T, Hq]
+    bound = (2.0 ** -7 + 2.0 ** -15) * np.abs(qp * kp).sum(-1) / np.sqrt(128.0) + 1e-5  # [B, T, Hq]
     err = np.abs(to_np(lse) - ref_lse)  # [B, Hq, T]
     assert np.all(err <= bound.transpose(0, 2, 1)), (err - bound.transpose(0, 2, 1)).max()
 

@@ -1,10 +1,14 @@
 """Plant plausible mistakes in the oracle (on the CPU) and confirm the pins catch
-each one: a wrong RoPE sign, adjacent-pair RoPE, a missing eps, mean-centering,
-h mod Hkv head mapping, an off-by-one causal mask, a missing 1/sqrt(d) scale,
-a base-2 logsumexp, in the chunked prefill a mask without the cached-prefix
-offset or cached keys rotated a second time, and in the variants a sliding window
-one key too wide, attention_scaling applied to cos only, and a caller's inv_freq
-ignored, and in the varlen batch one causal mask over the whole packed token axis."""
+each one: a wrong RoPE sign, adjacent-pair RoPE, RoPE frequencies theta^(-i/d), RoPE
+before QK-Norm, a missing eps, eps outside the square root, mean-centering, bf16 ties
+rounded away from zero, a KV cache kept unrounded, h mod Hkv head mapping, an off-by-one
+causal mask, a missing 1/sqrt(d) scale, a base-2 logsumexp, in decode the new token
+rotated one position late or its value never appended, a paged gather that ignores the
+block table, in the chunked prefill a mask without the cached-prefix offset or cached
+keys rotated a second time, in the variants a sliding window one key too wide,
+attention_scaling applied to cos only and a caller's inv_freq ignored, in the varlen
+batch one causal mask over the whole packed token axis or the cached prefixes dropped,
+and in the merged projection the k and v blocks swapped."""
 import numpy as np
 import pytest
 
@@ -148,6 +152,81 @@ def _varlen_one_causal_axis(q, k, v, gq, gk, pos, cu_seqlens, theta, eps, k_pref
 
 _ORIG_PREFILL = A.prefill_ref
 
+def _inv_freq_half_exponent(d, theta):
+    # theta^(-i/d) instead of theta^(-2i/d)
+    i = np.arange(d // 2, dtype=np.float64)
+    return np.power(np.float64(theta), -i / d)
+
+
+def _norm_eps_outside_root(x, g, eps):
+    x = np.asarray(x, dtype=np.float64)
+    return g * x / (np.sqrt(np.mean(x * x, axis=-1, keepdims=True)) + eps)
+
+
+def _prologue_rope_before_norm(x, g, pos, theta, eps, staged=False, inv_freq=None, scaling=1.0):
+    # RoPE first, then QK-Norm: the per-channel gain lands on rotated channels
+    y = A.rms_norm(A.rope(x, pos, theta, inv_freq, scaling), g, eps) * scaling
+    return A.bf16_round(y.astype(np.float32).astype(np.float64)) if staged else y
+
+
+def _bf16_ties_away(x):
+    # round to nearest with ties away from zero instead of ties to even
+    x = np.asarray(x, dtype=np.float64).astype(np.float32)
+    b = x.view(np.uint32).astype(np.uint64)
+    b = ((b + 0x8000) & 0xFFFF0000).astype(np.uint32)
+    return b.view(np.float32).astype(np.float64)
+
+
+def _cache_not_rounded(k_hist, k_norm_w, theta, eps, inv_freq=None, scaling=1.0):
+    # the cache keeps the fp64 keys instead of their bf16 storage values
+    L = np.asarray(k_hist).shape[0]
+    return A.qk_prologue(k_hist, k_norm_w, np.arange(L), theta, eps, inv_freq=inv_freq, scaling=scaling)
+
+
+def _decode_one_position_late(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, theta, eps,
+                              seqs=None, staged=False, window=0, inv_freq=None, scaling=1.0):
+    # the new token is rotated at L + 1 (positions counted from one) instead of at L
+    q = np.asarray(q, dtype=np.float64)
+    N, Hq, d = q.shape
+    G = Hq // np.asarray(k_new).shape[1]
+    outs, lses = [], []
+    for n in (range(N) if seqs is None else seqs):
+        L = int(cache_lens[n])
+        qp = A.qk_prologue(q[n][None], q_norm_w, np.array([L + 1]), theta, eps, staged, inv_freq, scaling)[0]
+        kn = A.qk_prologue(np.asarray(k_new[n], dtype=np.float64)[None], k_norm_w, np.array([L + 1]), theta, eps,
+                           staged, inv_freq, scaling)[0]
+        kc, vc = np.asarray(k_cache[n], dtype=np.float64), np.asarray(v_cache[n], dtype=np.float64)
+        o, ls = np.zeros((Hq, d)), np.zeros(Hq)
+        for h in range(Hq):
+            keys = np.concatenate([kc[h // G, :L], kn[h // G][None]], axis=0)
+            vals = np.concatenate([vc[h // G, :L], np.asarray(v_new[n], dtype=np.float64)[h // G][None]], axis=0)
+            oo, ll = A._attend(qp[h][None], keys, vals, np.array([L]), window)
+            o[h], ls[h] = oo[0], ll[0]
+        outs.append(o)
+        lses.append(ls)
+    return np.stack(outs), np.stack(lses)
+
+
+def _decode_drops_new_value(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, theta, eps, **kw):
+    # the new token's value is never appended: its slot reads as zeros
+    return _ORIG_DECODE(q, k_new, np.zeros_like(np.asarray(v_new, dtype=np.float64)), q_norm_w, k_norm_w, k_cache,
+                        v_cache, cache_lens, theta, eps, **kw)
+
+
+def _paged_gather_ignores_table(pages, block_table_row, n, page_size):
+    # block index taken as the page index, as if the table were the identity
+    return _ORIG_GATHER(pages, list(range(len(block_table_row))), n, page_size)
+
+
+def _varlen_drops_prefixes(q, k, v, gq, gk, pos, cu_seqlens, theta, eps, k_prefix=None, v_prefix=None, **kw):
+    # the cached prefixes are ignored: every sequence attends to its new tokens only
+    return _ORIG_VARLEN(q, k, v, gq, gk, pos, cu_seqlens, theta, eps, **kw)
+
+
+_ORIG_DECODE = A.decode_ref
+_ORIG_GATHER = A.paged_gather
+
+
 MUTANTS = [
     ("rope", _rope_wrong_sign),
     ("rope", _rope_adjacent_pairs),
@@ -164,6 +243,15 @@ MUTANTS = [
     ("chunk_prefill_ref", _chunk_no_offset),
     ("chunk_prefill_ref", _chunk_rerotates_cache),
     ("varlen_prefill_ref", _varlen_one_causal_axis),
+    ("rope_inv_freq", _inv_freq_half_exponent),
+    ("rms_norm", _norm_eps_outside_root),
+    ("qk_prologue", _prologue_rope_before_norm),
+    ("bf16_round", _bf16_ties_away),
+    ("build_cache_k", _cache_not_rounded),
+    ("decode_ref", _decode_one_position_late),
+    ("decode_ref", _decode_drops_new_value),
+    ("paged_gather", _paged_gather_ignores_table),
+    ("varlen_prefill_ref", _varlen_drops_prefixes),
 ]
 
 
