@@ -215,6 +215,29 @@ def test_decode_and_prologue_argument_checks():
     assert r == qa.ERR_UNSUPPORTED
 
 
+def test_size_limits_are_rejected_before_any_launch():
+    """Past the 32-bit element ranges the kernels index with, calls return UNSUPPORTED at
+    the host checks.  (Only the rejected side of each limit is exercised here: a call just
+    inside it would go on to launch kernels on the fake pointers.)"""
+    lib = qa.lib()
+    # prefill: T * Hq query rows of d elements must stay below 2^31 elements
+    T = (1 << 24) // 16 + 1
+    need = qa.prefill_workspace_size(1, T, 16, 8)
+    assert _prefill_ex(T=T, ws=FAKE, ws_bytes=need) == qa.ERR_UNSUPPORTED
+    # decode: N * Hkv * Lmax cache rows must fit a 32-bit row index
+    r = lib.qwen3_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 64, 32, 8, 128, 1 << 22,
+                              1e6, 1e-6, FAKE, 1 << 40, None)
+    assert r == qa.ERR_UNSUPPORTED
+    # decode: at most 65535 sequences (a grid dimension)
+    r = lib.qwen3_attn_decode(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 65536, 32, 8, 128, 16,
+                              1e6, 1e-6, FAKE, 1 << 40, None)
+    assert r == qa.ERR_UNSUPPORTED
+    # the no-allocation decode refuses requests beyond its fixed region before anything else
+    r = lib.qwen3_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 4096, 32, 8, 128,
+                                      32769, 1e6, 1e-6, None)
+    assert r == qa.ERR_WORKSPACE
+
+
 def test_binding_refuses_cpu_tensors():
     q = torch.zeros(1, 128, 16, 128, dtype=torch.bfloat16)
     k = torch.zeros(1, 128, 8, 128, dtype=torch.bfloat16)
