@@ -247,6 +247,14 @@ def test_binding_refuses_cpu_tensors():
         qa.prefill(q, k, k, w, w, pos)
 
 
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library the binding raises; there is no fallback implementation."""
+    monkeypatch.setattr(qa, "_lib", None)
+    monkeypatch.setattr(qa, "LIB_PATH", str(tmp_path / "libqwen3attn.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        qa.lib()
+
+
 def test_wait_limit_roundtrip():
     old = qa.set_wait_limit(123456)
     assert qa.set_wait_limit(old) == 123456
