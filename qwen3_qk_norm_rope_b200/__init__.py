@@ -202,6 +202,8 @@ def prefill(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, eps: floa
     """Causal GQA prefill with the QK-Norm+RoPE prologue.  q [B,T,Hq,d], k/v [B,T,Hkv,d] bf16,
     gains [d] fp32, pos [B,T] int32.  Returns out [B,T,Hq,d] bf16 (and writes lse [B,Hq,T]
     fp32 and the caches [B,Hkv,Tcap,d] when given)."""
+    if (k_cache is None) != (v_cache is None):
+        raise ValueError("k_cache and v_cache are given together or not at all")
     dev = q.device
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]

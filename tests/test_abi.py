@@ -245,6 +245,8 @@ def test_binding_refuses_cpu_tensors():
     pos = torch.arange(128, dtype=torch.int32)[None]
     with pytest.raises(ValueError):
         qa.prefill(q, k, k, w, w, pos)
+    with pytest.raises(ValueError, match="together"):
+        qa.prefill(q, k, k, w, w, pos, v_cache=torch.zeros(1, 8, 128, 128, dtype=torch.bfloat16))
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
