@@ -288,10 +288,15 @@ def prefill_simple(q, k, v, q_norm_w, k_norm_w, pos, *, theta: float = 1.0e6, ep
     dev = q.device
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, torch.bfloat16, tuple(t.shape), dev)
+    _need(q, "q", torch.bfloat16, (B, T, Hq, d), dev)
+    _need(k, "k", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(v, "v", torch.bfloat16, (B, T, Hkv, d), dev)
+    _need(q_norm_w, "q_norm_w", torch.float32, (d,), dev)
+    _need(k_norm_w, "k_norm_w", torch.float32, (d,), dev)
+    _need(pos, "pos", torch.int32, (B, T), dev)
     if out is None:
         out = torch.empty((B, T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, (B, T, Hq, d), dev)
     _check(lib().qwen3_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w), _ptr(pos),
                                     _ptr(out), B, T, Hq, Hkv, d, theta, eps, _stream(dev)), "qwen3_attn_prefill")
     return out
