@@ -260,3 +260,50 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
 def test_wait_limit_roundtrip():
     old = qa.set_wait_limit(123456)
     assert qa.set_wait_limit(old) == 123456
+
+
+def _c_param_kind(decl: str) -> str:
+    """The ctypes kind a C parameter declaration marshals as."""
+    d = " ".join(decl.replace("const ", "").split())
+    if d == "void":
+        return "none"
+    if "qwen3_attn_variant*" in d.replace(" *", "*"):
+        return "variant*"
+    if "qwen3_paged_kv*" in d.replace(" *", "*"):
+        return "paged*"
+    if "*" in d or d.startswith("qwen3_stream_t"):
+        return "int*" if d.replace(" *", "*").startswith("int*") else "ptr"
+    base = d.rsplit(" ", 1)[0] if " " in d else d
+    # size_t and uint64_t are one 64-bit unsigned type here (ctypes aliases them too)
+    return {"int": "int", "float": "float", "size_t": "u64", "long long": "longlong",
+            "uint64_t": "u64", "double": "double"}[base]
+
+
+def _ctypes_kind(t) -> str:
+    if t is ctypes.POINTER(qa.Variant):
+        return "variant*"
+    if t is ctypes.POINTER(qa.PagedKV):
+        return "paged*"
+    if t is ctypes.POINTER(ctypes.c_int):
+        return "int*"
+    return {ctypes.c_void_p: "ptr", ctypes.c_int: "int", ctypes.c_float: "float", ctypes.c_size_t: "u64",
+            ctypes.c_longlong: "longlong", ctypes.c_uint64: "u64", ctypes.c_double: "double"}[t]
+
+
+def test_binding_signatures_match_the_header():
+    """Every argument list the ctypes binding declares has the header's arity and kinds (a
+    mismatch would pass garbage across the ABI without any error), and so does every
+    return type."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"#[^\n]*", "", text)
+    decls = re.findall(r"([\w\s\*]+?)\b(qwen3_\w+)\s*\(([^)]*)\)\s*;", text)
+    assert len(decls) == len(qa.SIGNATURES)
+    ret_kind = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p,
+                "void": None, "uint64_t": ctypes.c_uint64}
+    for ret, name, params in decls:
+        res, args = qa.SIGNATURES[name]
+        ret = " ".join(ret.split()).replace(" *", "*")
+        assert res is ret_kind[ret], (name, ret)
+        kinds = [_c_param_kind(p) for p in params.split(",")]
+        kinds = [k for k in kinds if k != "none"]
+        assert kinds == [_ctypes_kind(a) for a in args], name
