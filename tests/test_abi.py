@@ -307,3 +307,13 @@ def test_binding_signatures_match_the_header():
         kinds = [_c_param_kind(p) for p in params.split(",")]
         kinds = [k for k in kinds if k != "none"]
         assert kinds == [_ctypes_kind(a) for a in args], name
+
+
+def test_status_codes_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    codes = {name: int(val) for name, val in re.findall(r"\b(QWEN3_(?:OK|ERR_\w+))\s*=\s*(\d+)", text)}
+    assert codes == {"QWEN3_OK": qa.OK, "QWEN3_ERR_INVALID_ARG": qa.ERR_INVALID_ARG,
+                     "QWEN3_ERR_UNSUPPORTED": qa.ERR_UNSUPPORTED, "QWEN3_ERR_CUDA": qa.ERR_CUDA,
+                     "QWEN3_ERR_DEVICE_TIMEOUT": qa.ERR_DEVICE_TIMEOUT, "QWEN3_ERR_WORKSPACE": qa.ERR_WORKSPACE}
+    # and each has its own message
+    assert len({qa.status_string(c) for c in codes.values()}) == len(codes)
