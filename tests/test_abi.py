@@ -317,3 +317,14 @@ def test_status_codes_match_the_header():
                      "QWEN3_ERR_DEVICE_TIMEOUT": qa.ERR_DEVICE_TIMEOUT, "QWEN3_ERR_WORKSPACE": qa.ERR_WORKSPACE}
     # and each has its own message
     assert len({qa.status_string(c) for c in codes.values()}) == len(codes)
+
+
+def test_noalloc_region_limit():
+    """The no-allocation decode's fixed region (48 MiB) holds the split-KV partials of up to
+    92 sequences of 32 heads at Lmax 32769, the batched-decode workload's 64 among them."""
+    region = 48 << 20
+    assert qa.decode_workspace_size(64, 32, 32769) <= region
+    assert qa.decode_workspace_size(92, 32, 32769) <= region < qa.decode_workspace_size(93, 32, 32769)
+    r = qa.lib().qwen3_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 93, 32, 8,
+                                           128, 32769, 1e6, 1e-6, None)
+    assert r == qa.ERR_WORKSPACE
