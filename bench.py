@@ -1,16 +1,19 @@
 """Benchmark of the Qwen3 attention core on B200: prints ONE JSON line.
 
 One step is one pass of the whole hot path over one batch of synthetic input:
-  * prefill of the Qwen3-0.6B-shaped workload (B=2, T=2048, Hq=16, Hkv=8, d=128):
-    QK-Norm + RoPE prologue and causal GQA attention, and
+  * prefill of the long-context wide-GQA workload (B=1, T=32768, Hq=64, Hkv=4, d=128), the
+    largest prefill that fits one GPU: QK-Norm + RoPE prologue and causal GQA attention, and
   * one batched decode step (64 sequences, cached lengths ~ U[1024, 32768], Hq=32,
     Hkv=8): append of the new normed/rotated key, split-KV attention, LSE combine.
 `value` is the prefill throughput in TFLOP/s (causal flops 4*B*Hq*d*T(T+1)/2; the
 prologue is counted as free work); the decode throughput in GB/s rides along under
-"decode".  Inputs are resident in HBM before the timed region; L2 is flushed (a
-256 MiB write) before every step, outside the per-step CUDA-event windows.
+"decode", and the Qwen3-0.6B- and 4B-shaped prefills, each timed alone over as many
+calls, under "prefill_shapes".  Inputs are resident in HBM before the timed region; L2 is
+flushed (a 256 MiB write) before every step and every call, outside the per-call CUDA-event
+windows.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py --prefill qwen3-0.6b          # another prefill workload in the step
     python bench.py --workload chunked-prefill    # the chunked-prefill call alone
     python bench.py --workload qkv-proj           # the merged qkv projection + QK-Norm/RoPE
     python bench.py --workload varlen-prefill     # a ragged batch of prompts on one token axis
@@ -42,6 +45,10 @@ from synthetic import CHUNK_SHAPES, DECODE_SHAPES, PREFILL_SHAPES, QKV_SHAPES, V
     decode_step_inputs, prefill_inputs, qkv_proj_inputs, varlen_inputs  # noqa: E402
 
 METRIC = "causal GQA attn TFLOP/s (+QK-Norm/RoPE) % bf16 peak; decode HBM GB/s"
+# The step's prefill: the largest single-GPU prefill workload (B=1, T=32768, Hq=64, Hkv=4).
+HEADLINE_PREFILL = "long-wide-gqa"
+# Prefill workloads timed beside the step, each alone, reported under "prefill_shapes".
+OTHER_PREFILLS = ("qwen3-0.6b", "qwen3-4b")
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 
@@ -155,7 +162,8 @@ class ClockSampler:
 class Workload:
     """Device-resident inputs of one step, built once."""
 
-    def __init__(self, dev: torch.device, seed: int = 0, prefill: str = "qwen3-0.6b", decode_seqs: int = 64):
+    def __init__(self, dev: torch.device, seed: int = 0, prefill: str = HEADLINE_PREFILL, decode_seqs: int = 64,
+                 others=()):
         import dataclasses
 
         import qwen3_qk_norm_rope_b200 as qa
@@ -163,6 +171,16 @@ class Workload:
         self.qa = qa
         self.dev = dev
         self.ps = PREFILL_SHAPES[prefill]
+        # the other prefill workloads, timed alone: (shape, device inputs, out, workspace)
+        self.others = []
+        for name in others:
+            if name == prefill:
+                continue
+            sh = PREFILL_SHAPES[name]
+            t = {k: v.to(dev) for k, v in prefill_inputs(sh, seed=seed).items()}
+            self.others.append((name, sh, t, torch.empty_like(t["q"]),
+                                torch.empty(qa.prefill_workspace_size(sh.B, sh.T, sh.Hq, sh.Hkv), dtype=torch.uint8,
+                                            device=dev)))
         full = DECODE_SHAPES["batched-decode"]
         self.ds = full if decode_seqs == full.N else dataclasses.replace(
             full, name=f"first {decode_seqs} sequences of the {full.name}", N=decode_seqs)
@@ -217,6 +235,10 @@ class Workload:
     def flush_l2(self):
         self.flush.fill_(1.0)
 
+    def prefill_other(self, i: int):
+        _, _, t, out, ws = self.others[i]
+        self.qa.prefill(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], out=out, workspace=ws)
+
     # launches of this library's kernels per step: prefill (prologue + attention) and
     # decode (append + split-KV attention + combine)
     LAUNCHES_PER_STEP = 5
@@ -236,6 +258,25 @@ def time_steps(w: Workload, steps: int):
     pre = sum(e[0].elapsed_time(e[1]) for e in ev)
     dec = sum(e[1].elapsed_time(e[2]) for e in ev)
     return pre, dec
+
+
+def time_other_prefills(w: Workload, steps: int, warmup: int):
+    """Each other prefill workload alone: `warmup` untimed calls, then `steps` calls with L2
+    flushed before each, outside the per-call CUDA-event windows.  Milliseconds per call."""
+    res = []
+    for i in range(len(w.others)):
+        for _ in range(warmup):
+            w.flush_l2()
+            w.prefill_other(i)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for j in range(steps):
+            w.flush_l2()
+            ev[j][0].record()
+            w.prefill_other(i)
+            ev[j][1].record()
+        torch.cuda.synchronize(w.dev)
+        res.append(sum(e[0].elapsed_time(e[1]) for e in ev) / steps)
+    return res
 
 
 def time_e2e(w: Workload, steps: int):
@@ -282,18 +323,20 @@ def oracle_threads() -> int:
         return os.cpu_count()
 
 
-def prefill_oracle(batch_rows: int = 2, seed: int = 0):
-    """The fp64 oracle on the Qwen3-0.6B-shaped prefill with its inputs built once: the
-    returned run(rows) times one oracle call on the last `rows` query rows (every head) of
-    the first `batch_rows` batch rows and returns its seconds, causal flops and a
-    description of the sample."""
+def prefill_oracle(name: str = HEADLINE_PREFILL, batch_rows: int = 1, seed: int = 0):
+    """The fp64 oracle on a prefill workload with its inputs built once: the returned
+    run(rows) times one oracle call on the last `rows` query rows (every head) of the first
+    `batch_rows` batch rows and returns its seconds, causal flops and a description of the
+    sample.  run.full_flops is the whole workload's causal flops."""
     import oracle
     from synthetic import as_f64
 
-    ps = PREFILL_SHAPES["qwen3-0.6b"]
+    ps = PREFILL_SHAPES[name]
+    batch_rows = min(batch_rows, ps.B)
     inp = prefill_inputs(ps, seed=seed)
     args = (as_f64(inp["q"][:batch_rows]), as_f64(inp["k"][:batch_rows]), as_f64(inp["v"][:batch_rows]),
             as_f64(inp["q_norm_w"]), as_f64(inp["k_norm_w"]), inp["pos"][:batch_rows].numpy(), ps.theta, ps.eps)
+    del inp
 
     def run(rows: int) -> dict:
         sel = np.arange(ps.T - rows, ps.T)
@@ -303,9 +346,10 @@ def prefill_oracle(batch_rows: int = 2, seed: int = 0):
         flops = batch_rows * 4.0 * ps.Hq * ps.d * float((sel + 1).sum())
         return {"seconds": secs, "flops": flops,
                 "sample": (f"prefill: last {rows} of {ps.T} query rows x {ps.Hq} heads of {batch_rows} of {ps.B} "
-                           f"batch rows of the Qwen3-0.6B-shaped workload ({flops:.3g} causal flops)")}
+                           f"batch rows of the {ps.name} ({flops:.3g} causal flops)")}
 
     run.max_rows = ps.T
+    run.full_flops = ps.causal_flops()
     return run
 
 
@@ -333,18 +377,21 @@ def decode_oracle_sample(decode_seqs: int = 16, seed: int = 0) -> dict:
             "sample": f"decode: first {decode_seqs} of 64 sequences ({int(lens[sel].sum())} cached tokens)"}
 
 
-def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seqs: int = 16, seed: int = 0):
+def cpu_oracle_sample(name: str = HEADLINE_PREFILL, rows_per_head: int = 512, batch_rows: int = 1,
+                      decode_seqs: int = 16, seed: int = 0):
     """The fp64 oracle, as it stands, on a bounded sample of the same workload: the last
     `rows_per_head` query rows (every head) of the first `batch_rows` batch rows of the
-    Qwen3-0.6B-shaped prefill (the defaults are the whole prefill), and the first
-    `decode_seqs` sequences of the batched decode.  Returns TFLOP/s on the prefill sample,
-    GB/s on the decode sample, the seconds each took and the BLAS thread count."""
-    pre = prefill_oracle(batch_rows, seed)(rows_per_head)
+    prefill `name`, and the first `decode_seqs` sequences of the batched decode.  Returns
+    TFLOP/s on the prefill sample, the whole prefill's time extrapolated from it by the
+    exact flop ratio, GB/s on the decode sample, the seconds each took and the BLAS thread
+    count."""
+    run = prefill_oracle(name, batch_rows, seed)
+    pre = run(min(rows_per_head, run.max_rows))
     dec = decode_oracle_sample(decode_seqs, seed) if decode_seqs > 0 else \
         {"seconds": 0.0, "gbs": 0.0, "sample": "no decode"}
     return {"tflops": pre["flops"] / pre["seconds"] / 1e12, "gbs": dec["gbs"], "t_prefill_s": pre["seconds"],
             "t_decode_s": dec["seconds"], "threads": oracle_threads(), "sample": pre["sample"] + "; " + dec["sample"],
-            "flops": pre["flops"]}
+            "flops": pre["flops"], "prefill_full_s_extrapolated": pre["seconds"] * run.full_flops / pre["flops"]}
 
 
 # The reference arm times the oracle for about this many seconds in all (warm-up and timed
@@ -352,11 +399,11 @@ def cpu_oracle_sample(rows_per_head: int = 2048, batch_rows: int = 2, decode_seq
 REFERENCE_BUDGET_S = 120.0
 
 
-def reference_steps(run, steps: int, warmup: int):
+def reference_steps(run, steps: int, warmup: int, budget_s: float = REFERENCE_BUDGET_S):
     """The reference arm's loop over an oracle whose inputs are already built: calibrate its
     cost per query row from two sample sizes (so a fixed per-call cost is not taken for a
     per-row one), size each step's sample so that `warmup` + `steps` calls take about
-    REFERENCE_BUDGET_S seconds (one row at least), then run the untimed warm-up calls and
+    `budget_s` seconds (one row at least), then run the untimed warm-up calls and
     the timed steps.  Only the oracle calls themselves are timed.  Returns the timed
     seconds, the flops, the rows per step and the last step's sample description."""
     lo, hi = min(8, run.max_rows), min(264, run.max_rows)
@@ -364,7 +411,7 @@ def reference_steps(run, steps: int, warmup: int):
     t_hi = min(run(hi)["seconds"] for _ in range(2))
     per_row = max((t_hi - t_lo) / max(hi - lo, 1), 1e-7)
     fixed = max(t_lo - lo * per_row, 0.0)
-    per_step = REFERENCE_BUDGET_S / max(steps + warmup, 1)
+    per_step = budget_s / max(steps + warmup, 1)
     rows = int(max(1, min(run.max_rows, (per_step - fixed) / per_row)))
     for _ in range(warmup):
         run(rows)
@@ -930,20 +977,21 @@ def max_over_ranks(world, vals, dev):
 
 
 def run_reference(args, world, rank):
-    """The reference arm: the fp64 oracle on the host cores, as it stands.  Its inputs are
-    built once; each step is the oracle's prefill of the last rows (every head) of one batch
-    row of the Qwen3-0.6B-shaped workload, sized so that the warm-up and the K steps take
-    about two minutes of oracle time.  The oracle's decode of one sequence takes longer
-    than such a step, so its GB/s comes from one separate call."""
+    """The reference arm: the fp64 oracle on the host cores, as it stands, on the step's
+    prefill workload.  Its inputs are built once; each step is the oracle's prefill of the
+    last rows (every head) of the workload, sized so that the warm-up and the K steps take
+    about `--reference-budget` seconds of oracle time.  The oracle's decode of one sequence
+    takes longer than such a step, so its GB/s comes from one separate call."""
     if rank != 0:
         return
-    secs, flops, rows, sample = reference_steps(prefill_oracle(batch_rows=1), args.steps, args.warmup)
+    secs, flops, rows, sample = reference_steps(prefill_oracle(args.prefill, batch_rows=1), args.steps, args.warmup,
+                                                args.reference_budget)
     dec = decode_oracle_sample(decode_seqs=1)
     value = flops / secs / 1e12
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_dict(),
+            "data": "synthetic", "config": config_dict(PREFILL_SHAPES[args.prefill]),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
                              "sample": f"per step, {sample}; {dec['sample']} once, outside the steps"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -952,14 +1000,15 @@ def run_reference(args, world, rank):
 
 
 def config_dict(ps=None, ds=None):
-    ps = ps or PREFILL_SHAPES["qwen3-0.6b"]
+    ps = ps or PREFILL_SHAPES[HEADLINE_PREFILL]
     ds = ds or DECODE_SHAPES["batched-decode"]
     return {"workload": f"{ps.name} + {ds.name}",
             "prefill": {"B": ps.B, "T": ps.T, "Hq": ps.Hq, "Hkv": ps.Hkv, "d": ps.d, "causal": True},
             "decode": {"N": ds.N, "Hq": ds.Hq, "Hkv": ds.Hkv, "d": ds.d, "L": f"U[{ds.lmin},{ds.lmax}]",
                        "Lmax": ds.cache_capacity},
             "rope_theta": ps.theta, "rms_eps": ps.eps, "seed": 0,
-            "l2": "flushed before every step (256 MiB write, outside the timed windows); decode K/V 4.4 GB > L2",
+            "l2": "flushed before every step and every call (256 MiB write, outside the timed windows); "
+                  "decode K/V 4.4 GB > L2",
             "parallelism": "replicas (one independent workload per GPU)"}
 
 
@@ -971,12 +1020,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--prefill", default="qwen3-0.6b", choices=sorted(PREFILL_SHAPES),
-                    help="prefill workload of the step (profiling of the other shapes)")
+    ap.add_argument("--prefill", default=HEADLINE_PREFILL, choices=sorted(PREFILL_SHAPES),
+                    help="prefill workload of the step (default: the long-context wide-GQA prefill)")
+    ap.add_argument("--no-other-prefills", action="store_true",
+                    help="skip timing the other prefill workloads beside the step")
+    ap.add_argument("--reference-budget", type=float, default=REFERENCE_BUDGET_S,
+                    help="--impl reference: seconds of oracle time for the warm-up and timed steps together")
     ap.add_argument("--decode-seqs", type=int, default=64,
                     help="decode the first n of the 64 sequences (small cases for ncu captures)")
     ap.add_argument("--workload", default="step", choices=["step", "chunked-prefill", "qkv-proj", "varlen-prefill"],
-                    help="step: 0.6B prefill + batched decode (default); chunked-prefill: the chunk call alone; "
+                    help="step: long-context prefill + batched decode (default); chunked-prefill: the chunk call alone; "
                          "qkv-proj: the merged projection with the QK-Norm/RoPE epilogue; varlen-prefill: a "
                          "ragged batch of prompts packed on one token axis")
     ap.add_argument("--qkv", default="qwen3-0.6b-qkv", choices=sorted(QKV_SHAPES),
@@ -1007,7 +1060,8 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    w = Workload(dev, prefill=args.prefill, decode_seqs=args.decode_seqs)
+    w = Workload(dev, prefill=args.prefill, decode_seqs=args.decode_seqs,
+                 others=() if args.no_other_prefills else OTHER_PREFILLS)
     for _ in range(args.warmup):
         w.flush_l2()
         w.prefill()
@@ -1022,7 +1076,12 @@ def main():
     st, site = w.qa.device_status(clear=True, device=dev)
     if st != w.qa.OK:
         raise RuntimeError(f"device status {w.qa.status_string(st)} at site {site}")
-    pre_ms, dec_ms = max_over_ranks(world, [pre_ms, dec_ms], dev)
+    other_ms = time_other_prefills(w, args.steps, args.warmup)
+    st, site = w.qa.device_status(clear=True, device=dev)
+    if st != w.qa.OK:
+        raise RuntimeError(f"device status {w.qa.status_string(st)} at site {site}")
+    res = max_over_ranks(world, [pre_ms, dec_ms] + other_ms, dev)
+    pre_ms, dec_ms, other_ms = res[0], res[1], res[2:]
     e2e = None
     if not args.no_e2e:
         e_pre, e_tot, h2d, d2h = time_e2e(w, max(1, min(args.steps, 200)))
@@ -1061,13 +1120,20 @@ def main():
                        "bytes": dbytes, "tflops": world * decode_flops(w.lens, w.ds.Hq) / dec_s / 1e12},
             "roofline": rl_dec if dominant_is_decode else rl_pre,
             "roofline_other": rl_pre if dominant_is_decode else rl_dec,
+            "prefill_shapes": {
+                name: {"workload": sh.name, "value": world * sh.causal_flops() / (ms * 1e-3) / 1e12,
+                       "unit": "TFLOP/s", "ms": ms,
+                       "frac_of_peak": sh.causal_flops() / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                       "calls": K, "timing": "alone, L2 flushed before each call, CUDA events"}
+                for (name, sh, *_), ms in zip(w.others, other_ms)},
             "gpu_launches": Workload.LAUNCHES_PER_STEP * K,
             "clocks": clocks, "e2e": e2e}
     if world == 1 and not args.no_cpu_baseline:
-        cb = cpu_oracle_sample(rows_per_head=2048, batch_rows=2, decode_seqs=16)
+        cb = cpu_oracle_sample(args.prefill, rows_per_head=512, batch_rows=1, decode_seqs=16)
         line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
                                 "sample": cb["sample"], "decode_gbs": cb["gbs"],
-                                "seconds": cb["t_prefill_s"] + cb["t_decode_s"]}
+                                "seconds": cb["t_prefill_s"] + cb["t_decode_s"],
+                                "prefill_full_s_extrapolated": cb["prefill_full_s_extrapolated"]}
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -214,8 +214,13 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
  *   - Limit: qwen3_attn_decode_workspace_size(N, Hq, d, Lmax) must not exceed
  *     QWEN3_ATTN_NOALLOC_SCRATCH_BYTES (64 sequences x 32 heads x Lmax 32769 need 34.9
  *     MB); larger requests return QWEN3_ERR_WORKSPACE and launch nothing.
- *   - The first call on a device looks up the region's device address (with that device
- *     current); make that first call before any stream capture.
+ *   - The region's device address belongs to one CUDA context.  The first call in a
+ *     context (the device's primary context, or another context the caller made current)
+ *     looks that address up and keeps it for that context; after a device reset the new
+ *     context's first call looks it up again.  Make the first call in a context before any
+ *     stream capture in it.
+ *   - Argument checks come first: a bad argument returns what qwen3_attn_decode returns
+ *     for it, before the region is looked up.
  *   - Every call on a device shares the one region, and a call leaves its partials there.
  *     Nothing in it needs to start at zero (each split writes its partial before the
  *     combine reads it).  Calls whose kernels overlap on the GPU (other streams, other
@@ -419,6 +424,23 @@ uint64_t qwen3_attn_set_wait_limit(uint64_t ns);
  * written).  0 turns it off.  No memory outside the call's own buffers is touched.
  */
 void qwen3_attn_set_fault_injection(int flags);
+
+/*
+ * qwen3_attn_set_softmax_path - test hook choosing the prefill softmax of later launches
+ * (every prefill, chunk, paged and varlen call).  Both paths compute the same softmax
+ * ("Assembling a large model from scratch", Attention.forward: fp32 softmax over the masked
+ * scores; the online logsumexp of "Qwen3 Architecture Layer-by-Layer", Liger fused linear
+ * cross-entropy); they differ in the reference exponent only.
+ *   QWEN3_SOFTMAX_AUTO (0, the default): a launch whose gains bound every logit
+ *       (sqrt(d) * max|g_q| * max|g_k| * attention_scaling^2 * log2(e) <= 60) uses that
+ *       bound as a fixed reference; larger gains take the running-max path.
+ *   QWEN3_SOFTMAX_RUNNING_MAX (1): every launch takes the running-max path (a row max per
+ *       key tile, lazy rescale of the accumulator), whatever the gains.
+ * Returns the previous setting, or -1 (nothing changed) for any other value.
+ */
+#define QWEN3_SOFTMAX_AUTO 0
+#define QWEN3_SOFTMAX_RUNNING_MAX 1
+int qwen3_attn_set_softmax_path(int path);
 
 /* Library version string. */
 const char* qwen3_attn_version(void);

@@ -68,6 +68,7 @@ SIGNATURES = {
     "qwen3_attn_device_status": (_I, [_P, _I, ctypes.POINTER(ctypes.c_int)]),
     "qwen3_attn_set_wait_limit": (_U64, [_U64]),
     "qwen3_attn_set_fault_injection": (None, [_I]),
+    "qwen3_attn_set_softmax_path": (_I, [_I]),
     "qwen3_attn_version": (ctypes.c_char_p, []),
 }
 
@@ -542,6 +543,19 @@ def set_wait_limit(ns: int) -> int:
 
 def set_fault_injection(flags: int) -> None:
     lib().qwen3_attn_set_fault_injection(int(flags))
+
+
+SOFTMAX_AUTO, SOFTMAX_RUNNING_MAX = 0, 1
+
+
+def set_softmax_path(path: int) -> int:
+    """Test hook: SOFTMAX_RUNNING_MAX sends every later prefill launch down the running-max
+    softmax whatever its gains; SOFTMAX_AUTO (the default) lets the gains' logit bound
+    choose.  Returns the previous setting."""
+    old = int(lib().qwen3_attn_set_softmax_path(int(path)))
+    if old < 0:
+        raise ValueError(f"unknown softmax path {path}")
+    return old
 
 
 def version() -> str:

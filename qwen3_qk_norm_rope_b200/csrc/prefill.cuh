@@ -52,6 +52,7 @@ struct PrefillParams {
   float rope_scale;  // attention_scaling that scaled q' and k' (enters the logit bound squared)
   WaitCfg wait;
   int fault;
+  int force_rmax;  // nonzero: the running-max softmax whatever the logit bound (a test hook)
   // Varlen batches (the kVar instance): the entry list {qoff, T, start, koff}, {pair, b}
   // and its item count, both written on the device; B is then the sequence count, T the
   // packed token count N, and `out` [N, Hq, d] takes the rows of tiles that end past their
@@ -372,7 +373,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // units) at most 60, p = 2^(s*scale*log2(e) - bnd) lies in [2^-120, 1] for every key, so
     // a fixed reference needs no row max, no rescale and can neither overflow nor go
     // subnormal; l and O stay bounded by the key count.  Larger gains take the running-max
-    // path.  The choice is uniform per CTA.
+    // path (and so does every launch while the host's test hook forces it).  The choice is
+    // uniform per CTA.
     float bnd;
     {
       float gq = fabsf(p.q_norm_w[row]), gk = fabsf(p.k_norm_w[row]);
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       gk = fmaxf(fmaxf(red[1], red[3]), fmaxf(red[5], red[7]));
       bnd = gq * gk * p.rope_scale * p.rope_scale * (11.3137085f * (1.0f + 0.0078125f) * 1.44269504f);
     }
-    const bool fast = bnd <= 60.0f;
+    const bool fast = bnd <= 60.0f && p.force_rmax == 0;
     uint32_t s_cnt = 0, o_cnt = 0;
     bool ok = true;
     // The tensor core may start the next item (its Q' tiles arrive by TMA) while this

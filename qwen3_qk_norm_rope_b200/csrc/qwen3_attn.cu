@@ -35,6 +35,7 @@ uint64_t initial_wait_ns() {
 uint64_t g_wait_ns = initial_wait_ns();
 uint64_t g_launch_id = 0;
 int g_fault = 0;
+int g_softmax_path = QWEN3_SOFTMAX_AUTO;
 std::mutex g_mu;
 
 q3::WaitCfg next_wait_cfg() {
@@ -291,6 +292,14 @@ void qwen3_attn_set_fault_injection(int flags) {
   g_fault = flags;
 }
 
+int qwen3_attn_set_softmax_path(int path) {
+  if (path != QWEN3_SOFTMAX_AUTO && path != QWEN3_SOFTMAX_RUNNING_MAX) return -1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int old = g_softmax_path;
+  g_softmax_path = path;
+  return old;
+}
+
 int qwen3_attn_device_status(qwen3_stream_t stream, int clear, int* site) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return QWEN3_ERR_CUDA;
   int h[2] = {0, 0};
@@ -534,6 +543,7 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   {
     std::lock_guard<std::mutex> lk(g_mu);
     p.fault = g_fault;
+    p.force_rmax = g_softmax_path == QWEN3_SOFTMAX_RUNNING_MAX ? 1 : 0;
   }
   return launch_fmha(mq, mk, mv, mo, p, static_cast<int>(n_items), var.window > 0, false, s);
 }
@@ -599,6 +609,27 @@ int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf1
 
 namespace {
 
+// The host checks of a decode call's tensors and sizes (every one but the workspace's).
+int decode_check(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
+                 const float* k_norm_w, const qwen3_bf16* k_cache, const qwen3_bf16* v_cache,
+                 const int32_t* cache_lens, const qwen3_bf16* out, const float* lse, int N, int Hq, int Hkv, int d,
+                 int Lmax, float eps, bool paged) {
+  if (q == nullptr || k_new == nullptr || v_new == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
+      k_cache == nullptr || v_cache == nullptr || cache_lens == nullptr || out == nullptr)
+    return QWEN3_ERR_INVALID_ARG;
+  if (N <= 0 || Lmax <= 0) return QWEN3_ERR_INVALID_ARG;
+  const int st = check_common(Hq, Hkv, d);
+  if (st != QWEN3_OK) return st;
+  if (Hq / Hkv > 16 || N > 65535 || Hkv > 65535) return QWEN3_ERR_UNSUPPORTED;
+  if (!paged && static_cast<long long>(N) * Hkv * Lmax > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
+      !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) ||
+      !aligned(cache_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return QWEN3_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
+  return QWEN3_OK;
+}
+
 // With `pg`, the cache is paged (k_cache, v_cache unused; Lmax = max_blocks * page).
 int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* v_new, const float* q_norm_w,
                 const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
@@ -609,19 +640,9 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
     v_cache = pg->v;
     Lmax = pg->max_blocks * pg->page;
   }
-  if (q == nullptr || k_new == nullptr || v_new == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
-      k_cache == nullptr || v_cache == nullptr || cache_lens == nullptr || out == nullptr)
-    return QWEN3_ERR_INVALID_ARG;
-  if (N <= 0 || Lmax <= 0) return QWEN3_ERR_INVALID_ARG;
-  int st = check_common(Hq, Hkv, d);
+  int st = decode_check(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq, Hkv, d,
+                        Lmax, eps, pg != nullptr);
   if (st != QWEN3_OK) return st;
-  if (Hq / Hkv > 16 || N > 65535 || Hkv > 65535) return QWEN3_ERR_UNSUPPORTED;
-  if (pg == nullptr && static_cast<long long>(N) * Hkv * Lmax > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_cache, 16) ||
-      !aligned(v_cache, 16) || !aligned(out, 16) || !aligned(q_norm_w, 8) || !aligned(k_norm_w, 8) ||
-      !aligned(cache_lens, 4) || (lse != nullptr && !aligned(lse, 4)))
-    return QWEN3_ERR_INVALID_ARG;
-  if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
   if (workspace == nullptr || ws_bytes < qwen3_attn_decode_workspace_size(N, Hq, d, Lmax)) return QWEN3_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
@@ -829,25 +850,71 @@ int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
 // declares statically instead of a caller workspace (see qwen3_attn_decode_noalloc in
 // include/qwen3_attn.h).  In host code `g_noalloc_scratch` names a host-side stand-in, not
 // device memory, so it is never passed to a kernel directly: its device address is looked
-// up once per device with cudaGetSymbolAddress, with that device current.
+// up with cudaGetSymbolAddress while the caller's context is current.
+//
+// A __device__ variable's address belongs to one CUDA context (the module is loaded into
+// each context separately, and again after a device reset recreates the primary context),
+// so the address is cached per context, keyed by the driver's context id, which is unique
+// for the life of the process and never reused by a later context.
 namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[QWEN3_ATTN_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of this device's scratch region, or nullptr when the lookup failed.
-void* noalloc_scratch_for_current_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+// Id of the calling thread's current context; false when there is none (or no driver).
+bool current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    (void)cudaGetLastError();
+  });
+  if (get_current == nullptr || get_id == nullptr) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+constexpr int kNoallocCacheSlots = 64;
+std::mutex g_noalloc_mu;
+unsigned long long g_noalloc_ctx[kNoallocCacheSlots] = {};
+void* g_noalloc_ptr[kNoallocCacheSlots] = {};
+int g_noalloc_next = 0;
+
+// Device address of the scratch region in the current context, or nullptr when the lookup
+// failed (the runtime's error state is cleared, so the failure does not surface in a later
+// call's launch check).
+void* noalloc_scratch_for_current_context() {
+  unsigned long long id = 0;
+  bool have_id = current_context_id(&id);
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    g_noalloc_ptr[dev] = ptr;
+  if (have_id)
+    for (int i = 0; i < kNoallocCacheSlots; ++i)
+      if (g_noalloc_ptr[i] != nullptr && g_noalloc_ctx[i] == id) return g_noalloc_ptr[i];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
   }
-  return g_noalloc_ptr[dev];
+  // the lookup makes the device's primary context current if none was
+  if (!have_id) have_id = current_context_id(&id);
+  if (have_id) {
+    g_noalloc_ctx[g_noalloc_next] = id;
+    g_noalloc_ptr[g_noalloc_next] = ptr;
+    g_noalloc_next = (g_noalloc_next + 1) % kNoallocCacheSlots;
+  }
+  return ptr;
 }
 
 }  // namespace
@@ -857,9 +924,17 @@ extern "C" int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* 
                                          qwen3_bf16* v_cache, const int32_t* cache_lens, qwen3_bf16* out,
                                          float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta,
                                          float eps, qwen3_stream_t stream) {
+  // every argument check of qwen3_attn_decode comes before the region's lookup, so a bad
+  // argument reports what qwen3_attn_decode reports for it
+  Variant var;
+  int st = theta_variant(theta, var);
+  if (st != QWEN3_OK) return st;
+  st = decode_check(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq, Hkv, d, Lmax,
+                    eps, false);
+  if (st != QWEN3_OK) return st;
   const size_t need = qwen3_attn_decode_workspace_size(N, Hq, d, Lmax);
   if (need > QWEN3_ATTN_NOALLOC_SCRATCH_BYTES) return QWEN3_ERR_WORKSPACE;
-  void* scratch = noalloc_scratch_for_current_device();
+  void* scratch = noalloc_scratch_for_current_context();
   if (scratch == nullptr) return QWEN3_ERR_CUDA;
   return qwen3_attn_decode(q, k_new, v_new, q_norm_w, k_norm_w, k_cache, v_cache, cache_lens, out, lse, N, Hq,
                            Hkv, d, Lmax, theta, eps, scratch, QWEN3_ATTN_NOALLOC_SCRATCH_BYTES, stream);
@@ -1052,6 +1127,7 @@ int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, c
   {
     std::lock_guard<std::mutex> lk(g_mu);
     p.fault = g_fault;
+    p.force_rmax = g_softmax_path == QWEN3_SOFTMAX_RUNNING_MAX ? 1 : 0;
   }
   p.vl_ent = ent;
   p.vl_n_items = n_items;

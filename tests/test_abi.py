@@ -319,6 +319,46 @@ def test_status_codes_match_the_header():
     assert len({qa.status_string(c) for c in codes.values()}) == len(codes)
 
 
+def test_noalloc_checks_arguments_before_the_region_lookup():
+    """A bad argument gets the status qwen3_attn_decode gives it, whether or not a device is
+    there to look the region up on; a call whose lookup failed (no device here) leaves no
+    error behind for the next call's checks."""
+    f = qa.lib().qwen3_attn_decode_noalloc
+    dec = qa.lib().qwen3_attn_decode
+    args = [FAKE] * 9 + [None, 8, 32, 8, 128, 4096, 1e6, 1e-6, None]
+    bad_ptr = list(args)
+    bad_ptr[0] = None
+    assert f(*bad_ptr) == qa.ERR_INVALID_ARG
+    bad_d = list(args)
+    bad_d[13] = 64
+    assert f(*bad_d) == qa.ERR_UNSUPPORTED == dec(*(bad_d[:17] + [FAKE, 1 << 30, None]))
+    bad_g = list(args)
+    bad_g[11] = 24
+    assert f(*bad_g) == qa.ERR_UNSUPPORTED
+    if not torch.cuda.is_available():
+        assert f(*args) == qa.ERR_CUDA  # the lookup itself needs a device
+        assert f(*bad_ptr) == qa.ERR_INVALID_ARG
+        assert f(*args) == qa.ERR_CUDA
+
+
+def test_softmax_path_constants_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    vals = {name: int(val) for name, val in re.findall(r"#define\s+(QWEN3_SOFTMAX_\w+)\s+(\d+)", text)}
+    assert vals == {"QWEN3_SOFTMAX_AUTO": qa.SOFTMAX_AUTO, "QWEN3_SOFTMAX_RUNNING_MAX": qa.SOFTMAX_RUNNING_MAX}
+
+
+def test_softmax_path_hook_returns_the_previous_setting_and_refuses_unknown_values():
+    """Host-side only: the hook records the setting for later launches and launches nothing."""
+    assert qa.set_softmax_path(qa.SOFTMAX_RUNNING_MAX) == qa.SOFTMAX_AUTO
+    try:
+        assert qa.set_softmax_path(qa.SOFTMAX_RUNNING_MAX) == qa.SOFTMAX_RUNNING_MAX
+        with pytest.raises(ValueError):
+            qa.set_softmax_path(7)
+        assert qa.lib().qwen3_attn_set_softmax_path(-3) == -1
+    finally:
+        assert qa.set_softmax_path(qa.SOFTMAX_AUTO) == qa.SOFTMAX_RUNNING_MAX
+
+
 def test_noalloc_region_limit():
     """The no-allocation decode's fixed region (48 MiB) holds the split-KV partials of up to
     92 sequences of 32 heads at Lmax 32769, the batched-decode workload's 64 among them."""

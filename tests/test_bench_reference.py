@@ -40,7 +40,8 @@ def test_reference_steps_clamp_the_sample():
 
 def test_reference_arm_json_line():
     res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
-                          "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+                          "--warmup", "3", "--reference-budget", "8"], capture_output=True, text=True, timeout=900,
+                         cwd=ROOT)
     assert res.returncode == 0, res.stderr[-2000:]
     line = json.loads(res.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s"

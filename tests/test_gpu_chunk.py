@@ -10,7 +10,7 @@ import torch
 import oracle
 import qwen3_qk_norm_rope_b200 as qa
 from synthetic import CHUNK_SHAPES, ChunkShape, PrefillShape, as_f64, chunk_inputs, prefill_inputs
-from tests.gpu_common import assert_status_ok, compare, dev, prefill_gpu, to_np
+from tests.gpu_common import MAX_TOL, MEAN_TOL, assert_status_ok, chunk_lse_bound, compare, dev, prefill_gpu, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -152,3 +152,9 @@ def test_chunk_large_gains_running_max_path():
     _, _, ref_st, st_lse = _oracle(inp, shape, kc, vc)
     # the same staged comparison and gain-scaled LSE bound as the prefill large-gains test
     compare(to_np(out), to_np(lse), ref_st, st_lse, st_lse, "chunk large gains (staged)", lse_tol=1e-3 * 1.6 ** 2)
+    # and against the pure oracle, with the bounds of the prefill large-gains test
+    ref, ref_lse, _, _ = _oracle(inp, shape, kc, vc)
+    g2 = 1.6 ** 2
+    bound = chunk_lse_bound(inp, shape.start, as_f64(kc[:, :, :shape.start]), theta=shape.theta, eps=shape.eps)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "chunk large gains (pure)", lse_tol=1e-3 * g2,
+            max_tol=MAX_TOL * g2, mean_tol=MEAN_TOL * g2, lse_pure_bound=bound)

@@ -9,7 +9,7 @@ import torch
 import oracle
 import qwen3_qk_norm_rope_b200 as qa
 from synthetic import PREFILL_SHAPES, PrefillShape, as_f64, prefill_inputs
-from tests.gpu_common import (assert_status_ok, check_lse_straddle, compare, dev, prefill_gpu,
+from tests.gpu_common import (MAX_TOL, MEAN_TOL, assert_status_ok, check_lse_straddle, compare, dev, prefill_gpu,
                               prefill_lse_bound, prefill_oracle, to_np)
 
 pytestmark = pytest.mark.gpu
@@ -164,3 +164,10 @@ def test_prefill_large_gains_take_the_running_max_path():
             as_f64(inp["k_norm_w"]), inp["pos"].numpy(), 1e6, 1e-6)
     ref_st, st_lse = oracle.prefill_ref(*args, staged=True)
     compare(to_np(out), to_np(lse), ref_st, st_lse, st_lse, "large gains (staged)", lse_tol=1e-3 * 1.6 ** 2)
+    # Against the pure oracle: the logit error of that rounding grows with the gain product,
+    # so the output bounds are the default ones times 1.6^2, and every row's LSE is held to
+    # the rigorous per-row bound, which follows the gains by construction.
+    ref, ref_lse = oracle.prefill_ref(*args)
+    g2 = 1.6 ** 2
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "large gains (pure)", lse_tol=1e-3 * g2,
+            max_tol=MAX_TOL * g2, mean_tol=MEAN_TOL * g2, lse_pure_bound=prefill_lse_bound(inp, np.arange(700)))

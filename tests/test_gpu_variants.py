@@ -10,7 +10,8 @@ import oracle
 import qwen3_qk_norm_rope_b200 as qa
 from synthetic import ChunkShape, DecodeShape, PrefillShape, as_f64, chunk_inputs, decode_history, \
     decode_step_inputs, prefill_inputs
-from tests.gpu_common import (LSE_PURE_TOL, LSE_TOL, MAX_TOL, MEAN_TOL, assert_status_ok, compare, dev, to_np)
+from tests.gpu_common import (LSE_PURE_TOL, LSE_TOL, MAX_TOL, MEAN_TOL, assert_status_ok, compare, dev,
+                              prefill_lse_bound, to_np)
 
 pytestmark = pytest.mark.gpu
 NAN16 = 0x7FC1
@@ -102,9 +103,18 @@ def test_prefill_sliding_window(B, T, Hq, Hkv, window):
 def test_prefill_window_running_max_path():
     """Large gains take the running-max softmax, where the first key tiles of an item can be
     wholly outside some rows' windows (no max yet for those rows)."""
-    out, lse, _, _, ref_st, st_lse = _prefill_case(2, 800, 16, 8, seed=41, window=200, gain_mul=1.6)
+    out, lse, ref, ref_lse, ref_st, st_lse = _prefill_case(2, 800, 16, 8, seed=41, window=200, gain_mul=1.6)
     compare(to_np(out), to_np(lse), ref_st, st_lse, st_lse, "window 200, large gains (staged)",
             lse_tol=SINGLE_LOGIT_LSE_TOL * 1.6 ** 2)
+    # against the pure oracle: the default output bounds times the gain product 1.6^2, and
+    # the LSE of every row within the rigorous per-row bound over the keys in its window
+    inp = prefill_inputs(PrefillShape("variant", 2, 800, 16, 8), seed=41)
+    inp["q_norm_w"] = inp["q_norm_w"] * 1.6
+    inp["k_norm_w"] = inp["k_norm_w"] * 1.6
+    g2 = 1.6 ** 2
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "window 200, large gains (pure)",
+            lse_tol=SINGLE_LOGIT_LSE_TOL * g2, max_tol=MAX_TOL * g2, mean_tol=MEAN_TOL * g2,
+            lse_pure_bound=prefill_lse_bound(inp, np.arange(800), window=200))
 
 
 def test_prefill_rope_variant():

@@ -4,17 +4,21 @@ that must not call cudaMalloc on its hot path).  Its split-KV partials live in t
 library's fixed device region instead of a caller workspace.
 
 It is checked through the C ABI against qwen3_attn_decode, the entry point that takes a
-caller workspace, on two calls in a row with different lengths, so contents the first
-call leaves in the shared region cannot leak into the second.  This file is collected
-last so that a run stopping at the first failure has already run every other test.
+caller workspace, on three calls in a row with different sizes (the last one smaller, so
+its partials sit in a region the earlier calls left full of their own), so contents a call
+leaves in the shared region cannot leak into the next.  Both entry points run the same
+kernels with the same split layout, so their outputs must agree bit for bit.  One sequence
+is also checked against the fp64 oracle.  This file is collected last so that a run
+stopping at the first failure has already run every other test.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import qwen3_qk_norm_rope_b200 as qa
-from synthetic import DECODE_SHAPES, decode_step_inputs
-from tests.gpu_common import MAX_TOL, MEAN_TOL, assert_status_ok, dev
+from synthetic import DECODE_SHAPES, as_f64, decode_step_inputs
+from tests.gpu_common import LSE_PURE_TOL, LSE_TOL, MAX_TOL, MEAN_TOL, assert_status_ok, dev, to_np
 
 pytestmark = pytest.mark.gpu
 
@@ -47,16 +51,41 @@ def _both(t, kc, vc):
     return out, lse, ref, lse_ref
 
 
-def test_decode_noalloc_matches_workspace_entry_point_on_two_calls():
-    Lmax = 32769
-    runs = [(_case(16, [int(x) for x in np.random.default_rng(1).integers(1024, 32768, 16)], Lmax, 3)),
-            (_case(9, [0, 1, 63, 1023, 1024, 4095, 20000, 32767, 32768], Lmax, 4))]
+def test_decode_noalloc_matches_workspace_entry_point_on_successive_calls():
+    runs = [(_case(16, [int(x) for x in np.random.default_rng(1).integers(1024, 32768, 16)], 32769, 3)),
+            (_case(9, [0, 1, 63, 1023, 1024, 4095, 20000, 32767, 32768], 32769, 4)),
+            (_case(5, [700, 2047, 0, 3000, 4095], 4096, 5))]
     for i, (t, kc, vc) in enumerate(runs):
         out, lse, ref, lse_ref = _both(t, kc, vc)
-        err = (out.float() - ref.float()).abs()
         assert torch.isfinite(out.float()).all(), f"call {i}: non-finite output"
-        assert err.max().item() <= MAX_TOL and err.mean().item() <= MEAN_TOL, f"call {i}: {err.max().item():.3e}"
-        assert (lse - lse_ref).abs().max().item() <= 1e-3, f"call {i}: lse"
+        assert torch.equal(out, ref), f"call {i}: out differs, max {(out.float() - ref.float()).abs().max().item():.3e}"
+        assert torch.equal(lse, lse_ref), f"call {i}: lse differs"
+
+
+def test_decode_noalloc_against_the_oracle():
+    """One sequence of a no-allocation call against the fp64 oracle over the same cache
+    contents (random bf16 keys and values read back from the device, the appended slot
+    included)."""
+    t, kc, vc = _case(4, [5000, 1500, 32768, 1], 32769, 6)
+    shape = DECODE_SHAPES["batched-decode"]
+    out = torch.full_like(t["q"], float("nan"))
+    lse = torch.full((4, shape.Hq), float("nan"), dtype=torch.float32, device=out.device)
+    qa.decode_noalloc(t["q"], t["k_new"], t["v_new"], t["q_norm_w"], t["k_norm_w"], kc, vc, t["cache_lens"],
+                      out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    for n, L in enumerate([5000, 1500, 32768, 1]):
+        kh = as_f64(kc[n, :, :L].cpu())
+        vh = as_f64(vc[n, :, :L].cpu())
+        q, kn, vn = (as_f64(t[k][n:n + 1].cpu()) for k in ("q", "k_new", "v_new"))
+        args = (q, kn, vn, as_f64(t["q_norm_w"].cpu()), as_f64(t["k_norm_w"].cpu()), [kh], [vh], [L], shape.theta,
+                shape.eps)
+        ref, ref_lse = oracle.decode_ref(*args)
+        _, st_lse = oracle.decode_ref(*args, staged=True)
+        err = np.abs(to_np(out[n:n + 1]) - ref)
+        assert err.max() <= MAX_TOL and err.mean() <= MEAN_TOL, f"seq {n} L={L}: {err.max():.3e}"
+        assert np.abs(to_np(lse[n:n + 1]) - st_lse).max() <= LSE_TOL
+        assert np.abs(to_np(lse[n:n + 1]) - ref_lse).max() <= LSE_PURE_TOL
 
 
 def test_decode_noalloc_rejects_requests_beyond_its_region():
