@@ -8,6 +8,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
@@ -19,6 +21,15 @@
 namespace {
 
 using q3::kD;
+
+// A named NVTX range around each compute entry point, so a profiler's timeline shows the
+// library's calls by name (header-only NVTX: nothing happens unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 constexpr int kDecodeSplit = 1024;  // keys per split-KV CTA
 constexpr int kMaxDevices = 64;
@@ -340,6 +351,7 @@ int qwen3_qk_norm_rope_variant(const qwen3_bf16* x, const float* w, const int32_
                                const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
                                int write_at_pos, const qwen3_attn_variant* variant, float eps,
                                qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_qk_norm_rope_variant");
   Variant var;
   const int sv = make_variant(variant, var);
   if (sv != QWEN3_OK) return sv;
@@ -358,6 +370,7 @@ int qwen3_qk_norm_rope_variant(const qwen3_bf16* x, const float* w, const int32_
 int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, qwen3_bf16* dst,
                        const qwen3_bf16* v_src, qwen3_bf16* v_dst, int B, int T, int H, int d, int Tcap,
                        int write_at_pos, float theta, float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_qk_norm_rope");
   const qwen3_attn_variant v = {theta, nullptr, 1.0f, 0};
   return qwen3_qk_norm_rope_variant(x, w, pos, dst, v_src, v_dst, B, T, H, d, Tcap, write_at_pos, &v, eps, stream);
 }
@@ -554,6 +567,7 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
                           const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, float* lse,
                           qwen3_bf16* k_cache, qwen3_bf16* v_cache, int Tcap, void* workspace, size_t ws_bytes,
                           int B, int T, int Hq, int Hkv, int d, float theta, float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill_ex");
   Variant var;
   const int sv = theta_variant(theta, var);
   if (sv != QWEN3_OK) return sv;
@@ -566,6 +580,7 @@ int qwen3_attn_prefill_variant(const qwen3_bf16* q, const qwen3_bf16* k, const q
                                qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap, void* workspace,
                                size_t ws_bytes, int B, int T, int Hq, int Hkv, int d,
                                const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill_variant");
   Variant var;
   const int sv = make_variant(variant, var);
   if (sv != QWEN3_OK) return sv;
@@ -578,6 +593,7 @@ int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
                              qwen3_bf16* k_cache, qwen3_bf16* v_cache, int start, int Tcap, void* workspace,
                              size_t ws_bytes, int B, int T, int Hq, int Hkv, int d, float theta, float eps,
                              qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill_chunk");
   if (k_cache == nullptr || v_cache == nullptr) return QWEN3_ERR_INVALID_ARG;
   Variant var;
   const int sv = theta_variant(theta, var);
@@ -589,6 +605,7 @@ int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
 int qwen3_attn_prefill(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, const float* q_norm_w,
                        const float* k_norm_w, const int32_t* pos, qwen3_bf16* out, int B, int T, int Hq, int Hkv,
                        int d, float theta, float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill");
   if (q == nullptr || k == nullptr || v == nullptr || q_norm_w == nullptr || k_norm_w == nullptr ||
       pos == nullptr || out == nullptr || B <= 0 || T <= 0)
     return QWEN3_ERR_INVALID_ARG;
@@ -715,6 +732,7 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
                       const float* k_norm_w, qwen3_bf16* k_cache, qwen3_bf16* v_cache, const int32_t* cache_lens,
                       qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta, float eps,
                       void* workspace, size_t ws_bytes, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_decode");
   Variant var;
   const int sv = theta_variant(theta, var);
   if (sv != QWEN3_OK) return sv;
@@ -727,6 +745,7 @@ int qwen3_attn_decode_paged(const qwen3_bf16* q, const qwen3_bf16* k_new, const 
                             const int32_t* cache_lens, qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d,
                             const qwen3_attn_variant* variant, float eps, void* workspace, size_t ws_bytes,
                             qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_decode_paged");
   Variant var;
   int st = make_variant(variant, var);
   if (st != QWEN3_OK) return st;
@@ -742,6 +761,7 @@ int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
                              const qwen3_paged_kv* kv, int start, void* workspace, size_t ws_bytes, int B, int T,
                              int Hq, int Hkv, int d, const qwen3_attn_variant* variant, float eps,
                              qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill_paged");
   Variant var;
   int st = make_variant(variant, var);
   if (st != QWEN3_OK) return st;
@@ -762,6 +782,7 @@ int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const
                              qwen3_bf16* v_out, int M, int hidden, int Hq, int Hkv, int d,
                              const qwen3_attn_variant* variant, float eps, void* workspace, size_t ws_bytes,
                              qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_qkv_proj_norm_rope");
   Variant var;
   int st = make_variant(variant, var);
   if (st != QWEN3_OK) return st;
@@ -836,6 +857,7 @@ int qwen3_attn_decode_variant(const qwen3_bf16* q, const qwen3_bf16* k_new, cons
                               const int32_t* cache_lens, qwen3_bf16* out, float* lse, int N, int Hq, int Hkv, int d,
                               int Lmax, const qwen3_attn_variant* variant, float eps, void* workspace,
                               size_t ws_bytes, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_decode_variant");
   Variant var;
   const int sv = make_variant(variant, var);
   if (sv != QWEN3_OK) return sv;
@@ -924,6 +946,7 @@ extern "C" int qwen3_attn_decode_noalloc(const qwen3_bf16* q, const qwen3_bf16* 
                                          qwen3_bf16* v_cache, const int32_t* cache_lens, qwen3_bf16* out,
                                          float* lse, int N, int Hq, int Hkv, int d, int Lmax, float theta,
                                          float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_decode_noalloc");
   // every argument check of qwen3_attn_decode comes before the region's lookup, so a bad
   // argument reports what qwen3_attn_decode reports for it
   Variant var;
@@ -1150,6 +1173,7 @@ int qwen3_attn_prefill_varlen(const qwen3_bf16* q, const qwen3_bf16* k, const qw
                               float* lse, const qwen3_paged_kv* kv, const int32_t* ctx_lens, long long key_cap,
                               void* workspace, size_t ws_bytes, int B, int N, int Hq, int Hkv, int d,
                               const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream) {
+  NvtxRange nvtx_range("qwen3_attn_prefill_varlen");
   Variant var;
   int st = make_variant(variant, var);
   if (st != QWEN3_OK) return st;
