@@ -93,6 +93,27 @@ def decode_traffic(lens: np.ndarray):
     return DECODE_TRAFFIC["bytes_per_cached_token"] * float(lens.astype(np.int64).sum())
 
 
+# DRAM traffic of the prefill attention kernel per launch on a workload (dram__bytes_read.sum
+# + dram__bytes_write.sum of one ncu capture of that launch), valid only for the kernel
+# source it was measured on.  Refreshed with each new capture.
+PREFILL_TRAFFIC = {"src_sha256": None, "bytes": {}}
+
+
+def prefill_src_sha256() -> str:
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("prefill.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "qwen3_qk_norm_rope_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def prefill_traffic(ps):
+    if PREFILL_TRAFFIC["src_sha256"] is None or PREFILL_TRAFFIC["src_sha256"] != prefill_src_sha256():
+        return None
+    return PREFILL_TRAFFIC["bytes"].get(ps.name)
+
+
 def decode_flops(lens: np.ndarray, Hq: int, d: int = 128) -> float:
     return 4.0 * Hq * d * float((lens.astype(np.int64) + 1).sum())
 
@@ -426,6 +447,19 @@ def reference_steps(run, steps: int, warmup: int, budget_s: float = REFERENCE_BU
 
 # ------------------------------------------------------------------------------ chunked prefill
 CHUNK_METRIC = "chunked-prefill causal GQA attn TFLOP/s (+QK-Norm/RoPE, cache append) % bf16 peak"
+SHORT_CHUNK_METRIC = "short-chunk prefill over a long cached prefix: HBM GB/s (K/V read, +QK-Norm/RoPE, cache append)"
+CHUNKS = {"second": "qwen3-4b-second-chunk", "short": "qwen3-4b-short-chunk"}
+
+
+def chunk_bytes(cs) -> float:
+    """Algorithmic HBM bytes of a chunked prefill: every cached and new key and value row
+    read once by the attention (start + T keys of Hkv heads), the new q, k, v read and the
+    new k', v written to the cache, and out written."""
+    d2 = cs.d * 2
+    kv_read = 2.0 * cs.B * (cs.start + cs.T) * cs.Hkv * d2
+    new_in = cs.B * cs.T * (cs.Hq + 2 * cs.Hkv) * d2
+    new_out = cs.B * cs.T * (2 * cs.Hkv + cs.Hq) * d2
+    return kv_read + new_in + new_out
 
 
 def paged_copy(caches, n: int, page: int, seed: int, dev):
@@ -453,6 +487,7 @@ class ChunkWorkload:
     LAUNCHES_PER_STEP = 2  # K prologue (cache append) + attention
 
     def __init__(self, dev: torch.device, name: str = "qwen3-4b-second-chunk", seed: int = 0, page: int = 0):
+        self.name = name
         import qwen3_qk_norm_rope_b200 as qa
 
         self.qa, self.dev, self.page = qa, dev, page
@@ -467,12 +502,16 @@ class ChunkWorkload:
         qa.qk_norm_rope(inp["k_hist"].to(dev), self.t["k_norm_w"], pos, self.kc, v_src=inp["v_hist"].to(dev),
                         v_dst=self.vc, theta=cs.theta, eps=cs.eps)
         self.out = torch.empty_like(self.t["q"])
-        self.ws = torch.empty(qa.prefill_workspace_size(cs.B, cs.T, cs.Hq, cs.Hkv), dtype=torch.uint8, device=dev)
+        self.ws = torch.empty(qa.prefill_chunk_workspace_size(cs.B, cs.start, cs.T, cs.Hq, cs.Hkv), dtype=torch.uint8,
+                              device=dev)
         if page:
             # the same caches in pages of `page` tokens, dealt to the rows in a seeded random order
             self.k_pages, self.v_pages, self.table = paged_copy([self.kc, self.vc], Tcap, page, seed, dev)
             self.ws = torch.empty(qa.prefill_paged_workspace_size(cs.B, cs.start, cs.T, cs.Hq, cs.Hkv),
                                   dtype=torch.uint8, device=dev)
+        # the call splits the key axis when the shapes give its workspace split partials
+        self.split = (qa.prefill_chunk_workspace_size(cs.B, cs.start, cs.T, cs.Hq, cs.Hkv) >
+                      qa.prefill_workspace_size(cs.B, cs.T, cs.Hq, cs.Hkv))
         self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
         torch.cuda.synchronize(dev)
         st, site = qa.device_status(clear=True, device=dev)
@@ -528,29 +567,38 @@ def chunk_oracle(name: str = "qwen3-4b-second-chunk", seed: int = 0):
 def cpu_oracle_chunk_sample(name: str = "qwen3-4b-second-chunk", rows: int = 512, seed: int = 0):
     """The oracle's chunked prefill on the last `rows` new rows (every head) of the chunk."""
     res = chunk_oracle(name, seed)(rows)
-    return dict(res, tflops=res["flops"] / res["seconds"] / 1e12, threads=oracle_threads())
+    return dict(res, tflops=res["flops"] / res["seconds"] / 1e12, threads=oracle_threads(), rows=rows)
 
 
 def run_chunk(args, world, rank, local):
+    name = CHUNKS[args.chunk]
+    cs = CHUNK_SHAPES[name]
+    short = args.chunk == "short"
     if args.impl == "reference":
         if rank != 0:
             return
-        secs, flops, _, sample = reference_steps(chunk_oracle(), args.steps, args.warmup)
+        run = chunk_oracle(name)
+        secs, flops, rows, sample = reference_steps(run, args.steps, args.warmup, args.reference_budget)
         value = flops / secs / 1e12
-        cs = CHUNK_SHAPES["qwen3-4b-second-chunk"]
-        line = {"impl": "reference", "metric": CHUNK_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        unit = "TFLOP/s"
+        if short:
+            # GB/s over the rows the oracle ran: the whole chunk's bytes scaled by its rows
+            value = chunk_bytes(cs) * rows / cs.T * args.steps / secs / 1e9
+            unit = "GB/s"
+        line = {"impl": "reference", "metric": SHORT_CHUNK_METRIC if short else CHUNK_METRIC, "value": value,
+                "unit": unit, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": {"workload": cs.name},
-                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle_threads(), "kind": "oracle",
+                "cpu_baseline": {"value": value, "unit": unit, "cores": oracle_threads(), "kind": "oracle",
                                  "sample": "per step, " + sample},
-                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
-    w = ChunkWorkload(dev, page=args.paged)
+    w = ChunkWorkload(dev, name=name, page=args.paged)
     for _ in range(args.warmup):
         w.flush.fill_(1.0)
         w.step()
@@ -595,22 +643,46 @@ def run_chunk(args, world, rank, local):
     flops = w.cs.causal_flops()
     per_s = ms * 1e-3 / K
     achieved = flops / per_s / 1e12
-    line = {"metric": CHUNK_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": w.config(),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops"], "traffic": None,
-                         "kernel": "chunked-prefill call (K prologue + cache append + attention)" if not w.page
-                         else "paged chunked-prefill call (K prologue into pages + gather + attention)",
-                         "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
-            "gpu_launches": (ChunkWorkload.LAUNCHES_PER_STEP + (1 if w.page else 0)) * K, "clocks": clk.summary(),
-            "e2e": {"value": world * flops * e_steps / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
-                    "ms_per_step": e_ms / e_steps}}
+    launches = ChunkWorkload.LAUNCHES_PER_STEP + (1 if w.split else 0)
+    kernel = ("chunked-prefill call (K prologue + cache append + attention)" if not w.page
+              else "paged chunked-prefill call (K prologue into pages + attention reading the pages in place)")
+    if w.split:
+        kernel = kernel[:-1] + " with a key-axis split + logsumexp combine)"
+    e2e_flops = world * flops * e_steps / (e_ms * 1e-3) / 1e12
+    if short:
+        # HBM bound: the K/V read of the whole prefix dominates the bytes
+        nbytes = chunk_bytes(w.cs)
+        gbs = nbytes / per_s / 1e9
+        line = {"metric": SHORT_CHUNK_METRIC, "value": world * gbs, "unit": "GB/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": w.config(),
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": kernel,
+                             "algorithmic_bytes": nbytes, "peak_source": peak_src},
+                "tflops": world * achieved, "gpu_launches": launches * K, "clocks": clk.summary(),
+                "e2e": {"value": world * nbytes * e_steps / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
+                        "ms_per_step": e_ms / e_steps}}
+    else:
+        line = {"metric": CHUNK_METRIC, "value": world * achieved, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+                "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": w.config(),
+                "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                             "frac": achieved / peaks["bf16_tflops"], "traffic": None, "kernel": kernel,
+                             "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
+                "gpu_launches": launches * K, "clocks": clk.summary(),
+                "e2e": {"value": e2e_flops, "unit": "TFLOP/s",
+                        "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_h.numel() * 2),
+                        "ms_per_step": e_ms / e_steps}}
     if world == 1 and not args.no_cpu_baseline:
-        cb = cpu_oracle_chunk_sample(rows=2048)
-        line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
-                                "sample": cb["sample"], "seconds": cb["seconds"]}
+        cb = cpu_oracle_chunk_sample(name, rows=min(2048, w.cs.T))
+        if short:
+            gb = chunk_bytes(w.cs) * cb["rows"] / w.cs.T / cb["seconds"] / 1e9
+            line["cpu_baseline"] = {"value": gb, "unit": "GB/s", "cores": cb["threads"], "kind": "oracle",
+                                    "sample": cb["sample"], "seconds": cb["seconds"]}
+        else:
+            line["cpu_baseline"] = {"value": cb["tflops"], "unit": "TFLOP/s", "cores": cb["threads"], "kind": "oracle",
+                                    "sample": cb["sample"], "seconds": cb["seconds"]}
     print(json.dumps(line), flush=True)
 
 
@@ -925,9 +997,10 @@ def run_varlen(args, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": None,
                          "kernel": "varlen prefill call (metadata + QK prologue + attention)" if not cached
-                         else "paged varlen prefill call (metadata + QK prologue into pages + gather + attention)",
+                         else "paged varlen prefill call (metadata + QK prologue into pages + attention reading the "
+                              "pages in place)",
                          "algorithmic_flops": flops, "peak_source": peak_src + " burst"},
-            "gpu_launches": (4 if cached else 3) * K, "clocks": clk.summary(),
+            "gpu_launches": 3 * K, "clocks": clk.summary(),
             "e2e": {"value": world * flops * max(1, min(K, 100)) / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                     "ms_per_step": e_ms / max(1, min(K, 100))}}
@@ -1032,6 +1105,8 @@ def main():
                     help="step: long-context prefill + batched decode (default); chunked-prefill: the chunk call alone; "
                          "qkv-proj: the merged projection with the QK-Norm/RoPE epilogue; varlen-prefill: a "
                          "ragged batch of prompts packed on one token axis")
+    ap.add_argument("--chunk", default="second", choices=sorted(CHUNKS),
+                    help="chunked-prefill: second (4096 new tokens over 4096 cached) or short (16 over 32752)")
     ap.add_argument("--qkv", default="qwen3-0.6b-qkv", choices=sorted(QKV_SHAPES),
                     help="the qkv-proj workload's shape")
     ap.add_argument("--varlen", default="qwen3-4b-varlen", choices=sorted(VARLEN_SHAPES),
@@ -1107,10 +1182,19 @@ def main():
               "frac": dbytes / dec_s / 1e9 / peaks["hbm_gbs"], "traffic": decode_traffic(w.lens),
               "kernel": "decode call (append + split-KV attention + combine)",
               "algorithmic_bytes": dbytes, "peak_source": peak_src}
-    rl_pre = {"bound": "tensor", "achieved": w.ps.causal_flops() / pre_s / 1e12, "peak": peaks["bf16_tflops"],
-              "unit": "TFLOP/s", "frac": w.ps.causal_flops() / pre_s / 1e12 / peaks["bf16_tflops"],
-              "traffic": None, "kernel": "prefill call (K prologue + attention)",
-              "algorithmic_flops": w.ps.causal_flops(), "peak_source": peak_src + " burst"}
+    # The step's prefill runs back to back for the whole timed region.  When the clock samples
+    # taken during it show the power cap, its denominator is the dense bf16 peak measured
+    # under the same cap (the sustained figure); otherwise the burst figure.  Both fractions
+    # are reported.
+    capped = bool(clocks) and "sw_power_cap" in clocks.get("reasons", [])
+    pre_tf = w.ps.causal_flops() / pre_s / 1e12
+    peak_pre = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
+    rl_pre = {"bound": "tensor", "achieved": pre_tf, "peak": peak_pre, "unit": "TFLOP/s", "frac": pre_tf / peak_pre,
+              "traffic": prefill_traffic(w.ps), "kernel": "prefill call (K prologue + attention)",
+              "algorithmic_flops": w.ps.causal_flops(),
+              "peak_source": peak_src + (" sustained (sw_power_cap seen in the timed region)" if capped else " burst"),
+              "frac_of_burst": pre_tf / peaks["bf16_tflops"],
+              "frac_of_sustained": pre_tf / peaks["bf16_tflops_sustained"]}
     line = {"metric": METRIC, "value": tflops, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",

@@ -163,7 +163,13 @@ int qwen3_attn_prefill_ex(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_
  *   start     cached tokens, the same for every batch row; 0 <= start and
  *             start + T <= Tcap, else QWEN3_ERR_INVALID_ARG.
  *   workspace, ws_bytes  at least qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d) bytes,
- *             else QWEN3_ERR_WORKSPACE.
+ *             else QWEN3_ERR_WORKSPACE.  With
+ *             qwen3_attn_prefill_chunk_workspace_size(B, start, T, Hq, Hkv, d) bytes, a chunk
+ *             whose work items are few next to the SMs (a short chunk over a long prefix)
+ *             splits the key axis: each run of keys leaves its O/l and LSE as partials in the
+ *             workspace and one more kernel merges them by logsumexp weight (the online
+ *             logsumexp of "Qwen3 Architecture Layer-by-Layer", Liger fused linear
+ *             cross-entropy).  With less, the call runs unsplit.  Sliding windows never split.
  * Other errors as in qwen3_attn_prefill_ex.  The caches must not alias q, k, v or out.
  */
 int qwen3_attn_prefill_chunk(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
@@ -302,12 +308,16 @@ int qwen3_attn_decode_paged(const qwen3_bf16* q, const qwen3_bf16* k_new, const 
 /*
  * qwen3_attn_prefill_paged - chunked prefill over a paged cache: T new tokens per batch row
  * after `start` cached ones (start = 0: a fresh prompt).  The new keys (normed, rotated) and
- * values are written into their pages at key indices start..start+T-1.  The row's first
- * start + T keys are then gathered from the pages into the workspace, where the attention
- * kernel reads them, as for qwen3_attn_prefill_chunk.  The gather costs a read and a write
- * of those keys, small next to the attention's arithmetic.  start + T <=
- * max_blocks * page_size.  Workspace:
- * qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d) bytes.
+ * values are written into their pages at key indices start..start+T-1.  The attention
+ * kernel then reads the row's start + T keys and values in place, one TMA box per page (or
+ * per 128 rows of a larger page), as qwen3_attn_prefill_chunk reads a contiguous cache.
+ * Pages under 64 keys would take too many small boxes: their keys and values are first
+ * gathered into the workspace, where the attention kernel reads them.
+ * start + T <= max_blocks * page_size.  A key index below start + T whose block-table entry
+ * is out of range is recorded as QWEN3_ERR_INVALID_ARG in the device status word (read in
+ * place, its rows are not read; gathered, they are zero) and the call's outputs for that row
+ * are undefined.  Workspace: qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d)
+ * bytes.
  */
 int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v,
                              const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
@@ -317,8 +327,11 @@ int qwen3_attn_prefill_paged(const qwen3_bf16* q, const qwen3_bf16* k, const qwe
                              int B, int T, int Hq, int Hkv, int d,
                              const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream);
 
-/* Scratch bytes qwen3_attn_prefill_paged needs: K and V of start + T keys per row, Q', and
- * alignment slack; 0 when a size is not positive (start may be 0). */
+/* Scratch bytes qwen3_attn_prefill_paged needs: K and V of start + T keys per row (used
+ * for pages under 64 keys only), Q', the partials of a key-axis split when its work items
+ * are few (as for qwen3_attn_prefill_chunk_workspace_size), and alignment slack; 0 when a
+ * size is not positive (start may be 0).  A smaller workspace that still holds all but the
+ * split partials runs the call unsplit. */
 size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d);
 
 /*
@@ -342,8 +355,9 @@ size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, 
  *              to its key indices ctx_lens[b] .. ctx_lens[b] + T_b - 1, and its queries see
  *              its ctx_lens[b] cached keys first, as in qwen3_attn_prefill_paged.
  *   ctx_lens   [B] int32 device array of cached keys per sequence, or NULL (all 0).
- *   key_cap    with kv: a bound on the sum over sequences of ctx_lens[b] + T_b (the
- *              workspace holds that many gathered keys and values).
+ *   key_cap    with kv: a bound (> 0) on the sum over sequences of ctx_lens[b] + T_b.  The
+ *              attention reads every sequence's keys and values in its own pages; pages
+ *              under 64 keys are gathered first, into key_cap rows of the workspace.
  * The lengths stay on the device: the host reads none of them.  A sequence whose metadata
  * is out of range (offsets outside [0, N] or decreasing, a negative ctx_lens, keys past
  * max_blocks * page_size, or keys past key_cap) is recorded as QWEN3_ERR_INVALID_ARG in
@@ -359,7 +373,8 @@ int qwen3_attn_prefill_varlen(const qwen3_bf16* q, const qwen3_bf16* k, const qw
                               const qwen3_attn_variant* variant, float eps, qwen3_stream_t stream);
 
 /* Scratch bytes qwen3_attn_prefill_varlen needs: the sequence metadata and work list, Q',
- * and K' and V for N rows (key_cap = 0) or key_cap rows; 0 for an unsupported shape. */
+ * and K' and V for N rows (key_cap = 0) or key_cap rows (used for pages under 64 keys
+ * only); 0 for an unsupported shape. */
 size_t qwen3_attn_prefill_varlen_workspace_size(int B, int N, long long key_cap, int Hq, int Hkv, int d);
 
 /*
@@ -393,6 +408,16 @@ size_t qwen3_qkv_proj_workspace_size(int M);
  * (normed, rotated keys) + B*T*Hq*d*2 (normed, rotated queries), plus alignment slack;
  * 0 when a size is not positive. */
 size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d);
+
+/*
+ * qwen3_attn_prefill_chunk_workspace_size - workspace bytes of a chunked prefill (or a
+ * prefill_variant with caches) of T new tokens over `start` cached ones that let it split
+ * the key axis when its work items are few: qwen3_attn_prefill_workspace_size plus the
+ * split partials (fp32 O/l and LSEs of every new row and query head, for each run of
+ * keys).  Equal to qwen3_attn_prefill_workspace_size when the shapes give no split.
+ * 0 for invalid sizes.
+ */
+size_t qwen3_attn_prefill_chunk_workspace_size(int B, int start, int T, int Hq, int Hkv, int d);
 
 /* Scratch bytes qwen3_attn_decode needs (split-KV partial outputs and logsumexps). */
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax);

@@ -62,6 +62,7 @@ SIGNATURES = {
     "qwen3_qkv_proj_norm_rope": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _V, _F, _P, _Z, _P]),
     "qwen3_qkv_proj_workspace_size": (_Z, [_I]),
     "qwen3_attn_prefill_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "qwen3_attn_prefill_chunk_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "qwen3_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_kv_cache_bytes": (_Z, [_I, _I, _I, _I]),
     "qwen3_attn_status_string": (ctypes.c_char_p, [_I]),
@@ -144,6 +145,11 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, shape: tuple, device: 
 
 def prefill_workspace_size(B: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
     return int(lib().qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d))
+
+
+def prefill_chunk_workspace_size(B: int, start: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
+    """Workspace of a chunk over `start` cached tokens, room for a key-axis split included."""
+    return int(lib().qwen3_attn_prefill_chunk_workspace_size(B, start, T, Hq, Hkv, d))
 
 
 def prefill_paged_workspace_size(B: int, start: int, T: int, Hq: int, Hkv: int, d: int = HEAD_DIM) -> int:
@@ -266,7 +272,8 @@ def prefill_chunk(q, k, v, q_norm_w, k_norm_w, pos, k_cache, v_cache, start: int
     if lse is not None:
         _need(lse, "lse", torch.float32, (B, Hq, T), dev)
     if workspace is None:
-        workspace = torch.empty(prefill_workspace_size(B, T, Hq, Hkv, d), dtype=torch.uint8, device=dev)
+        workspace = torch.empty(prefill_chunk_workspace_size(B, start, T, Hq, Hkv, d), dtype=torch.uint8,
+                                device=dev)
     ws_bytes = workspace.numel() * workspace.element_size()
     if _is_default(inv_freq, attention_scaling, window):
         _check(lib().qwen3_attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(q_norm_w), _ptr(k_norm_w),

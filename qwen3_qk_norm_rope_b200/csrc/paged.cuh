@@ -4,9 +4,11 @@
 //
 // A pool holds num_pages pages of `page` tokens for all KV heads, [num_pages, Hkv, page, d]
 // bf16; key index j of batch row b lives in page block_table[b, j / page] at offset
-// j % page.  The decode split kernel reads pages directly (decode.cuh); this file holds the
-// gather that copies a row's first n keys out of the pages into the contiguous layout
-// [B, Hkv, n, d], which the prefill attention kernel then reads.
+// j % page.  The decode split kernel and the prefill attention kernel read pages of 64 keys
+// or more in place; this file holds the gather for smaller pages, which copies a row's first
+// n keys out of the pages into the contiguous layout [B, Hkv, n, d] that the prefill
+// attention kernel then reads (a 128-key tile of 16-key pages would take 16 TMA boxes of
+// 2 KB per operand, and the TMA box rate, not the bytes, would then bound the prefill).
 #pragma once
 #include "common.cuh"
 

@@ -60,6 +60,19 @@ struct PrefillParams {
   const int4* vl_ent;
   const int* vl_n_items;
   uint4* out;
+  // Key-axis split (the kSplit instance): every (pair, batch row, KV head) is n_split items,
+  // split s taking the s-th of n_split contiguous runs of the pair's key tiles.  Each item
+  // leaves its rows' O/l (fp32) and LSE as partials, [B*T, Hq, n_split, d] and
+  // [B*T, Hq, n_split], for prefill_split_combine_kernel.
+  int n_split;
+  float* part_o;
+  float* part_lse;
+  // Keys and values read in place from page pools (block_table != nullptr): tmK and tmV are
+  // 2-D maps over the pools as rows of d, [num_pages * Hkv * page, d], with boxes of
+  // min(page, 128) rows, and key j of batch row (or sequence) r lies in page
+  // block_table[r, j >> log2_page] at row j & (page - 1).
+  const int* block_table;
+  int max_blocks, log2_page, num_pages;
 };
 
 constexpr uint32_t kPfTile = 32768;  // 128 rows x 128 bf16
@@ -75,7 +88,8 @@ constexpr uint32_t kPfStage = kPfBar + 1024;
 constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
                    kBOFull = 96, kBQFull = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
                    kBRed = 144,     // 2 groups x 4 warps x (max|g_q|, max|g_k|): 64 bytes
-                   kBQEmpty = 208;  // [X]: the last S_X MMA of an item has read Q'_X
+                   kBQEmpty = 208,  // [X]: the last S_X MMA of an item has read Q'_X
+                   kBTail = 224;    // a paged V tile past the keys' end has landed (zeroed after)
 constexpr uint32_t kPrefillSmemBytes = kPfStage + 2 * kPfBox + 1024;  // + slack to align the base to 1024
 constexpr int kPrefillThreads = 320;
 constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
@@ -127,6 +141,26 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, const Item
   return ti;
 }
 
+// The key tiles an item reads: from tile lo on, nX[X] of them for its query tile X (0 when
+// the item has no tile X).  A split item takes its own run of the pair's tiles: split s of n
+// covers tiles [s*N/n, (s+1)*N/n) of the N the pair reads, and tile X reads the part of that
+// run below its own count.
+template <bool kWin, bool kSplit>
+__device__ __forceinline__ void item_tiles(const PrefillParams& p, const ItemSeq& sq, int pair, int split, int& lo,
+                                           int (&nX)[2]) {
+  lo = item_lo<kWin>(p, sq, pair);
+  nX[0] = tile_info(p, sq, 2 * pair, lo).nkv;
+  nX[1] = tile_info(p, sq, 2 * pair + 1, lo).nkv;
+  if constexpr (kSplit) {
+    const int n = max(nX[0], nX[1]);
+    const int j0 = static_cast<int>(static_cast<long long>(split) * n / p.n_split);
+    const int j1 = static_cast<int>(static_cast<long long>(split + 1) * n / p.n_split);
+    nX[0] = max(0, min(nX[0], j1) - j0);
+    nX[1] = max(0, min(nX[1], j1) - j0);
+    lo += j0;
+  }
+}
+
 // Item this CTA takes in round k: snake order (left to right in even rounds, right to left
 // in odd ones) over the heaviest-first numbering, so the heaviest and lightest items of
 // consecutive rounds land on the same CTA.
@@ -153,9 +187,17 @@ __device__ __forceinline__ int item_count(const PrefillParams& p) {
 
 // Work item -> (pair, batch coordinate, KV head, sequence).  A varlen item reads its entry
 // (two independent 16-byte loads); its batch coordinate is 0 (the packed axis is one row).
-template <bool kVar>
+template <bool kVar, bool kSplit = false>
 __device__ __forceinline__ void item_fetch(const PrefillParams& p, int item, int& pair, int& b, int& hkv,
-                                           ItemSeq& sq) {
+                                           ItemSeq& sq, int& split, int* seq_index = nullptr) {
+  split = 0;
+  if constexpr (kSplit) {
+    // the n_split items of one pair are adjacent: the heaviest-first order of pairs stays
+    split = item % p.n_split;
+    item_coords(p, item / p.n_split, pair, b, hkv);
+    sq = ItemSeq{0, p.T, p.start, 0};
+    return;
+  }
   if constexpr (kVar) {
     const int e = item / p.Hkv;
     hkv = item - e * p.Hkv;
@@ -164,15 +206,63 @@ __device__ __forceinline__ void item_fetch(const PrefillParams& p, int item, int
     sq = ItemSeq{a.x, a.y, a.z, a.w};
     pair = c.x;
     b = 0;
+    if (seq_index != nullptr) *seq_index = c.y;
   } else {
     item_coords(p, item, pair, b, hkv);
     sq = ItemSeq{0, p.T, p.start, 0};
   }
 }
 
+// Paged-cache loads.  They run in the producer warp only, and their code shares the
+// instruction cache with the softmax warps' hot loop: unrolled at each of their three call
+// sites they cost the prefill a third of its speed in instruction fetch stalls, so the
+// copies are issued by one out-of-line function.
+//
+// The block-table entries of the boxes of a 128-key tile, for the boxes that start before
+// the row's key count nk (boxes of R = min(page, 128) rows, each inside one page): only the
+// loads, into registers, so the producer issues them a tile ahead of their use.  Entries
+// past the table are -1.  Returns the box count.
+__device__ __forceinline__ int paged_tile_fetch(const PrefillParams& p, const int* table_row, int key0, int nk,
+                                                int (&pg)[8]) {
+  const int R = min(1 << p.log2_page, 128);
+  const int nsub = min(128 / R, (nk - key0 + R - 1) / R);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int blk = (key0 + i * R) >> p.log2_page;
+    pg[i] = (i < nsub && blk < p.max_blocks) ? __ldg(table_row + blk) : -1;
+  }
+  return nsub;
+}
+
+// The loads of one 128-key tile (two 64-dim halves) into `dst`, signalled on `bar`: one box
+// per entry g0..g7 below nsub, none for an out-of-range page (recorded as an invalid
+// argument).  The barrier's expected bytes are set after the copies are issued, as the sum
+// of what they carry; its phase cannot complete before that arrival.
+__device__ __noinline__ void paged_tile_issue(const PrefillParams& p, uint32_t dst, const CUtensorMap* map,
+                                              uint32_t bar, int nsub, int key0, int hkv, int g0, int g1, int g2,
+                                              int g3, int g4, int g5, int g6, int g7) {
+  const int R = min(1 << p.log2_page, 128);
+  const int pg[8] = {g0, g1, g2, g3, g4, g5, g6, g7};
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= nsub) break;
+    if (pg[i] < 0 || pg[i] >= p.num_pages) {
+      record_error(QWEN3_ERR_INVALID_ARG, kSitePagedTable);
+      continue;
+    }
+    const int row = ((pg[i] * p.Hkv + hkv) << p.log2_page) | ((key0 + i * R) & ((1 << p.log2_page) - 1));
+    tma_load_2d(dst + i * R * 128, map, bar, 0, row);
+    tma_load_2d(dst + kPfBox + i * R * 128, map, bar, 64, row);
+    bytes += static_cast<uint32_t>(R) * 256u;
+  }
+  mbar_arrive_expect_tx(bar, bytes);
+}
+
 // kWin: a sliding window is set (p.window > 0); the full-causal instance carries none of its
-// masks or bookkeeping.  kVar: a varlen batch (items from the device's entry list).
-template <bool kWin, bool kVar>
+// masks or bookkeeping.  kVar: a varlen batch (items from the device's entry list).  kSplit:
+// a key-axis split (a uniform batch, no window), whose items write partials.
+template <bool kWin, bool kVar, bool kSplit = false>
 __global__ void __launch_bounds__(kPrefillThreads, 1)
     fmha_prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -199,6 +289,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       mbar_init(bar + kBQEmpty + 8 * s, 1);
     }
     mbar_init(bar + kBDone, 1);
+    mbar_init(bar + kBTail, 1);
     *abort_flag = 0;
     mbar_init_fence();
     fence_proxy_async_smem();
@@ -220,16 +311,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tma_prefetch_map(&tmV);
       griddep_wait();  // Q', K' (and a cache's V) come from the prologue kernel before this one
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last[2] = {-1, -1};
-      uint32_t it = 0, q_use[2] = {0, 0};
+      uint32_t it = 0, q_use[2] = {0, 0}, tail_use = 0;
       bool ok = true;
       const int n_items = item_count<kVar>(p);
       for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-        int pair, b, hkv;
+        int pair, b, hkv, split, lo, nX[2], seq = 0;
         ItemSeq sq;
-        item_fetch<kVar>(p, item, pair, b, hkv, sq);
-        const int lo = item_lo<kWin>(p, sq, pair);
-        const int nX[2] = {tile_info(p, sq, 2 * pair, lo).nkv, tile_info(p, sq, 2 * pair + 1, lo).nkv};
+        item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split, &seq);
+        item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+        // a paged cache: the row's block table (a varlen sequence's own row) and key count
+        const int* table_row =
+            p.block_table != nullptr ? p.block_table + static_cast<long long>(kVar ? seq : b) * p.max_blocks : nullptr;
+        const int nk = sq.start + sq.T;
+        // the first tile's block-table entries; each later tile's are fetched one tile ahead
         const int n = max(nX[0], nX[1]);
+        int pg_next[8] = {-1, -1, -1, -1, -1, -1, -1, -1}, nsub_next = 0;
+        if (table_row != nullptr && n > 0) nsub_next = paged_tile_fetch(p, table_row, lo * 128, nk, pg_next);
         for (int X = 0; X < 2 && ok; ++X) {
           if (nX[X] == 0) continue;
           // buffer X is free once the previous item's last S_X MMA has completed
@@ -252,22 +349,69 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             ok = false;
             break;
           }
-          if (!(p.fault != 0 && it == 0)) {
-            mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
-            tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, sq.koff + (lo + j) * 128, hkv, b);
-            tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, sq.koff + (lo + j) * 128, hkv,
-                        b);
-            k_last[st] = static_cast<int>(it);
+          const int key0 = (lo + j) * 128;
+          if (table_row == nullptr) {
+            if (!(p.fault != 0 && it == 0)) {
+              mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
+              tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, sq.koff + key0, hkv, b);
+              tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, sq.koff + key0, hkv, b);
+              k_last[st] = static_cast<int>(it);
+            }
+            if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
+            tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, sq.koff + key0, hkv, b);
+            tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, sq.koff + key0, hkv, b);
+            v_last[st] = static_cast<int>(it);
+          } else {
+            // In place from the pages: one box per page (or per 128 rows of a larger page),
+            // none for the part of the tile past the keys' end.  The bytes the barrier waits
+            // for are those of the boxes issued.
+            int pg[8];
+            const int nsub = nsub_next;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pg[i] = pg_next[i];
+            if (j + 1 < n) nsub_next = paged_tile_fetch(p, table_row, key0 + 128, nk, pg_next);
+            if (!(p.fault != 0 && it == 0)) {
+              paged_tile_issue(p, sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
+                               pg[2], pg[3], pg[4], pg[5], pg[6], pg[7]);
+              k_last[st] = static_cast<int>(it);
+            }
+            if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
+              ok = false;
+              break;
+            }
+            if (key0 + 128 <= nk) {
+              paged_tile_issue(p, sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
+                               pg[2], pg[3], pg[4], pg[5], pg[6], pg[7]);
+            } else {
+              // The tile runs past the keys' end: its rows from there on hold whatever the page
+              // (or an earlier use of this buffer) left, NaN included, and P = 0 there would
+              // still carry NaN into P.V.  Load on the private barrier, zero those rows, then
+              // release the tile to the MMA issuer.
+              paged_tile_issue(p, sV + st * kPfTile, &tmV, bar + kBTail, nsub, key0, hkv, pg[0], pg[1], pg[2],
+                               pg[3], pg[4], pg[5], pg[6], pg[7]);
+              if (!mbar_wait(bar + kBTail, tail_use & 1, p.wait, abort_flag, kSitePrefillVFull)) {
+                // the copies still land in this CTA's shared memory: wait for them regardless
+                mbar_wait(bar + kBTail, tail_use & 1, p.wait, nullptr, kSitePrefillDrain);
+                ok = false;
+                break;
+              }
+              ++tail_use;
+#pragma unroll 1
+              for (int r = nk - key0; r < 128; ++r)
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                  st_shared_v4(sV + st * kPfTile + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+                  st_shared_v4(sV + st * kPfTile + kPfBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+                }
+              fence_proxy_async_smem();
+              mbar_arrive(bar + kBVFull + 8 * st);
+            }
+            v_last[st] = static_cast<int>(it);
           }
-          if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
-          tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, sq.koff + (lo + j) * 128, hkv, b);
-          tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, sq.koff + (lo + j) * 128, hkv,
-                      b);
-          v_last[st] = static_cast<int>(it);
         }
       }
       // Every issued copy must land before this CTA's shared memory is released.
@@ -286,13 +430,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       bool ok = true;
       const int n_items = item_count<kVar>(p);
       for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-        int pair, b, hkv;
+        int pair, b, hkv, split, lo, nX[2];
         ItemSeq sq;
-        item_fetch<kVar>(p, item, pair, b, hkv, sq);
-        const int lo = item_lo<kWin>(p, sq, pair);
-        const int nX[2] = {tile_info(p, sq, 2 * pair, lo).nkv, tile_info(p, sq, 2 * pair + 1, lo).nkv};
+        item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split);
+        item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
         const int n = max(nX[0], nX[1]);
-        if (kVar && n == 0) continue;  // an empty entry (none is built; the producer skips it too)
+        if ((kVar || kSplit) && n == 0) continue;  // an item with no tile (the producer skips it too)
         for (int X = 0; X < 2 && ok; ++X)
           if (nX[X] > 0) {
             ok = mbar_wait(bar + kBQFull + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQFull);
@@ -401,12 +544,24 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // waits for a P that is only written after this epilogue.
     const int n_items = item_count<kVar>(p);
     for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-      int pair, b, hkv;
+      int pair, b, hkv, split, lo, nX[2];
       ItemSeq sq;
-      item_fetch<kVar>(p, item, pair, b, hkv, sq);
-      const int lo = item_lo<kWin>(p, sq, pair);
-      const TileInfo ti = tile_info(p, sq, 2 * pair + X, lo);
-      if (ti.nkv == 0) continue;  // this item has no tile X
+      item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split);
+      item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+      TileInfo ti;
+      ti.t0 = (2 * pair + X) * p.P;
+      ti.nkv = nX[X];
+      if (ti.nkv == 0) {
+        // This item has no tile X.  A split's run may hold no key a tile's rows see: its
+        // partials are still written, as no contribution (LSE -inf), for the combine.
+        if constexpr (kSplit) {
+          const int t_row = ti.t0 + (row >> p.log2G);
+          if (t_row < sq.T)
+            p.part_lse[((static_cast<long long>(b) * p.T + t_row) * p.Hq + hkv * G + (row & (G - 1))) * p.n_split +
+                       split] = -INFINITY;
+        }
+        continue;
+      }
       const int t0 = ti.t0;
 
       const int t_row = t0 + (row >> p.log2G);
@@ -496,7 +651,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         // columns.  P occupies S columns [0,64): chunk c of P (columns [16c,16c+16)) only
         // overwrites S columns that chunks 0..c have already read.
         // a row whose keys so far all lie outside its window has no max yet: p = 0 for it
-        const float mref = (kWin && m_new == -INFINITY) ? 0.0f : m_new;
+        const float mref = ((kWin || kSplit) && m_new == -INFINITY) ? 0.0f : m_new;
         const uint64_t sl2x2 = f2pack(sl2, sl2), negm2 = f2pack(-mref, -mref);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -560,6 +715,27 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tc_fence_after();
       const int h = hkv * G + (row & (G - 1));
       const bool valid = t_row < sq.T;
+      if constexpr (kSplit) {
+        // This run of keys' O/l (fp32) and its LSE, for the combine kernel.  A row that saw no
+        // key of the run (l = 0) leaves O = 0 and LSE = -inf, which the combine weighs by 0.
+        const float inv_lp = l > 0.f ? 1.0f / l : 0.f;
+        const long long slot = ((static_cast<long long>(b) * p.T + t_row) * p.Hq + h) * p.n_split + split;
+        float4* dst = reinterpret_cast<float4*>(p.part_o + slot * kD);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          tmem_ld32(tO + c * 32, r);
+          if (valid) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              dst[c * 8 + u] = make_float4(__uint_as_float(r[4 * u]) * inv_lp, __uint_as_float(r[4 * u + 1]) * inv_lp,
+                                           __uint_as_float(r[4 * u + 2]) * inv_lp,
+                                           __uint_as_float(r[4 * u + 3]) * inv_lp);
+          }
+        }
+        if (valid) p.part_lse[slot] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+        continue;
+      }
       const float inv_l = 1.0f / l;
       // O/l in two 64-dim halves through this group's staging box.  Row r of the tile is row r
       // of the box [P positions][G heads][64 dims], so one tiled store writes the half to
@@ -623,6 +799,55 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge of the key-split partials of a prefill: per (row of the token axis, query head),
+// lse = log sum_s exp(lse_s) and out = sum_s exp(lse_s - lse) O_s (the online logsumexp of
+// "Qwen3 Architecture Layer-by-Layer", Liger fused linear cross-entropy, across runs of
+// keys).  One warp per (token, head): lane s holds run s's LSE (n_split <= 32) for the
+// max and the weights, and lane i owns output dims 4i..4i+3; the runs' partial rows are
+// read eight at a time so their loads overlap.
+struct SplitCombineParams {
+  const float* part_o;    // [B*T, Hq, n_split, d]
+  const float* part_lse;  // [B*T, Hq, n_split]
+  uint2* out;             // [B*T, Hq, d] bf16
+  float* lse;             // [B, Hq, T] or nullptr
+  int B, T, Hq, n_split;
+};
+
+__global__ void __launch_bounds__(256) prefill_split_combine_kernel(const __grid_constant__ SplitCombineParams p) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // (b*T + t)*Hq + h
+  if (row >= static_cast<long long>(p.B) * p.T * p.Hq) return;
+  const int lane = threadIdx.x & 31;
+  const float mine = lane < p.n_split ? p.part_lse[row * p.n_split + lane] : -INFINITY;
+  float M = mine;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const float kLog2e = 1.44269504088896341f;
+  // a run with no key this row sees has LSE -inf: weight 0, and its O is never read
+  const float w = (mine == -INFINITY || M == -INFINITY) ? 0.f : ex2((mine - M) * kLog2e);
+  const float z = warp_sum(w);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  const float4* po = reinterpret_cast<const float4*>(p.part_o + row * p.n_split * kD) + lane;
+#pragma unroll 8
+  for (int s = 0; s < p.n_split; ++s) {
+    const float ws = __shfl_sync(0xffffffffu, w, s);
+    const float4 o = po[s * (kD / 4)];  // read even when unused, so the loads overlap
+    if (ws != 0.f) {                     // an unused run's row may hold anything, NaN included
+      acc.x += ws * o.x;
+      acc.y += ws * o.y;
+      acc.z += ws * o.z;
+      acc.w += ws * o.w;
+    }
+  }
+  const float inv = z > 0.f ? 1.0f / z : 0.f;
+  p.out[row * (kD / 4) + lane] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
+  if (p.lse != nullptr && lane == 0) {
+    const long long bt = row / p.Hq;
+    const int h = static_cast<int>(row - bt * p.Hq);
+    const long long b = bt / p.T, t = bt - b * p.T;
+    p.lse[(b * p.Hq + h) * p.T + t] = M + logf(z);
   }
 }
 

@@ -48,13 +48,17 @@ struct PrologueParams {
 
 constexpr int kPrologueHeads = 8;  // head vectors of one token in flight per warp
 
-// One warp per token (b, t): its position and the sin/cos of its 64 angles are computed
-// once and shared by the token's H key heads (and, for the prefill, its Hq query heads),
-// whose loads are issued a batch at a time before any arithmetic.  Each warp's work is a
-// fixed chain of dependent loads, so the kernel takes as many chain times as it has waves:
-// at most 64 registers a thread keeps 4 blocks (32 warps) resident per SM, which holds the
-// 4096 tokens of a B=2, T=2048 prefill in one wave (at 80 registers only 3 blocks fit and
-// 68 blocks ran as a second wave).
+// One warp per token (b, t): its position and the sin/cos of its 64 angles are computed once
+// and shared by the token's H key heads (and, for the prefill, its Hq query heads), whose
+// loads are issued a batch at a time before any arithmetic.  Each warp's work is a fixed
+// chain of dependent loads, so the kernel takes as many chain times as it has waves: at most
+// 64 registers a thread keeps 4 blocks (32 warps) resident per SM, which holds the 4096
+// tokens of a B=2, T=2048 prefill in one wave (at 80 registers only 3 blocks fit and 68
+// blocks ran as a second wave).  kPerBatch: one warp per batch of kPrologueHeads head vectors
+// of a token instead (its key batches, then its query batches), for calls whose tokens are
+// few enough that all their batches fit one wave: the batches then run side by side rather
+// than as one chain per token.
+template <bool kPerBatch>
 __global__ void __launch_bounds__(256, 4) qk_norm_rope_kernel(const __grid_constant__ PrologueParams p) {
   // The RoPE constants go through shared memory once per block: read from parameter space
   // with a lane-dependent index they would serialise.
@@ -72,7 +76,18 @@ __global__ void __launch_bounds__(256, 4) qk_norm_rope_kernel(const __grid_const
   const float2 gb = reinterpret_cast<const float2*>(p.w)[32 + lane];
   const float hi0 = s_rope[2 * lane], hi1 = s_rope[2 * lane + 1];
   const float lo0 = s_rope[kHalf + 2 * lane], lo1 = s_rope[kHalf + 2 * lane + 1];
-  for (int bt = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); bt < ntok; bt += nwarps) {
+  const int nbk = (p.H + kPrologueHeads - 1) / kPrologueHeads;
+  const int nb = kPerBatch ? nbk + (p.xq != nullptr ? (p.Hq + kPrologueHeads - 1) / kPrologueHeads : 0) : 1;
+  // units: ntok (one per token), or ntok * nb <= 32 warps per SM (one per batch of heads)
+  const int nunits = ntok * nb;
+  for (int unit = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); unit < nunits; unit += nwarps) {
+    const int bt = kPerBatch ? unit / nb : unit;
+    // the head batches of this unit: all of them, or key batch ub, or query batch ub - nbk
+    const int ub = kPerBatch ? unit - bt * nb : -1;
+    const int k_lo = ub < 0 ? 0 : (ub < nbk ? ub * kPrologueHeads : p.H);
+    const int k_hi = ub < 0 ? p.H : k_lo + kPrologueHeads;
+    const int q_lo = ub < 0 ? 0 : (ub < nbk ? p.Hq : (ub - nbk) * kPrologueHeads);
+    const int q_hi = ub < 0 ? p.Hq : q_lo + kPrologueHeads;
     const int b = bt / p.T;
     const int t = bt - b * p.T;
     const int ps = p.pos[bt];
@@ -126,7 +141,7 @@ __global__ void __launch_bounds__(256, 4) qk_norm_rope_kernel(const __grid_const
     c0 *= p.rope_scale;
     s1 *= p.rope_scale;
     c1 *= p.rope_scale;
-    for (int h0 = 0; kv_write && h0 < p.H; h0 += kPrologueHeads) {
+    for (int h0 = k_lo; kv_write && h0 < min(k_hi, p.H); h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
       uint2 vv[kPrologueHeads];
 #pragma unroll
@@ -161,7 +176,7 @@ __global__ void __launch_bounds__(256, 4) qk_norm_rope_kernel(const __grid_const
     const float2 qa = reinterpret_cast<const float2*>(p.wq)[lane];
     const float2 qb = reinterpret_cast<const float2*>(p.wq)[32 + lane];
     const int G = 1 << p.log2G;
-    for (int h0 = 0; h0 < p.Hq; h0 += kPrologueHeads) {
+    for (int h0 = q_lo; h0 < min(q_hi, p.Hq); h0 += kPrologueHeads) {
       uint32_t ua[kPrologueHeads], ub[kPrologueHeads];
 #pragma unroll
       for (int u = 0; u < kPrologueHeads; ++u) {

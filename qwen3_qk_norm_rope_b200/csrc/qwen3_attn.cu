@@ -12,8 +12,8 @@
 
 #include "common.cuh"
 #include "decode.cuh"
-#include "prefill.cuh"
 #include "paged.cuh"
+#include "prefill.cuh"
 #include "prologue.cuh"
 #include "qkv_proj.cuh"
 #include "varlen.cuh"
@@ -179,6 +179,8 @@ int ensure_kernel_attrs() {
       cudaFuncSetAttribute(q3::fmha_prefill_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(q3::fmha_prefill_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kPrefillSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::fmha_prefill_kernel<false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -208,6 +210,38 @@ int num_sms() {
 size_t kspace_bytes(int B, int T, int Hkv, int d) {
   return (static_cast<size_t>(B) * Hkv * T * d * 2 + 255) & ~static_cast<size_t>(255);
 }
+
+// Key-axis split of a prefill whose work items are few next to the SMs (a short chunk over
+// a long cached prefix): the number of runs its keys are cut into, 1 for no split.  It is
+// fixed by the shapes alone, so the workspace size that holds the partials is known on the
+// host: about kSplitTarget items in all, each run at least 4 key tiles, at most 32 runs.
+constexpr int kSplitTarget = 128;
+int split_count(int B, int start, int T, int Hq, int Hkv, int window) {
+  if (window > 0 || B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 1;
+  const int G = Hq / Hkv;
+  if (G > 128) return 1;
+  const long long P = 128 / G;
+  const long long n_pairs = ((T + P - 1) / P + 1) / 2;
+  const long long items = static_cast<long long>(B) * Hkv * n_pairs;
+  const long long tiles = (static_cast<long long>(start) + T + 127) / 128;
+  if (items * 2 > kSplitTarget || tiles < 8) return 1;
+  long long n = std::min<long long>(kSplitTarget / items, tiles / 4);
+  n = std::min<long long>(n, 32);
+  return n >= 2 ? static_cast<int>(n) : 1;
+}
+
+// Bytes of the split partials: O/l fp32 [B*T, Hq, n, d] and LSEs [B*T, Hq, n], each
+// 256-byte aligned.
+size_t split_bytes(int B, int T, int Hq, int n) {
+  if (n <= 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * T * Hq * n;
+  return ((rows * kD * 4 + 255) & ~static_cast<size_t>(255)) + ((rows * 4 + 255) & ~static_cast<size_t>(255));
+}
+
+// Pages of at least this many keys are read in place by the prefill attention kernel (one
+// TMA box per page per 64-dim half); smaller ones are gathered first, since a tile of them
+// would take too many small boxes.
+constexpr int kInPlaceMinPage = 64;
 
 int check_common(int Hq, int Hkv, int d) {
   if (Hq <= 0 || Hkv <= 0) return QWEN3_ERR_INVALID_ARG;
@@ -266,10 +300,19 @@ int launch_prologue(const void* x, const float* w, const int32_t* pos, void* dst
   const long long ntok = static_cast<long long>(B) * T;
   if (ntok > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   const int warps = 8;
-  long long blocks = (ntok + warps - 1) / warps;  // one warp per token
+  // A warp per token, or per batch of a token's heads when that still fits one wave of
+  // resident warps (32 per SM): few tokens then run their batches side by side.
+  const long long nb = (H + q3::kPrologueHeads - 1) / q3::kPrologueHeads +
+                       (q.xq != nullptr ? (q.Hq + q3::kPrologueHeads - 1) / q3::kPrologueHeads : 0);
+  const bool per_batch = nb > 1 && ntok * nb <= static_cast<long long>(num_sms()) * 32;
+  const long long units = per_batch ? ntok * nb : ntok;
+  long long blocks = (units + warps - 1) / warps;
   const long long cap = static_cast<long long>(num_sms()) * 16;  // grid-stride beyond 16 blocks per SM
   if (blocks > cap) blocks = cap;
-  q3::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
+  if (per_batch)
+    q3::qk_norm_rope_kernel<true><<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
+  else
+    q3::qk_norm_rope_kernel<false><<<static_cast<unsigned>(blocks), warps * 32, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
@@ -331,8 +374,16 @@ size_t qwen3_attn_prefill_workspace_size(int B, int T, int Hq, int Hkv, int d) {
 
 size_t qwen3_attn_prefill_paged_workspace_size(int B, int start, int T, int Hq, int Hkv, int d) {
   if (B <= 0 || start < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return 0;
-  // K and V of the row's first start + T keys gathered out of the pages, then Q'
-  return 2 * kspace_bytes(B, start + T, Hkv, d) + kspace_bytes(B, T, Hq, d) + 256;
+  // K and V of the row's first start + T keys gathered out of pages under kInPlaceMinPage
+  // keys (pages of that size or more are read in place and leave this region unused), Q',
+  // then the partials of a key-axis split
+  return 2 * kspace_bytes(B, start + T, Hkv, d) + kspace_bytes(B, T, Hq, d) +
+         split_bytes(B, T, Hq, split_count(B, start, T, Hq, Hkv, 0)) + 256;
+}
+
+size_t qwen3_attn_prefill_chunk_workspace_size(int B, int start, int T, int Hq, int Hkv, int d) {
+  if (B <= 0 || start < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return 0;
+  return qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d) + split_bytes(B, T, Hq, split_count(B, start, T, Hq, Hkv, 0));
 }
 
 size_t qwen3_attn_decode_workspace_size(int N, int Hq, int d, int Lmax) {
@@ -378,14 +429,15 @@ int qwen3_qk_norm_rope(const qwen3_bf16* x, const float* w, const int32_t* pos, 
 namespace {
 
 // Prefill of T new tokens per batch row after `start` cached ones (start > 0 needs the caches).
-// With `pg`, the cache is paged: the new keys and values go into the pages, and the row's
-// first start + T keys are gathered from the pages into the workspace for the attention.
+// With `pg`, the cache is paged: the new keys and values go into the pages, and the attention
+// kernel reads the row's start + T keys and values there, page by page.
 // The attention kernel, persistent (one CTA per SM, fewer for fewer items), as a
 // programmatic dependent launch: its CTAs may be scheduled while the kernel before it
 // finishes; they set up (barriers, TMEM, tensor maps, the logit bound) and wait
 // (griddepcontrol.wait) before their first load of Q', K' or the cache.
 int launch_fmha(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-                const q3::PrefillParams& p, int max_items, bool window, bool varlen, cudaStream_t s) {
+                const q3::PrefillParams& p, int max_items, bool window, bool varlen, cudaStream_t s,
+                bool split = false) {
   const int grid = max_items < num_sms() ? max_items : num_sms();
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
@@ -398,7 +450,9 @@ int launch_fmha(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap&
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   cudaError_t le;
-  if (varlen)
+  if (split)
+    le = cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false, false, true>, mq, mk, mv, mo, p);
+  else if (varlen)
     le = window ? cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<true, true>, mq, mk, mv, mo, p)
                 : cudaLaunchKernelEx(&cfg, q3::fmha_prefill_kernel<false, true>, mq, mk, mv, mo, p);
   else
@@ -435,12 +489,16 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     return QWEN3_ERR_INVALID_ARG;
   if (use_cache && (!aligned(k_cache, 16) || !aligned(v_cache, 16))) return QWEN3_ERR_INVALID_ARG;
   if (!(eps >= 0.f)) return QWEN3_ERR_INVALID_ARG;
-  const size_t need = pg != nullptr ? qwen3_attn_prefill_paged_workspace_size(B, start, T, Hq, Hkv, d)
-                                    : qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d);
-  if (workspace == nullptr || need == 0 || ws_bytes < need) return QWEN3_ERR_WORKSPACE;
+  // A key-axis split when the work items are few; its partials follow the other regions
+  // of the workspace, and a workspace without room for them runs the call unsplit.
+  int n_split = split_count(B, start, T, Hq, Hkv, var.window);
+  const bool in_place = pg != nullptr && pg->page >= kInPlaceMinPage;
+  const size_t base = pg == nullptr ? qwen3_attn_prefill_workspace_size(B, T, Hq, Hkv, d)
+                      : in_place    ? kspace_bytes(B, T, Hq, d) + 256  // Q' only: K, V are read in place
+                                    : 2 * kspace_bytes(B, start + T, Hkv, d) + kspace_bytes(B, T, Hq, d) + 256;
+  if (workspace == nullptr || base == 0 || ws_bytes < base) return QWEN3_ERR_WORKSPACE;
+  if (ws_bytes < base + split_bytes(B, T, Hq, n_split)) n_split = 1;
   if (static_cast<long long>(T) * Hq > (1LL << 31) / kD || static_cast<long long>(B) * Hkv > 65535LL * 1024)
-    return QWEN3_ERR_UNSUPPORTED;
-  if (pg != nullptr && static_cast<long long>(B) * Hkv * (static_cast<long long>(start) + T) > (1LL << 31) / kD)
     return QWEN3_ERR_UNSUPPORTED;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = ensure_kernel_attrs()) != QWEN3_OK) return st;
@@ -465,33 +523,37 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     if (st != QWEN3_OK) return st;
   } else {
     // Paged: K' and V of the new tokens into their pages (keys start..start+T-1), Q' into the
-    // workspace; then the row's first start + T keys and values out of the pages into the
+    // workspace.  The attention kernel then reads the row's start + T keys and values in
+    // place, page by page; pages under kInPlaceMinPage keys are first gathered into the
     // workspace, [B, Hkv, start + T, d] each, where the attention reads them.
     const int n = start + T;
-    qdst = reinterpret_cast<qwen3_bf16*>(w0 + 2 * kspace_bytes(B, n, Hkv, d));
+    qdst = reinterpret_cast<qwen3_bf16*>(in_place ? w0 : w0 + 2 * kspace_bytes(B, n, Hkv, d));
     pq.dstq = qdst;
     st = launch_prologue(k, k_norm_w, pos, pg->k, v, pg->v, B, T, Hkv, 1, 0, var, eps, s, pq, pg, start);
     if (st != QWEN3_OK) return st;
-    kdst = reinterpret_cast<qwen3_bf16*>(w0);
-    vsrc = reinterpret_cast<qwen3_bf16*>(w0 + kspace_bytes(B, n, Hkv, d));
-    Tc = n;
-    q3::GatherParams gp;
-    gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
-    gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
-    gp.block_table = pg->table;
-    gp.k_out = reinterpret_cast<uint4*>(kdst);
-    gp.v_out = reinterpret_cast<uint4*>(vsrc);
-    gp.B = B;
-    gp.Hkv = Hkv;
-    gp.n = n;
-    gp.max_blocks = pg->max_blocks;
-    gp.log2_page = pg->log2_page;
-    gp.num_pages = pg->num_pages;
-    const long long chunks = static_cast<long long>(B) * n * Hkv * 16;
-    long long blocks = (chunks + 255) / 256;
-    if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
-    q3::paged_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
-    if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+    if (!in_place) {
+      if (static_cast<long long>(B) * Hkv * n > (1LL << 31) / kD) return QWEN3_ERR_UNSUPPORTED;
+      kdst = reinterpret_cast<qwen3_bf16*>(w0);
+      vsrc = reinterpret_cast<qwen3_bf16*>(w0 + kspace_bytes(B, n, Hkv, d));
+      Tc = n;
+      q3::GatherParams gp;
+      gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
+      gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
+      gp.block_table = pg->table;
+      gp.k_out = reinterpret_cast<uint4*>(kdst);
+      gp.v_out = reinterpret_cast<uint4*>(vsrc);
+      gp.B = B;
+      gp.Hkv = Hkv;
+      gp.n = n;
+      gp.max_blocks = pg->max_blocks;
+      gp.log2_page = pg->log2_page;
+      gp.num_pages = pg->num_pages;
+      const long long chunks = static_cast<long long>(B) * n * Hkv * 16;
+      long long blocks = (chunks + 255) / 256;
+      if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
+      q3::paged_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
+      if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+    }
   }
 
   // 2. Tensor maps.  The key-axis extent is start + T (not Tcap) so slots past the new tokens
@@ -516,7 +578,15 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     const cuuint64_t qstr[3] = {kD * 2ull, TG * kD * 2ull, static_cast<cuuint64_t>(Hkv) * TG * kD * 2ull};
     if (!make_map(&mq, qdst, 4, qdims, qstr, box)) return QWEN3_ERR_CUDA;
   }
-  {
+  if (in_place) {
+    // the page pools as rows of d, boxes of one page (or 128 rows of a larger page)
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD),
+                                static_cast<cuuint64_t>(pg->num_pages) * Hkv * pg->page};
+    const cuuint64_t str[1] = {kD * 2ull};
+    const cuuint32_t pbox[2] = {64, static_cast<cuuint32_t>(std::min(pg->page, 128))};
+    if (!make_map(&mk, pg->k, 2, dims, str, pbox) || !make_map(&mv, pg->v, 2, dims, str, pbox))
+      return QWEN3_ERR_CUDA;
+  } else {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), static_cast<cuuint64_t>(start) + T,
                                 static_cast<cuuint64_t>(Hkv), static_cast<cuuint64_t>(B)};
     const cuuint64_t str[3] = {kD * 2ull, static_cast<cuuint64_t>(Tc) * kD * 2ull,
@@ -558,7 +628,37 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     p.fault = g_fault;
     p.force_rmax = g_softmax_path == QWEN3_SOFTMAX_RUNNING_MAX ? 1 : 0;
   }
-  return launch_fmha(mq, mk, mv, mo, p, static_cast<int>(n_items), var.window > 0, false, s);
+  if (in_place) {
+    p.block_table = pg->table;
+    p.max_blocks = pg->max_blocks;
+    p.log2_page = pg->log2_page;
+    p.num_pages = pg->num_pages;
+  }
+  p.n_split = n_split;
+  if (n_split <= 1) return launch_fmha(mq, mk, mv, mo, p, static_cast<int>(n_items), var.window > 0, false, s);
+
+  // 4. Key-axis split: every item leaves partials, which one more kernel merges.
+  const uintptr_t pbase = (w0 + base - 256 + 255) & ~static_cast<uintptr_t>(255);
+  const size_t rows = static_cast<size_t>(B) * T * Hq * n_split;
+  p.part_o = reinterpret_cast<float*>(pbase);
+  p.part_lse = reinterpret_cast<float*>(pbase + ((rows * kD * 4 + 255) & ~static_cast<size_t>(255)));
+  const long long split_items = n_items * n_split;
+  if (split_items > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  p.n_items = static_cast<int>(split_items);
+  if ((st = launch_fmha(mq, mk, mv, mo, p, static_cast<int>(split_items), false, false, s, true)) != QWEN3_OK)
+    return st;
+  q3::SplitCombineParams c;
+  c.part_o = p.part_o;
+  c.part_lse = p.part_lse;
+  c.out = reinterpret_cast<uint2*>(out);
+  c.lse = lse;
+  c.B = B;
+  c.T = T;
+  c.Hq = Hq;
+  c.n_split = n_split;
+  const long long nrow = static_cast<long long>(B) * T * Hq;
+  q3::prefill_split_combine_kernel<<<static_cast<unsigned>((nrow + 7) / 8), 256, 0, s>>>(c);
+  return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
 }  // namespace
@@ -969,8 +1069,9 @@ namespace {
 
 // Workspace regions of a varlen prefill, each 256-byte aligned: the checked metadata
 // (seq [B], the entry list, the item count, rank scratch), Q' [Hkv, N*G, d], and K' and V
-// [Hkv, rows, d] with rows = N (fresh prompts: the tokens' own keys) or key_cap (a cache:
-// every sequence's cached and new keys, gathered out of the pages).
+// [Hkv, rows, d] with rows = N (fresh prompts: the tokens' own keys) or key_cap (a cache
+// in pages under kInPlaceMinPage keys: every sequence's cached and new keys, gathered out of
+// the pages; larger pages are read in place and leave these rows unused).
 struct VarlenLayout {
   size_t seq = 0, ent = 0, n_items = 0, np = 0, sbase = 0, qp = 0, kp = 0, vp = 0, total = 0;
   int two_p = 0, n_lvl = 0, max_entries = 0;
@@ -989,7 +1090,7 @@ bool varlen_layout(int B, int N, long long key_cap, int Hq, int Hkv, VarlenLayou
   const long long max_entries = static_cast<long long>(L.n_lvl) + B;
   if (max_entries * Hkv > 0x7fffffffLL) return false;
   L.max_entries = static_cast<int>(max_entries);
-  L.rows = key_cap > 0 ? key_cap : N;
+  L.rows = key_cap > 0 ? key_cap : N;  // pages of kInPlaceMinPage keys or more leave these rows unused
   size_t o = 0;
   L.seq = o;
   o = align256(o + static_cast<size_t>(B) * 16);
@@ -1083,25 +1184,28 @@ int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, c
     vl.seq = seq;
     st = launch_prologue(k, k_norm_w, pos, pg->k, v, pg->v, 1, N, Hkv, 1, 0, var, eps, s, pq, pg, 0, vl);
     if (st != QWEN3_OK) return st;
-    // 3. Every sequence's keys and values, cached and new, out of the pages.
-    q3::VarlenGatherParams gp{};
-    gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
-    gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
-    gp.block_table = pg->table;
-    gp.seq = seq;
-    gp.k_out = reinterpret_cast<uint4*>(kp);
-    gp.v_out = reinterpret_cast<uint4*>(vp);
-    gp.key_cap = key_cap;
-    gp.B = B;
-    gp.Hkv = Hkv;
-    gp.max_blocks = pg->max_blocks;
-    gp.log2_page = pg->log2_page;
-    gp.num_pages = pg->num_pages;
-    const long long chunks = key_cap * Hkv * 16;
-    long long blocks = (chunks + 255) / 256;
-    if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
-    q3::varlen_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
-    if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+    // 3. The attention kernel reads every sequence's cached and new keys in place, page by
+    //    page; pages under kInPlaceMinPage keys are first gathered into the workspace.
+    if (pg->page < kInPlaceMinPage) {
+      q3::VarlenGatherParams gp{};
+      gp.k_pages = reinterpret_cast<const uint4*>(pg->k);
+      gp.v_pages = reinterpret_cast<const uint4*>(pg->v);
+      gp.block_table = pg->table;
+      gp.seq = seq;
+      gp.k_out = reinterpret_cast<uint4*>(kp);
+      gp.v_out = reinterpret_cast<uint4*>(vp);
+      gp.key_cap = key_cap;
+      gp.B = B;
+      gp.Hkv = Hkv;
+      gp.max_blocks = pg->max_blocks;
+      gp.log2_page = pg->log2_page;
+      gp.num_pages = pg->num_pages;
+      const long long chunks = key_cap * Hkv * 16;
+      long long blocks = (chunks + 255) / 256;
+      if (blocks > static_cast<long long>(num_sms()) * 32) blocks = static_cast<long long>(num_sms()) * 32;
+      q3::varlen_gather_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(gp);
+      if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
+    }
   }
 
   // 4. Tensor maps over the packed layouts (batch coordinate 0).
@@ -1122,7 +1226,15 @@ int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, c
     const cuuint64_t qstr[3] = {kD * 2ull, NG * kD * 2ull, static_cast<cuuint64_t>(Hkv) * NG * kD * 2ull};
     if (!make_map(&mq, qp, 4, qdims, qstr, box)) return QWEN3_ERR_CUDA;
   }
-  {
+  const bool in_place = pg != nullptr && pg->page >= kInPlaceMinPage;
+  if (in_place) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD),
+                                static_cast<cuuint64_t>(pg->num_pages) * Hkv * pg->page};
+    const cuuint64_t str[1] = {kD * 2ull};
+    const cuuint32_t pbox[2] = {64, static_cast<cuuint32_t>(std::min(pg->page, 128))};
+    if (!make_map(&mk, pg->k, 2, dims, str, pbox) || !make_map(&mv, pg->v, 2, dims, str, pbox))
+      return QWEN3_ERR_CUDA;
+  } else {
     const cuuint64_t R = static_cast<cuuint64_t>(L.rows);
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kD), R, static_cast<cuuint64_t>(Hkv), 1};
     const cuuint64_t str[3] = {kD * 2ull, R * kD * 2ull, static_cast<cuuint64_t>(Hkv) * R * kD * 2ull};
@@ -1155,6 +1267,12 @@ int varlen_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, c
   p.vl_ent = ent;
   p.vl_n_items = n_items;
   p.out = reinterpret_cast<uint4*>(out);
+  if (in_place) {
+    p.block_table = pg->table;
+    p.max_blocks = pg->max_blocks;
+    p.log2_page = pg->log2_page;
+    p.num_pages = pg->num_pages;
+  }
   return launch_fmha(mq, mk, mv, mo, p, p.n_items, var.window > 0, true, s);
 }
 

@@ -12,11 +12,13 @@
 //
 // varlen_setup_kernel, one CTA:
 //   1. validates each sequence (0 <= cu[b] <= cu[b+1] <= N, ctx >= 0, keys within what the
-//      block table addresses, gathered keys within the workspace); an invalid sequence is
-//      recorded in the status word and treated as empty;
+//      block table addresses, the running sum of keys within key_cap); an invalid sequence
+//      is recorded in the status word and treated as empty;
 //   2. seq[b] = {qoff, T, start, koff}: first token, new tokens, cached keys, and the first
-//      row of the sequence's keys in the gathered key layout (a running sum of ctx + T;
-//      without a cache the keys are the tokens themselves, koff = qoff);
+//      row of the sequence's keys on the key axis the attention reads (without a cache the
+//      keys are the tokens themselves, koff = qoff; with a paged cache the keys are read in
+//      the sequence's own pages and koff is the running sum of ctx + T, kept for the key_cap
+//      check);
 //   3. the entry list: sequence b has np_b = ceil(T_b / 2P) pairs of query tiles (P token
 //      positions per 128-row tile), and its pair p reads about c_b + (p + 1) 2P keys (its
 //      cached ones and the new ones up to the pair's diagonal).  Entries go by that count,
@@ -49,7 +51,7 @@ struct VarlenParams {
   int* n_items;     // [1] out
   int* np;          // scratch [B]: pairs of each sequence
   int* sbase;       // scratch [B]: its first entry in sequence order
-  long long key_cap;  // key rows of the gathered layout (cache), 0 without a cache
+  long long key_cap;  // with a cache: the bound on the sum of every sequence's keys; 0 without
   int B, N, two_p, Hkv, max_entries;
   int max_keys;       // keys one sequence may address (cache: max_blocks * page_size)
 };
@@ -102,7 +104,7 @@ __global__ void __launch_bounds__(kVarlenThreads, 1) varlen_setup_kernel(const _
     if (p.key_cap > 0) {
       kb = koff;
       koff += keys;
-      if (ok && kb + keys > p.key_cap) ok = false;  // more keys than the workspace holds
+      if (ok && kb + keys > p.key_cap) ok = false;  // more keys than the caller's bound
     }
     if (!ok) {  // treated as empty; koff keeps its running value, so koff stays nondecreasing
       record_error(QWEN3_ERR_INVALID_ARG, kSiteVarlenMeta);

@@ -113,6 +113,9 @@ DECODE_SHAPES = {
 CHUNK_SHAPES = {
     "qwen3-4b-second-chunk": ChunkShape("Qwen3-4B-shaped chunked prefill B=1 start=4096 T=4096 Hq=32 Hkv=8",
                                         1, 4096, 4096, 32, 8),
+    # a few new tokens over a long cached prefix (the prefix fills the 32768-token context)
+    "qwen3-4b-short-chunk": ChunkShape("Qwen3-4B-shaped short chunk B=1 start=32752 T=16 Hq=32 Hkv=8",
+                                       1, 32752, 16, 32, 8),
 }
 
 

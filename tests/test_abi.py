@@ -154,6 +154,7 @@ def test_paged_argument_checks():
                 qa.PagedKV((1 << 20) + 2, 1 << 20, 1 << 20, 100, 64, 40)):  # misaligned pool
         assert dec(ctypes.byref(bad)) == qa.ERR_INVALID_ARG
         assert pre(ctypes.byref(bad)) == qa.ERR_INVALID_ARG
+    # room to gather the start + T keys and values (pages under 64 keys), and Q'
     assert qa.prefill_paged_workspace_size(2, 100, 300, 16, 8) >= 2 * 2 * 8 * 400 * 256 + 2 * 300 * 16 * 256
     assert qa.prefill_paged_workspace_size(2, -1, 300, 16, 8) == 0
 
@@ -179,7 +180,8 @@ def test_varlen_argument_checks():
     assert pre(cu=ctypes.c_void_p((1 << 20) + 2)) == qa.ERR_INVALID_ARG  # misaligned offsets
     assert pre(B=0) == qa.ERR_INVALID_ARG and pre(N=0) == qa.ERR_INVALID_ARG
     assert pre(Hq=12) == qa.ERR_UNSUPPORTED and pre(d=64) == qa.ERR_UNSUPPORTED
-    # metadata, entry list and level scratch, Q' [N, Hq, d], K' and V [N, Hkv, d] (or key_cap rows)
+    # metadata, entry list and level scratch, Q' [N, Hq, d], K' and V [N, Hkv, d] (or key_cap
+    # rows, for gathering pages under 64 keys)
     n = qa.prefill_varlen_workspace_size(4, 1000, 16, 8)
     assert n >= 1000 * (16 + 2 * 8) * 128 * 2 + 4 * 16
     m = qa.prefill_varlen_workspace_size(4, 1000, 16, 8, key_cap=5000)
@@ -368,3 +370,24 @@ def test_noalloc_region_limit():
     r = qa.lib().qwen3_attn_decode_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 93, 32, 8,
                                            128, 32769, 1e6, 1e-6, None)
     assert r == qa.ERR_WORKSPACE
+
+
+def test_chunk_workspace_sizes_hold_the_key_split_partials():
+    """The key-axis split's partials are sized on the host from the shapes alone: none for a
+    chunk with many work items, fp32 O/l and an LSE per (new row, query head, run of keys)
+    for a short chunk over a long prefix (the runs: about 128 items in all, each at least 4
+    key tiles, at most 32)."""
+    base = qa.prefill_workspace_size(1, 16, 32, 8)
+    # 16 new tokens, G = 4: one pair item per KV head, 8 items; 235 key tiles -> 16 runs
+    rows = 1 * 16 * 32 * 16
+    want = base + ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    assert qa.prefill_chunk_workspace_size(1, 30000, 16, 32, 8) == want
+    # many items (the 4B-shaped second chunk): no split, no extra bytes
+    assert qa.prefill_chunk_workspace_size(1, 4096, 4096, 32, 8) == qa.prefill_workspace_size(1, 4096, 32, 8)
+    # a short prefix: fewer than 8 key tiles, no split
+    assert qa.prefill_chunk_workspace_size(1, 500, 16, 32, 8) == qa.prefill_workspace_size(1, 16, 32, 8)
+    # the paged prefill's workspace carries the same partials after its gathered K, V and Q'
+    def al(x):
+        return (x + 255) // 256 * 256
+    paged = 2 * al(30016 * 8 * 256) + al(16 * 32 * 256) + 256
+    assert qa.prefill_paged_workspace_size(1, 30000, 16, 32, 8) == paged + (want - base)

@@ -158,3 +158,66 @@ def test_chunk_large_gains_running_max_path():
     bound = chunk_lse_bound(inp, shape.start, as_f64(kc[:, :, :shape.start]), theta=shape.theta, eps=shape.eps)
     compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "chunk large gains (pure)", lse_tol=1e-3 * g2,
             max_tol=MAX_TOL * g2, mean_tol=MEAN_TOL * g2, lse_pure_bound=bound)
+
+
+SHORT_OVER_LONG = [
+    # (T, start): a few new tokens over a long cached prefix, the case the key-axis split is
+    # for: B * Hkv work items are far below the SM count, each with ~235 key tiles
+    (1, 30000),
+    (16, 30011),
+    (64, 29950),
+]
+
+
+@pytest.mark.parametrize("T,start", SHORT_OVER_LONG)
+def test_short_chunk_over_long_prefix_splits_the_keys(T, start):
+    """The key-axis split (each run of keys leaves O/l and its LSE; one more kernel merges
+    them by logsumexp weight) against the oracle, and against the same call run unsplit
+    (a workspace without room for the partials)."""
+    shape = ChunkShape("short chunk", 1, start, T, 32, 8)
+    assert qa.prefill_chunk_workspace_size(1, start, T, 32, 8) > qa.prefill_workspace_size(1, T, 32, 8)
+    inp = chunk_inputs(shape, seed=T)
+    kc, vc = _caches(inp, shape, start + T + 7)
+    out, lse, kca, vca = _run(inp, shape, kc, vc)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, f"short chunk T{T} over {start}, key split")
+    _check_caches(inp, shape, kc, vc, kca, vca)
+    # unsplit: the plain prefill workspace has no room for the partials
+    d = dev()
+    t = {k: inp[k].to(d) for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
+    lse1 = torch.empty_like(lse)
+    ws = torch.empty(qa.prefill_workspace_size(1, T, 32, 8), dtype=torch.uint8, device=d)
+    out1 = qa.prefill_chunk(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], kc.to(d), vc.to(d), start,
+                            lse=lse1, workspace=ws)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    compare(to_np(out1), to_np(lse1), ref, ref_lse, st_lse, f"short chunk T{T} over {start}, unsplit")
+    diff = (out.float() - out1.float()).abs()
+    assert diff.max().item() <= 2e-2 and (lse - lse1).abs().max().item() <= 1e-3
+
+
+def test_short_chunk_key_split_running_max_path():
+    shape = ChunkShape("short chunk", 1, 20000, 48, 16, 4)
+    inp = chunk_inputs(shape, seed=5)
+    kc, vc = _caches(inp, shape, 20100)
+    old = qa.set_softmax_path(qa.SOFTMAX_RUNNING_MAX)
+    try:
+        out, lse, _, _ = _run(inp, shape, kc, vc)
+    finally:
+        qa.set_softmax_path(old)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "short chunk over 20000, key split, running max")
+
+
+@pytest.mark.parametrize("start,T,Hq,Hkv", [(0, 1024, 2, 1), (200, 1000, 4, 2)])
+def test_key_split_with_runs_a_pair_does_not_reach(start, T, Hq, Hkv):
+    """Few work items split into runs of the longest pair's key tiles; the lightest pairs
+    read fewer tiles than there are runs, so some of their runs hold no key at all and leave
+    an empty partial (LSE -inf) that the combine must weigh by zero."""
+    shape = ChunkShape("split, empty runs", 1, start, T, Hq, Hkv)
+    assert qa.prefill_chunk_workspace_size(1, start, T, Hq, Hkv) > qa.prefill_workspace_size(1, T, Hq, Hkv)
+    inp = chunk_inputs(shape, seed=start + 3)
+    kc, vc = _caches(inp, shape, start + T)
+    out, lse, _, _ = _run(inp, shape, kc, vc)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, f"key split, empty runs, start {start} T {T} Hq {Hq}")
