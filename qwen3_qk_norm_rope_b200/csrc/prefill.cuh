@@ -67,6 +67,17 @@ struct PrefillParams {
   int n_split;
   float* part_o;
   float* part_lse;
+  // dual != 0 (only with ring3): an item is two runs of one pair, 2s for tile A and 2s + 1
+  // for tile B, and both tiles are the pair's single query tile (one Q' buffer, read by both
+  // S MMAs), so the CTA's two softmax groups overlap on it.
+  int dual;
+  // ring3 != 0 (the kSplit instance, when every pair has a single query tile: T * G <= 128):
+  // a K/V ring of three stages instead of two, for more bytes in flight per CTA.
+  int ring3;
+  // kv_early != 0: the keys and values before `start` that tmK and tmV cover were written
+  // before the kernel ahead of this one began (a contiguous cache), so the producer may load
+  // them before waiting for that kernel.
+  int kv_early;
   // Keys and values read in place from page pools (block_table != nullptr): tmK and tmV are
   // 2-D maps over the pools as rows of d, [num_pages * Hkv * page, d], with boxes of
   // min(page, 128) rows, and key j of batch row (or sequence) r lies in page
@@ -84,13 +95,35 @@ constexpr uint32_t kPfBar = 6 * kPfTile;
 // Output staging, one 128-row x 64-dim box (16 KB, 128B-swizzled) per softmax group: the
 // epilogue writes half of O/l there and one thread stores it to `out` with a tiled bulk copy.
 constexpr uint32_t kPfStage = kPfBar + 1024;
-// barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage
-constexpr uint32_t kBKFull = 0, kBKEmpty = 16, kBVFull = 32, kBVEmpty = 48, kBSFull = 64, kBPReady = 80,
-                   kBOFull = 96, kBQFull = 112, kBDone = 128, kBTmemSlot = 136, kBAbort = 140,
-                   kBRed = 144,     // 2 groups x 4 warps x (max|g_q|, max|g_k|): 64 bytes
-                   kBQEmpty = 208,  // [X]: the last S_X MMA of an item has read Q'_X
-                   kBTail = 224;    // a paged V tile past the keys' end has landed (zeroed after)
+// barrier block (byte offsets from kPfBar); [X] = tile A (0) or B (1), [s] = ring stage (up to 3)
+constexpr uint32_t kBKFull = 0, kBKEmpty = 24, kBVFull = 48, kBVEmpty = 72, kBSFull = 96, kBPReady = 112,
+                   kBOFull = 128, kBQFull = 144, kBQEmpty = 160,  // [X]: an item's last S_X MMA has read Q'_X
+                   kBDone = 176,
+                   kBTail = 184,  // a paged V tile past the keys' end has landed (zeroed after)
+                   kBTmemSlot = 192, kBAbort = 196,
+                   kBRed = 200;  // 2 groups x 4 warps x (max|g_q|, max|g_k|): 64 bytes
 constexpr uint32_t kPrefillSmemBytes = kPfStage + 2 * kPfBox + 1024;  // + slack to align the base to 1024
+
+// K/V ring stage s.  Stages 0 and 1 sit in the K and V regions.  A third stage, used when
+// every item has a single query tile (ring3), takes Q'_B's buffer for K and the output
+// staging for V: such items load Q' into buffer A only, and a split's epilogue writes its
+// partials straight from tensor memory.
+__device__ __forceinline__ uint32_t k_stage(uint32_t sb, int s) {
+  return s < 2 ? sb + kPfK + s * kPfTile : sb + kPfQ + kPfTile;
+}
+__device__ __forceinline__ uint32_t v_stage(uint32_t sb, int s) {
+  return s < 2 ? sb + kPfV + s * kPfTile : sb + kPfStage;
+}
+// Stage and phase bit of the t-th K/V load in a ring of R (2 or 3) stages.
+__device__ __forceinline__ void ring_pos(uint32_t t, int R, int& s, uint32_t& ph) {
+  if (R == 2) {
+    s = static_cast<int>(t & 1);
+    ph = (t >> 1) & 1;
+  } else {
+    s = static_cast<int>(t % 3u);
+    ph = (t / 3u) & 1;
+  }
+}
 constexpr int kPrefillThreads = 320;
 constexpr uint32_t kTmPOff = 0;  // P within S: chunk c of P lands on S columns already read
 constexpr float kLn2 = 0.693147180559945309f;
@@ -141,24 +174,45 @@ __device__ __forceinline__ TileInfo tile_info(const PrefillParams& p, const Item
   return ti;
 }
 
-// The key tiles an item reads: from tile lo on, nX[X] of them for its query tile X (0 when
-// the item has no tile X).  A split item takes its own run of the pair's tiles: split s of n
-// covers tiles [s*N/n, (s+1)*N/n) of the N the pair reads, and tile X reads the part of that
-// run below its own count.
+// The key tiles an item reads: from tile lo[X] on, nX[X] of them for its query tile X (0
+// when the item has no tile X).  A split item takes its own run of the pair's tiles: split
+// s of n covers tiles [s*N/n, (s+1)*N/n) of the N the pair reads, and tile X reads the part
+// of that run below its own tile count.  A dual item (one query tile per pair) takes run s
+// of n/2 and gives its first half to tile A and the rest to tile B, which holds the same
+// query rows.
 template <bool kWin, bool kSplit>
-__device__ __forceinline__ void item_tiles(const PrefillParams& p, const ItemSeq& sq, int pair, int split, int& lo,
-                                           int (&nX)[2]) {
-  lo = item_lo<kWin>(p, sq, pair);
-  nX[0] = tile_info(p, sq, 2 * pair, lo).nkv;
-  nX[1] = tile_info(p, sq, 2 * pair + 1, lo).nkv;
+__device__ __forceinline__ void item_tiles(const PrefillParams& p, const ItemSeq& sq, int pair, int split,
+                                           int (&lo)[2], int (&nX)[2]) {
+  const int l0 = item_lo<kWin>(p, sq, pair);
+  nX[0] = tile_info(p, sq, 2 * pair, l0).nkv;
+  nX[1] = tile_info(p, sq, 2 * pair + 1, l0).nkv;
+  lo[0] = lo[1] = l0;
   if constexpr (kSplit) {
-    const int n = max(nX[0], nX[1]);
-    const int j0 = static_cast<int>(static_cast<long long>(split) * n / p.n_split);
-    const int j1 = static_cast<int>(static_cast<long long>(split + 1) * n / p.n_split);
-    nX[0] = max(0, min(nX[0], j1) - j0);
-    nX[1] = max(0, min(nX[1], j1) - j0);
-    lo += j0;
+    if (p.dual) {
+      const int runs = p.n_split / 2, N = nX[0];
+      const int j0 = static_cast<int>(static_cast<long long>(split) * N / runs);
+      const int j1 = static_cast<int>(static_cast<long long>(split + 1) * N / runs);
+      const int m = (j1 - j0 + 1) / 2;
+      lo[0] = l0 + j0;
+      nX[0] = m;
+      lo[1] = l0 + j0 + m;
+      nX[1] = j1 - j0 - m;
+    } else {
+      const int n = max(nX[0], nX[1]);
+      const int j0 = static_cast<int>(static_cast<long long>(split) * n / p.n_split);
+      const int j1 = static_cast<int>(static_cast<long long>(split + 1) * n / p.n_split);
+      nX[0] = max(0, min(nX[0], j1) - j0);
+      nX[1] = max(0, min(nX[1], j1) - j0);
+      lo[0] = lo[1] = l0 + j0;
+    }
   }
+}
+
+// A dual item's K/V loads interleave its tiles: A0, B0, A1, B1, ..., and A's last when it
+// has one more.  The u-th load's query tile X and step j.
+__device__ __forceinline__ void dual_load(int u, int nB, int& X, int& j) {
+  X = u < 2 * nB ? (u & 1) : 0;
+  j = u < 2 * nB ? (u >> 1) : u - nB;
 }
 
 // Item this CTA takes in round k: snake order (left to right in even rounds, right to left
@@ -192,9 +246,10 @@ __device__ __forceinline__ void item_fetch(const PrefillParams& p, int item, int
                                            ItemSeq& sq, int& split, int* seq_index = nullptr) {
   split = 0;
   if constexpr (kSplit) {
-    // the n_split items of one pair are adjacent: the heaviest-first order of pairs stays
-    split = item % p.n_split;
-    item_coords(p, item / p.n_split, pair, b, hkv);
+    // the items of one pair are adjacent: the heaviest-first order of pairs stays
+    const int per = p.dual ? p.n_split / 2 : p.n_split;
+    split = item % per;
+    item_coords(p, item / per, pair, b, hkv);
     sq = ItemSeq{0, p.T, p.start, 0};
     return;
   }
@@ -271,17 +326,21 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
   uint8_t* sgen = smem_raw + (sb - raw);
-  const uint32_t sK = sb + kPfK, sV = sb + kPfV, bar = sb + kPfBar;
+  const uint32_t bar = sb + kPfBar;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sgen + kPfBar + kBAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + kPfBar + kBTmemSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // A split's combine kernel, launched next, may be scheduled now: it waits for this grid.
+  if constexpr (kSplit) griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(bar + kBKFull + 8 * s, 1);
       mbar_init(bar + kBKEmpty + 8 * s, 1);
       mbar_init(bar + kBVFull + 8 * s, 1);
       mbar_init(bar + kBVEmpty + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar + kBSFull + 8 * s, 1);
       mbar_init(bar + kBPReady + 8 * s, 128);
       mbar_init(bar + kBOFull + 8 * s, 1);
@@ -309,26 +368,67 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       tma_prefetch_map(&tmQ);
       tma_prefetch_map(&tmK);
       tma_prefetch_map(&tmV);
+      int k_last[3] = {-1, -1, -1}, v_last[3] = {-1, -1, -1}, q_last[2] = {-1, -1};
+      const int R = kSplit && p.ring3 != 0 ? 3 : 2;  // K/V ring stages
+      const int n_items = item_count<kVar>(p);
+      // The first item's first K/V tiles of a contiguous cache that lie wholly before the new
+      // keys were written by earlier calls, not by the prologue: they are loaded into the
+      // empty ring before waiting for the prologue, so their latency overlaps it.
+      int pre = 0;
+      if constexpr (!kVar) {
+        const int item0 = round_item(0);
+        if (p.kv_early != 0 && p.block_table == nullptr && item0 < n_items) {
+          int pair, b, hkv, split, lo[2], nX[2];
+          ItemSeq sq;
+          item_fetch<false, kSplit>(p, item0, pair, b, hkv, sq, split);
+          item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+          const bool dual = kSplit && p.dual != 0;
+          const int n = dual ? nX[0] + nX[1] : max(nX[0], nX[1]);
+          for (; pre < min(n, R); ++pre) {
+            int X = 0, j = pre;
+            if (dual) dual_load(pre, nX[1], X, j);
+            const int key0 = ((X != 0 ? lo[1] : lo[0]) + j) * 128;
+            if (key0 + 128 > sq.start) break;  // keys from here on may come from the prologue
+            const uint32_t sKs = k_stage(sb, pre), sVs = v_stage(sb, pre);
+            if (!(p.fault != 0 && pre == 0)) {
+              mbar_arrive_expect_tx(bar + kBKFull + 8 * pre, kPfTile);
+              tma_load_4d(sKs, &tmK, bar + kBKFull + 8 * pre, 0, sq.koff + key0, hkv, b);
+              tma_load_4d(sKs + kPfBox, &tmK, bar + kBKFull + 8 * pre, 64, sq.koff + key0, hkv, b);
+              k_last[pre] = pre;
+            }
+            mbar_arrive_expect_tx(bar + kBVFull + 8 * pre, kPfTile);
+            tma_load_4d(sVs, &tmV, bar + kBVFull + 8 * pre, 0, sq.koff + key0, hkv, b);
+            tma_load_4d(sVs + kPfBox, &tmV, bar + kBVFull + 8 * pre, 64, sq.koff + key0, hkv, b);
+            v_last[pre] = pre;
+          }
+        }
+      }
       griddep_wait();  // Q', K' (and a cache's V) come from the prologue kernel before this one
-      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1}, q_last[2] = {-1, -1};
       uint32_t it = 0, q_use[2] = {0, 0}, tail_use = 0;
       bool ok = true;
-      const int n_items = item_count<kVar>(p);
       for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-        int pair, b, hkv, split, lo, nX[2], seq = 0;
+        int pair, b, hkv, split, lo[2], nX[2], seq = 0;
         ItemSeq sq;
         item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split, &seq);
         item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+        const bool dual = kSplit && p.dual != 0;
         // a paged cache: the row's block table (a varlen sequence's own row) and key count
         const int* table_row =
             p.block_table != nullptr ? p.block_table + static_cast<long long>(kVar ? seq : b) * p.max_blocks : nullptr;
         const int nk = sq.start + sq.T;
+        // K/V loads: one per step, shared by both tiles, or one per tile of a dual item
+        const int n = dual ? nX[0] + nX[1] : max(nX[0], nX[1]);
+        // first key of the u-th load
+        auto load_key = [&](int u) {
+          int X = 0, j = u;
+          if (dual) dual_load(u, nX[1], X, j);
+          return ((X != 0 ? lo[1] : lo[0]) + j) * 128;
+        };
         // the first tile's block-table entries; each later tile's are fetched one tile ahead
-        const int n = max(nX[0], nX[1]);
         int pg_next[8] = {-1, -1, -1, -1, -1, -1, -1, -1}, nsub_next = 0;
-        if (table_row != nullptr && n > 0) nsub_next = paged_tile_fetch(p, table_row, lo * 128, nk, pg_next);
+        if (table_row != nullptr && n > 0) nsub_next = paged_tile_fetch(p, table_row, load_key(0), nk, pg_next);
         for (int X = 0; X < 2 && ok; ++X) {
-          if (nX[X] == 0) continue;
+          if (nX[X] == 0 || (dual && X == 1)) continue;  // a dual item's tiles share buffer A
           // buffer X is free once the previous item's last S_X MMA has completed
           if (q_use[X] >= 1 &&
               !mbar_wait(bar + kBQEmpty + 8 * X, (q_use[X] - 1) & 1, p.wait, abort_flag, kSitePrefillQEmpty)) {
@@ -343,27 +443,32 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
           q_last[X] = static_cast<int>(q_use[X]++);
         }
         for (int j = 0; j < n && ok; ++j, ++it) {
-          const int st = it & 1;
-          const uint32_t ph = (it >> 1) & 1;
-          if (it >= 2 && !mbar_wait(bar + kBKEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillKEmpty)) {
+          if (k == 0 && j < pre) continue;  // loaded before the prologue's results were awaited
+          int st;
+          uint32_t ph;
+          ring_pos(it, R, st, ph);
+          const uint32_t sKs = k_stage(sb, st), sVs = v_stage(sb, st);
+          if (it >= static_cast<uint32_t>(R) &&
+              !mbar_wait(bar + kBKEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillKEmpty)) {
             ok = false;
             break;
           }
-          const int key0 = (lo + j) * 128;
+          const int key0 = load_key(j);
           if (table_row == nullptr) {
             if (!(p.fault != 0 && it == 0)) {
               mbar_arrive_expect_tx(bar + kBKFull + 8 * st, kPfTile);
-              tma_load_4d(sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, 0, sq.koff + key0, hkv, b);
-              tma_load_4d(sK + st * kPfTile + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, sq.koff + key0, hkv, b);
+              tma_load_4d(sKs, &tmK, bar + kBKFull + 8 * st, 0, sq.koff + key0, hkv, b);
+              tma_load_4d(sKs + kPfBox, &tmK, bar + kBKFull + 8 * st, 64, sq.koff + key0, hkv, b);
               k_last[st] = static_cast<int>(it);
             }
-            if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
+            if (it >= static_cast<uint32_t>(R) &&
+                !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
               ok = false;
               break;
             }
             mbar_arrive_expect_tx(bar + kBVFull + 8 * st, kPfTile);
-            tma_load_4d(sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, 0, sq.koff + key0, hkv, b);
-            tma_load_4d(sV + st * kPfTile + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, sq.koff + key0, hkv, b);
+            tma_load_4d(sVs, &tmV, bar + kBVFull + 8 * st, 0, sq.koff + key0, hkv, b);
+            tma_load_4d(sVs + kPfBox, &tmV, bar + kBVFull + 8 * st, 64, sq.koff + key0, hkv, b);
             v_last[st] = static_cast<int>(it);
           } else {
             // In place from the pages: one box per page (or per 128 rows of a larger page),
@@ -373,25 +478,26 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const int nsub = nsub_next;
 #pragma unroll
             for (int i = 0; i < 8; ++i) pg[i] = pg_next[i];
-            if (j + 1 < n) nsub_next = paged_tile_fetch(p, table_row, key0 + 128, nk, pg_next);
+            if (j + 1 < n) nsub_next = paged_tile_fetch(p, table_row, load_key(j + 1), nk, pg_next);
             if (!(p.fault != 0 && it == 0)) {
-              paged_tile_issue(p, sK + st * kPfTile, &tmK, bar + kBKFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
+              paged_tile_issue(p, sKs, &tmK, bar + kBKFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
                                pg[2], pg[3], pg[4], pg[5], pg[6], pg[7]);
               k_last[st] = static_cast<int>(it);
             }
-            if (it >= 2 && !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
+            if (it >= static_cast<uint32_t>(R) &&
+                !mbar_wait(bar + kBVEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSitePrefillVEmpty)) {
               ok = false;
               break;
             }
             if (key0 + 128 <= nk) {
-              paged_tile_issue(p, sV + st * kPfTile, &tmV, bar + kBVFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
+              paged_tile_issue(p, sVs, &tmV, bar + kBVFull + 8 * st, nsub, key0, hkv, pg[0], pg[1],
                                pg[2], pg[3], pg[4], pg[5], pg[6], pg[7]);
             } else {
               // The tile runs past the keys' end: its rows from there on hold whatever the page
               // (or an earlier use of this buffer) left, NaN included, and P = 0 there would
               // still carry NaN into P.V.  Load on the private barrier, zero those rows, then
               // release the tile to the MMA issuer.
-              paged_tile_issue(p, sV + st * kPfTile, &tmV, bar + kBTail, nsub, key0, hkv, pg[0], pg[1], pg[2],
+              paged_tile_issue(p, sVs, &tmV, bar + kBTail, nsub, key0, hkv, pg[0], pg[1], pg[2],
                                pg[3], pg[4], pg[5], pg[6], pg[7]);
               if (!mbar_wait(bar + kBTail, tail_use & 1, p.wait, abort_flag, kSitePrefillVFull)) {
                 // the copies still land in this CTA's shared memory: wait for them regardless
@@ -404,8 +510,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               for (int r = nk - key0; r < 128; ++r)
 #pragma unroll 1
                 for (int c = 0; c < 8; ++c) {
-                  st_shared_v4(sV + st * kPfTile + r * 128 + c * 16, 0u, 0u, 0u, 0u);
-                  st_shared_v4(sV + st * kPfTile + kPfBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+                  st_shared_v4(sVs + r * 128 + c * 16, 0u, 0u, 0u, 0u);
+                  st_shared_v4(sVs + kPfBox + r * 128 + c * 16, 0u, 0u, 0u, 0u);
                 }
               fence_proxy_async_smem();
               mbar_arrive(bar + kBVFull + 8 * st);
@@ -415,10 +521,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
       }
       // Every issued copy must land before this CTA's shared memory is released.
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < 2; ++s)
         if (q_last[s] >= 0) mbar_wait(bar + kBQFull + 8 * s, q_last[s] & 1, p.wait, nullptr, kSitePrefillDrain);
-        if (k_last[s] >= 0) mbar_wait(bar + kBKFull + 8 * s, (k_last[s] >> 1) & 1, p.wait, nullptr, kSitePrefillDrain);
-        if (v_last[s] >= 0) mbar_wait(bar + kBVFull + 8 * s, (v_last[s] >> 1) & 1, p.wait, nullptr, kSitePrefillDrain);
+      for (int s = 0; s < R; ++s) {
+        int st;
+        uint32_t ph;
+        if (k_last[s] >= 0) {
+          ring_pos(static_cast<uint32_t>(k_last[s]), R, st, ph);
+          mbar_wait(bar + kBKFull + 8 * s, ph, p.wait, nullptr, kSitePrefillDrain);
+        }
+        if (v_last[s] >= 0) {
+          ring_pos(static_cast<uint32_t>(v_last[s]), R, st, ph);
+          mbar_wait(bar + kBVFull + 8 * s, ph, p.wait, nullptr, kSitePrefillDrain);
+        }
       }
     }
   } else if (warp == 1) {
@@ -428,22 +543,72 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
       constexpr uint32_t kIdPV = idesc_bf16(128, 128, true);   // B = V, dims contiguous (MN-major)
       uint32_t it = 0, q_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
       bool ok = true;
+      const int R = kSplit && p.ring3 != 0 ? 3 : 2;  // K/V ring stages
       const int n_items = item_count<kVar>(p);
       for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-        int pair, b, hkv, split, lo, nX[2];
+        int pair, b, hkv, split, lo[2], nX[2];
         ItemSeq sq;
         item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split);
         item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+        const bool dual = kSplit && p.dual != 0;
         const int n = max(nX[0], nX[1]);
         if ((kVar || kSplit) && n == 0) continue;  // an item with no tile (the producer skips it too)
-        for (int X = 0; X < 2 && ok; ++X)
+        for (int X = 0; X < (dual ? 1 : 2) && ok; ++X)
           if (nX[X] > 0) {
             ok = mbar_wait(bar + kBQFull + 8 * X, q_cnt[X] & 1, p.wait, abort_flag, kSitePrefillQFull);
             ++q_cnt[X];
           }
         if (!ok) break;
+        if (dual) {
+          // A dual item: each tile has its own K/V loads, taken in the producer's order, and
+          // both read Q' buffer A.  Step j issues PV_X(j-1) then S_X(j), for X = A, B.
+          const int nB = nX[1];
+          for (int j = 0; j <= n && ok; ++j) {
+            for (int X = 0; X < 2 && ok; ++X) {
+              int st;
+              uint32_t ph;
+              if (j >= 1 && j - 1 < nX[X]) {
+                ring_pos(it + (j - 1 < nB ? 2 * (j - 1) + X : nB + j - 1), R, st, ph);
+                ok = mbar_wait(bar + kBVFull + 8 * st, ph, p.wait, abort_flag, kSitePrefillVFull) &&
+                     mbar_wait(bar + kBPReady + 8 * X, p_cnt[X] & 1, p.wait, abort_flag, kSitePrefillPReady);
+                ++p_cnt[X];
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t sVs = v_stage(sb, st);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                  tc_mma_ts(tmem + tm_o(X), tmem + tm_s(X) + kTmPOff + kk * 8,
+                            smem_desc_sw128(sVs + kk * 2048, kPfBox, 1024), kIdPV, (j > 1 || kk > 0) ? 1u : 0u);
+                if (j == nX[X]) tc_commit(bar + kBOFull + 8 * X);
+                tc_commit(bar + kBVEmpty + 8 * st);
+              }
+              if (j < nX[X]) {
+                ring_pos(it + (j < nB ? 2 * j + X : nB + j), R, st, ph);
+                ok = mbar_wait(bar + kBKFull + 8 * st, ph, p.wait, abort_flag, kSitePrefillKFull);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t sKs = k_stage(sb, st);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
+                  tc_mma_ss(tmem + tm_s(X), smem_desc_sw128(sb + kPfQ + koff, 16, 1024),
+                            smem_desc_sw128(sKs + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+                }
+                tc_commit(bar + kBSFull + 8 * X);
+                // the item's last S MMA (B's, or A's when A has one tile more) frees buffer A
+                if (j == nX[X] - 1 && (X == 1) == (nB == nX[0])) tc_commit(bar + kBQEmpty);
+                tc_commit(bar + kBKEmpty + 8 * st);
+              }
+            }
+          }
+          it += nX[0] + nX[1];
+          continue;
+        }
         // j = 0: S_A(0), S_B(0)
-        ok = mbar_wait(bar + kBKFull + 8 * (it & 1), (it >> 1) & 1, p.wait, abort_flag, kSitePrefillKFull);
+        int sc;
+        uint32_t pc;
+        ring_pos(it, R, sc, pc);
+        ok = mbar_wait(bar + kBKFull + 8 * sc, pc, p.wait, abort_flag, kSitePrefillKFull);
         if (!ok) break;
         tc_fence_after();
         for (int X = 0; X < 2; ++X)
@@ -452,20 +617,22 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
               tc_mma_ss(tmem + tm_s(X), smem_desc_sw128(sb + kPfQ + X * kPfTile + koff, 16, 1024),
-                        smem_desc_sw128(sK + (it & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+                        smem_desc_sw128(k_stage(sb, sc) + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
             }
             tc_commit(bar + kBSFull + 8 * X);
             if (nX[X] == 1) tc_commit(bar + kBQEmpty + 8 * X);  // the item's last S_X
           }
-        tc_commit(bar + kBKEmpty + 8 * (it & 1));
+        tc_commit(bar + kBKEmpty + 8 * sc);
         // j >= 1: PV_X(j-1) then S_X(j), for X = A, B
         for (int j = 1; j <= n && ok; ++j) {
-          const uint32_t prev = it + j - 1, cur = it + j;
+          const int sp = sc;  // stage and phase of tile j-1
+          const uint32_t pv = pc;
           if (j < n) {
-            ok = mbar_wait(bar + kBKFull + 8 * (cur & 1), (cur >> 1) & 1, p.wait, abort_flag, kSitePrefillKFull);
+            ring_pos(it + j, R, sc, pc);
+            ok = mbar_wait(bar + kBKFull + 8 * sc, pc, p.wait, abort_flag, kSitePrefillKFull);
             if (!ok) break;
           }
-          ok = mbar_wait(bar + kBVFull + 8 * (prev & 1), (prev >> 1) & 1, p.wait, abort_flag, kSitePrefillVFull);
+          ok = mbar_wait(bar + kBVFull + 8 * sp, pv, p.wait, abort_flag, kSitePrefillVFull);
           if (!ok) break;
           for (int X = 0; X < 2; ++X) {
             if (j - 1 < nX[X]) {
@@ -476,7 +643,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk)
                 tc_mma_ts(tmem + tm_o(X), tmem + tm_s(X) + kTmPOff + kk * 8,
-                          smem_desc_sw128(sV + (prev & 1) * kPfTile + kk * 2048, kPfBox, 1024), kIdPV,
+                          smem_desc_sw128(v_stage(sb, sp) + kk * 2048, kPfBox, 1024), kIdPV,
                           (j > 1 || kk > 0) ? 1u : 0u);
               if (j == nX[X]) tc_commit(bar + kBOFull + 8 * X);
             }
@@ -485,15 +652,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
               for (int kk = 0; kk < 8; ++kk) {
                 const uint32_t koff = (kk >> 2) * kPfBox + (kk & 3) * 32;
                 tc_mma_ss(tmem + tm_s(X), smem_desc_sw128(sb + kPfQ + X * kPfTile + koff, 16, 1024),
-                          smem_desc_sw128(sK + (cur & 1) * kPfTile + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
+                          smem_desc_sw128(k_stage(sb, sc) + koff, 16, 1024), kIdQK, kk > 0 ? 1u : 0u);
               }
               tc_commit(bar + kBSFull + 8 * X);
               if (j == nX[X] - 1) tc_commit(bar + kBQEmpty + 8 * X);  // the item's last S_X
             }
           }
           if (!ok) break;
-          tc_commit(bar + kBVEmpty + 8 * (prev & 1));
-          if (j < n) tc_commit(bar + kBKEmpty + 8 * (cur & 1));
+          tc_commit(bar + kBVEmpty + 8 * sp);
+          if (j < n) tc_commit(bar + kBKEmpty + 8 * sc);
         }
         it += n;
       }
@@ -544,12 +711,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // waits for a P that is only written after this epilogue.
     const int n_items = item_count<kVar>(p);
     for (int k = 0, item = round_item(0); item < n_items && ok; item = round_item(++k)) {
-      int pair, b, hkv, split, lo, nX[2];
+      int pair, b, hkv, split, lo[2], nX[2];
       ItemSeq sq;
       item_fetch<kVar, kSplit>(p, item, pair, b, hkv, sq, split);
       item_tiles<kWin, kSplit>(p, sq, pair, split, lo, nX);
+      const bool dual = kSplit && p.dual != 0;
+      if (dual) split = 2 * split + X;  // this tile's run: the index of its partials
       TileInfo ti;
-      ti.t0 = (2 * pair + X) * p.P;
+      ti.t0 = (dual ? 2 * pair : 2 * pair + X) * p.P;
       ti.nkv = nX[X];
       if (ti.nkv == 0) {
         // This item has no tile X.  A split's run may hold no key a tile's rows see: its
@@ -563,6 +732,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         continue;
       }
       const int t0 = ti.t0;
+      const int lo_x = (kSplit && X != 0) ? lo[1] : lo[0];  // the tiles differ only in a dual item
 
       const int t_row = t0 + (row >> p.log2G);
       const int lim = sq.start + min(t_row, sq.T - 1);  // last key index this row may see
@@ -574,7 +744,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const int kv0 = (lo + j) * 128;
+        const int kv0 = (lo_x + j) * 128;
         // some key of this tile lies past some row's limit, or before some row's window
         const bool diag = kv0 + 127 > sq.start + t0 || (kWin && kv0 < sq.start + t0 + p.P - p.window);
         if (fast) {
@@ -805,9 +975,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 // Merge of the key-split partials of a prefill: per (row of the token axis, query head),
 // lse = log sum_s exp(lse_s) and out = sum_s exp(lse_s - lse) O_s (the online logsumexp of
 // "Qwen3 Architecture Layer-by-Layer", Liger fused linear cross-entropy, across runs of
-// keys).  One warp per (token, head): lane s holds run s's LSE (n_split <= 32) for the
-// max and the weights, and lane i owns output dims 4i..4i+3; the runs' partial rows are
-// read eight at a time so their loads overlap.
+// keys).  One block of four warps per (token, head): every warp reads the row's LSEs (lane s
+// holds run s, n_split <= 32) for the max and the weights, and warp g merges runs 8g..8g+7,
+// lane i owning output dims 4i..4i+3; the four partial sums meet in shared memory.  All of a
+// lane's loads are independent, so a block waits for about one round trip to L2, where the
+// attention kernel just left the partials.  A programmatic dependent launch: its blocks may
+// be scheduled while that kernel runs and wait (griddep_wait) before their first read.
 struct SplitCombineParams {
   const float* part_o;    // [B*T, Hq, n_split, d]
   const float* part_lse;  // [B*T, Hq, n_split]
@@ -815,31 +988,52 @@ struct SplitCombineParams {
   float* lse;             // [B, Hq, T] or nullptr
   int B, T, Hq, n_split;
 };
+constexpr int kCombineWarps = 4;  // runs per warp: 32 / kCombineWarps
 
-__global__ void __launch_bounds__(256) prefill_split_combine_kernel(const __grid_constant__ SplitCombineParams p) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);  // (b*T + t)*Hq + h
-  if (row >= static_cast<long long>(p.B) * p.T * p.Hq) return;
-  const int lane = threadIdx.x & 31;
-  const float mine = lane < p.n_split ? p.part_lse[row * p.n_split + lane] : -INFINITY;
+__global__ void __launch_bounds__(kCombineWarps * 32) prefill_split_combine_kernel(
+    const __grid_constant__ SplitCombineParams p) {
+  constexpr int kPer = 32 / kCombineWarps;
+  __shared__ float4 part[kCombineWarps][32];
+  griddep_wait();
+  const long long row = blockIdx.x;  // (b*T + t)*Hq + h
+  const int g = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = p.n_split;
+  const float mine = lane < n ? p.part_lse[row * n + lane] : -INFINITY;
+  const float4* po = reinterpret_cast<const float4*>(p.part_o + row * n * kD) + lane;
+  float4 o[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int s = g * kPer + i;
+    o[i] = s < n ? po[s * (kD / 4)] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float M = mine;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  for (int x = 16; x > 0; x >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, x));
   const float kLog2e = 1.44269504088896341f;
-  // a run with no key this row sees has LSE -inf: weight 0, and its O is never read
+  // a run with no key this row sees has LSE -inf: weight 0, and its O is never used
   const float w = (mine == -INFINITY || M == -INFINITY) ? 0.f : ex2((mine - M) * kLog2e);
-  const float z = warp_sum(w);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  const float4* po = reinterpret_cast<const float4*>(p.part_o + row * p.n_split * kD) + lane;
-#pragma unroll 8
-  for (int s = 0; s < p.n_split; ++s) {
-    const float ws = __shfl_sync(0xffffffffu, w, s);
-    const float4 o = po[s * (kD / 4)];  // read even when unused, so the loads overlap
-    if (ws != 0.f) {                     // an unused run's row may hold anything, NaN included
-      acc.x += ws * o.x;
-      acc.y += ws * o.y;
-      acc.z += ws * o.z;
-      acc.w += ws * o.w;
-    }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    // an unused run's row may hold anything, NaN included: selected away, not multiplied by 0
+    const float ws = __shfl_sync(0xffffffffu, w, g * kPer + i);
+    const bool use = ws != 0.f;
+    acc.x += use ? ws * o[i].x : 0.f;
+    acc.y += use ? ws * o[i].y : 0.f;
+    acc.z += use ? ws * o[i].z : 0.f;
+    acc.w += use ? ws * o[i].w : 0.f;
+  }
+  part[g][lane] = acc;
+  __syncthreads();
+  if (g != 0) return;
+  const float z = warp_sum(w);
+#pragma unroll
+  for (int j = 1; j < kCombineWarps; ++j) {
+    const float4 a = part[j][lane];
+    acc.x += a.x;
+    acc.y += a.y;
+    acc.z += a.z;
+    acc.w += a.w;
   }
   const float inv = z > 0.f ? 1.0f / z : 0.f;
   p.out[row * (kD / 4) + lane] = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));

@@ -215,7 +215,13 @@ size_t kspace_bytes(int B, int T, int Hkv, int d) {
 // a long cached prefix): the number of runs its keys are cut into, 1 for no split.  It is
 // fixed by the shapes alone, so the workspace size that holds the partials is known on the
 // host: about kSplitTarget items in all, each run at least 4 key tiles, at most 32 runs.
+// When every (batch row, KV head) has a single query tile (T <= 128 / G, single_qtile), the
+// kernel's K/V ring takes a third stage, and with kDualRuns an item takes two runs, one per
+// softmax group, so the count is even and twice the items'.
 constexpr int kSplitTarget = 128;
+constexpr bool kDualRuns = true;
+bool single_qtile(int T, int Hq, int Hkv) { return static_cast<long long>(T) * (Hq / Hkv) <= 128; }
+bool dual_split(int T, int Hq, int Hkv) { return kDualRuns && single_qtile(T, Hq, Hkv); }
 int split_count(int B, int start, int T, int Hq, int Hkv, int window) {
   if (window > 0 || B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 1;
   const int G = Hq / Hkv;
@@ -224,7 +230,14 @@ int split_count(int B, int start, int T, int Hq, int Hkv, int window) {
   const long long n_pairs = ((T + P - 1) / P + 1) / 2;
   const long long items = static_cast<long long>(B) * Hkv * n_pairs;
   const long long tiles = (static_cast<long long>(start) + T + 127) / 128;
-  if (items * 2 > kSplitTarget || tiles < 8) return 1;
+  if (tiles < 8) return 1;
+  if (dual_split(T, Hq, Hkv)) {
+    if (items > kSplitTarget) return 1;
+    long long n = std::min<long long>(2 * kSplitTarget / items, tiles / 4);
+    n = std::min<long long>(n, 32) & ~1LL;
+    return n >= 2 ? static_cast<int>(n) : 1;
+  }
+  if (items * 2 > kSplitTarget) return 1;
   long long n = std::min<long long>(kSplitTarget / items, tiles / 4);
   n = std::min<long long>(n, 32);
   return n >= 2 ? static_cast<int>(n) : 1;
@@ -634,6 +647,9 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
     p.log2_page = pg->log2_page;
     p.num_pages = pg->num_pages;
   }
+  // A contiguous cache's keys and values before `start` come from earlier calls; a gathered
+  // copy of pages is written by this call's gather kernel.
+  p.kv_early = (pg == nullptr && use_cache) ? 1 : 0;
   p.n_split = n_split;
   if (n_split <= 1) return launch_fmha(mq, mk, mv, mo, p, static_cast<int>(n_items), var.window > 0, false, s);
 
@@ -642,7 +658,9 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   const size_t rows = static_cast<size_t>(B) * T * Hq * n_split;
   p.part_o = reinterpret_cast<float*>(pbase);
   p.part_lse = reinterpret_cast<float*>(pbase + ((rows * kD * 4 + 255) & ~static_cast<size_t>(255)));
-  const long long split_items = n_items * n_split;
+  p.dual = dual_split(T, Hq, Hkv) ? 1 : 0;  // n_split is even then
+  p.ring3 = single_qtile(T, Hq, Hkv) ? 1 : 0;
+  const long long split_items = n_items * (p.dual ? n_split / 2 : n_split);
   if (split_items > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
   p.n_items = static_cast<int>(split_items);
   if ((st = launch_fmha(mq, mk, mv, mo, p, static_cast<int>(split_items), false, false, s, true)) != QWEN3_OK)
@@ -657,7 +675,20 @@ int prefill_impl(const qwen3_bf16* q, const qwen3_bf16* k, const qwen3_bf16* v, 
   c.Hq = Hq;
   c.n_split = n_split;
   const long long nrow = static_cast<long long>(B) * T * Hq;
-  q3::prefill_split_combine_kernel<<<static_cast<unsigned>((nrow + 7) / 8), 256, 0, s>>>(c);
+  cudaLaunchConfig_t cfg = {};
+  if (nrow > 0x7fffffffLL) return QWEN3_ERR_UNSUPPORTED;
+  cfg.gridDim = dim3(static_cast<unsigned>(nrow));  // a block per (token, head)
+  cfg.blockDim = dim3(q3::kCombineWarps * 32);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, q3::prefill_split_combine_kernel, c) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 

@@ -376,12 +376,24 @@ def test_chunk_workspace_sizes_hold_the_key_split_partials():
     """The key-axis split's partials are sized on the host from the shapes alone: none for a
     chunk with many work items, fp32 O/l and an LSE per (new row, query head, run of keys)
     for a short chunk over a long prefix (the runs: about 128 items in all, each at least 4
-    key tiles, at most 32)."""
+    key tiles, at most 32; a chunk with one query tile per KV head takes two runs per item)."""
+    def parts(T, n):
+        rows = 1 * T * 32 * n
+        return ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+
+    # 64 new tokens, G = 4: two query tiles, one pair item per KV head, 8 items; 235 key
+    # tiles -> 16 runs
+    assert qa.prefill_chunk_workspace_size(1, 30000, 64, 32, 8) == qa.prefill_workspace_size(1, 64, 32, 8) + parts(64, 16)
+    # 16 new tokens: a single query tile (64 rows), so two runs per item -> 32 runs
     base = qa.prefill_workspace_size(1, 16, 32, 8)
-    # 16 new tokens, G = 4: one pair item per KV head, 8 items; 235 key tiles -> 16 runs
-    rows = 1 * 16 * 32 * 16
-    want = base + ((rows * 128 * 4 + 255) // 256) * 256 + ((rows * 4 + 255) // 256) * 256
+    want = base + parts(16, 32)
     assert qa.prefill_chunk_workspace_size(1, 30000, 16, 32, 8) == want
+    # a single query tile over 40 key tiles: runs of at least 4 tiles, an even count -> 10
+    assert qa.prefill_chunk_workspace_size(1, 5000, 16, 32, 8) == base + parts(16, 10)
+    # 32 KV heads of one query tile each: 2 * 128 / 32 = 8 runs
+    assert qa.prefill_chunk_workspace_size(1, 30000, 16, 128, 32) == \
+        qa.prefill_workspace_size(1, 16, 128, 32) + ((16 * 128 * 8 * 512 + 255) // 256 * 256) + \
+        ((16 * 128 * 8 * 4 + 255) // 256 * 256)
     # many items (the 4B-shaped second chunk): no split, no extra bytes
     assert qa.prefill_chunk_workspace_size(1, 4096, 4096, 32, 8) == qa.prefill_workspace_size(1, 4096, 32, 8)
     # a short prefix: fewer than 8 key tiles, no split

@@ -196,6 +196,33 @@ def test_short_chunk_over_long_prefix_splits_the_keys(T, start):
     assert diff.max().item() <= 2e-2 and (lse - lse1).abs().max().item() <= 1e-3
 
 
+@pytest.mark.parametrize("B,start,T,Hq,Hkv", [(1, 5200, 16, 32, 8), (2, 8000, 16, 32, 8), (1, 20000, 1, 64, 4),
+                                             (1, 3000, 128, 8, 8), (3, 1500, 5, 16, 2)])
+def test_single_query_tile_chunk_takes_two_runs_per_item(B, start, T, Hq, Hkv):
+    """A chunk whose every KV head has a single query tile (T * G <= 128): each work item
+    takes two runs of keys, one per softmax group over the same query rows.  Against the
+    oracle, and against the same call run unsplit.  5200 + 16 keys make 41 tiles in 5 item
+    runs, the last of 9 tiles, so its halves differ in length."""
+    shape = ChunkShape("single query tile", B, start, T, Hq, Hkv)
+    assert T * (Hq // Hkv) <= 128
+    assert qa.prefill_chunk_workspace_size(B, start, T, Hq, Hkv) > qa.prefill_workspace_size(B, T, Hq, Hkv)
+    inp = chunk_inputs(shape, seed=start + T + B)
+    kc, vc = _caches(inp, shape, start + T + 3)
+    out, lse, _, _ = _run(inp, shape, kc, vc)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, f"one query tile B{B} T{T} over {start}, two runs per item")
+    d = dev()
+    t = {k: inp[k].to(d) for k in ("q", "k", "v", "q_norm_w", "k_norm_w", "pos")}
+    lse1 = torch.empty_like(lse)
+    ws = torch.empty(qa.prefill_workspace_size(B, T, Hq, Hkv), dtype=torch.uint8, device=d)
+    out1 = qa.prefill_chunk(t["q"], t["k"], t["v"], t["q_norm_w"], t["k_norm_w"], t["pos"], kc.to(d), vc.to(d), start,
+                            lse=lse1, workspace=ws)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    diff = (out.float() - out1.float()).abs()
+    assert diff.max().item() <= 2e-2 and (lse - lse1).abs().max().item() <= 1e-3
+
+
 def test_short_chunk_key_split_running_max_path():
     shape = ChunkShape("short chunk", 1, 20000, 48, 16, 4)
     inp = chunk_inputs(shape, seed=5)
@@ -207,6 +234,17 @@ def test_short_chunk_key_split_running_max_path():
         qa.set_softmax_path(old)
     ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
     compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "short chunk over 20000, key split, running max")
+    # a single query tile per KV head: two runs per item on the running-max path
+    shape = ChunkShape("short chunk", 1, 20000, 16, 16, 4)
+    inp = chunk_inputs(shape, seed=6)
+    kc, vc = _caches(inp, shape, 20020)
+    old = qa.set_softmax_path(qa.SOFTMAX_RUNNING_MAX)
+    try:
+        out, lse, _, _ = _run(inp, shape, kc, vc)
+    finally:
+        qa.set_softmax_path(old)
+    ref, ref_lse, _, st_lse = _oracle(inp, shape, kc, vc)
+    compare(to_np(out), to_np(lse), ref, ref_lse, st_lse, "one query tile over 20000, two runs per item, running max")
 
 
 @pytest.mark.parametrize("start,T,Hq,Hkv", [(0, 1024, 2, 1), (200, 1000, 4, 2)])

@@ -126,7 +126,8 @@ def test_decode_paged_equals_contiguous():
     assert torch.equal(out_c, out_p)
 
 
-@pytest.mark.parametrize("start,T,page", [(0, 300, 64), (777, 300, 16), (1000, 129, 256)])
+@pytest.mark.parametrize("start,T,page", [(0, 300, 64), (777, 300, 16), (1000, 129, 256), (5000, 32, 64),
+                                          (3000, 20, 16), (4090, 7, 256)])
 def test_prefill_paged(start, T, page):
     shape = ChunkShape("paged chunk", 2, start, T, 16, 8)
     inp = chunk_inputs(shape, seed=start + T)
