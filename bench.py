@@ -96,8 +96,8 @@ def decode_traffic(lens: np.ndarray):
 # DRAM traffic of the prefill attention kernel per launch on a workload (dram__bytes_read.sum
 # + dram__bytes_write.sum of one ncu capture of that launch), valid only for the kernel
 # source it was measured on.  Refreshed with each new capture.
-PREFILL_TRAFFIC = {"src_sha256": "73072760887affb1bce678e7ada38eab1c6dd95d0eb206c338b5cd4ebce134c2",
-                   "bytes": {"long-context wide-GQA prefill B=1 T=32768 Hq=64 Hkv=4": 1.254633e9 + 0.521545216e9}}
+PREFILL_TRAFFIC = {"src_sha256": "9bb0814517d2b15eb41681e1cdb1a8f53d0d1d314898fccbedcaa03ebe37c3d0",
+                   "bytes": {"long-context wide-GQA prefill B=1 T=32768 Hq=64 Hkv=4": 1.22407e9 + 0.51934e9}}
 
 
 def prefill_src_sha256() -> str:
