@@ -8,7 +8,9 @@
 // start = cache.length, and the tril(diagonal=S-T) mask with T = 1).
 //
 // Split kernel: one CTA per (split of `split` keys, KV head, sequence); CTAs past a
-// sequence's end exit at once, so the host never needs the lengths.  Warp 4 streams 64-key
+// sequence's end exit at once, so the host never needs the lengths.  It is a programmatic
+// dependent launch after the append: only the chunk holding slot L waits for the append's
+// results (griddepcontrol.wait); the rest of the cache was written by earlier calls.  Warp 4 streams 64-key
 // chunks of K and V (two 64x64 128B-swizzled TMA boxes each) into a 3-stage ring.  Warps
 // 0-3 each take 16 keys of every chunk: S = q'K^T and O += P V as mma.sync m16n8k16 (rows =
 // the G <= 16 query heads of the group), an exp2 online softmax in registers, then the four
@@ -136,6 +138,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const uint32_t ph = (u / kDcStages) & 1;
         if (u >= kDcStages && !mbar_wait(bar + kDcBEmpty + 8 * st, ph ^ 1, p.wait, abort_flag, kSiteDecodeEmpty))
           break;
+        // slot L, the new token's key and value, comes from the append kernel before this one
+        if (tok0 + c * 64 + 63 >= L) griddep_wait();
         const uint32_t dst = sb + st * kDcStage;
         const uint32_t fb = bar + kDcBFull + 8 * st;
         if (p.block_table == nullptr) {
@@ -361,6 +365,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
     p.part_o[(hq * p.n_split_max + s_idx) * kD + dcol] = acc / Lsum;
     if (dcol == 0) p.part_lse[hq * p.n_split_max + s_idx] = (M + log2f(Lsum)) * 0.693147180559945309f;
   }
+  // The combine kernel may be scheduled once every CTA has got here or exited: it waits for
+  // this grid's partials (griddepcontrol.wait) before reading them.
+  griddep_launch_dependents();
 }
 
 struct CombineParams {
@@ -373,8 +380,10 @@ struct CombineParams {
   int window;  // as in DecodeParams: splits wholly before the window wrote nothing
 };
 
-// One CTA of 128 threads per (sequence, query head); thread i owns output dim i.
+// One CTA of 128 threads per (sequence, query head); thread i owns output dim i.  A
+// programmatic dependent launch after the split kernel, whose partials it waits for.
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ CombineParams p) {
+  griddep_wait();
   const int hq = blockIdx.x;  // n * Hq + head
   const int n = hq / p.Hq;
   const int L = p.cache_lens[n];
@@ -383,10 +392,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   const int s0 = p.window > 0 ? max(0, L - p.window + 1) / p.split : 0;  // the first one in the window
   const float* lse_s = p.part_lse + static_cast<long long>(hq) * p.n_split_max;
   float M = -INFINITY;
+#pragma unroll 8
   for (int s = s0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
   const float kLog2e = 1.44269504088896341f;
   float z = 0.f, acc = 0.f;
   const float* po = p.part_o + static_cast<long long>(hq) * p.n_split_max * kD + threadIdx.x;
+#pragma unroll 8
   for (int s = s0; s < ns; ++s) {
     const float w = ex2d((lse_s[s] - M) * kLog2e);
     z += w;

@@ -836,7 +836,22 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   p.max_blocks = pg != nullptr ? pg->max_blocks : 0;
   p.log2_page = pg != nullptr ? pg->log2_page : 0;
   p.num_pages = pg != nullptr ? pg->num_pages : 0;
-  q3::decode_split_kernel<<<dim3(ns, Hkv, N), q3::kDecodeThreads, q3::kDecodeSmemBytes, s>>>(mk, mv, p);
+  // Both launches below are programmatic dependent launches (see the kernels): the split
+  // kernel overlaps the append, the combine the split kernel's last CTAs.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ns, Hkv, N);
+  cfg.blockDim = dim3(q3::kDecodeThreads);
+  cfg.dynamicSmemBytes = q3::kDecodeSmemBytes;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, q3::decode_split_kernel, mk, mv, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
   if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
 
   // 3. Logsumexp combine of the splits.
@@ -851,7 +866,13 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   c.split = kDecodeSplit;
   c.n_split_max = ns;
   c.window = var.window;
-  q3::decode_combine_kernel<<<N * Hq, 128, 0, s>>>(c);
+  cfg.gridDim = dim3(N * Hq);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, q3::decode_combine_kernel, c) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
