@@ -74,8 +74,8 @@ def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
 # DRAM traffic of the decode split-KV kernel per cached token (dram__bytes_read.sum +
 # dram__bytes_write.sum of one ncu capture of a smaller case, divided by its cached tokens),
 # valid only for the kernel source it was measured on.  Refreshed with each new capture.
-DECODE_TRAFFIC = {"src_sha256": "65820a30e1e2921678f67e2648cdf0c555a6a54bee07c421d033d25db85efed8",
-                  "bytes_per_cached_token": (630.653696e6 + 6.289664e6) / 153639}
+DECODE_TRAFFIC = {"src_sha256": "e9ed9214854a024560e1affa2f7c6a31576ecbae86d27716a02ecffc6b4527b9",
+                  "bytes_per_cached_token": (630.648576e6 + 5.422592e6) / 153639}
 
 
 def decode_src_sha256() -> str:
