@@ -223,8 +223,7 @@ int qwen3_attn_decode(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_
  *   - The region's device address belongs to one CUDA context.  The first call in a
  *     context (the device's primary context, or another context the caller made current)
  *     looks that address up and keeps it for that context; after a device reset the new
- *     context's first call looks it up again.  Make the first call in a context before any
- *     stream capture in it.
+ *     context's first call looks it up again.
  *   - Argument checks come first: a bad argument returns what qwen3_attn_decode returns
  *     for it, before the region is looked up.
  *   - Every call on a device shares the one region, and a call leaves its partials there.
