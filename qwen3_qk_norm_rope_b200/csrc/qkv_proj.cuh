@@ -43,7 +43,9 @@ struct QkvParams {
   WaitCfg wait;
 };
 
-constexpr int kQkvThreads = 192;
+// warp 0: TMA producer; warp 1: MMA issuer; warps 2-9: epilogue, two warps per TMEM lane
+// quadrant, one for each of a tile's two heads
+constexpr int kQkvThreads = 320;
 constexpr int kQkvStages = 4;
 constexpr uint32_t kQkA = 16384;                  // 128 tokens x 64 bf16
 constexpr uint32_t kQkB = 32768;                  // 256 columns x 64 bf16
@@ -110,7 +112,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar + kQbAccFull + 8 * b, 1);
-      mbar_init(bar + kQbAccEmpty + 8 * b, 128);
+      mbar_init(bar + kQbAccEmpty + 8 * b, 256);
     }
     mbar_init(bar + kQbDone, 1);
     *abort_flag = 0;
@@ -200,6 +202,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
   } else {
     // ------------------------------------------------------------------ epilogue
     const int wq = warp & 3;
+    const int hh = (warp - 2) >> 2;  // which of the tile's two heads this warp takes
     const int row = wq * 32 + lane;  // token row of the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float* sg = reinterpret_cast<const float*>(sgen + kQkGain);
@@ -213,7 +216,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const long long m = static_cast<long long>(mt) * 128 + row;
-      for (int hh = 0; hh < 2; ++hh) {
+      {
         const int h = nt * 2 + hh;  // head index in [q heads | k heads | v heads]
         uint32_t y[128];
 #pragma unroll
@@ -223,10 +226,9 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) y[c * 32 + i] = r[i];
         }
-        if (hh == 1) {  // both heads are in registers or stored: the accumulator is free
-          tc_fence_before();
-          mbar_arrive(bar + kQbAccEmpty + 8 * buf);
-        }
+        // this head is in registers: once both heads' warps are here the accumulator is free
+        tc_fence_before();
+        mbar_arrive(bar + kQbAccEmpty + 8 * buf);
         if (h >= p.n_heads || m >= p.M) continue;
         uint4* dst;
         if (h < p.Hq + p.Hkv) {
