@@ -187,7 +187,9 @@ int ensure_kernel_attrs() {
                            q3::kDecodeSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           q3::kQkvSmemBytes) != cudaSuccess)
+                           q3::kQkvSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::qkv_proj_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kQkv2SmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   done[dev] = true;
   return QWEN3_OK;
@@ -970,15 +972,6 @@ int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const
     q3::qkv_rope_table_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(rp);
     if (cudaGetLastError() != cudaSuccess) return QWEN3_ERR_CUDA;
   }
-  CUtensorMap mx, mw;
-  {
-    const cuuint64_t xd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(M)};
-    const cuuint64_t xs[1] = {static_cast<cuuint64_t>(hidden) * 2ull};
-    const cuuint32_t xb[2] = {64, 128};
-    const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(n_heads) * kD};
-    const cuuint32_t wb[2] = {64, 256};
-    if (!make_map(&mx, x, 2, xd, xs, xb) || !make_map(&mw, w_qkv, 2, wd, xs, wb)) return QWEN3_ERR_CUDA;
-  }
   q3::QkvParams p;
   p.q_norm_w = q_norm_w;
   p.k_norm_w = k_norm_w;
@@ -999,6 +992,29 @@ int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const
   p.n_k = (hidden + 63) / 64;
   p.eps = eps;
   p.wait = next_wait_cfg();
+  // Two SMs per MMA: tiles of 256 tokens (a pair of 128-token tiles) x 256 columns, one
+  // cluster of two CTAs per SM pair.  Each SM then loads a third less per K chunk, which
+  // pays once a pair's run is long (128 K chunks or more: hidden >= 2048 at 4096 tokens);
+  // on shorter runs the one-SM kernel's shorter ring fill and simpler handoffs win.
+  p.n_mp = (n_mt + 1) / 2;
+  p.n_tiles2 = p.n_mp * p.n_nt;
+  const int pairs = num_sms() / 2;
+  const long long pair_run = pairs >= 1 ? static_cast<long long>((p.n_tiles2 + pairs - 1) / pairs) * p.n_k : 0;
+  const cuuint64_t xd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(M)};
+  const cuuint64_t xs[1] = {static_cast<cuuint64_t>(hidden) * 2ull};
+  const cuuint32_t xb[2] = {64, 128};
+  const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(n_heads) * kD};
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, x, 2, xd, xs, xb)) return QWEN3_ERR_CUDA;
+  if (pair_run >= 128) {
+    const cuuint32_t wb2[2] = {64, 128};  // each CTA of a pair loads half of a column tile
+    if (!make_map(&mw, w_qkv, 2, wd, xs, wb2)) return QWEN3_ERR_CUDA;
+    const int grid2 = 2 * (p.n_tiles2 < pairs ? p.n_tiles2 : pairs);
+    q3::qkv_proj_pair_kernel<<<grid2, q3::kQkvThreads, q3::kQkv2SmemBytes, s>>>(mx, mw, p);
+    if (cudaGetLastError() == cudaSuccess) return QWEN3_OK;
+  }
+  const cuuint32_t wb[2] = {64, 256};
+  if (!make_map(&mw, w_qkv, 2, wd, xs, wb)) return QWEN3_ERR_CUDA;
   const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
   q3::qkv_proj_kernel<<<grid, q3::kQkvThreads, q3::kQkvSmemBytes, s>>>(mx, mw, p);
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;

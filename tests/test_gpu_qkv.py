@@ -60,6 +60,41 @@ def test_qkv_proj_full_size():
     _check(got, ref, shape.name)
 
 
+@pytest.mark.parametrize("M,hidden,Hq,Hkv", [
+    (300, 8192, 4, 2),   # three token tiles: the last pair's second CTA has no rows
+    (200, 8200, 3, 3),   # an odd head count, and hidden off the 64-chunk
+    (2400, 4096, 16, 8),  # three pair tiles per SM pair, 19 token tiles, rows off the tile
+])
+def test_qkv_proj_long_k_runs(M, hidden, Hq, Hkv):
+    """Runs of 128 K chunks or more per SM pair, which the library computes with both SMs of
+    a pair on each MMA (M = 256 rows split across the two CTAs, each holding half of the
+    tile's weight rows)."""
+    shape = QkvShape("qkv long K", M, hidden, Hq, Hkv)
+    got, ref = _run(shape, seed=M + hidden + 1)
+    _check(got, ref, f"M{M} hidden{hidden} Hq{Hq} Hkv{Hkv}")
+
+
+def test_qkv_proj_full_size_4b_sampled_rows():
+    """The 4B-shaped projection (M=8192, hidden=2560, 48 heads) at full size, checked on 640
+    sampled token rows (every row's output depends on that row alone): rows of both CTAs of
+    several SM pairs, the first and the last token tile."""
+    shape = QKV_SHAPES["qwen3-4b-qkv"]
+    inp = qkv_proj_inputs(shape, seed=3)
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items()}
+    q, k, v = qa.qkv_proj_norm_rope(t["x"], t["w_qkv"], t["q_norm_w"], t["k_norm_w"], t["pos"], shape.Hq, shape.Hkv)
+    torch.cuda.synchronize()
+    assert_status_ok()
+    rng = np.random.default_rng(9)
+    rows = np.unique(np.concatenate([np.arange(128), np.arange(shape.M - 128, shape.M),
+                                     rng.choice(shape.M, size=384, replace=False)]))
+    ref = oracle.qkv_proj_norm_rope_ref(as_f64(inp["x"])[rows], as_f64(inp["w_qkv"]), as_f64(inp["q_norm_w"]),
+                                        as_f64(inp["k_norm_w"]), inp["pos"].numpy()[rows], shape.Hq, shape.Hkv,
+                                        THETA, EPS)
+    got = tuple(to_np(a)[rows] for a in (q, k, v))
+    _check(got, ref, shape.name + " (sampled rows)")
+
+
 def test_qkv_proj_rope_variant_and_positions():
     shape = QkvShape("qkv variant", 384, 256, 8, 4)
     i = np.arange(64, dtype=np.float64)
