@@ -466,6 +466,23 @@ void qwen3_attn_set_fault_injection(int flags);
 #define QWEN3_SOFTMAX_RUNNING_MAX 1
 int qwen3_attn_set_softmax_path(int path);
 
+/*
+ * qwen3_attn_set_sm_pairs - test hook choosing how later qkv projections
+ * (qwen3_qkv_proj_norm_rope) use the SMs.  The projection has a variant in which the two
+ * SMs of a pair share every tensor-core MMA (tcgen05 with cta_group::2, a cluster of two
+ * CTAs, each loading its own token rows and half of the tile's weight rows).  It computes
+ * the same results as the one-SM kernel, in the same precision.
+ *   QWEN3_SM_PAIRS_AUTO (0, the default): SM pairs when each pair's run of tiles reaches
+ *       128 K chunks of 64 (hidden >= 2048 at 4096 tokens), one SM per tile otherwise.
+ *   QWEN3_SM_PAIRS_OFF (1): one SM per tile.
+ *   QWEN3_SM_PAIRS_ALWAYS (2): SM pairs whatever the size.
+ * Returns the previous setting, or -1 (nothing changed) for any other value.
+ */
+#define QWEN3_SM_PAIRS_AUTO 0
+#define QWEN3_SM_PAIRS_OFF 1
+#define QWEN3_SM_PAIRS_ALWAYS 2
+int qwen3_attn_set_sm_pairs(int mode);
+
 /* Library version string. */
 const char* qwen3_attn_version(void);
 

@@ -70,6 +70,7 @@ SIGNATURES = {
     "qwen3_attn_set_wait_limit": (_U64, [_U64]),
     "qwen3_attn_set_fault_injection": (None, [_I]),
     "qwen3_attn_set_softmax_path": (_I, [_I]),
+    "qwen3_attn_set_sm_pairs": (_I, [_I]),
     "qwen3_attn_version": (ctypes.c_char_p, []),
 }
 
@@ -562,6 +563,19 @@ def set_softmax_path(path: int) -> int:
     old = int(lib().qwen3_attn_set_softmax_path(int(path)))
     if old < 0:
         raise ValueError(f"unknown softmax path {path}")
+    return old
+
+
+SM_PAIRS_AUTO, SM_PAIRS_OFF, SM_PAIRS_ALWAYS = 0, 1, 2
+
+
+def set_sm_pairs(mode: int) -> int:
+    """Test hook: how later qkv projections use the SMs.  SM_PAIRS_AUTO (the default) pairs
+    SMs on each MMA for long K runs, SM_PAIRS_OFF keeps one SM per tile, SM_PAIRS_ALWAYS
+    pairs them whatever the size.  Returns the previous setting."""
+    old = int(lib().qwen3_attn_set_sm_pairs(int(mode)))
+    if old < 0:
+        raise ValueError(f"unknown SM-pair mode {mode}")
     return old
 
 

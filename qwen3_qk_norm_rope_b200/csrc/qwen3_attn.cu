@@ -47,6 +47,7 @@ uint64_t g_wait_ns = initial_wait_ns();
 uint64_t g_launch_id = 0;
 int g_fault = 0;
 int g_softmax_path = QWEN3_SOFTMAX_AUTO;
+int g_sm_pairs = QWEN3_SM_PAIRS_AUTO;
 std::mutex g_mu;
 
 q3::WaitCfg next_wait_cfg() {
@@ -366,6 +367,14 @@ int qwen3_attn_set_softmax_path(int path) {
   std::lock_guard<std::mutex> lk(g_mu);
   const int old = g_softmax_path;
   g_softmax_path = path;
+  return old;
+}
+
+int qwen3_attn_set_sm_pairs(int mode) {
+  if (mode != QWEN3_SM_PAIRS_AUTO && mode != QWEN3_SM_PAIRS_OFF && mode != QWEN3_SM_PAIRS_ALWAYS) return -1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int old = g_sm_pairs;
+  g_sm_pairs = mode;
   return old;
 }
 
@@ -1000,13 +1009,18 @@ int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const
   p.n_tiles2 = p.n_mp * p.n_nt;
   const int pairs = num_sms() / 2;
   const long long pair_run = pairs >= 1 ? static_cast<long long>((p.n_tiles2 + pairs - 1) / pairs) * p.n_k : 0;
+  int pairs_mode;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    pairs_mode = g_sm_pairs;
+  }
   const cuuint64_t xd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(M)};
   const cuuint64_t xs[1] = {static_cast<cuuint64_t>(hidden) * 2ull};
   const cuuint32_t xb[2] = {64, 128};
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(n_heads) * kD};
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, 2, xd, xs, xb)) return QWEN3_ERR_CUDA;
-  if (pair_run >= 128) {
+  if (pairs >= 1 && pairs_mode != QWEN3_SM_PAIRS_OFF && (pair_run >= 128 || pairs_mode == QWEN3_SM_PAIRS_ALWAYS)) {
     const cuuint32_t wb2[2] = {64, 128};  // each CTA of a pair loads half of a column tile
     if (!make_map(&mw, w_qkv, 2, wd, xs, wb2)) return QWEN3_ERR_CUDA;
     const int grid2 = 2 * (p.n_tiles2 < pairs ? p.n_tiles2 : pairs);

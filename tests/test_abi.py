@@ -361,6 +361,25 @@ def test_softmax_path_hook_returns_the_previous_setting_and_refuses_unknown_valu
         assert qa.set_softmax_path(qa.SOFTMAX_AUTO) == qa.SOFTMAX_RUNNING_MAX
 
 
+def test_sm_pairs_constants_match_the_header():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    vals = {name: int(val) for name, val in re.findall(r"#define\s+(QWEN3_SM_PAIRS_\w+)\s+(\d+)", text)}
+    assert vals == {"QWEN3_SM_PAIRS_AUTO": qa.SM_PAIRS_AUTO, "QWEN3_SM_PAIRS_OFF": qa.SM_PAIRS_OFF,
+                    "QWEN3_SM_PAIRS_ALWAYS": qa.SM_PAIRS_ALWAYS}
+
+
+def test_sm_pairs_hook_returns_the_previous_setting_and_refuses_unknown_values():
+    """Host-side only: the hook records the setting for later qkv projections."""
+    assert qa.set_sm_pairs(qa.SM_PAIRS_OFF) == qa.SM_PAIRS_AUTO
+    try:
+        assert qa.set_sm_pairs(qa.SM_PAIRS_ALWAYS) == qa.SM_PAIRS_OFF
+        with pytest.raises(ValueError):
+            qa.set_sm_pairs(3)
+        assert qa.lib().qwen3_attn_set_sm_pairs(-1) == -1
+    finally:
+        assert qa.set_sm_pairs(qa.SM_PAIRS_AUTO) == qa.SM_PAIRS_ALWAYS
+
+
 def test_noalloc_region_limit():
     """The no-allocation decode's fixed region (48 MiB) holds the split-KV partials of up to
     92 sequences of 32 heads at Lmax 32769, the batched-decode workload's 64 among them."""

@@ -43,12 +43,23 @@ def _check(got, ref, what):
         assert err.mean() <= 2.0 ** -9 * np.mean(np.abs(r)) + 1e-4 * rms, f"{what} {name}: mean {err.mean():.3e}"
 
 
+@pytest.fixture
+def sm_pairs(request):
+    """The SM-pair setting for the test (the default rule, or one kernel forced), restored after."""
+    old = qa.set_sm_pairs(request.param)
+    yield request.param
+    qa.set_sm_pairs(old)
+
+
+@pytest.mark.parametrize("sm_pairs", [qa.SM_PAIRS_AUTO, qa.SM_PAIRS_ALWAYS], indirect=True, ids=["auto", "pairs"])
 @pytest.mark.parametrize("M,hidden,Hq,Hkv", [
     (300, 256, 4, 2),    # M off the 128-row tile, hidden a few chunks
     (128, 200, 3, 3),    # an odd head count (the last tile holds one head), hidden off the 64-chunk
     (1000, 512, 16, 8),  # several token tiles per CTA run
 ])
-def test_qkv_proj_small(M, hidden, Hq, Hkv):
+def test_qkv_proj_small(M, hidden, Hq, Hkv, sm_pairs):
+    """Short K runs take the one-SM kernel by default; forced, the SM-pair kernel on the same
+    shapes (a single token tile, whose pair partner has no rows; an odd head count)."""
     shape = QkvShape("qkv small", M, hidden, Hq, Hkv)
     got, ref = _run(shape, seed=M + hidden)
     _check(got, ref, f"M{M} hidden{hidden} Hq{Hq} Hkv{Hkv}")
@@ -65,10 +76,11 @@ def test_qkv_proj_full_size():
     (200, 8200, 3, 3),   # an odd head count, and hidden off the 64-chunk
     (2400, 4096, 16, 8),  # three pair tiles per SM pair, 19 token tiles, rows off the tile
 ])
-def test_qkv_proj_long_k_runs(M, hidden, Hq, Hkv):
-    """Runs of 128 K chunks or more per SM pair, which the library computes with both SMs of
-    a pair on each MMA (M = 256 rows split across the two CTAs, each holding half of the
-    tile's weight rows)."""
+@pytest.mark.parametrize("sm_pairs", [qa.SM_PAIRS_AUTO, qa.SM_PAIRS_OFF], indirect=True, ids=["auto", "one-sm"])
+def test_qkv_proj_long_k_runs(M, hidden, Hq, Hkv, sm_pairs):
+    """Runs of 128 K chunks or more per SM pair, which the library computes by default with
+    both SMs of a pair on each MMA (M = 256 rows split across the two CTAs, each holding half
+    of the tile's weight rows); forced, the one-SM kernel on the same shapes."""
     shape = QkvShape("qkv long K", M, hidden, Hq, Hkv)
     got, ref = _run(shape, seed=M + hidden + 1)
     _check(got, ref, f"M{M} hidden{hidden} Hq{Hq} Hkv{Hkv}")
