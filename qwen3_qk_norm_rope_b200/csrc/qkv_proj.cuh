@@ -26,7 +26,9 @@
 //              RoPE table ([64][128] float2, 64 KB, built by qkv_rope_table_kernel): for one
 //              frequency the 32 rows of a warp are one coalesced 256-byte read, and the
 //              table stays in L2 for all the tile's column tiles.  Left out of shared
-//              memory, it leaves room for a fourth stage.
+//              memory, it leaves room for a fourth stage.  The GEMM is a programmatic
+//              dependent launch after the table kernel: its loads and MMAs start at once,
+//              and only the epilogue warps wait for the table (griddep_wait).
 //
 // qkv_proj_pair_kernel is the same GEMM on SM pairs (tcgen05 cta_group::2): a cluster of two
 // CTAs computes a 256-token x 256-column tile with M=256 MMAs, each CTA loading its own 128
@@ -78,6 +80,9 @@ struct QkvRopeParams {
 };
 
 __global__ void __launch_bounds__(256) qkv_rope_table_kernel(const __grid_constant__ QkvRopeParams p) {
+  // The projection launched next may start now: only its epilogue reads this table, and it
+  // waits for this grid first (griddep_wait).
+  griddep_launch_dependents();
   const long long total = static_cast<long long>(p.n_mt) * 64 * 128;
   for (long long e = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
        e += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(kQkvThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue
+    griddep_wait();  // the RoPE table, written by the kernel launched before this one
     const int wq = warp & 3;
     const int hh = (warp - 2) >> 2;  // which of the tile's two heads this warp takes
     const int row = wq * 32 + lane;  // token row of the tile = TMEM lane
@@ -487,6 +493,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kQkvThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
+    griddep_wait();  // the RoPE table, written by the kernel launched before this one
     const int wq = warp & 3;
     const int hh = (warp - 2) >> 2;  // which of the tile's two heads this warp takes
     const int row = wq * 32 + lane;  // token row of this CTA's tile = TMEM lane

@@ -1020,17 +1020,35 @@ int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv, const
   const cuuint64_t wd[2] = {static_cast<cuuint64_t>(hidden), static_cast<cuuint64_t>(n_heads) * kD};
   CUtensorMap mx, mw;
   if (!make_map(&mx, x, 2, xd, xs, xb)) return QWEN3_ERR_CUDA;
+  // The GEMM is a programmatic dependent launch after the RoPE-table kernel: everything
+  // before that kernel has completed once it starts, and the GEMM reads the table only
+  // after griddep_wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(q3::kQkvThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (pairs >= 1 && pairs_mode != QWEN3_SM_PAIRS_OFF && (pair_run >= 128 || pairs_mode == QWEN3_SM_PAIRS_ALWAYS)) {
     const cuuint32_t wb2[2] = {64, 128};  // each CTA of a pair loads half of a column tile
     if (!make_map(&mw, w_qkv, 2, wd, xs, wb2)) return QWEN3_ERR_CUDA;
-    const int grid2 = 2 * (p.n_tiles2 < pairs ? p.n_tiles2 : pairs);
-    q3::qkv_proj_pair_kernel<<<grid2, q3::kQkvThreads, q3::kQkv2SmemBytes, s>>>(mx, mw, p);
-    if (cudaGetLastError() == cudaSuccess) return QWEN3_OK;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (p.n_tiles2 < pairs ? p.n_tiles2 : pairs)));
+    cfg.dynamicSmemBytes = q3::kQkv2SmemBytes;
+    if (cudaLaunchKernelEx(&cfg, q3::qkv_proj_pair_kernel, mx, mw, p) == cudaSuccess &&
+        cudaGetLastError() == cudaSuccess)
+      return QWEN3_OK;
+    (void)cudaGetLastError();
   }
   const cuuint32_t wb[2] = {64, 256};
   if (!make_map(&mw, w_qkv, 2, wd, xs, wb)) return QWEN3_ERR_CUDA;
-  const int grid = static_cast<int>(n_tiles < num_sms() ? n_tiles : num_sms());
-  q3::qkv_proj_kernel<<<grid, q3::kQkvThreads, q3::kQkvSmemBytes, s>>>(mx, mw, p);
+  cfg.gridDim = dim3(static_cast<unsigned>(n_tiles < num_sms() ? n_tiles : num_sms()));
+  cfg.dynamicSmemBytes = q3::kQkvSmemBytes;
+  if (cudaLaunchKernelEx(&cfg, q3::qkv_proj_kernel, mx, mw, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return QWEN3_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? QWEN3_OK : QWEN3_ERR_CUDA;
 }
 
