@@ -56,6 +56,7 @@ def sm_pairs(request):
     (300, 256, 4, 2),    # M off the 128-row tile, hidden a few chunks
     (128, 200, 3, 3),    # an odd head count (the last tile holds one head), hidden off the 64-chunk
     (1000, 512, 16, 8),  # several token tiles per CTA run
+    (1, 64, 1, 1),       # one token, one head of each kind, one K chunk
 ])
 def test_qkv_proj_small(M, hidden, Hq, Hkv, sm_pairs):
     """Short K runs take the one-SM kernel by default; forced, the SM-pair kernel on the same
@@ -84,6 +85,27 @@ def test_qkv_proj_long_k_runs(M, hidden, Hq, Hkv, sm_pairs):
     shape = QkvShape("qkv long K", M, hidden, Hq, Hkv)
     got, ref = _run(shape, seed=M + hidden + 1)
     _check(got, ref, f"M{M} hidden{hidden} Hq{Hq} Hkv{Hkv}")
+
+
+@pytest.mark.parametrize("M,hidden,Hq,Hkv", [(300, 2048, 4, 2), (4096, 1024, 16, 8)])
+def test_qkv_proj_sm_pair_and_one_sm_kernels_agree_bit_for_bit(M, hidden, Hq, Hkv):
+    """Both kernels multiply the same bf16 operands in the same K order into fp32 and apply
+    the same epilogue, so they must return identical bits."""
+    shape = QkvShape("qkv kernels", M, hidden, Hq, Hkv)
+    inp = qkv_proj_inputs(shape, seed=17)
+    d = dev()
+    t = {k: v.to(d) for k, v in inp.items()}
+    res = {}
+    for mode in (qa.SM_PAIRS_OFF, qa.SM_PAIRS_ALWAYS):
+        old = qa.set_sm_pairs(mode)
+        try:
+            res[mode] = qa.qkv_proj_norm_rope(t["x"], t["w_qkv"], t["q_norm_w"], t["k_norm_w"], t["pos"], Hq, Hkv)
+            torch.cuda.synchronize()
+            assert_status_ok()
+        finally:
+            qa.set_sm_pairs(old)
+    for name, a, b in zip("qkv", res[qa.SM_PAIRS_OFF], res[qa.SM_PAIRS_ALWAYS]):
+        assert torch.equal(a, b), f"{name}: max diff {(a.float() - b.float()).abs().max().item():.3e}"
 
 
 def test_qkv_proj_full_size_4b_sampled_rows():
