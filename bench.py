@@ -86,8 +86,8 @@ def decode_bytes(lens: np.ndarray, Hq: int, Hkv: int, d: int = 128) -> int:
 # DRAM traffic of the decode split-KV kernel per cached token (dram__bytes_read.sum +
 # dram__bytes_write.sum of one ncu capture of a smaller case, divided by its cached tokens),
 # valid only for the kernel source it was measured on.  Refreshed with each new capture.
-DECODE_TRAFFIC = {"src_sha256": "e9ed9214854a024560e1affa2f7c6a31576ecbae86d27716a02ecffc6b4527b9",
-                  "bytes_per_cached_token": (630.648576e6 + 5.422592e6) / 153639}
+DECODE_TRAFFIC = {"src_sha256": "9c02d49265cc31c08af603737c19fb9d763c26ee719b5caaedf0dad97588df61",
+                  "bytes_per_cached_token": (630.657280e6 + 5.152512e6) / 153639}
 
 
 def decode_src_sha256() -> str:

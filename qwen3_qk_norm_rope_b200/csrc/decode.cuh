@@ -10,9 +10,9 @@
 // Split kernel: one CTA per (split of `split` keys, KV head, sequence); CTAs past a
 // sequence's end exit at once, so the host never needs the lengths.  It is a programmatic
 // dependent launch after the append: only the chunk holding slot L waits for the append's
-// results (griddepcontrol.wait); the rest of the cache was written by earlier calls.  Warp 4 streams 64-key
-// chunks of K and V (two 64x64 128B-swizzled TMA boxes each) into a 3-stage ring.  Warps
-// 0-3 each take 16 keys of every chunk: S = q'K^T and O += P V as mma.sync m16n8k16 (rows =
+// results (griddepcontrol.wait); the rest of the cache was written by earlier calls.  Warp 4
+// streams 64-key chunks of K and V (two 64x64 128B-swizzled TMA boxes each, or per page for
+// smaller pages) into a 3-stage ring.  Warps 0-3 each take 16 keys of every chunk: S = q'K^T and O += P V as mma.sync m16n8k16 (rows =
 // the G <= 16 query heads of the group), an exp2 online softmax in registers, then the four
 // warps merge their (max, sum, O) and write the split's normalised O and its LSE.
 // The work per key is 4*G*d flops against 4*d bytes, so this path is bound by HBM
@@ -77,7 +77,26 @@ __device__ __forceinline__ float ex2d(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// A chunk of K (or V) in shared memory: key r's two 64-dim halves are the 128-byte lines
+// 2r and 2r+1, as one TMA box {64 dims, 2 halves, keys} writes them, 128B-swizzled (the
+// 16-byte piece c of line l sits at piece c ^ (l mod 8)).
+__device__ __forceinline__ uint32_t dc_line_offset(uint32_t row, uint32_t half, uint32_t piece) {
+  const uint32_t l = 2u * row + half;
+  return l * 128u + ((piece ^ (l & 7u)) << 4);
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(m), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 
+// kLines: the chunk layout of pages under 64 keys, where one TMA box per page brings both
+// 64-dim halves of its keys (key r's halves are the 128-byte lines 2r and 2r+1), half as
+// many boxes as one per half.  Otherwise each half is its own 64-key plane, one box each:
+// its ldmatrix reads are free of bank conflicts, which the interleaved lines are not.
+template <bool kLines>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ DecodeParams p) {
@@ -171,11 +190,17 @@ __global__ void __launch_bounds__(kDecodeThreads)
           mbar_arrive_expect_tx(fb, bytes);
           for (int i = 0; i < nb; ++i) {
             if (rows[i] < 0) continue;
-            const uint32_t off = static_cast<uint32_t>(i * br) * 128u;
-            tma_load_2d(dst + off, &tmK, fb, 0, rows[i]);
-            tma_load_2d(dst + kDcBox + off, &tmK, fb, 64, rows[i]);
-            tma_load_2d(dst + kDcChunk + off, &tmV, fb, 0, rows[i]);
-            tma_load_2d(dst + kDcChunk + kDcBox + off, &tmV, fb, 64, rows[i]);
+            if constexpr (kLines) {
+              const uint32_t off = static_cast<uint32_t>(i * br) * 256u;  // br keys of both halves
+              tma_load_3d(dst + off, &tmK, fb, 0, 0, rows[i]);
+              tma_load_3d(dst + kDcChunk + off, &tmV, fb, 0, 0, rows[i]);
+            } else {
+              const uint32_t off = static_cast<uint32_t>(i * br) * 128u;
+              tma_load_2d(dst + off, &tmK, fb, 0, rows[i]);
+              tma_load_2d(dst + kDcBox + off, &tmK, fb, 64, rows[i]);
+              tma_load_2d(dst + kDcChunk + off, &tmV, fb, 0, rows[i]);
+              tma_load_2d(dst + kDcChunk + kDcBox + off, &tmV, fb, 64, rows[i]);
+            }
           }
         }
         last[st] = u;
@@ -249,9 +274,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         // Slots past the sequence hold stale cache contents: zero their V rows so that
         // P = 0 never meets a non-finite value in P.V.
         for (int t = valid + (lane >> 3); t < 16; t += 4) {
-          const uint32_t rowoff = static_cast<uint32_t>(tw + t) * 128u + (lane & 7) * 16u;
+          const uint32_t rowoff = static_cast<uint32_t>(tw + t) * (kLines ? 256u : 128u) + (lane & 7) * 16u;
           st_shared_v4(sVc + rowoff, 0u, 0u, 0u, 0u);
-          st_shared_v4(sVc + kDcBox + rowoff, 0u, 0u, 0u, 0u);
+          st_shared_v4(sVc + (kLines ? 128u : kDcBox) + rowoff, 0u, 0u, 0u, 0u);
         }
         __syncwarp();
       }
@@ -263,7 +288,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const uint32_t tok = tw + ((mi >> 1) << 3) + mr;
         const uint32_t chunk = ((kk & 3) << 1) + (mi & 1);
         uint32_t b0, b1, b2, b3;
-        ldsm_x4(sKc + (kk >> 2) * kDcBox + sw128_offset(tok, chunk), b0, b1, b2, b3);
+        ldsm_x4(sKc + (kLines ? dc_line_offset(tok, kk >> 2, chunk) : (kk >> 2) * kDcBox + sw128_offset(tok, chunk)),
+                b0, b1, b2, b3);
         mma_bf16_16816(sa, qa[kk], b0, b1);
         mma_bf16_16816(sbk, qa[kk], b2, b3);
       }
@@ -316,7 +342,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
         const uint32_t tok = tw + ((mi & 1) << 3) + mr;
         const uint32_t chunk = ((nb2 & 3) << 1) + (mi >> 1);
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sVc + (nb2 >> 2) * kDcBox + sw128_offset(tok, chunk), b0, b1, b2, b3);
+        ldsm_x4_t(
+            sVc + (kLines ? dc_line_offset(tok, nb2 >> 2, chunk) : (nb2 >> 2) * kDcBox + sw128_offset(tok, chunk)), b0,
+            b1, b2, b3);
         mma_bf16_16816(o[2 * nb2], pa, b0, b1);
         mma_bf16_16816(o[2 * nb2 + 1], pa, b2, b3);
       }

@@ -184,7 +184,9 @@ int ensure_kernel_attrs() {
       cudaFuncSetAttribute(q3::fmha_prefill_kernel<false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kPrefillSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
-  if (cudaFuncSetAttribute(q3::decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(q3::decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           q3::kDecodeSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(q3::decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            q3::kDecodeSmemBytes) != cudaSuccess)
     return QWEN3_ERR_CUDA;
   if (cudaFuncSetAttribute(q3::qkv_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -820,10 +822,22 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   CUtensorMap mk, mv;
   const cuuint64_t rows = pg != nullptr ? static_cast<cuuint64_t>(pg->num_pages) * Hkv * pg->page
                                         : static_cast<cuuint64_t>(N) * Hkv * Lmax;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
-  const cuuint64_t str[1] = {kD * 2ull};
-  const cuuint32_t box[2] = {64, pg != nullptr ? static_cast<cuuint32_t>(std::min(pg->page, 64)) : 64u};
-  if (!make_map(&mk, k_cache, 2, dims, str, box) || !make_map(&mv, v_cache, 2, dims, str, box)) return QWEN3_ERR_CUDA;
+  // Pages under 64 keys: rows of d viewed as two 64-dim halves, so that one box {64, 2, page}
+  // brings a page's keys with both halves.  Otherwise boxes of {64 dims, 64 keys or a page}.
+  const bool lines = pg != nullptr && pg->page < 64;
+  if (lines) {
+    const cuuint64_t dims[3] = {64, 2, rows};
+    const cuuint64_t str[2] = {128, kD * 2ull};
+    const cuuint32_t box[3] = {64, 2, static_cast<cuuint32_t>(pg->page)};
+    if (!make_map(&mk, k_cache, 3, dims, str, box) || !make_map(&mv, v_cache, 3, dims, str, box))
+      return QWEN3_ERR_CUDA;
+  } else {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kD), rows};
+    const cuuint64_t str[1] = {kD * 2ull};
+    const cuuint32_t box[2] = {64, pg != nullptr ? static_cast<cuuint32_t>(std::min(pg->page, 64)) : 64u};
+    if (!make_map(&mk, k_cache, 2, dims, str, box) || !make_map(&mv, v_cache, 2, dims, str, box))
+      return QWEN3_ERR_CUDA;
+  }
   q3::DecodeParams p;
   p.q = reinterpret_cast<const uint32_t*>(q);
   p.q_norm_w = q_norm_w;
@@ -859,7 +873,8 @@ int decode_impl(const qwen3_bf16* q, const qwen3_bf16* k_new, const qwen3_bf16* 
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, q3::decode_split_kernel, mk, mv, p) != cudaSuccess) {
+  if ((lines ? cudaLaunchKernelEx(&cfg, q3::decode_split_kernel<true>, mk, mv, p)
+             : cudaLaunchKernelEx(&cfg, q3::decode_split_kernel<false>, mk, mv, p)) != cudaSuccess) {
     (void)cudaGetLastError();
     return QWEN3_ERR_CUDA;
   }
