@@ -361,6 +361,34 @@ def test_softmax_path_hook_returns_the_previous_setting_and_refuses_unknown_valu
         assert qa.set_softmax_path(qa.SOFTMAX_AUTO) == qa.SOFTMAX_RUNNING_MAX
 
 
+def test_qkv_projection_argument_checks():
+    """Host-side only: every call fails a check made before any device work."""
+    var, _ = qa.make_variant()
+
+    def qkv(**kw):
+        a = dict(x=FAKE, w=FAKE, gq=FAKE, gk=FAKE, pos=FAKE, qo=FAKE, ko=FAKE, vo=FAKE, M=300, hidden=256, Hq=4,
+                 Hkv=2, d=128, var=ctypes.byref(var), eps=1e-6, ws=FAKE, ws_bytes=0)
+        a.update(kw)
+        return qa.lib().qwen3_qkv_proj_norm_rope(a["x"], a["w"], a["gq"], a["gk"], a["pos"], a["qo"], a["ko"],
+                                                  a["vo"], a["M"], a["hidden"], a["Hq"], a["Hkv"], a["d"],
+                                                  a["var"], a["eps"], a["ws"], a["ws_bytes"], None)
+
+    need = qa.qkv_proj_workspace_size(300)
+    assert need >= ((300 + 127) // 128) * 64 * 128 * 8  # the RoPE table, (cos, sin) per row and frequency
+    assert qkv(ws_bytes=need - 1) == qa.ERR_WORKSPACE  # every other argument passes its checks
+    assert qkv(ws=None, ws_bytes=need) == qa.ERR_WORKSPACE
+    assert qkv(x=None, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qkv(vo=None, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qkv(var=None, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qkv(M=0, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qkv(Hkv=0, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qkv(d=64, ws_bytes=need) == qa.ERR_UNSUPPORTED
+    assert qkv(hidden=100, ws_bytes=need) == qa.ERR_UNSUPPORTED  # rows must be 16-byte multiples for TMA
+    assert qkv(x=ctypes.c_void_p((1 << 20) + 8), ws_bytes=need) == qa.ERR_INVALID_ARG  # misaligned
+    assert qkv(eps=-1.0, ws_bytes=need) == qa.ERR_INVALID_ARG
+    assert qa.qkv_proj_workspace_size(0) == 0
+
+
 def test_sm_pairs_constants_match_the_header():
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
     vals = {name: int(val) for name, val in re.findall(r"#define\s+(QWEN3_SM_PAIRS_\w+)\s+(\d+)", text)}
