@@ -450,11 +450,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kQkvThreads, 1)
         }
       }
       // The leader's barriers count both CTAs' copies: once they complete, nothing either
-      // CTA issued is still in flight.
-      if (leader)
+      // CTA issued is still in flight.  After an abort the odd CTA may have issued a few
+      // copies beyond the leader's last phase; it gives them a bounded pause to land.
+      if (leader) {
         for (int s = 0; s < kQk2Stages; ++s)
           if (last[s] >= 0)
             mbar_wait(bar + kQ2Full + 8 * s, (last[s] / kQk2Stages) & 1, p.wait, nullptr, kSiteQkvDrain);
+      } else if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 50000u) {
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer (leader)
