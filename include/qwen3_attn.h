@@ -392,6 +392,13 @@ size_t qwen3_attn_prefill_varlen_workspace_size(int B, int N, long long key_cap,
  *             tokens), else QWEN3_ERR_WORKSPACE.
  * q_out and k_out are the normed, rotated vectors the attention entry points compute
  * themselves from raw q and k.
+ * All pointers are device pointers the caller owns: x, w_qkv and the outputs 16-byte
+ * aligned, the gains 8-byte, pos 4-byte.  The call is asynchronous on `stream` (two
+ * launches: the RoPE table, then the GEMM, on one SM per tile or, for long K runs, on SM
+ * pairs; see qwen3_attn_set_sm_pairs).  Errors: QWEN3_ERR_INVALID_ARG for a null pointer,
+ * a non-positive size, a misaligned pointer, eps < 0 or an invalid variant;
+ * QWEN3_ERR_UNSUPPORTED for d != 128, hidden not a multiple of 8 or sizes past the 32-bit
+ * index range; QWEN3_ERR_WORKSPACE as above; QWEN3_ERR_CUDA when a launch fails.
  */
 int qwen3_qkv_proj_norm_rope(const qwen3_bf16* x, const qwen3_bf16* w_qkv,
                              const float* q_norm_w, const float* k_norm_w, const int32_t* pos,
