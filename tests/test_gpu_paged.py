@@ -37,7 +37,7 @@ def _scatter(pool, table_row, keys, page):
         pool[int(table_row[j // page]), :, j % page] = keys[:, j]
 
 
-@pytest.mark.parametrize("page,window", [(16, 0), (64, 0), (256, 0), (128, 700)])
+@pytest.mark.parametrize("page,window", [(16, 0), (32, 0), (64, 0), (256, 0), (128, 700), (16, 700)])
 def test_decode_paged(page, window):
     shape = DecodeShape("paged decode", 5, 32, 8)
     lens = [3000, page - 1, 1023, 4095, 100]
@@ -97,11 +97,13 @@ def test_decode_paged(page, window):
     assert torch.equal(va.view(torch.int16)[mask], before_v.view(torch.int16)[mask])
 
 
-def test_decode_paged_equals_contiguous():
-    """The same caches, once contiguous and once in pages, give the same bits."""
+@pytest.mark.parametrize("page", [64, 16])
+def test_decode_paged_equals_contiguous(page):
+    """The same caches, once contiguous and once in pages, give the same bits (pages under
+    64 keys are read one box per page for both 64-dim halves, larger ones a box per half)."""
     shape = DecodeShape("paged vs contiguous", 3, 32, 8)
     lens = [2500, 64, 1000]
-    page, Lmax = 64, 2560
+    Lmax = 2560
     max_blocks = Lmax // page
     blocks = [(L + 1 + page - 1) // page for L in lens]
     table, _ = _tables(3, blocks, max_blocks, sum(blocks), seed=9)
